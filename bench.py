@@ -1,0 +1,436 @@
+"""Benchmark of the neighbor-rebuild hot path on B200.
+
+One step = one pass of the whole path over the 10.24M-atom salt solution
+(rc 5.75 A, skin 0.5 A, 160 neighbors per row, 64 features):
+    Hilbert sort -> neighbor list (padded) -> skin check -> edge aggregation
+with every input resident in HBM when the timed region starts.  The value is
+atoms per second over all ranks (weak scaling: with --gpus N each rank runs
+an independent replica of the same workload, there is no collective in the
+data path).
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle
+instead (a deliberately plain program, on the host cores, on a bounded
+sample of the workload).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "atoms/s for full neighbor rebuild at 10.24M atoms (1 B200); % of HBM roofline"
+WORKLOAD_CFG = 4
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock samples during the timed region."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self._stop = threading.Event()
+        self._proc = None
+
+    def __enter__(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self._proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + q,
+                                           "--format=csv,noheader,nounits", "-lms", "100"],
+                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except (OSError, FileNotFoundError):
+            self._proc = None
+        return self
+
+    def _read(self):
+        for line in self._proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 7:
+                self.samples.append(parts)
+
+    def __exit__(self, *a):
+        if self._proc is not None:
+            self._proc.terminate()
+            try:
+                self._proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self._proc.kill()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for s in self.samples for k in range(4) if s[3 + k].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+def _dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, world: int, device=None) -> float:
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- CUDA arm
+
+
+class Step:
+    """All device buffers of one replica and the step itself, through the C ABI."""
+
+    def __init__(self, s, device, pad_fill=True):
+        import torch
+        import space_filling_curve_b200 as tess
+        self.tess = tess
+        self.s = s
+        self.n = s.n
+        self.box = s.box
+        self.dev = device
+        n, cap, F = s.n, s.cap, s.F
+        self.pos3 = torch.from_numpy(s.pos).to(device)
+        self.ws_sort = torch.empty(tess.tess_hilbert_sort_workspace(n), dtype=torch.uint8, device=device)
+        self.ws_nbr = torch.empty(tess.tess_build_neighbors_workspace(n, s.box, s.rc, s.skin), dtype=torch.uint8,
+                                  device=device)
+        self.perm = torch.empty(n, dtype=torch.int32, device=device)
+        self.keys = torch.empty(n, dtype=torch.int32, device=device)
+        self.pos_sorted = torch.empty((n, 4), dtype=torch.float32, device=device)
+        self.status = torch.empty(1, dtype=torch.int32, device=device)
+        self.nbr = torch.empty((n, cap), dtype=torch.int32, device=device)
+        self.counts = torch.empty(n, dtype=torch.int32, device=device)
+        self.overflow = torch.empty(1, dtype=torch.int32, device=device)
+        self.rebuild = torch.empty(1, dtype=torch.int32, device=device)
+        self.maxd = torch.empty(1, dtype=torch.float64, device=device)
+        g = torch.Generator(device=device)
+        g.manual_seed(s.seed)
+        # features live in the sorted index space (produced there by the model)
+        self.feat = torch.randn((n, F), generator=g, device=device, dtype=torch.float32)
+        self.out = torch.empty((n, F), dtype=torch.float32, device=device)
+        self.pad_fill = pad_fill
+        # the next frame of the trajectory, in the sorted order of frame 0
+        t1 = next(iter(s.trajectory(1, condition=False)))[1]
+        self.frame1 = torch.from_numpy(t1).to(device)
+        self.pos_next = torch.empty((n, 4), dtype=torch.float32, device=device)
+        self.run()
+        torch.cuda.synchronize()
+        self.pos_next.zero_()
+        self.pos_next[:, :3] = self.frame1[self.perm.long()]
+        torch.cuda.synchronize()
+
+    def run(self):
+        import ctypes
+        tess = self.tess
+        P = lambda t: ctypes.c_void_p(t.data_ptr())
+        import torch
+        st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        s = self.s
+        c = tess.tess_hilbert_sort(P(self.pos3), self.n, s.box, 10, P(self.ws_sort), self.ws_sort.numel(),
+                                   P(self.perm), P(self.keys), P(self.pos_sorted), P(self.status), st)
+        assert c == 0, c
+        c = tess.tess_build_neighbors(P(self.pos_sorted), self.n, s.box, s.rc, s.skin, s.cap,
+                                      0 if self.pad_fill else tess.TESS_NO_PAD_FILL, P(self.ws_nbr),
+                                      self.ws_nbr.numel(), P(self.nbr), P(self.counts), P(self.overflow), st)
+        assert c == 0, c
+        c = tess.tess_skin_check(P(self.pos_next), P(self.pos_sorted), self.n, s.box, s.skin, P(self.rebuild),
+                                 P(self.maxd), st)
+        assert c == 0, c
+        c = tess.tess_edge_aggregate(P(self.pos_sorted), self.n, s.box, s.rc, P(self.nbr), P(self.counts), s.cap,
+                                     P(self.feat), s.F, P(self.out), None, None, None, st)
+        assert c == 0, c
+
+
+def _algorithmic_bytes(n, mean_count, F):
+    """Minimum bytes each stage must move (per launch), from the per-atom
+    figures of the design notes."""
+    return {
+        "hilbert_keys": n * (16 + 8),
+        "key_sort": n * 12,
+        "cell_binning": n * 28,
+        "pair_search": n * (16 + 4 * mean_count + 4),
+        "skin_check": n * 32,
+        "edge_aggregate": n * (4 * F + 4 * F + 16 + 4 * mean_count + 4),
+    }
+
+
+def run_cuda(args, world, rank, local):
+    import torch
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    import synth
+    import space_filling_curve_b200 as tess
+    s = synth.system(args.config)
+    step = Step(s, dev, pad_fill=not args.no_pad_fill)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step.run()
+    torch.cuda.synchronize()
+    ov = int(step.overflow.item())
+    counts = step.counts
+    mean_count = float(counts.double().mean().item())
+    pairs = float(counts.double().sum().item())
+
+    launches0 = tess.tess_kernel_launch_count()
+    tess.tess_stage_times()          # clear
+    tess.tess_stage_timing(True)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for k in range(args.steps):
+            flush.zero_()
+            evs[k][0].record()
+            step.run()
+            evs[k][1].record()
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    tess.tess_stage_timing(False)
+    stages = tess.tess_stage_times()
+    launches = tess.tess_kernel_launch_count() - launches0
+    ms = sum(a.elapsed_time(b) for a, b in evs)
+    ms_max = max_over_ranks(ms, world, dev)
+    n_total = sum_over_ranks(float(s.n * args.steps), world, dev)
+    value = n_total / (ms_max / 1e3)
+
+    # e2e: through the C ABI with host buffers (pinned), copies inside the timed region
+    host_pos = torch.from_numpy(s.pos).pin_memory()
+    host_perm = torch.empty(s.n, dtype=torch.int32).pin_memory()
+    host_counts = torch.empty(s.n, dtype=torch.int32).pin_memory()
+    host_flags = torch.empty(2, dtype=torch.int32).pin_memory()
+    flags_d = torch.empty(2, dtype=torch.int32, device=dev)
+    e2e_steps = max(1, min(args.steps, 5))
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        step.pos3.copy_(host_pos, non_blocking=True)
+        step.run()
+        flags_d[0:1].copy_(step.overflow)
+        flags_d[1:2].copy_(step.rebuild)
+        host_perm.copy_(step.perm, non_blocking=True)
+        host_counts.copy_(step.counts, non_blocking=True)
+        host_flags.copy_(flags_d, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_val = sum_over_ranks(float(s.n * e2e_steps), world, dev) / (e2e_ms / 1e3)
+
+    peak, peak_kind = _peaks()
+    nbytes = _algorithmic_bytes(s.n, mean_count, s.F)
+    stage_ms = {k: (v[0] / max(v[1], 1)) for k, v in stages.items() if v[1] > 0}
+    dom = max(stage_ms, key=stage_ms.get)
+    achieved = nbytes[dom] / (stage_ms[dom] / 1e3) / 1e9
+    traffic = _traffic_from_profile(dom)
+    clocks = clk.summary()
+
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": value,
+            "unit": "atoms/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_max / args.steps,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic (seeded salt-solution generator; no dataset)",
+            "config": {
+                "workload": "salt-10.24M: %d atoms, box %.3f A cubic, rc %.2f, skin %.2f, cap %d, F %d; step = "
+                            "hilbert_sort + build_neighbors (pad-filled) + skin_check + edge_aggregate"
+                            % (s.n, s.box[0], s.rc, s.skin, s.cap, s.F),
+                "atoms": s.n,
+                "pad_fill": not args.no_pad_fill,
+                "l2": "flushed between timed steps (256 MB write); each step also moves ~9 GB",
+                "parallelism": "replicas (no collective in the data path)",
+                "mean_neighbors": mean_count,
+                "pairs_listed": pairs,
+                "overflow": ov,
+            },
+            "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+            "rebuild_atoms_per_s": s.n / ((stage_ms.get("hilbert_keys", 0) + stage_ms.get("key_sort", 0)
+                                           + stage_ms.get("cell_binning", 0) + stage_ms.get("pair_search", 0)) / 1e3),
+            "pairs_per_s": pairs / (stage_ms.get("pair_search", float("nan")) / 1e3),
+            "roofline": {
+                "bound": "hbm",
+                "kernel": dom,
+                "achieved": achieved,
+                "peak": peak,
+                "peak_kind": peak_kind,
+                "unit": "GB/s",
+                "frac": achieved / peak,
+                "traffic": traffic,
+                "algorithmic_bytes": nbytes[dom],
+            },
+            "rebuild_roofline": _rebuild_roofline(s.n, mean_count, stage_ms, peak),
+            "e2e": {"value": e2e_val, "unit": "atoms/s", "steps": e2e_steps, "h2d_bytes_per_step": s.n * 12,
+                    "d2h_bytes_per_step": s.n * 8 + 8},
+            "gpu_launches": launches,
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(args)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def _rebuild_roofline(n, mean_count, stage_ms, peak):
+    t = sum(stage_ms.get(k, 0.0) for k in ("hilbert_keys", "key_sort", "cell_binning", "pair_search"))
+    b = n * (24 + 12 + 36 + 28 + 16 + 4 * mean_count + 4)
+    return {"ms": t, "algorithmic_bytes": b, "achieved_gbs": b / (t / 1e3) / 1e9 if t else None,
+            "frac": (b / (t / 1e3) / 1e9) / peak if t else None}
+
+
+def _traffic_from_profile(kernel_stage):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary (profiles/<stage>_traffic.json), or None."""
+    path = os.path.join(ROOT, "profiles", "%s_traffic.json" % kernel_stage)
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d.get("bytes_per_launch_full_size")
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------- oracle arm
+
+
+def _oracle_step(s, feat):
+    """One step of the path on the CPU oracle (sort, list, skin, aggregate)."""
+    import oracle
+    perm, keys, ps, nbr, cnt, ov = oracle.rebuild(s.pos, s.box, s.rc, s.skin, s.cap)
+    oracle.skin_check(ps, ps, s.box, s.skin)
+    oracle.edge_aggregate(ps, s.box, s.rc, nbr, cnt, feat)
+    return int(cnt.sum())
+
+
+def _sample_system(budget_steps: int):
+    """The bounded sample the oracle runs: the same salt-solution generator
+    and parameters at 1.024M atoms (config 3), or 98k atoms (config 2) when
+    many steps are asked for."""
+    import synth
+    return synth.system(3 if budget_steps <= 6 else 2)
+
+
+def cpu_baseline(args):
+    import oracle
+    s = _sample_system(1)
+    feat = s.features()
+    t = time.perf_counter()
+    _oracle_step(s, feat)
+    dt = time.perf_counter() - t
+    return {"value": s.n / dt, "unit": "atoms/s", "cores": oracle.get_threads(), "kind": "oracle",
+            "sample": "one full step (sort, cell-list Verlet list, skin check, aggregation) of %s "
+                      "(%d atoms, same generator and rc/skin/cap/F family as the 10.24M workload), %.1f s"
+                      % (s.name, s.n, dt)}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    import oracle
+    s = _sample_system(args.steps + args.warmup)
+    feat = s.features()
+    for _ in range(args.warmup):
+        _oracle_step(s, feat)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        _oracle_step(s, feat)
+    dt = time.perf_counter() - t
+    value = s.n * args.steps / dt
+    sample = "%s (%d atoms) per step, the plain CPU oracle on %d host threads" % (s.name, s.n, oracle.get_threads())
+    line = {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": value,
+        "unit": "atoms/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded salt-solution generator; no dataset)",
+        "config": {"workload": "salt-10.24M (sampled: %s)" % s.name, "atoms": s.n},
+        "cpu_baseline": {"value": value, "unit": "atoms/s", "cores": oracle.get_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "atoms/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["tess", "reference"], default="tess")
+    ap.add_argument("--config", type=int, default=WORKLOAD_CFG)
+    ap.add_argument("--no-pad-fill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    world, rank, local = _dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+    else:
+        run_cuda(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,196 @@
+/*
+ * tess.h -- C ABI of the B200 neighbor-rebuild library (libtess.so).
+ *
+ * The library implements the per-rebuild neighbor pipeline of an
+ * equivariant message-passing molecular-dynamics runtime, as described in
+ * "Ab Initio Accuracy Beyond the Cutoff: Distributed Message-Passing
+ * Equivariant Attention at Tens-of-Millions-of-Atom Scale" (Tessera),
+ * abstract:
+ *   - atoms are sorted along a space-filling curve (here the 3-D Hilbert
+ *     curve)                                          -> tess_hilbert_sort
+ *   - a neighbor list with fixed shapes between rebuilds, found by a
+ *     three-level search (tile, cell, pair)           -> tess_build_neighbors
+ *   - a conservative neighbor skin decides when to rebuild -> tess_skin_check
+ *   - each message-passing layer aggregates one-hop neighbor features
+ *     within the cutoff (review of arXiv 2505.06711, "load-bearing
+ *     attack" paragraph)                              -> tess_edge_aggregate
+ *
+ * Conventions (all entry points):
+ *   - Array pointers are DEVICE pointers owned by the caller.  The library
+ *     allocates nothing; scratch memory is a caller-provided workspace whose
+ *     size the *_workspace query returns.  Workspaces must be 256-byte
+ *     aligned; float4-layout arrays ([n,4] float) must be 16-byte aligned.
+ *   - Every call is asynchronous on the given stream and does no host
+ *     synchronisation.  The return value reports argument errors and launch
+ *     errors (cudaGetLastError) only; conditions found on the device are
+ *     written to caller-provided int32 words.
+ *   - The periodic box is orthorhombic with its origin at 0; positions are
+ *     expected in [0, L) per axis.
+ *   - Indices are int32: n <= 2^31 - 1.  n_max for a workspace is the n the
+ *     workspace was sized for.
+ */
+#ifndef TESS_H
+#define TESS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same underlying type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* tess_stream_t;
+
+typedef enum {
+    TESS_OK = 0,
+    TESS_ERR_INVALID_ARG = 1,        /* n <= 0, null pointer, bad parameter, misalignment */
+    TESS_ERR_BOX_TOO_SMALL = 2,      /* some box length below 2 (rc + skin) */
+    TESS_ERR_WORKSPACE_TOO_SMALL = 3,/* ws_bytes below the workspace query */
+    TESS_ERR_CUDA = 4                /* a kernel launch failed */
+} tess_status;
+
+/* Orthorhombic periodic box lengths (Angstrom, or any unit used throughout). */
+typedef struct {
+    float lx, ly, lz;
+} tess_box;
+
+/* Bits of the device status words (overflow / dev_status arguments). */
+#define TESS_DEV_OVERFLOW   1   /* some neighbor count exceeded max_neighbors */
+#define TESS_DEV_BAD_INPUT  2   /* some position outside [0, L) or not finite (clamped into the grid) */
+#define TESS_DEV_TIMEOUT    4   /* an inter-block wait gave up; outputs of that call are invalid */
+
+/* tess_build_neighbors flags */
+#define TESS_NO_PAD_FILL    1   /* leave slots >= min(count, max_neighbors) unwritten */
+
+/* Human-readable name of a status code (static string). */
+const char* tess_status_string(tess_status s);
+
+/* Library version string (static). */
+const char* tess_version(void);
+
+/* Number of kernels this process has launched through the library so far (a
+ * diagnostic counter; thread-safe). */
+long long tess_kernel_launch_count(void);
+
+/* ---------------------------------------------------------------------------
+ * Hilbert sort -- "sorts atoms along a space-filling curve" (Tessera,
+ * abstract).
+ *
+ * Each coordinate is quantised on a grid of 2^bits cells per axis: the scale
+ * s = 2^bits / L is one fp32 division, the cell is floor(x * s) with x * s a
+ * single fp32 multiply, clamped into [0, 2^bits - 1] (values below 0 or NaN
+ * give 0).  The key is the 3-D Hilbert index of the cell (Skilling's
+ * transform, "Programming the Hilbert curve", 2004; x is axis 0), 3*bits bits.
+ * Atoms are ordered by key, ties by ascending input index, so the result is
+ * unique.
+ *
+ *   pos          [n,3] float, input order (12-byte rows)
+ *   bits         1..10 (10: a 1024^3 grid)
+ *   ws, ws_bytes scratch of at least tess_hilbert_sort_workspace(n) bytes
+ *   perm         [n] int32 out: perm[k] = input index of the atom at rank k
+ *   keys_sorted  [n] uint32 out, nullable: key of the atom at rank k
+ *   pos_sorted   [n,4] float out, nullable: (x, y, z, 0) of the atom at rank k
+ *   dev_status   [1] int32 out, nullable: 0, or TESS_DEV_* bits
+ *                (BAD_INPUT, TIMEOUT)
+ * Errors: INVALID_ARG (n <= 0, null pos/perm/ws, bits outside 1..10, a
+ * non-positive or non-finite box length, misaligned pos_sorted),
+ * WORKSPACE_TOO_SMALL, CUDA.
+ * ------------------------------------------------------------------------- */
+size_t tess_hilbert_sort_workspace(int n);
+tess_status tess_hilbert_sort(const float* pos, int n, tess_box box, int bits,
+                              void* ws, size_t ws_bytes,
+                              int32_t* perm, uint32_t* keys_sorted, float* pos_sorted,
+                              int32_t* dev_status, tess_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Verlet neighbor list at rs = rc + skin -- "fixes workload shapes between
+ * rebuilds", "three-level neighbor search" (Tessera, abstract).
+ *
+ * Row i lists every j != i whose minimum-image distance to i is below rs
+ * (strictly), computed in fp32.  The list is full (j in row i iff i in row
+ * j) and lives in the index space of `pos` (pass the Hilbert-sorted
+ * positions for locality; any order gives the same sets).  Within a row
+ * the order is unspecified but deterministic for a given input.
+ *
+ *   pos            [n,4] float (x, y, z, ignored), 16-byte aligned
+ *   rc, skin       cutoff and skin (rc > 0, skin >= 0); rs = rc + skin in fp32
+ *   max_neighbors  row capacity cap >= 1
+ *   flags          0 or TESS_NO_PAD_FILL
+ *   ws, ws_bytes   scratch of at least tess_build_neighbors_workspace(...)
+ *   nbr            [n, cap] int32 out: row i in nbr[i*cap .. i*cap+cap);
+ *                  the first min(counts[i], cap) slots hold neighbors, the
+ *                  rest are -1 (not written under TESS_NO_PAD_FILL)
+ *   counts         [n] int32 out: TRUE neighbor count (may exceed cap; then
+ *                  which cap neighbors are stored is unspecified)
+ *   overflow       [1] int32 out: 0, or TESS_DEV_OVERFLOW if any count > cap,
+ *                  or'ed with TESS_DEV_BAD_INPUT if a position is outside
+ *                  [0, L) or not finite (its list is then unspecified)
+ * Errors: INVALID_ARG, BOX_TOO_SMALL (some L_d < 2 * rs, where the minimum
+ * image is not unique), WORKSPACE_TOO_SMALL, CUDA.
+ * ------------------------------------------------------------------------- */
+size_t tess_build_neighbors_workspace(int n, tess_box box, float rc, float skin);
+tess_status tess_build_neighbors(const float* pos, int n, tess_box box, float rc, float skin,
+                                 int max_neighbors, int flags, void* ws, size_t ws_bytes,
+                                 int32_t* nbr, int32_t* counts, int32_t* overflow,
+                                 tess_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Skin check -- "a conservative neighbor skin preserves topology across
+ * updates" (Tessera, abstract).  Rebuild when some atom has moved more than
+ * skin/2 since the reference frame: max_i |minimg(r_i - r_i^ref)|^2 >
+ * (skin/2)^2.  Displacements, squares and the threshold are fp64 (each
+ * operation one IEEE rounding: (dx*dx + dy*dy) + dz*dz), so the flag and
+ * the maximum are exact functions of the fp32 inputs.
+ *
+ *   pos, pos_ref  [n,4] float, same index order, 16-byte aligned
+ *   rebuild       [1] int32 out: 1 to rebuild, else 0
+ *   max_disp2     [1] double out, nullable: the maximum squared displacement
+ * Errors: INVALID_ARG (n <= 0, null, skin < 0, misaligned), CUDA.
+ * ------------------------------------------------------------------------- */
+tess_status tess_skin_check(const float* pos, const float* pos_ref, int n, tess_box box, float skin,
+                            int32_t* rebuild, double* max_disp2, tess_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Edge geometry and one-hop aggregation -- each message-passing layer
+ * aggregates one-hop neighbor features within the cutoff (review of arXiv
+ * 2505.06711, "load-bearing attack" paragraph); "Fused kernels" (Tessera,
+ * abstract).
+ *
+ * For row i and each of its first min(counts[i], cap) listed j (entries < 0
+ * skipped): r_ij = minimg(r_j - r_i), r = |r_ij|, f_c(r) = (cos(pi r / rc) +
+ * 1) / 2 for r < rc else 0, unit = r_ij / r (0 if r = 0), and
+ *     out[i, f] = sum_j f_c(r_ij) * feat[j, f]       (fp32 accumulation)
+ *
+ *   pos          [n,4] float, 16-byte aligned
+ *   nbr, counts  the list from tess_build_neighbors (cap = max_neighbors)
+ *   feat         [n, F] float, row-major;  out  [n, F] float
+ *   edge_vec     [n, cap, 4] float out, nullable: (rx, ry, rz, r)
+ *   edge_fc      [n, cap] float out, nullable: f_c
+ *   edge_unit    [n, cap, 4] float out, nullable: (ux, uy, uz, 0)
+ *   Unused slots of the edge arrays are written 0.
+ * Errors: INVALID_ARG (n <= 0, F < 1, cap < 1, rc <= 0, null, misaligned),
+ * BOX_TOO_SMALL (some L_d < 2 rc), CUDA.
+ * ------------------------------------------------------------------------- */
+tess_status tess_edge_aggregate(const float* pos, int n, tess_box box, float rc,
+                                const int32_t* nbr, const int32_t* counts, int max_neighbors,
+                                const float* feat, int F, float* out,
+                                float* edge_vec, float* edge_fc, float* edge_unit,
+                                tess_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Stage timing (diagnostic).  When enabled, each entry point records CUDA
+ * events on its stream around its kernels; tess_stage_times adds the elapsed
+ * times of all recorded calls per stage (this synchronises on the events)
+ * and clears them.  Stages: 0 hilbert keys, 1 key sort, 2 cell binning,
+ * 3 pair search, 4 skin check, 5 edge aggregate.  Returns the number of
+ * stages written (<= max_stages).  ms_out[k] = total milliseconds,
+ * calls_out[k] (nullable) = number of timed calls.
+ * ------------------------------------------------------------------------- */
+void tess_stage_timing(int enable);
+int tess_stage_times(double* ms_out, long long* calls_out, int max_stages);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TESS_H */

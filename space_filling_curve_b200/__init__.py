@@ -1,0 +1,276 @@
+"""B200-native neighbor-rebuild library: Python binding of libtess.so.
+
+The C ABI (``include/tess.h``) is the product; this module only marshals
+arguments.  Every step of the path runs in the library's CUDA kernels on the
+caller's current CUDA stream; PyTorch provides device memory and streams.
+
+Two layers:
+  * ``tess_*`` -- one-to-one ctypes bindings with the C names and arguments
+    (raw device pointers as ints, ``tess_box`` as three floats).
+  * ``hilbert_sort``, ``build_neighbors``, ``skin_check``, ``edge_aggregate``
+    -- the same calls taking torch CUDA tensors; outputs and workspaces are
+    allocated with torch when not given.
+
+There is no CPU fallback: if the CUDA library is missing or a tensor is not
+on a CUDA device, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "TessError", "lib", "library_path", "Box",
+    "tess_status_string", "tess_version", "tess_kernel_launch_count",
+    "tess_hilbert_sort_workspace", "tess_hilbert_sort",
+    "tess_build_neighbors_workspace", "tess_build_neighbors",
+    "tess_skin_check", "tess_edge_aggregate", "tess_stage_timing", "tess_stage_times",
+    "hilbert_sort", "build_neighbors", "skin_check", "edge_aggregate",
+    "TESS_DEV_OVERFLOW", "TESS_DEV_BAD_INPUT", "TESS_DEV_TIMEOUT", "TESS_NO_PAD_FILL", "STAGES",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libtess.so")
+
+TESS_DEV_OVERFLOW = 1
+TESS_DEV_BAD_INPUT = 2
+TESS_DEV_TIMEOUT = 4
+TESS_NO_PAD_FILL = 1
+STAGES = ("hilbert_keys", "key_sort", "cell_binning", "pair_search", "skin_check", "edge_aggregate")
+_STATUS = {0: "ok", 1: "invalid argument", 2: "box too small", 3: "workspace too small", 4: "CUDA launch error"}
+
+
+class TessError(RuntimeError):
+    """A library call returned a non-zero tess_status."""
+
+    def __init__(self, fn: str, code: int):
+        super().__init__("%s failed: %s (status %d)" % (fn, _STATUS.get(code, "unknown"), code))
+        self.code = code
+
+
+class Box(ctypes.Structure):
+    _fields_ = [("lx", ctypes.c_float), ("ly", ctypes.c_float), ("lz", ctypes.c_float)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libtess.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(library_path):
+        raise ImportError("libtess.so is not built (run `python space_filling_curve_b200/build.py` "
+                          "or __graft_entry__.build()): there is no fallback path")
+    L = ctypes.CDLL(library_path)
+    P, i32, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.tess_status_string.argtypes = [i32]
+    L.tess_status_string.restype = ctypes.c_char_p
+    L.tess_version.restype = ctypes.c_char_p
+    L.tess_kernel_launch_count.restype = ctypes.c_longlong
+    L.tess_hilbert_sort_workspace.argtypes = [i32]
+    L.tess_hilbert_sort_workspace.restype = sz
+    L.tess_hilbert_sort.argtypes = [P, i32, Box, i32, P, sz, P, P, P, P, P]
+    L.tess_hilbert_sort.restype = i32
+    L.tess_build_neighbors_workspace.argtypes = [i32, Box, f32, f32]
+    L.tess_build_neighbors_workspace.restype = sz
+    L.tess_build_neighbors.argtypes = [P, i32, Box, f32, f32, i32, i32, P, sz, P, P, P, P]
+    L.tess_build_neighbors.restype = i32
+    L.tess_skin_check.argtypes = [P, P, i32, Box, f32, P, P, P]
+    L.tess_skin_check.restype = i32
+    L.tess_edge_aggregate.argtypes = [P, i32, Box, f32, P, P, i32, P, i32, P, P, P, P, P]
+    L.tess_edge_aggregate.restype = i32
+    L.tess_stage_timing.argtypes = [i32]
+    L.tess_stage_times.argtypes = [P, P, i32]
+    L.tess_stage_times.restype = i32
+    _lib = L
+    return L
+
+
+def _box(box) -> Box:
+    if isinstance(box, Box):
+        return box
+    lx, ly, lz = (float(v) for v in box)
+    return Box(lx, ly, lz)
+
+
+# ------------------------------------------------------------------ raw C names
+
+
+def tess_status_string(code: int) -> str:
+    return lib().tess_status_string(int(code)).decode()
+
+
+def tess_version() -> str:
+    return lib().tess_version().decode()
+
+
+def tess_kernel_launch_count() -> int:
+    return int(lib().tess_kernel_launch_count())
+
+
+def tess_hilbert_sort_workspace(n: int) -> int:
+    return int(lib().tess_hilbert_sort_workspace(int(n)))
+
+
+def tess_hilbert_sort(pos, n, box, bits, ws, ws_bytes, perm, keys_sorted, pos_sorted, dev_status, stream) -> int:
+    return int(lib().tess_hilbert_sort(pos, n, _box(box), bits, ws, ws_bytes, perm, keys_sorted, pos_sorted,
+                                       dev_status, stream))
+
+
+def tess_build_neighbors_workspace(n, box, rc, skin) -> int:
+    return int(lib().tess_build_neighbors_workspace(int(n), _box(box), float(rc), float(skin)))
+
+
+def tess_build_neighbors(pos, n, box, rc, skin, max_neighbors, flags, ws, ws_bytes, nbr, counts, overflow,
+                         stream) -> int:
+    return int(lib().tess_build_neighbors(pos, n, _box(box), rc, skin, max_neighbors, flags, ws, ws_bytes, nbr,
+                                          counts, overflow, stream))
+
+
+def tess_skin_check(pos, pos_ref, n, box, skin, rebuild, max_disp2, stream) -> int:
+    return int(lib().tess_skin_check(pos, pos_ref, n, _box(box), skin, rebuild, max_disp2, stream))
+
+
+def tess_edge_aggregate(pos, n, box, rc, nbr, counts, max_neighbors, feat, F, out, edge_vec, edge_fc, edge_unit,
+                        stream) -> int:
+    return int(lib().tess_edge_aggregate(pos, n, _box(box), rc, nbr, counts, max_neighbors, feat, F, out, edge_vec,
+                                         edge_fc, edge_unit, stream))
+
+
+def tess_stage_timing(enable: bool) -> None:
+    lib().tess_stage_timing(1 if enable else 0)
+
+
+def tess_stage_times() -> dict:
+    """{stage name: (total ms, calls)} since the last read (synchronises)."""
+    ms = (ctypes.c_double * len(STAGES))()
+    calls = (ctypes.c_longlong * len(STAGES))()
+    k = lib().tess_stage_times(ctypes.cast(ms, ctypes.c_void_p), ctypes.cast(calls, ctypes.c_void_p), len(STAGES))
+    return {STAGES[i]: (float(ms[i]), int(calls[i])) for i in range(k)}
+
+
+# ------------------------------------------------------------------ torch layer
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    torch = _torch()
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(name, t, dtype=None, shape_tail=None):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor (no CPU path)" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError("%s must be %s" % (name, dtype))
+    if shape_tail is not None and (t.dim() != 2 or t.shape[1] != shape_tail):
+        raise ValueError("%s must be [n, %d]" % (name, shape_tail))
+
+
+def _check(fn, code):
+    if code != 0:
+        raise TessError(fn, code)
+
+
+def _workspace(nbytes, device, ws=None):
+    torch = _torch()
+    if ws is not None and ws.numel() * ws.element_size() >= nbytes:
+        return ws
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+def hilbert_sort(pos, box, bits: int = 10, *, ws=None, perm=None, keys_sorted=None, pos_sorted=None,
+                 dev_status=None, want_keys: bool = True, want_pos: bool = True, stream=None):
+    """Order atoms along the 3-D Hilbert curve.  ``pos``: float32 [n, 3]
+    CUDA tensor.  Returns (perm int32 [n], keys uint32->int32 view [n] or
+    None, pos_sorted float32 [n, 4] or None, dev_status int32 [1])."""
+    torch = _torch()
+    _need_cuda("pos", pos, torch.float32, 3)
+    n = pos.shape[0]
+    dev = pos.device
+    ws = _workspace(tess_hilbert_sort_workspace(n), dev, ws)
+    perm = torch.empty(n, dtype=torch.int32, device=dev) if perm is None else perm
+    if want_keys and keys_sorted is None:
+        keys_sorted = torch.empty(n, dtype=torch.int32, device=dev)
+    if want_pos and pos_sorted is None:
+        pos_sorted = torch.empty((n, 4), dtype=torch.float32, device=dev)
+    dev_status = torch.empty(1, dtype=torch.int32, device=dev) if dev_status is None else dev_status
+    code = tess_hilbert_sort(_ptr(pos), n, box, bits, _ptr(ws), ws.numel() * ws.element_size(), _ptr(perm),
+                             _ptr(keys_sorted), _ptr(pos_sorted), _ptr(dev_status), _stream(stream))
+    _check("tess_hilbert_sort", code)
+    return perm, keys_sorted, pos_sorted, dev_status
+
+
+def build_neighbors(pos4, box, rc: float, skin: float, max_neighbors: int, *, pad_fill: bool = True, ws=None,
+                    nbr=None, counts=None, overflow=None, stream=None):
+    """Padded Verlet list at rc + skin.  ``pos4``: float32 [n, 4] CUDA
+    tensor.  Returns (nbr int32 [n, cap], counts int32 [n], overflow int32 [1])."""
+    torch = _torch()
+    _need_cuda("pos4", pos4, torch.float32, 4)
+    n = pos4.shape[0]
+    dev = pos4.device
+    ws = _workspace(tess_build_neighbors_workspace(n, box, rc, skin), dev, ws)
+    nbr = torch.empty((n, max_neighbors), dtype=torch.int32, device=dev) if nbr is None else nbr
+    counts = torch.empty(n, dtype=torch.int32, device=dev) if counts is None else counts
+    overflow = torch.empty(1, dtype=torch.int32, device=dev) if overflow is None else overflow
+    flags = 0 if pad_fill else TESS_NO_PAD_FILL
+    code = tess_build_neighbors(_ptr(pos4), n, box, float(rc), float(skin), int(max_neighbors), flags, _ptr(ws),
+                                ws.numel() * ws.element_size(), _ptr(nbr), _ptr(counts), _ptr(overflow),
+                                _stream(stream))
+    _check("tess_build_neighbors", code)
+    return nbr, counts, overflow
+
+
+def skin_check(pos4, ref4, box, skin: float, *, rebuild=None, max_disp2=None, stream=None):
+    """Rebuild flag (int32 [1]) and max squared displacement (float64 [1])."""
+    torch = _torch()
+    _need_cuda("pos4", pos4, torch.float32, 4)
+    _need_cuda("ref4", ref4, torch.float32, 4)
+    if pos4.shape != ref4.shape:
+        raise ValueError("pos4 and ref4 must have the same shape")
+    dev = pos4.device
+    rebuild = torch.empty(1, dtype=torch.int32, device=dev) if rebuild is None else rebuild
+    max_disp2 = torch.empty(1, dtype=torch.float64, device=dev) if max_disp2 is None else max_disp2
+    code = tess_skin_check(_ptr(pos4), _ptr(ref4), pos4.shape[0], box, float(skin), _ptr(rebuild), _ptr(max_disp2),
+                           _stream(stream))
+    _check("tess_skin_check", code)
+    return rebuild, max_disp2
+
+
+def edge_aggregate(pos4, box, rc: float, nbr, counts, feat, *, out=None, edges: bool = False, stream=None):
+    """out[i] = sum_j f_c(|r_ij|) feat[j] over row i.  With ``edges`` also
+    returns edge_vec [n, cap, 4], edge_fc [n, cap], edge_unit [n, cap, 4]."""
+    torch = _torch()
+    _need_cuda("pos4", pos4, torch.float32, 4)
+    _need_cuda("nbr", nbr, torch.int32)
+    _need_cuda("counts", counts, torch.int32)
+    _need_cuda("feat", feat, torch.float32)
+    n, cap = nbr.shape
+    F = feat.shape[1]
+    dev = pos4.device
+    out = torch.empty((n, F), dtype=torch.float32, device=dev) if out is None else out
+    ev = ef = eu = None
+    if edges:
+        ev = torch.empty((n, cap, 4), dtype=torch.float32, device=dev)
+        ef = torch.empty((n, cap), dtype=torch.float32, device=dev)
+        eu = torch.empty((n, cap, 4), dtype=torch.float32, device=dev)
+    code = tess_edge_aggregate(_ptr(pos4), n, box, float(rc), _ptr(nbr), _ptr(counts), cap, _ptr(feat), F,
+                               _ptr(out), _ptr(ev), _ptr(ef), _ptr(eu), _stream(stream))
+    _check("tess_edge_aggregate", code)
+    if edges:
+        return out, ev, ef, eu
+    return out

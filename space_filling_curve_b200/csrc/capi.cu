@@ -1,0 +1,143 @@
+// capi.cu -- the extern "C" boundary of libtess.so (declared in tess.h).
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+
+namespace tess {
+
+std::atomic<long long> g_launches{0};
+
+size_t hilbert_sort_workspace(int n);
+tess_status hilbert_sort(const float* pos, int n, tess_box box, int bits, void* ws, size_t ws_bytes, int32_t* perm,
+                         uint32_t* keys_sorted, float* pos_sorted, int32_t* dev_status, cudaStream_t s);
+size_t build_neighbors_workspace(int n, tess_box box, float rc, float skin);
+tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, float skin, int cap, int flags,
+                            void* ws, size_t ws_bytes, int32_t* nbr, int32_t* counts, int32_t* overflow,
+                            cudaStream_t s);
+tess_status skin_check(const float* pos, const float* pos_ref, int n, tess_box box, float skin, int32_t* rebuild,
+                       double* max_disp2, cudaStream_t s);
+tess_status edge_aggregate(const float* pos, int n, tess_box box, float rc, const int32_t* nbr, const int32_t* counts,
+                           int cap, const float* feat, int F, float* out, float* edge_vec, float* edge_fc,
+                           float* edge_unit, cudaStream_t s);
+
+// ---------------------------------------------------------------- stage timing
+
+namespace {
+struct Timing {
+    std::mutex mu;
+    bool enabled = false;
+    struct Rec {
+        int stage;
+        cudaEvent_t a, b;
+    };
+    std::vector<Rec> recs;
+};
+Timing& timing() {
+    static Timing t;
+    return t;
+}
+}  // namespace
+
+StageScope::StageScope(int stage_, cudaStream_t s_) : stage(stage_), s(s_) {
+    Timing& t = timing();
+    std::lock_guard<std::mutex> g(t.mu);
+    if (!t.enabled) return;
+    cudaEventCreate(&a);
+    cudaEventCreate(&b);
+    cudaEventRecord(a, s);
+}
+
+StageScope::~StageScope() {
+    if (!a) return;
+    cudaEventRecord(b, s);
+    Timing& t = timing();
+    std::lock_guard<std::mutex> g(t.mu);
+    t.recs.push_back({stage, a, b});
+}
+
+}  // namespace tess
+
+using namespace tess;
+
+extern "C" {
+
+const char* tess_status_string(tess_status s) {
+    switch (s) {
+        case TESS_OK: return "ok";
+        case TESS_ERR_INVALID_ARG: return "invalid argument";
+        case TESS_ERR_BOX_TOO_SMALL: return "box too small: some length below twice the cutoff radius";
+        case TESS_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case TESS_ERR_CUDA: return "CUDA launch error";
+    }
+    return "unknown status";
+}
+
+const char* tess_version(void) { return "tess-b200 0.1 (sm_100a)"; }
+
+long long tess_kernel_launch_count(void) { return g_launches.load(); }
+
+size_t tess_hilbert_sort_workspace(int n) { return hilbert_sort_workspace(n); }
+
+tess_status tess_hilbert_sort(const float* pos, int n, tess_box box, int bits, void* ws, size_t ws_bytes,
+                              int32_t* perm, uint32_t* keys_sorted, float* pos_sorted, int32_t* dev_status,
+                              tess_stream_t stream) {
+    return hilbert_sort(pos, n, box, bits, ws, ws_bytes, perm, keys_sorted, pos_sorted, dev_status,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t tess_build_neighbors_workspace(int n, tess_box box, float rc, float skin) {
+    return build_neighbors_workspace(n, box, rc, skin);
+}
+
+tess_status tess_build_neighbors(const float* pos, int n, tess_box box, float rc, float skin, int max_neighbors,
+                                 int flags, void* ws, size_t ws_bytes, int32_t* nbr, int32_t* counts,
+                                 int32_t* overflow, tess_stream_t stream) {
+    return build_neighbors(pos, n, box, rc, skin, max_neighbors, flags, ws, ws_bytes, nbr, counts, overflow,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+tess_status tess_skin_check(const float* pos, const float* pos_ref, int n, tess_box box, float skin,
+                            int32_t* rebuild, double* max_disp2, tess_stream_t stream) {
+    return skin_check(pos, pos_ref, n, box, skin, rebuild, max_disp2, reinterpret_cast<cudaStream_t>(stream));
+}
+
+tess_status tess_edge_aggregate(const float* pos, int n, tess_box box, float rc, const int32_t* nbr,
+                                const int32_t* counts, int max_neighbors, const float* feat, int F, float* out,
+                                float* edge_vec, float* edge_fc, float* edge_unit, tess_stream_t stream) {
+    return edge_aggregate(pos, n, box, rc, nbr, counts, max_neighbors, feat, F, out, edge_vec, edge_fc, edge_unit,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+void tess_stage_timing(int enable) {
+    Timing& t = timing();
+    std::lock_guard<std::mutex> g(t.mu);
+    t.enabled = enable != 0;
+}
+
+int tess_stage_times(double* ms_out, long long* calls_out, int max_stages) {
+    Timing& t = timing();
+    std::vector<Timing::Rec> recs;
+    {
+        std::lock_guard<std::mutex> g(t.mu);
+        recs.swap(t.recs);
+    }
+    const int ns = std::min<int>(max_stages, ST_COUNT);
+    for (int k = 0; k < ns; ++k) {
+        ms_out[k] = 0.0;
+        if (calls_out) calls_out[k] = 0;
+    }
+    for (auto& r : recs) {
+        float ms = 0.f;
+        cudaEventSynchronize(r.b);
+        if (cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess && r.stage < ns) {
+            ms_out[r.stage] += ms;
+            if (calls_out) calls_out[r.stage] += 1;
+        }
+        cudaEventDestroy(r.a);
+        cudaEventDestroy(r.b);
+    }
+    return ns;
+}
+
+}  // extern "C"

@@ -1,0 +1,68 @@
+// common.cuh -- shared helpers of the CUDA library (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <cmath>
+
+#include "tess.h"
+
+namespace tess {
+
+constexpr unsigned FULL = 0xffffffffu;
+
+// Number of kernels launched through the library (diagnostic).
+extern std::atomic<long long> g_launches;
+inline void count_launch(long long k = 1) { g_launches.fetch_add(k, std::memory_order_relaxed); }
+
+// Stage ids for the optional event timing.
+enum Stage { ST_KEYS = 0, ST_SORT = 1, ST_CELLS = 2, ST_PAIRS = 3, ST_SKIN = 4, ST_EDGE = 5, ST_COUNT = 6 };
+
+// Records an event pair around a stage when stage timing is enabled.
+struct StageScope {
+    int stage;
+    cudaStream_t s;
+    cudaEvent_t a = nullptr, b = nullptr;
+    StageScope(int stage_, cudaStream_t s_);
+    ~StageScope();
+};
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Bump allocator over a caller-provided workspace.
+struct Carve {
+    char* base;
+    size_t off = 0;
+    explicit Carve(void* p) : base(static_cast<char*>(p)) {}
+    template <class T>
+    T* take(size_t count) {
+        off = align_up(off, 256);
+        T* p = reinterpret_cast<T*>(base ? base + off : nullptr);
+        off += sizeof(T) * count;
+        return p;
+    }
+};
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline bool finite_pos(float x) { return std::isfinite(x) && x > 0.0f; }
+
+inline tess_status launch_status() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? TESS_OK : TESS_ERR_CUDA;
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+    unsigned m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+__device__ __forceinline__ int floor_div(int a, int b) {
+    int q = a / b;
+    return (a % b != 0 && ((a < 0) != (b < 0))) ? q - 1 : q;
+}
+
+}  // namespace tess

@@ -1,0 +1,536 @@
+// neighbors.cu -- fixed-capacity Verlet list at rs = rc + skin ("fixes
+// workload shapes between rebuilds", "three-level neighbor search",
+// Tessera, abstract).
+//
+// Level 0 (binning, deterministic):
+//   cell_count     cell id per atom, warp-aggregated histogram
+//   scan_*         exclusive scan of the cell counts -> cell_start
+//   cell_scatter   atom indices into their cells (any order within a cell)
+//   cell_order     within each cell, order by atom index and write the
+//                  positions in cell order as float4 (x, y, z, index bits)
+// Levels 1-3 (pair_search, one warp per tile of 32 consecutive atoms, lane =
+// atom i):
+//   1. tile: bounding box of the 32 atoms (Hilbert-consecutive, so compact)
+//   2. cells: every cell row overlapping box +- rs; each cell row is one
+//      contiguous range of the cell-ordered positions, shifted by its
+//      periodic image; candidates are culled against box +- rs and compacted
+//      (ballot + popc) into a shared-memory chunk
+//   3. pairs: every lane tests its atom against the chunk (broadcast reads)
+//      and appends accepted indices to its row in shared memory; the 32 rows
+//      are one contiguous block of the output and leave with 16-byte stores.
+#include "common.cuh"
+
+namespace tess {
+
+// ---------------------------------------------------------------- grid
+
+struct Grid {
+    int nc[3];
+    float inv_w[3];
+    long long ncell;
+};
+
+// Cells of width about rs/2 (the pair search adapts to any width), coarsened
+// when that would give more than ~2 cells per atom.
+static Grid make_grid(int n, tess_box box, float rs) {
+    Grid g{};
+    const float L[3] = {box.lx, box.ly, box.lz};
+    double w = (double)rs * 1.0001 / 2.0;
+    for (int it = 0; it < 64; ++it) {
+        long long tot = 1;
+        for (int d = 0; d < 3; ++d) {
+            long long c = (long long)std::floor((double)L[d] / w);
+            if (c < 1) c = 1;
+            if (c > (1 << 20)) c = 1 << 20;
+            g.nc[d] = (int)c;
+            tot *= c;
+        }
+        g.ncell = tot;
+        if (tot <= 2LL * n + 4096) break;
+        w *= 1.26;
+    }
+    for (int d = 0; d < 3; ++d) g.inv_w[d] = (float)g.nc[d] / L[d];   // fp32, shared by all kernels
+    return g;
+}
+
+__device__ __forceinline__ int cell_coord(float x, float inv_w, int nc) {
+    float f = floorf(__fmul_rn(x, inv_w));
+    f = fminf(fmaxf(f, 0.0f), (float)(nc - 1));     // NaN -> 0
+    return (int)f;
+}
+
+// ---------------------------------------------------------------- binning
+
+__global__ void cell_count_kernel(const float4* __restrict__ pos, int n, int3 nc, float3 inv_w, float3 L,
+                                  int* __restrict__ cell_id, int* __restrict__ cnt, int32_t* status) {
+    bool bad = false;
+    const int stride = gridDim.x * blockDim.x;
+    for (int base = blockIdx.x * blockDim.x; base < n; base += stride) {
+        const int i = base + threadIdx.x;
+        const bool valid = i < n;
+        int c = -1;
+        if (valid) {
+            const float4 p = pos[i];
+            bad |= !(p.x >= 0.0f && p.x < L.x && p.y >= 0.0f && p.y < L.y && p.z >= 0.0f && p.z < L.z);
+            const int cx = cell_coord(p.x, inv_w.x, nc.x);
+            const int cy = cell_coord(p.y, inv_w.y, nc.y);
+            const int cz = cell_coord(p.z, inv_w.z, nc.z);
+            c = (cz * nc.y + cy) * nc.x + cx;
+            cell_id[i] = c;
+        }
+        const unsigned act = __ballot_sync(FULL, valid);
+        if (valid) {
+            const unsigned peers = __match_any_sync(act, c);
+            if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&cnt[c], __popc(peers));
+        }
+    }
+    if (__any_sync(FULL, bad) && (threadIdx.x & 31) == 0 && status) atomicOr(status, TESS_DEV_BAD_INPUT);
+}
+
+constexpr int SCAN_THREADS = 1024;
+constexpr int SCAN_ITEMS = 4;
+constexpr int SCAN_TILE = SCAN_THREADS * SCAN_ITEMS;
+
+__device__ __forceinline__ int block_scan_incl(int v, int* s_warp) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(FULL, v, o);
+        if (lane >= o) v += y;
+    }
+    if (lane == 31) s_warp[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        int w = (lane < (int)(blockDim.x >> 5)) ? s_warp[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int y = __shfl_up_sync(FULL, w, o);
+            if (lane >= o) w += y;
+        }
+        s_warp[lane] = w;
+    }
+    __syncthreads();
+    const int add = warp > 0 ? s_warp[warp - 1] : 0;
+    __syncthreads();
+    return v + add;
+}
+
+// per-tile sums of the counts
+__global__ __launch_bounds__(SCAN_THREADS) void scan_reduce_kernel(const int* __restrict__ cnt, long long m,
+                                                                   int* __restrict__ sums) {
+    __shared__ int s_warp[32];
+    const long long b = (long long)blockIdx.x * SCAN_TILE + (long long)threadIdx.x * SCAN_ITEMS;
+    int v = 0;
+#pragma unroll
+    for (int k = 0; k < SCAN_ITEMS; ++k) v += (b + k < m) ? cnt[b + k] : 0;
+    const int tot = block_scan_incl(v, s_warp);
+    if (threadIdx.x == blockDim.x - 1) sums[blockIdx.x] = tot;
+}
+
+// exclusive scan of the per-tile sums, one block, any length
+__global__ __launch_bounds__(SCAN_THREADS) void scan_sums_kernel(int* sums, long long nt) {
+    __shared__ int s_warp[32];
+    __shared__ int s_carry;
+    if (threadIdx.x == 0) s_carry = 0;
+    __syncthreads();
+    for (long long b = 0; b < nt; b += SCAN_THREADS) {
+        const long long k = b + threadIdx.x;
+        const int v = k < nt ? sums[k] : 0;
+        const int inc = block_scan_incl(v, s_warp);
+        const int carry = s_carry;
+        if (k < nt) sums[k] = carry + inc - v;
+        __syncthreads();
+        if (threadIdx.x == blockDim.x - 1) s_carry = carry + inc;
+        __syncthreads();
+    }
+}
+
+// cell_start[c] = exclusive prefix; cnt[c] reset to 0 for the scatter cursor
+__global__ __launch_bounds__(SCAN_THREADS) void scan_apply_kernel(int* __restrict__ cnt, long long m,
+                                                                  const int* __restrict__ sums,
+                                                                  int* __restrict__ cell_start) {
+    __shared__ int s_warp[32];
+    const long long b = (long long)blockIdx.x * SCAN_TILE + (long long)threadIdx.x * SCAN_ITEMS;
+    int v[SCAN_ITEMS];
+    int tot = 0;
+#pragma unroll
+    for (int k = 0; k < SCAN_ITEMS; ++k) {
+        v[k] = (b + k < m) ? cnt[b + k] : 0;
+        tot += v[k];
+    }
+    const int inc = block_scan_incl(tot, s_warp);
+    int run = sums[blockIdx.x] + inc - tot;
+#pragma unroll
+    for (int k = 0; k < SCAN_ITEMS; ++k) {
+        if (b + k < m) {
+            cell_start[b + k] = run;
+            cnt[b + k] = 0;
+        }
+        run += v[k];
+    }
+    if (b < m && b + SCAN_ITEMS >= m) cell_start[m] = run;   // the thread holding the last cell
+}
+
+__global__ void cell_scatter_kernel(const int* __restrict__ cell_id, int n, const int* __restrict__ cell_start,
+                                    int* __restrict__ cursor, int* __restrict__ slot_atom) {
+    const int stride = gridDim.x * blockDim.x;
+    for (int base = blockIdx.x * blockDim.x; base < n; base += stride) {
+        const int i = base + threadIdx.x;
+        const bool valid = i < n;
+        const int c = valid ? cell_id[i] : -1;
+        const unsigned act = __ballot_sync(FULL, valid);
+        if (valid) {
+            const unsigned peers = __match_any_sync(act, c);
+            const int lane = threadIdx.x & 31, leader = __ffs(peers) - 1;
+            int b0 = 0;
+            if (lane == leader) b0 = atomicAdd(&cursor[c], __popc(peers));
+            b0 = __shfl_sync(peers, b0, leader);
+            slot_atom[cell_start[c] + b0 + __popc(peers & lanemask_lt())] = i;
+        }
+    }
+}
+
+// Deterministic order inside each cell: the slot of atom i is the cell start
+// plus the number of atoms of the same cell with a smaller index.
+__global__ void cell_order_kernel(const int* __restrict__ slot_atom, int n, const int* __restrict__ cell_id,
+                                  const int* __restrict__ cell_start, const float4* __restrict__ pos,
+                                  float4* __restrict__ pos_cell) {
+    const int stride = gridDim.x * blockDim.x;
+    for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < n; k += stride) {
+        const int i = slot_atom[k];
+        const int c = cell_id[i];
+        const int b = cell_start[c], e = cell_start[c + 1];
+        int r = 0;
+        for (int s = b; s < e; ++s) r += slot_atom[s] < i;
+        const float4 p = pos[i];
+        pos_cell[b + r] = make_float4(p.x, p.y, p.z, __int_as_float(i));
+    }
+}
+
+// ---------------------------------------------------------------- pair search
+
+constexpr int PS_WARPS = 2;          // warps per block
+constexpr int PS_CHUNK = 256;        // culled candidates staged per warp before testing
+constexpr int PS_MAXSEG = 64;        // cell-row segments per table batch
+constexpr int PS_UNROLL = 4;         // candidate loads in flight per lane
+
+struct PairArgs {
+    const float4* pos;
+    const float4* pos_cell;
+    const int* cell_start;
+    int n;
+    int cap;
+    int pad_fill;
+    int3 nc;
+    float3 inv_w;
+    float3 L;
+    float rs2;
+    float reach;       // rs plus a margin that covers fp32 rounding of cell and box tests
+    int* nbr;
+    int* counts;
+    int32_t* status;
+};
+
+struct SegEntry {
+    int beg;
+    int pre;           // exclusive prefix of segment lengths within the batch
+    float sx, sy, sz, pad0, pad1, pad2;
+};
+
+__host__ __device__ constexpr size_t ps_warp_smem(int cap, bool rows_in_smem) {
+    return sizeof(float4) * PS_CHUNK + sizeof(SegEntry) * (PS_MAXSEG + 1) +
+           (rows_in_smem ? sizeof(int) * 32 * (size_t)cap : 0);
+}
+
+template <bool SMEM_ROWS>
+__global__ __launch_bounds__(PS_WARPS * 32, 8) void pair_search_kernel(PairArgs A) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned char* wbase = smem_raw + (size_t)warp * ps_warp_smem(A.cap, SMEM_ROWS);
+    float4* cand = reinterpret_cast<float4*>(wbase);
+    SegEntry* seg = reinterpret_cast<SegEntry*>(wbase + sizeof(float4) * PS_CHUNK);
+    int* rows = reinterpret_cast<int*>(wbase + sizeof(float4) * PS_CHUNK + sizeof(SegEntry) * (PS_MAXSEG + 1));
+    const int cap = A.cap;
+    const long long ntiles = ((long long)A.n + 31) / 32;
+
+    for (long long tile = (long long)blockIdx.x * PS_WARPS + warp; tile < ntiles;
+         tile += (long long)gridDim.x * PS_WARPS) {
+        const int base = (int)(tile * 32);
+        const int i = base + lane;
+        const bool valid = i < A.n;
+        const float nanf_ = __int_as_float(0x7fc00000);
+        float4 p = valid ? A.pos[i] : make_float4(nanf_, nanf_, nanf_, 0.f);
+
+        // level 1: tile bounding box
+        float lox = valid ? p.x : INFINITY, loy = valid ? p.y : INFINITY, loz = valid ? p.z : INFINITY;
+        float hix = valid ? p.x : -INFINITY, hiy = valid ? p.y : -INFINITY, hiz = valid ? p.z : -INFINITY;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+            lox = fminf(lox, __shfl_xor_sync(FULL, lox, o));
+            loy = fminf(loy, __shfl_xor_sync(FULL, loy, o));
+            loz = fminf(loz, __shfl_xor_sync(FULL, loz, o));
+            hix = fmaxf(hix, __shfl_xor_sync(FULL, hix, o));
+            hiy = fmaxf(hiy, __shfl_xor_sync(FULL, hiy, o));
+            hiz = fmaxf(hiz, __shfl_xor_sync(FULL, hiz, o));
+        }
+        // a non-finite position (invalid input) would make the box useless:
+        // fall back to the whole box for this tile
+        if (!(isfinite(lox) && isfinite(hix) && isfinite(loy) && isfinite(hiy) && isfinite(loz) && isfinite(hiz))) {
+            lox = loy = loz = 0.f;
+            hix = A.L.x; hiy = A.L.y; hiz = A.L.z;
+        }
+        // positions far outside the box (invalid input, flagged by the
+        // binning) must not blow up the cell ranges
+        lox = fmaxf(lox, -A.L.x); loy = fmaxf(loy, -A.L.y); loz = fmaxf(loz, -A.L.z);
+        hix = fminf(hix, 2.f * A.L.x); hiy = fminf(hiy, 2.f * A.L.y); hiz = fminf(hiz, 2.f * A.L.z);
+
+        if (SMEM_ROWS && A.pad_fill) {
+            int4* r4 = reinterpret_cast<int4*>(rows);
+            for (int e = lane; e < 8 * cap; e += 32) r4[e] = make_int4(-1, -1, -1, -1);
+        }
+        int* myrow = SMEM_ROWS ? rows + lane * cap : A.nbr + (size_t)(valid ? i : 0) * cap;
+        int cnt = 0;
+        int ncand = 0;
+
+        // level 3: test the staged chunk
+        auto flush = [&]() {
+            __syncwarp();
+            for (int c = 0; c < ncand; ++c) {
+                const float4 q = cand[c];
+                const float dx = q.x - p.x, dy = q.y - p.y, dz = q.z - p.z;
+                const float r2 = fmaf(dz, dz, fmaf(dy, dy, dx * dx));
+                const int j = __float_as_int(q.w);
+                if (r2 < A.rs2 && j != i) {
+                    if (SMEM_ROWS) myrow[min(cnt, cap - 1)] = j;
+                    else if (cnt < cap && valid) myrow[cnt] = j;
+                    ++cnt;
+                }
+            }
+            ncand = 0;
+            __syncwarp();
+        };
+
+        // level 2: cell rows overlapping the box +- reach
+        const int ux0 = (int)floorf((lox - A.reach) * A.inv_w.x), ux1 = (int)floorf((hix + A.reach) * A.inv_w.x);
+        const int uy0 = (int)floorf((loy - A.reach) * A.inv_w.y), uy1 = (int)floorf((hiy + A.reach) * A.inv_w.y);
+        const int uz0 = (int)floorf((loz - A.reach) * A.inv_w.z), uz1 = (int)floorf((hiz + A.reach) * A.inv_w.z);
+        const int ny = uy1 - uy0 + 1, nz = uz1 - uz0 + 1;
+        const int npieces = floor_div(ux1, A.nc.x) - floor_div(ux0, A.nc.x) + 1;
+        const int nseg = ny * nz * npieces;
+        const float reach2 = A.reach * A.reach;
+
+        for (int sb = 0; sb < nseg; sb += PS_MAXSEG) {
+            const int nb = min(PS_MAXSEG, nseg - sb);
+            // segment table: lane-parallel decode and bounds
+            int run = 0;
+            for (int s0 = 0; s0 < nb; s0 += 32) {
+                const int sl = s0 + lane;
+                int len = 0, beg = 0;
+                float sx = 0.f, sy = 0.f, sz = 0.f;
+                if (sl < nb) {
+                    const int s = sb + sl;
+                    const int piece = s % npieces;
+                    const int row = s / npieces;
+                    const int uy = uy0 + row % ny, uz = uz0 + row / ny;
+                    const int ky = floor_div(uy, A.nc.y), kz = floor_div(uz, A.nc.z);
+                    const int cy = uy - ky * A.nc.y, cz = uz - kz * A.nc.z;
+                    const int kx = floor_div(ux0, A.nc.x) + piece;
+                    const int xa = max(ux0, kx * A.nc.x) - kx * A.nc.x;
+                    const int xb = min(ux1, (kx + 1) * A.nc.x - 1) - kx * A.nc.x;
+                    const int rowbase = (cz * A.nc.y + cy) * A.nc.x;
+                    beg = A.cell_start[rowbase + xa];
+                    len = A.cell_start[rowbase + xb + 1] - beg;
+                    sx = (float)kx * A.L.x;
+                    sy = (float)ky * A.L.y;
+                    sz = (float)kz * A.L.z;
+                }
+                int inc = len;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(FULL, inc, o);
+                    if (lane >= o) inc += y;
+                }
+                if (sl < nb) {
+                    SegEntry& e = seg[sl];
+                    e.beg = beg;
+                    e.pre = run + inc - len;
+                    e.sx = sx; e.sy = sy; e.sz = sz;
+                }
+                run += __shfl_sync(FULL, inc, 31);
+            }
+            if (lane == 0) seg[nb].pre = run;
+            __syncwarp();
+            const int total = run;
+
+            int sc = 0;   // this lane's segment cursor
+            for (int t0 = 0; t0 < total; t0 += 32 * PS_UNROLL) {
+                if (ncand > PS_CHUNK - 32 * PS_UNROLL) flush();
+                float4 q[PS_UNROLL];
+                bool ok[PS_UNROLL];
+#pragma unroll
+                for (int u = 0; u < PS_UNROLL; ++u) {
+                    const int t = t0 + u * 32 + lane;
+                    ok[u] = t < total;
+                    if (ok[u]) {
+                        while (seg[sc + 1].pre <= t) ++sc;
+                        const SegEntry& e = seg[sc];
+                        const float4 c = A.pos_cell[e.beg + (t - e.pre)];
+                        q[u] = make_float4(c.x + e.sx, c.y + e.sy, c.z + e.sz, c.w);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < PS_UNROLL; ++u) {
+                    bool keep = false;
+                    if (ok[u]) {
+                        const float ex = fmaxf(fmaxf(lox - q[u].x, q[u].x - hix), 0.f);
+                        const float ey = fmaxf(fmaxf(loy - q[u].y, q[u].y - hiy), 0.f);
+                        const float ez = fmaxf(fmaxf(loz - q[u].z, q[u].z - hiz), 0.f);
+                        keep = fmaf(ez, ez, fmaf(ey, ey, ex * ex)) < reach2;
+                    }
+                    const unsigned bm = __ballot_sync(FULL, keep);
+                    if (keep) cand[ncand + __popc(bm & lanemask_lt())] = q[u];
+                    ncand += __popc(bm);
+                }
+            }
+            __syncwarp();
+        }
+        flush();
+
+        // write the tile's rows
+        if (valid) A.counts[i] = cnt;
+        const unsigned ov = __ballot_sync(FULL, valid && cnt > cap);
+        if (ov && lane == 0) atomicOr(A.status, TESS_DEV_OVERFLOW);
+        const int nvalid = min(32, A.n - base);
+        if (SMEM_ROWS) {
+            __syncwarp();
+            int* gdst = A.nbr + (size_t)base * cap;
+            if (A.pad_fill) {
+                const long long total = (long long)nvalid * cap;
+                const long long n4 = total / 4;
+                const int4* s4 = reinterpret_cast<const int4*>(rows);
+                int4* g4 = reinterpret_cast<int4*>(gdst);
+                for (long long e = lane; e < n4; e += 32) g4[e] = s4[e];
+                for (long long e = n4 * 4 + lane; e < total; e += 32) gdst[e] = rows[e];
+            } else {
+                for (int r = 0; r < nvalid; ++r) {
+                    const int m = min(__shfl_sync(FULL, cnt, r), cap);
+                    for (int e = lane; e < m; e += 32) gdst[(size_t)r * cap + e] = rows[r * cap + e];
+                }
+            }
+            __syncwarp();
+        } else if (A.pad_fill && valid) {
+            for (int e = min(cnt, cap); e < cap; ++e) myrow[e] = -1;
+        }
+    }
+}
+
+// ---------------------------------------------------------------- host
+
+struct NbrLayout {
+    int* cell_id;
+    int* cnt;
+    int* cell_start;
+    int* sums;
+    int* slot_atom;
+    float4* pos_cell;
+    int32_t* status;
+    size_t total;
+};
+
+static NbrLayout nbr_layout(void* ws, int n, const Grid& g) {
+    Carve c(ws);
+    NbrLayout L{};
+    const long long m = g.ncell;
+    L.cell_id = c.take<int>((size_t)n);
+    L.cnt = c.take<int>((size_t)m);
+    L.cell_start = c.take<int>((size_t)m + 1);
+    L.sums = c.take<int>((size_t)((m + SCAN_TILE - 1) / SCAN_TILE) + 1);
+    L.slot_atom = c.take<int>((size_t)n);
+    L.pos_cell = c.take<float4>((size_t)n);
+    L.status = c.take<int32_t>(1);
+    L.total = align_up(c.off, 256);
+    return L;
+}
+
+static bool box_ok(tess_box b) { return finite_pos(b.lx) && finite_pos(b.ly) && finite_pos(b.lz); }
+
+size_t build_neighbors_workspace(int n, tess_box box, float rc, float skin) {
+    if (n <= 0 || !box_ok(box) || !(rc > 0.f) || !(skin >= 0.f)) return 0;
+    const float rs = rc + skin;
+    return nbr_layout(nullptr, n, make_grid(n, box, rs)).total;
+}
+
+tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, float skin, int cap, int flags,
+                            void* ws, size_t ws_bytes, int32_t* nbr, int32_t* counts, int32_t* overflow,
+                            cudaStream_t s) {
+    if (n <= 0 || !pos || !ws || !nbr || !counts || !overflow || cap < 1) return TESS_ERR_INVALID_ARG;
+    if (!box_ok(box) || !(rc > 0.f) || !(skin >= 0.f) || !std::isfinite(rc) || !std::isfinite(skin))
+        return TESS_ERR_INVALID_ARG;
+    if ((flags & ~TESS_NO_PAD_FILL) != 0) return TESS_ERR_INVALID_ARG;
+    if (!aligned(pos, 16) || !aligned(ws, 256) || !aligned(nbr, 4) || !aligned(counts, 4)) return TESS_ERR_INVALID_ARG;
+    const float rs = rc + skin;
+    if (box.lx < 2.f * rs || box.ly < 2.f * rs || box.lz < 2.f * rs) return TESS_ERR_BOX_TOO_SMALL;
+    const Grid g = make_grid(n, box, rs);
+    NbrLayout L = nbr_layout(ws, n, g);
+    if (ws_bytes < L.total) return TESS_ERR_WORKSPACE_TOO_SMALL;
+
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const float4* pos4 = reinterpret_cast<const float4*>(pos);
+    const int3 nc = make_int3(g.nc[0], g.nc[1], g.nc[2]);
+    const float3 inv_w = make_float3(g.inv_w[0], g.inv_w[1], g.inv_w[2]);
+    const float3 Lb = make_float3(box.lx, box.ly, box.lz);
+    const long long m = g.ncell;
+    const long long scan_tiles = (m + SCAN_TILE - 1) / SCAN_TILE;
+
+    cudaMemsetAsync(overflow, 0, sizeof(int32_t), s);
+    {
+        StageScope sc(ST_CELLS, s);
+        cudaMemsetAsync(L.cnt, 0, sizeof(int) * (size_t)m, s);
+        const int blocks = (int)std::min<long long>(((long long)n + 255) / 256, (long long)sms * 16);
+        cell_count_kernel<<<blocks, 256, 0, s>>>(pos4, n, nc, inv_w, Lb, L.cell_id, L.cnt, overflow);
+        scan_reduce_kernel<<<(unsigned)scan_tiles, SCAN_THREADS, 0, s>>>(L.cnt, m, L.sums);
+        scan_sums_kernel<<<1, SCAN_THREADS, 0, s>>>(L.sums, scan_tiles);
+        scan_apply_kernel<<<(unsigned)scan_tiles, SCAN_THREADS, 0, s>>>(L.cnt, m, L.sums, L.cell_start);
+        cell_scatter_kernel<<<blocks, 256, 0, s>>>(L.cell_id, n, L.cell_start, L.cnt, L.slot_atom);
+        cell_order_kernel<<<blocks, 256, 0, s>>>(L.slot_atom, n, L.cell_id, L.cell_start, pos4, L.pos_cell);
+        count_launch(6);
+    }
+    {
+        StageScope sc(ST_PAIRS, s);
+        PairArgs A;
+        A.pos = pos4;
+        A.pos_cell = L.pos_cell;
+        A.cell_start = L.cell_start;
+        A.n = n;
+        A.cap = cap;
+        A.pad_fill = (flags & TESS_NO_PAD_FILL) ? 0 : 1;
+        A.nc = nc;
+        A.inv_w = inv_w;
+        A.L = Lb;
+        A.rs2 = rs * rs;
+        const float lmax = std::max(box.lx, std::max(box.ly, box.lz));
+        A.reach = rs + 1e-3f + 4e-6f * lmax;
+        A.nbr = nbr;
+        A.counts = counts;
+        A.status = overflow;
+        const long long ntiles = ((long long)n + 31) / 32;
+        const size_t smem_rows = ps_warp_smem(cap, true) * PS_WARPS;
+        const bool rows_ok = smem_rows <= 200 * 1024 && aligned(nbr, 16);
+        const size_t smem = rows_ok ? smem_rows : ps_warp_smem(cap, false) * PS_WARPS;
+        if (rows_ok) {
+            cudaFuncSetAttribute(pair_search_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            const long long blocks = (ntiles + PS_WARPS - 1) / PS_WARPS;
+            pair_search_kernel<true><<<(unsigned)std::min<long long>(blocks, 1LL << 30), PS_WARPS * 32, smem, s>>>(A);
+        } else {
+            cudaFuncSetAttribute(pair_search_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            const long long blocks = (ntiles + PS_WARPS - 1) / PS_WARPS;
+            pair_search_kernel<false><<<(unsigned)std::min<long long>(blocks, 1LL << 30), PS_WARPS * 32, smem, s>>>(A);
+        }
+        count_launch();
+    }
+    return launch_status();
+}
+
+}  // namespace tess

@@ -1,0 +1,69 @@
+"""The C ABI library loads on a machine without a GPU and exports every
+symbol that include/tess.h declares; host-side argument checks and
+workspace queries work without touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import space_filling_curve_b200 as tess
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "tess.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tess_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from space_filling_curve_b200 import build
+    build.build()
+    return tess.lib()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert len(names) >= 10
+    for name in names:
+        assert hasattr(lib, name), name
+    # and the Python binding carries the same names
+    for name in names:
+        assert hasattr(tess, name), name
+
+
+def test_status_strings_and_version(lib):
+    assert tess.tess_status_string(0) == "ok"
+    assert "workspace" in tess.tess_status_string(3)
+    assert "sm_100a" in tess.tess_version()
+
+
+def test_workspace_queries_are_host_only(lib):
+    box = (467.84283, 467.84283, 467.84283)
+    a = tess.tess_hilbert_sort_workspace(10_240_000)
+    b = tess.tess_build_neighbors_workspace(10_240_000, box, 5.75, 0.5)
+    assert a > 16 * 10_240_000 and b > 24 * 10_240_000
+    assert tess.tess_hilbert_sort_workspace(0) == 0
+    assert tess.tess_build_neighbors_workspace(10, box, -1.0, 0.5) == 0
+    # sized for 10.24M atoms, the buffers fit comfortably in 180 GB
+    assert a + b < 2 * 1024 ** 3
+
+
+def test_argument_errors_are_reported_before_any_launch(lib):
+    null = None
+    box = (30.0, 30.0, 30.0)
+    assert tess.tess_hilbert_sort(null, 10, box, 10, null, 0, null, null, null, null, null) == 1
+    assert tess.tess_hilbert_sort(ctypes.c_void_p(256), 10, box, 11, ctypes.c_void_p(256), 1 << 20,
+                                  ctypes.c_void_p(256), null, null, null, null) == 1
+    # box below 2 (rc + skin): rejected on the host
+    p = ctypes.c_void_p(256)
+    assert tess.tess_build_neighbors(p, 10, (12.0, 30.0, 30.0), 6.0, 0.5, 16, 0, p, 1 << 30, p, p, p, null) == 2
+    # workspace too small
+    assert tess.tess_build_neighbors(p, 10, box, 6.0, 0.5, 16, 0, p, 16, p, p, p, null) == 3
+    # unknown flag
+    assert tess.tess_build_neighbors(p, 10, box, 6.0, 0.5, 16, 8, p, 1 << 30, p, p, p, null) == 1
+    assert tess.tess_skin_check(p, p, 10, box, -0.5, p, null, null) == 1
+    assert tess.tess_edge_aggregate(p, 10, box, 6.0, p, p, 16, p, 0, p, null, null, null, null) == 1

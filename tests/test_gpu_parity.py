@@ -1,0 +1,300 @@
+"""GPU parity: the CUDA path through the C ABI against the oracle, element
+by element, on seeded inputs (configs 1-2, smaller systems of the same
+kinds, ragged sizes and edge cases).  Integer results (keys, permutations,
+neighbor sets, counts, flags) must match bit-exactly; aggregated features
+within 1e-5 relative error (condition-aware, see gpu_util.agg_error).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_util import agg_error, canon_rows, canon_rows_gpu, torch_cuda
+
+pytestmark = pytest.mark.gpu
+
+AGG_TOL = 1e-5
+
+
+def _tess():
+    import space_filling_curve_b200 as tess
+    return tess
+
+
+def _dev(a):
+    torch = torch_cuda()
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def _gpu_sort(pos, box, bits=10):
+    tess = _tess()
+    perm, keys, ps, st = tess.hilbert_sort(_dev(pos), box, bits)
+    torch_cuda().cuda.synchronize()
+    return perm.cpu().numpy(), keys.cpu().numpy().view(np.uint32), ps.cpu().numpy(), int(st.item())
+
+
+# ------------------------------------------------------------------ Hilbert sort
+
+
+@pytest.mark.parametrize("n", [1, 2, 31, 33, 4095, 4096, 4097, 12293])
+def test_sort_ragged_sizes(n):
+    rng = np.random.default_rng(n)
+    box = (40.0, 50.0, 60.0)
+    pos = (rng.uniform(0, 1, (n, 3)) * np.array(box)).astype(np.float32)
+    perm, keys, ps, st = _gpu_sort(pos, box)
+    operm, okeys = oracle.hilbert_sort(pos, box, 10)
+    assert st == 0
+    assert np.array_equal(keys, okeys)
+    assert np.array_equal(perm, operm)
+    assert np.array_equal(ps[:, :3], pos[operm]) and np.all(ps[:, 3] == 0)
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 5, 7, 8, 9, 10])
+def test_sort_every_width_with_ties(bits):
+    # a coarse grid forces long runs of equal keys: ties must keep input order
+    rng = np.random.default_rng(bits)
+    box = (31.0, 31.0, 31.0)
+    pos = (rng.uniform(0, 31.0, (20000, 3))).astype(np.float32)
+    perm, keys, _, _ = _gpu_sort(pos, box, bits)
+    operm, okeys = oracle.hilbert_sort(pos, box, bits)
+    assert np.array_equal(keys, okeys) and np.array_equal(perm, operm)
+
+
+def test_sort_grid_points_exhaustive_keys():
+    # every cell centre of a 2^6 grid: the GPU keys equal the oracle's index
+    bits = 6
+    g = np.stack(np.meshgrid(*[np.arange(64)] * 3, indexing="ij"), -1).reshape(-1, 3)
+    box = (64.0, 64.0, 64.0)
+    pos = (g + 0.5).astype(np.float32)
+    _, keys, _, _ = _gpu_sort(pos, box, bits)
+    okeys = oracle.hilbert_index_grid(g.astype(np.uint32), bits)
+    assert np.array_equal(np.sort(keys), np.sort(okeys))
+    perm, _, _, _ = _gpu_sort(pos, box, bits)
+    assert np.array_equal(okeys[perm], np.arange(64 ** 3, dtype=np.uint32))
+
+
+def test_sort_flags_out_of_box_input():
+    pos = np.array([[1, 1, 1], [-0.5, 2, 2], [3, 3, 40.0]], np.float32)
+    box = (30.0, 30.0, 30.0)
+    perm, keys, _, st = _gpu_sort(pos, box)
+    assert st & 2
+    operm, okeys = oracle.hilbert_sort(pos, box, 10)     # both clamp into the grid
+    assert np.array_equal(keys, okeys) and np.array_equal(perm, operm)
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3])
+def test_sort_configs(cfg):
+    s = synth.system(cfg)
+    perm, keys, ps, st = _gpu_sort(s.pos, s.box)
+    operm, okeys = oracle.hilbert_sort(s.pos, s.box, 10)
+    assert st == 0
+    assert np.array_equal(keys, okeys) and np.array_equal(perm, operm)
+
+
+# ------------------------------------------------------------------ neighbors
+
+
+def _gpu_list(pos4, box, rc, skin, cap, pad_fill=True):
+    tess = _tess()
+    nbr, cnt, ov = tess.build_neighbors(_dev(pos4), box, rc, skin, cap, pad_fill=pad_fill)
+    torch_cuda().cuda.synchronize()
+    return nbr, cnt, int(ov.item())
+
+
+def _check_list(pos4, box, rc, skin, cap, pad_fill=True, method="cells"):
+    nbr_d, cnt_d, ov = _gpu_list(pos4, box, rc, skin, cap, pad_fill)
+    fn = oracle.neighbors_cells if method == "cells" else oracle.neighbors_brute
+    onbr, ocnt, oov = fn(pos4, box, rc, skin, cap)
+    cnt = cnt_d.cpu().numpy()
+    assert np.array_equal(cnt, ocnt)
+    assert (ov & 1) == oov
+    rows = canon_rows_gpu(nbr_d, cnt_d)
+    full = ocnt <= cap
+    assert np.array_equal(rows[full], onbr[full])
+    if pad_fill:
+        nb = nbr_d.cpu().numpy()
+        slot = np.arange(cap)[None, :]
+        assert np.all(nb[slot >= np.minimum(cnt, cap)[:, None]] == -1)
+    if (~full).any():
+        # overflowing rows: whatever is stored must be true neighbors, distinct
+        nb = nbr_d.cpu().numpy()
+        for i in np.nonzero(~full)[0][:200]:
+            stored = nb[i, :cap]
+            truth = set(oracle.neighbors_of(pos4, box, rc, skin, int(i)).tolist())
+            assert len(set(stored.tolist())) == cap and set(stored.tolist()) <= truth
+    return nbr_d, cnt
+
+
+@pytest.mark.parametrize("cfg", [1, 2])
+def test_neighbors_configs_sorted_order(cfg):
+    s = synth.system(cfg)
+    perm, _ = oracle.hilbert_sort(s.pos, s.box, 10)
+    p4 = s.pos4()[perm]
+    _check_list(p4, s.box, s.rc, s.skin, s.cap)
+
+
+def test_neighbors_config3():
+    s = synth.system(3)
+    perm, _ = oracle.hilbert_sort(s.pos, s.box, 10)
+    _check_list(s.pos4()[perm], s.box, s.rc, s.skin, s.cap)
+
+
+def test_neighbors_unsorted_input_gives_the_same_sets():
+    s = synth.system(1)
+    _check_list(s.pos4(), s.box, s.rc, s.skin, s.cap, method="brute")
+
+
+@pytest.mark.parametrize("n", [1, 2, 31, 32, 33, 97, 1000])
+def test_neighbors_ragged(n):
+    rng = np.random.default_rng(100 + n)
+    L = 30.0
+    p = np.zeros((n, 4), np.float32)
+    p[:, :3] = rng.uniform(0, L, (n, 3))
+    _check_list(p, (L, L, L), 4.0, 0.5, 64, method="brute")
+
+
+def test_neighbors_no_pad_fill_and_overflow():
+    s = synth.system(1)
+    perm, _ = oracle.hilbert_sort(s.pos, s.box, 10)
+    p4 = s.pos4()[perm]
+    _check_list(p4, s.box, s.rc, s.skin, s.cap, pad_fill=False)
+    _check_list(p4, s.box, s.rc, s.skin, 40)                 # overflow: flag, true counts
+    _check_list(p4, s.box, s.rc, s.skin, 40, pad_fill=False)
+
+
+@pytest.mark.parametrize("L,rc", [(13.0, 6.0), (19.6, 6.0), (25.0, 5.75)])
+def test_neighbors_small_boxes(L, rc):
+    # boxes of 2 to 4 list radii: the cell range of a tile wraps onto itself
+    rng = np.random.default_rng(int(L * 10))
+    n = int(0.1 * L ** 3)
+    p = np.zeros((n, 4), np.float32)
+    p[:, :3] = rng.uniform(0, L, (n, 3))
+    p = p[oracle.hilbert_sort(p, (L, L, L), 10)[0]]
+    _check_list(p, (L, L, L), rc, 0.5, 256, method="brute")
+
+
+def test_neighbors_large_cap_global_rows():
+    # a cap too large for shared-memory rows takes the global-row path
+    s = synth.system(1)
+    perm, _ = oracle.hilbert_sort(s.pos, s.box, 10)
+    _check_list(s.pos4()[perm], s.box, s.rc, s.skin, 1024)
+
+
+def test_neighbors_box_errors():
+    tess = _tess()
+    p = _dev(np.zeros((10, 4), np.float32))
+    with pytest.raises(tess.TessError) as e:
+        tess.build_neighbors(p, (12.9, 30, 30), 6.0, 0.5, 16)
+    assert e.value.code == 2
+
+
+# ------------------------------------------------------------------ skin check + rebuild loop
+
+
+def _run_loop(s, steps, gpu=True):
+    """Step 0 build, then per step: skin check; on a flag rebuild (sort +
+    list) and reset the reference.  Returns flags and rebuild data."""
+    tess = _tess()
+    torch = torch_cuda()
+    flags, maxd = [], []
+    frames = [(0, s.pos)] + list(s.trajectory(steps))
+    perm = None
+    ref4 = None
+    for t, pos in frames:
+        if t == 0:
+            need = True
+        else:
+            cur4 = np.zeros((s.n, 4), np.float32)
+            cur4[:, :3] = pos[perm]
+            if gpu:
+                rb, md = tess.skin_check(_dev(cur4), ref4, s.box, s.skin)
+                f, m = int(rb.item()), float(md.item())
+            else:
+                f, m = oracle.skin_check(cur4, ref4, s.box, s.skin)
+            flags.append(f)
+            maxd.append(m)
+            need = bool(f)
+        if need:
+            if gpu:
+                perm_d, _, ps, _ = tess.hilbert_sort(_dev(pos), s.box)
+                torch.cuda.synchronize()
+                perm = perm_d.cpu().numpy()
+                ref4 = ps
+            else:
+                perm, _ = oracle.hilbert_sort(pos, s.box, 10)
+                ref4 = np.zeros((s.n, 4), np.float32)
+                ref4[:, :3] = pos[perm]
+    return flags, maxd
+
+
+@pytest.mark.parametrize("cfg,steps", [(1, 20), (2, 60)])
+def test_skin_flags_over_trajectory(cfg, steps):
+    s = synth.system(cfg)
+    gf, gm = _run_loop(s, steps, gpu=True)
+    of, om = _run_loop(s, steps, gpu=False)
+    assert gf == of
+    assert gm == om                 # fp64, same operations: exact
+    assert any(gf), "the trajectory should trigger at least one rebuild"
+
+
+def test_skin_hand_cases():
+    tess = _tess()
+    ref = np.zeros((3, 4), np.float32)
+    ref[:, :3] = [[5, 5, 5], [19.9, 5, 5], [10, 10, 10]]
+    cur = ref.copy()
+    cur[1, 0] = 0.05                 # +0.15 through the face
+    cur[2, 1] += np.float32(0.24)
+    rb, md = tess.skin_check(_dev(cur), _dev(ref), (20, 20, 20), 0.5)
+    f, m = oracle.skin_check(cur, ref, (20, 20, 20), 0.5)
+    assert int(rb.item()) == f == 0 and float(md.item()) == m
+    cur[2, 1] = ref[2, 1] + np.float32(0.26)
+    rb, md = tess.skin_check(_dev(cur), _dev(ref), (20, 20, 20), 0.5)
+    f, m = oracle.skin_check(cur, ref, (20, 20, 20), 0.5)
+    assert int(rb.item()) == f == 1 and float(md.item()) == m
+
+
+# ------------------------------------------------------------------ edge aggregate
+
+
+@pytest.mark.parametrize("cfg", [1, 2])
+def test_edge_aggregate_configs(cfg):
+    tess = _tess()
+    s = synth.system(cfg)
+    perm, _ = oracle.hilbert_sort(s.pos, s.box, 10)
+    p4 = s.pos4()[perm]
+    feat = s.features()[perm]
+    nbr_d, cnt_d, _ = tess.build_neighbors(_dev(p4), s.box, s.rc, s.skin, s.cap)
+    out, ev, ef, eu = tess.edge_aggregate(_dev(p4), s.box, s.rc, nbr_d, cnt_d, _dev(feat), edges=True)
+    nbr, cnt = nbr_d.cpu().numpy(), cnt_d.cpu().numpy()
+    ref = oracle.edge_aggregate(p4, s.box, s.rc, nbr, cnt, feat, edges=True)
+    err, plain = agg_error(out.cpu().numpy(), ref)
+    assert err <= AGG_TOL, (err, plain)
+    ev, ef, eu = ev.cpu().numpy(), ef.cpu().numpy(), eu.cpu().numpy()
+    assert np.allclose(ev[..., :3], ref["edge_vec"][..., :3], rtol=0, atol=2e-5)
+    r = ref["edge_vec"][..., 3]
+    assert np.all(np.abs(ev[..., 3] - r) <= 1e-6 * np.maximum(r, 1.0))
+    assert np.all(np.abs(ef - ref["edge_fc"]) <= 1e-6)
+    assert np.allclose(eu, ref["edge_unit"], rtol=0, atol=2e-6)
+
+
+@pytest.mark.parametrize("F", [1, 7, 32, 33, 64, 100, 128])
+def test_edge_aggregate_feature_widths(F):
+    tess = _tess()
+    s = synth.custom("uniform", 1500, rc=5.0, cap=128, F=F)
+    p4 = s.pos4()
+    feat = s.features()
+    nbr_d, cnt_d, _ = tess.build_neighbors(_dev(p4), s.box, s.rc, s.skin, s.cap)
+    out = tess.edge_aggregate(_dev(p4), s.box, s.rc, nbr_d, cnt_d, _dev(feat))
+    ref = oracle.edge_aggregate(p4, s.box, s.rc, nbr_d.cpu().numpy(), cnt_d.cpu().numpy(), feat)
+    err, _ = agg_error(out.cpu().numpy(), ref)
+    assert err <= AGG_TOL
+
+
+def test_edge_aggregate_constant_features_sum_fc():
+    tess = _tess()
+    s = synth.system(1)
+    p4 = s.pos4()
+    nbr_d, cnt_d, _ = tess.build_neighbors(_dev(p4), s.box, s.rc, s.skin, s.cap)
+    ones = _dev(np.ones((s.n, 1), np.float32) * np.float32(3.0))
+    out, ev, ef, eu = tess.edge_aggregate(_dev(p4), s.box, s.rc, nbr_d, cnt_d, ones, edges=True)
+    assert np.allclose(out.cpu().numpy()[:, 0], 3.0 * ef.cpu().numpy().astype(np.float64).sum(1), rtol=1e-5)
