@@ -209,10 +209,12 @@ __global__ void cell_order_kernel(const int* __restrict__ slot_atom, int n, cons
 
 // ---------------------------------------------------------------- pair search
 
-constexpr int PS_WARPS = 2;          // warps per block
+constexpr int PS_WARPS = 4;          // warps per block (each warp owns its tiles)
 constexpr int PS_CHUNK = 256;        // culled candidates staged per warp before testing
 constexpr int PS_MAXSEG = 64;        // cell-row segments per table batch
 constexpr int PS_UNROLL = 4;         // candidate loads in flight per lane
+constexpr int PS_RING = 16;          // per-lane staging of accepted indices
+constexpr int PS_GROUP = 8;          // accepted indices leave in aligned groups of 8 (32 bytes)
 
 struct PairArgs {
     const float4* pos;
@@ -221,6 +223,7 @@ struct PairArgs {
     int n;
     int cap;
     int pad_fill;
+    int vec_rows;      // rows can take 16-byte stores (cap % 4 == 0, 16-byte aligned nbr)
     int3 nc;
     float3 inv_w;
     float3 L;
@@ -237,29 +240,64 @@ struct SegEntry {
     float sx, sy, sz, pad0, pad1, pad2;
 };
 
-__host__ __device__ constexpr size_t ps_warp_smem(int cap, bool rows_in_smem) {
-    return sizeof(float4) * PS_CHUNK + sizeof(SegEntry) * (PS_MAXSEG + 1) +
-           (rows_in_smem ? sizeof(int) * 32 * (size_t)cap : 0);
+// Per-warp shared memory: candidates as pairs in structure-of-arrays form so
+// that one 16-byte read gives (x0, x1, y0, y1) and another (z0, z1, j0, j1),
+// ready for packed f32x2 arithmetic; the segment table; the index rings.
+struct PairWarpSmem {
+    float4 ca[PS_CHUNK / 2];
+    float4 cb[PS_CHUNK / 2];
+    SegEntry seg[PS_MAXSEG + 1];
+    int ring[32 * PS_RING];
+};
+
+__device__ __forceinline__ unsigned long long pk(float lo, float hi) {
+    return (unsigned long long)__float_as_uint(lo) | ((unsigned long long)__float_as_uint(hi) << 32);
+}
+__device__ __forceinline__ float pk_lo(unsigned long long v) { return __uint_as_float((unsigned)v); }
+__device__ __forceinline__ float pk_hi(unsigned long long v) { return __uint_as_float((unsigned)(v >> 32)); }
+__device__ __forceinline__ unsigned long long f2_sub(unsigned long long a, unsigned long long b) {
+    unsigned long long d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
+    unsigned long long d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
+                                                     unsigned long long c) {
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
 }
 
-template <bool SMEM_ROWS>
-__global__ __launch_bounds__(PS_WARPS * 32, 8) void pair_search_kernel(PairArgs A) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
+// Store one accepted index into slot `slot` of a candidate pair array.
+__device__ __forceinline__ void put_cand(PairWarpSmem& W, int slot, float4 q) {
+    float* a = reinterpret_cast<float*>(&W.ca[slot >> 1]) + (slot & 1);
+    float* b = reinterpret_cast<float*>(&W.cb[slot >> 1]) + (slot & 1);
+    a[0] = q.x;
+    a[2] = q.y;
+    b[0] = q.z;
+    b[2] = q.w;
+}
+
+__global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs A) {
+    __shared__ PairWarpSmem smem_w[PS_WARPS];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    unsigned char* wbase = smem_raw + (size_t)warp * ps_warp_smem(A.cap, SMEM_ROWS);
-    float4* cand = reinterpret_cast<float4*>(wbase);
-    SegEntry* seg = reinterpret_cast<SegEntry*>(wbase + sizeof(float4) * PS_CHUNK);
-    int* rows = reinterpret_cast<int*>(wbase + sizeof(float4) * PS_CHUNK + sizeof(SegEntry) * (PS_MAXSEG + 1));
+    PairWarpSmem& W = smem_w[warp];
+    int* ring = W.ring + lane * PS_RING;
     const int cap = A.cap;
     const long long ntiles = ((long long)A.n + 31) / 32;
+    const float nanf_ = __int_as_float(0x7fc00000);
 
     for (long long tile = (long long)blockIdx.x * PS_WARPS + warp; tile < ntiles;
          tile += (long long)gridDim.x * PS_WARPS) {
         const int base = (int)(tile * 32);
         const int i = base + lane;
         const bool valid = i < A.n;
-        const float nanf_ = __int_as_float(0x7fc00000);
-        float4 p = valid ? A.pos[i] : make_float4(nanf_, nanf_, nanf_, 0.f);
+        const float4 p = valid ? A.pos[i] : make_float4(nanf_, nanf_, nanf_, 0.f);
+        int* row = A.nbr + (size_t)(valid ? i : 0) * cap;
 
         // level 1: tile bounding box
         float lox = valid ? p.x : INFINITY, loy = valid ? p.y : INFINITY, loz = valid ? p.z : INFINITY;
@@ -273,38 +311,63 @@ __global__ __launch_bounds__(PS_WARPS * 32, 8) void pair_search_kernel(PairArgs 
             hiy = fmaxf(hiy, __shfl_xor_sync(FULL, hiy, o));
             hiz = fmaxf(hiz, __shfl_xor_sync(FULL, hiz, o));
         }
-        // a non-finite position (invalid input) would make the box useless:
-        // fall back to the whole box for this tile
+        // a tile with no finite position (invalid input) searches the whole box;
+        // positions far outside the box must not blow up the cell ranges
         if (!(isfinite(lox) && isfinite(hix) && isfinite(loy) && isfinite(hiy) && isfinite(loz) && isfinite(hiz))) {
             lox = loy = loz = 0.f;
             hix = A.L.x; hiy = A.L.y; hiz = A.L.z;
         }
-        // positions far outside the box (invalid input, flagged by the
-        // binning) must not blow up the cell ranges
         lox = fmaxf(lox, -A.L.x); loy = fmaxf(loy, -A.L.y); loz = fmaxf(loz, -A.L.z);
         hix = fminf(hix, 2.f * A.L.x); hiy = fminf(hiy, 2.f * A.L.y); hiz = fminf(hiz, 2.f * A.L.z);
 
-        if (SMEM_ROWS && A.pad_fill) {
-            int4* r4 = reinterpret_cast<int4*>(rows);
-            for (int e = lane; e < 8 * cap; e += 32) r4[e] = make_int4(-1, -1, -1, -1);
-        }
-        int* myrow = SMEM_ROWS ? rows + lane * cap : A.nbr + (size_t)(valid ? i : 0) * cap;
-        int cnt = 0;
-        int ncand = 0;
+        int cnt = 0;       // accepted so far (true count)
+        int done = 0;      // accepted indices already written to the row
+        int ncand = 0;     // staged candidates (warp-uniform)
+        const unsigned long long px2 = pk(p.x, p.x), py2 = pk(p.y, p.y), pz2 = pk(p.z, p.z);
 
-        // level 3: test the staged chunk
-        auto flush = [&]() {
-            __syncwarp();
-            for (int c = 0; c < ncand; ++c) {
-                const float4 q = cand[c];
-                const float dx = q.x - p.x, dy = q.y - p.y, dz = q.z - p.z;
-                const float r2 = fmaf(dz, dz, fmaf(dy, dy, dx * dx));
-                const int j = __float_as_int(q.w);
-                if (r2 < A.rs2 && j != i) {
-                    if (SMEM_ROWS) myrow[min(cnt, cap - 1)] = j;
-                    else if (cnt < cap && valid) myrow[cnt] = j;
-                    ++cnt;
+        // move complete groups of 8 accepted indices from the ring to the row
+        auto drain = [&](bool all) {
+            while (cnt - done >= PS_GROUP || (all && cnt > done)) {
+                const int k = min(cnt - done, PS_GROUP);
+                const int* src = ring + (done & (PS_RING - 1));
+                if (k == PS_GROUP && done + PS_GROUP <= cap && A.vec_rows) {
+                    const int4 a = *reinterpret_cast<const int4*>(src);
+                    const int4 b = *reinterpret_cast<const int4*>(src + 4);
+                    *reinterpret_cast<int4*>(row + done) = a;
+                    *reinterpret_cast<int4*>(row + done + 4) = b;
+                } else {
+                    for (int e = 0; e < k; ++e)
+                        if (done + e < cap) row[done + e] = src[e];
                 }
+                done += k;
+            }
+        };
+
+        // level 3: test the staged candidates, two at a time in f32x2
+        auto test_chunk = [&]() {
+            __syncwarp();
+            if (ncand & 1) {
+                if (lane == 0) put_cand(W, ncand, make_float4(nanf_, nanf_, nanf_, __int_as_float(-1)));
+                ++ncand;
+                __syncwarp();
+            }
+            const int npair = ncand >> 1;
+            for (int c = 0; c < npair; c += 2) {
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    if (c + u < npair) {
+                        const float4 a = W.ca[c + u];
+                        const float4 b = W.cb[c + u];
+                        const unsigned long long dx = f2_sub(pk(a.x, a.y), px2);
+                        const unsigned long long dy = f2_sub(pk(a.z, a.w), py2);
+                        const unsigned long long dz = f2_sub(pk(b.x, b.y), pz2);
+                        const unsigned long long r2 = f2_fma(dz, dz, f2_fma(dy, dy, f2_mul(dx, dx)));
+                        const int j0 = __float_as_int(b.z), j1 = __float_as_int(b.w);
+                        if (pk_lo(r2) < A.rs2 && j0 != i) ring[cnt++ & (PS_RING - 1)] = j0;
+                        if (pk_hi(r2) < A.rs2 && j1 != i) ring[cnt++ & (PS_RING - 1)] = j1;
+                    }
+                }
+                if (cnt - done >= PS_GROUP) drain(false);
             }
             ncand = 0;
             __syncwarp();
@@ -321,7 +384,6 @@ __global__ __launch_bounds__(PS_WARPS * 32, 8) void pair_search_kernel(PairArgs 
 
         for (int sb = 0; sb < nseg; sb += PS_MAXSEG) {
             const int nb = min(PS_MAXSEG, nseg - sb);
-            // segment table: lane-parallel decode and bounds
             int run = 0;
             for (int s0 = 0; s0 < nb; s0 += 32) {
                 const int sl = s0 + lane;
@@ -330,8 +392,8 @@ __global__ __launch_bounds__(PS_WARPS * 32, 8) void pair_search_kernel(PairArgs 
                 if (sl < nb) {
                     const int s = sb + sl;
                     const int piece = s % npieces;
-                    const int row = s / npieces;
-                    const int uy = uy0 + row % ny, uz = uz0 + row / ny;
+                    const int rw = s / npieces;
+                    const int uy = uy0 + rw % ny, uz = uz0 + rw / ny;
                     const int ky = floor_div(uy, A.nc.y), kz = floor_div(uz, A.nc.z);
                     const int cy = uy - ky * A.nc.y, cz = uz - kz * A.nc.z;
                     const int kx = floor_div(ux0, A.nc.x) + piece;
@@ -351,20 +413,20 @@ __global__ __launch_bounds__(PS_WARPS * 32, 8) void pair_search_kernel(PairArgs 
                     if (lane >= o) inc += y;
                 }
                 if (sl < nb) {
-                    SegEntry& e = seg[sl];
+                    SegEntry& e = W.seg[sl];
                     e.beg = beg;
                     e.pre = run + inc - len;
                     e.sx = sx; e.sy = sy; e.sz = sz;
                 }
                 run += __shfl_sync(FULL, inc, 31);
             }
-            if (lane == 0) seg[nb].pre = run;
+            if (lane == 0) W.seg[nb].pre = run;
             __syncwarp();
             const int total = run;
 
             int sc = 0;   // this lane's segment cursor
             for (int t0 = 0; t0 < total; t0 += 32 * PS_UNROLL) {
-                if (ncand > PS_CHUNK - 32 * PS_UNROLL) flush();
+                if (ncand > PS_CHUNK - 1 - 32 * PS_UNROLL) test_chunk();
                 float4 q[PS_UNROLL];
                 bool ok[PS_UNROLL];
 #pragma unroll
@@ -372,8 +434,8 @@ __global__ __launch_bounds__(PS_WARPS * 32, 8) void pair_search_kernel(PairArgs 
                     const int t = t0 + u * 32 + lane;
                     ok[u] = t < total;
                     if (ok[u]) {
-                        while (seg[sc + 1].pre <= t) ++sc;
-                        const SegEntry& e = seg[sc];
+                        while (W.seg[sc + 1].pre <= t) ++sc;
+                        const SegEntry& e = W.seg[sc];
                         const float4 c = A.pos_cell[e.beg + (t - e.pre)];
                         q[u] = make_float4(c.x + e.sx, c.y + e.sy, c.z + e.sz, c.w);
                     }
@@ -388,39 +450,28 @@ __global__ __launch_bounds__(PS_WARPS * 32, 8) void pair_search_kernel(PairArgs 
                         keep = fmaf(ez, ez, fmaf(ey, ey, ex * ex)) < reach2;
                     }
                     const unsigned bm = __ballot_sync(FULL, keep);
-                    if (keep) cand[ncand + __popc(bm & lanemask_lt())] = q[u];
+                    if (keep) put_cand(W, ncand + __popc(bm & lanemask_lt()), q[u]);
                     ncand += __popc(bm);
                 }
             }
             __syncwarp();
         }
-        flush();
+        test_chunk();
+        drain(true);
 
-        // write the tile's rows
-        if (valid) A.counts[i] = cnt;
+        if (valid) {
+            A.counts[i] = cnt;
+            if (A.pad_fill) {
+                int e = min(cnt, cap);
+                if (A.vec_rows) {
+                    for (; e < cap && (e & 3); ++e) row[e] = -1;
+                    for (; e + 4 <= cap; e += 4) *reinterpret_cast<int4*>(row + e) = make_int4(-1, -1, -1, -1);
+                }
+                for (; e < cap; ++e) row[e] = -1;
+            }
+        }
         const unsigned ov = __ballot_sync(FULL, valid && cnt > cap);
         if (ov && lane == 0) atomicOr(A.status, TESS_DEV_OVERFLOW);
-        const int nvalid = min(32, A.n - base);
-        if (SMEM_ROWS) {
-            __syncwarp();
-            int* gdst = A.nbr + (size_t)base * cap;
-            if (A.pad_fill) {
-                const long long total = (long long)nvalid * cap;
-                const long long n4 = total / 4;
-                const int4* s4 = reinterpret_cast<const int4*>(rows);
-                int4* g4 = reinterpret_cast<int4*>(gdst);
-                for (long long e = lane; e < n4; e += 32) g4[e] = s4[e];
-                for (long long e = n4 * 4 + lane; e < total; e += 32) gdst[e] = rows[e];
-            } else {
-                for (int r = 0; r < nvalid; ++r) {
-                    const int m = min(__shfl_sync(FULL, cnt, r), cap);
-                    for (int e = lane; e < m; e += 32) gdst[(size_t)r * cap + e] = rows[r * cap + e];
-                }
-            }
-            __syncwarp();
-        } else if (A.pad_fill && valid) {
-            for (int e = min(cnt, cap); e < cap; ++e) myrow[e] = -1;
-        }
     }
 }
 
@@ -506,6 +557,7 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
         A.n = n;
         A.cap = cap;
         A.pad_fill = (flags & TESS_NO_PAD_FILL) ? 0 : 1;
+        A.vec_rows = (cap % 4 == 0 && aligned(nbr, 16)) ? 1 : 0;
         A.nc = nc;
         A.inv_w = inv_w;
         A.L = Lb;
@@ -516,18 +568,8 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
         A.counts = counts;
         A.status = overflow;
         const long long ntiles = ((long long)n + 31) / 32;
-        const size_t smem_rows = ps_warp_smem(cap, true) * PS_WARPS;
-        const bool rows_ok = smem_rows <= 200 * 1024 && aligned(nbr, 16);
-        const size_t smem = rows_ok ? smem_rows : ps_warp_smem(cap, false) * PS_WARPS;
-        if (rows_ok) {
-            cudaFuncSetAttribute(pair_search_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            const long long blocks = (ntiles + PS_WARPS - 1) / PS_WARPS;
-            pair_search_kernel<true><<<(unsigned)std::min<long long>(blocks, 1LL << 30), PS_WARPS * 32, smem, s>>>(A);
-        } else {
-            cudaFuncSetAttribute(pair_search_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-            const long long blocks = (ntiles + PS_WARPS - 1) / PS_WARPS;
-            pair_search_kernel<false><<<(unsigned)std::min<long long>(blocks, 1LL << 30), PS_WARPS * 32, smem, s>>>(A);
-        }
+        const long long blocks = (ntiles + PS_WARPS - 1) / PS_WARPS;
+        pair_search_kernel<<<(unsigned)std::min<long long>(blocks, 1LL << 30), PS_WARPS * 32, 0, s>>>(A);
         count_launch();
     }
     return launch_status();

@@ -160,6 +160,109 @@ __global__ __launch_bounds__(EDGE_WARPS * 32) void edge_kernel(EdgeArgs A) {
     }
 }
 
+constexpr int EV_WARPS = 8;
+constexpr int EV_MAXCAP = 512;       // live edges of one row staged in shared memory
+constexpr int EV_GEO_UNROLL = 4;     // neighbor/position loads in flight per lane
+constexpr int EV_ACC_UNROLL = 4;     // feature rows in flight per lane group
+
+// Features as float4 (F % 4 == 0, F <= 128): LPE = F/4 lanes share one edge,
+// so a warp reads 32/LPE neighbor feature rows per instruction with 16-byte
+// loads.  Phase 1 computes the geometry of the whole row (one edge per lane,
+// several loads in flight) and compacts the live (j, f_c) pairs into shared
+// memory; phase 2 accumulates f_c * h_j with several rows in flight; the lane
+// groups are then summed with shuffles.
+template <int LPE>
+__global__ __launch_bounds__(EV_WARPS * 32) void edge_vec4_kernel(EdgeArgs A) {
+    constexpr int EPI = 32 / LPE;
+    __shared__ int2 s_edge[EV_WARPS][EV_MAXCAP];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int2* live_e = s_edge[warp];
+    const int g = lane / LPE, fl = lane % LPE;
+    const int F4 = A.F / 4;
+    const float4* feat4 = reinterpret_cast<const float4*>(A.feat);
+    float4* out4 = reinterpret_cast<float4*>(A.out);
+    const bool edges = A.edge_vec || A.edge_fc || A.edge_unit;
+    for (long long i = (long long)blockIdx.x * EV_WARPS + warp; i < A.n; i += (long long)gridDim.x * EV_WARPS) {
+        const float4 pi = A.pos[i];
+        const int m = max(min(A.counts[i], A.cap), 0);
+        const int limit = edges ? A.cap : m;
+        int nlive = 0;
+        for (int s0 = 0; s0 < limit; s0 += 32 * EV_GEO_UNROLL) {
+            int j[EV_GEO_UNROLL];
+            float4 pj[EV_GEO_UNROLL];
+#pragma unroll
+            for (int u = 0; u < EV_GEO_UNROLL; ++u) {
+                const int s = s0 + u * 32 + lane;
+                j[u] = (s < m) ? A.nbr[(size_t)i * A.cap + s] : -1;
+                if (j[u] >= A.n) j[u] = -1;
+            }
+#pragma unroll
+            for (int u = 0; u < EV_GEO_UNROLL; ++u)
+                if (j[u] >= 0) pj[u] = A.pos[j[u]];
+#pragma unroll
+            for (int u = 0; u < EV_GEO_UNROLL; ++u) {
+                const int s = s0 + u * 32 + lane;
+                float fc = 0.f;
+                if (j[u] >= 0) {
+                    const float dx = min_image_f(pj[u].x - pi.x, A.L.x);
+                    const float dy = min_image_f(pj[u].y - pi.y, A.L.y);
+                    const float dz = min_image_f(pj[u].z - pi.z, A.L.z);
+                    const float r = sqrtf(fmaf(dz, dz, fmaf(dy, dy, dx * dx)));
+                    fc = r < A.rc ? 0.5f * (cospif(r * A.inv_rc) + 1.0f) : 0.0f;
+                    if (edges) {
+                        const size_t e = (size_t)i * A.cap + s;
+                        const float inv_r = r > 0.f ? 1.0f / r : 0.f;
+                        if (A.edge_vec) A.edge_vec[e] = make_float4(dx, dy, dz, r);
+                        if (A.edge_fc) A.edge_fc[e] = fc;
+                        if (A.edge_unit) A.edge_unit[e] = make_float4(dx * inv_r, dy * inv_r, dz * inv_r, 0.f);
+                    }
+                } else if (edges && s < A.cap) {
+                    const size_t e = (size_t)i * A.cap + s;
+                    if (A.edge_vec) A.edge_vec[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (A.edge_fc) A.edge_fc[e] = 0.f;
+                    if (A.edge_unit) A.edge_unit[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+                const unsigned live = __ballot_sync(FULL, fc != 0.f);
+                if (fc != 0.f) live_e[nlive + __popc(live & lanemask_lt())] = make_int2(j[u], __float_as_int(fc));
+                nlive += __popc(live);
+            }
+        }
+        __syncwarp();
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int e0 = 0; e0 < nlive; e0 += EPI * EV_ACC_UNROLL) {
+            int2 ed[EV_ACC_UNROLL];
+            float4 h[EV_ACC_UNROLL];
+#pragma unroll
+            for (int u = 0; u < EV_ACC_UNROLL; ++u) {
+                const int e = e0 + u * EPI + g;
+                ed[u] = (e < nlive) ? live_e[e] : make_int2(-1, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < EV_ACC_UNROLL; ++u)
+                if (ed[u].x >= 0) h[u] = feat4[(size_t)ed[u].x * F4 + fl];
+#pragma unroll
+            for (int u = 0; u < EV_ACC_UNROLL; ++u) {
+                if (ed[u].x >= 0) {
+                    const float w = __int_as_float(ed[u].y);
+                    acc.x = fmaf(w, h[u].x, acc.x);
+                    acc.y = fmaf(w, h[u].y, acc.y);
+                    acc.z = fmaf(w, h[u].z, acc.z);
+                    acc.w = fmaf(w, h[u].w, acc.w);
+                }
+            }
+        }
+#pragma unroll
+        for (int o = LPE; o < 32; o <<= 1) {
+            acc.x += __shfl_xor_sync(FULL, acc.x, o);
+            acc.y += __shfl_xor_sync(FULL, acc.y, o);
+            acc.z += __shfl_xor_sync(FULL, acc.z, o);
+            acc.w += __shfl_xor_sync(FULL, acc.w, o);
+        }
+        if (g == 0) out4[(size_t)i * F4 + fl] = acc;
+        __syncwarp();
+    }
+}
+
 tess_status edge_aggregate(const float* pos, int n, tess_box box, float rc, const int32_t* nbr, const int32_t* counts,
                            int cap, const float* feat, int F, float* out, float* edge_vec, float* edge_fc,
                            float* edge_unit, cudaStream_t s) {
@@ -190,9 +293,23 @@ tess_status edge_aggregate(const float* pos, int n, tess_box box, float rc, cons
     StageScope sc(ST_EDGE, s);
     const long long rows_blocks = ((long long)n + EDGE_WARPS - 1) / EDGE_WARPS;
     const int blocks = (int)std::min<long long>(rows_blocks, (long long)sms * 64);
-    const bool vec2 = (F % 2 == 0) && aligned(feat, 8) && F >= 64;
-    if (vec2) edge_kernel<2><<<blocks, EDGE_WARPS * 32, 0, s>>>(A);
-    else edge_kernel<1><<<blocks, EDGE_WARPS * 32, 0, s>>>(A);
+    const bool vec4 = (F % 4 == 0) && F <= 128 && aligned(feat, 16) && aligned(out, 16) && cap <= EV_MAXCAP;
+    if (vec4) {
+        const int vblocks = (int)std::min<long long>(((long long)n + EV_WARPS - 1) / EV_WARPS, (long long)sms * 32);
+        switch (F / 4) {
+            case 1: edge_vec4_kernel<1><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
+            case 2: edge_vec4_kernel<2><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
+            case 4: edge_vec4_kernel<4><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
+            case 8: edge_vec4_kernel<8><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
+            case 16: edge_vec4_kernel<16><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
+            case 32: edge_vec4_kernel<32><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
+            default: edge_kernel<1><<<blocks, EDGE_WARPS * 32, 0, s>>>(A); break;
+        }
+    } else if ((F % 2 == 0) && aligned(feat, 8) && F >= 64) {
+        edge_kernel<2><<<blocks, EDGE_WARPS * 32, 0, s>>>(A);
+    } else {
+        edge_kernel<1><<<blocks, EDGE_WARPS * 32, 0, s>>>(A);
+    }
     count_launch();
     return launch_status();
 }
