@@ -213,8 +213,9 @@ constexpr int PS_WARPS = 4;          // warps per block (each warp owns its tile
 constexpr int PS_CHUNK = 256;        // culled candidates staged per warp before testing
 constexpr int PS_MAXSEG = 64;        // cell-row segments per table batch
 constexpr int PS_UNROLL = 4;         // candidate loads in flight per lane
-constexpr int PS_RING = 16;          // per-lane staging of accepted indices
+constexpr int PS_BUF = 32;           // per-lane staging of accepted indices (linear)
 constexpr int PS_GROUP = 8;          // accepted indices leave in aligned groups of 8 (32 bytes)
+constexpr int PS_TEST_UNROLL = 8;    // candidate pairs tested between fullness votes
 
 struct PairArgs {
     const float4* pos;
@@ -247,7 +248,7 @@ struct PairWarpSmem {
     float4 ca[PS_CHUNK / 2];
     float4 cb[PS_CHUNK / 2];
     SegEntry seg[PS_MAXSEG + 1];
-    int ring[32 * PS_RING];
+    int buf[32 * PS_BUF];
 };
 
 __device__ __forceinline__ unsigned long long pk(float lo, float hi) {
@@ -286,7 +287,7 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
     __shared__ PairWarpSmem smem_w[PS_WARPS];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     PairWarpSmem& W = smem_w[warp];
-    int* ring = W.ring + lane * PS_RING;
+    int* const buf = W.buf + lane * PS_BUF;
     const int cap = A.cap;
     const long long ntiles = ((long long)A.n + 31) / 32;
     const float nanf_ = __int_as_float(0x7fc00000);
@@ -320,30 +321,45 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
         lox = fmaxf(lox, -A.L.x); loy = fmaxf(loy, -A.L.y); loz = fmaxf(loz, -A.L.z);
         hix = fminf(hix, 2.f * A.L.x); hiy = fminf(hiy, 2.f * A.L.y); hiz = fminf(hiz, 2.f * A.L.z);
 
-        int cnt = 0;       // accepted so far (true count)
-        int done = 0;      // accepted indices already written to the row
+        int done = 0;      // accepted indices already written to the row (a multiple of 8 until the end)
+        int* wp = buf;     // next free slot of this lane's buffer
         int ncand = 0;     // staged candidates (warp-uniform)
         const unsigned long long px2 = pk(p.x, p.x), py2 = pk(p.y, p.y), pz2 = pk(p.z, p.z);
 
-        // move complete groups of 8 accepted indices from the ring to the row
+        // write the complete groups of 8 buffered indices to the row; with
+        // `all`, the remainder too.  The remainder of a partial drain moves
+        // to the front of the buffer.
         auto drain = [&](bool all) {
-            while (cnt - done >= PS_GROUP || (all && cnt > done)) {
-                const int k = min(cnt - done, PS_GROUP);
-                const int* src = ring + (done & (PS_RING - 1));
-                if (k == PS_GROUP && done + PS_GROUP <= cap && A.vec_rows) {
+            const int pend = (int)(wp - buf);
+            const int groups = pend / PS_GROUP;
+            for (int gi = 0; gi < groups; ++gi) {
+                const int* src = buf + gi * PS_GROUP;
+                if (done + PS_GROUP <= cap && A.vec_rows) {
                     const int4 a = *reinterpret_cast<const int4*>(src);
                     const int4 b = *reinterpret_cast<const int4*>(src + 4);
                     *reinterpret_cast<int4*>(row + done) = a;
                     *reinterpret_cast<int4*>(row + done + 4) = b;
                 } else {
-                    for (int e = 0; e < k; ++e)
+                    for (int e = 0; e < PS_GROUP; ++e)
                         if (done + e < cap) row[done + e] = src[e];
                 }
-                done += k;
+                done += PS_GROUP;
+            }
+            const int rest = pend - groups * PS_GROUP;
+            if (all) {
+                for (int e = 0; e < rest; ++e)
+                    if (done + e < cap) row[done + e] = buf[groups * PS_GROUP + e];
+                done += rest;
+                wp = buf;
+            } else {
+                for (int e = 0; e < rest; ++e) buf[e] = buf[groups * PS_GROUP + e];
+                wp = buf + rest;
             }
         };
 
-        // level 3: test the staged candidates, two at a time in f32x2
+        // level 3: test the staged candidates, two at a time in f32x2.  An
+        // accepted index is stored at the buffer pointer, which then advances
+        // (stores for rejected candidates are overwritten by the next one).
         auto test_chunk = [&]() {
             __syncwarp();
             if (ncand & 1) {
@@ -352,9 +368,11 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
                 __syncwarp();
             }
             const int npair = ncand >> 1;
-            for (int c = 0; c < npair; c += 2) {
+            for (int c = 0; c < npair; c += PS_TEST_UNROLL) {
+                // room for 2 * PS_TEST_UNROLL more in every lane's buffer?
+                if (__any_sync(FULL, (int)(wp - buf) > PS_BUF - 2 * PS_TEST_UNROLL)) drain(false);
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
+                for (int u = 0; u < PS_TEST_UNROLL; ++u) {
                     if (c + u < npair) {
                         const float4 a = W.ca[c + u];
                         const float4 b = W.cb[c + u];
@@ -363,11 +381,12 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
                         const unsigned long long dz = f2_sub(pk(b.x, b.y), pz2);
                         const unsigned long long r2 = f2_fma(dz, dz, f2_fma(dy, dy, f2_mul(dx, dx)));
                         const int j0 = __float_as_int(b.z), j1 = __float_as_int(b.w);
-                        if (pk_lo(r2) < A.rs2 && j0 != i) ring[cnt++ & (PS_RING - 1)] = j0;
-                        if (pk_hi(r2) < A.rs2 && j1 != i) ring[cnt++ & (PS_RING - 1)] = j1;
+                        *wp = j0;
+                        wp += (pk_lo(r2) < A.rs2 && j0 != i) ? 1 : 0;
+                        *wp = j1;
+                        wp += (pk_hi(r2) < A.rs2 && j1 != i) ? 1 : 0;
                     }
                 }
-                if (cnt - done >= PS_GROUP) drain(false);
             }
             ncand = 0;
             __syncwarp();
@@ -458,6 +477,7 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
         }
         test_chunk();
         drain(true);
+        const int cnt = done;
 
         if (valid) {
             A.counts[i] = cnt;

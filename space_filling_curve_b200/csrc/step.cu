@@ -77,13 +77,40 @@ struct EdgeArgs {
     float4* edge_unit;
     int n, cap, F;
     float3 L;
-    float rc, inv_rc;
+    float rc, inv_rc2;
 };
 
 __device__ __forceinline__ float min_image_f(float d, float L) {
     if (d > 0.5f * L) return d - L;
     if (d < -0.5f * L) return d + L;
     return d;
+}
+
+// Smooth cosine cutoff f_c = (cos(pi r / rc) + 1) / 2 for r < rc, as a
+// function of u = (r / rc)^2 in [0, 1): cos(pi sqrt(u)) is the Taylor series
+// sum_k (-pi^2 u)^k / (2k)!, which converges on the whole interval; eleven
+// terms leave a truncation error below 4e-9 at u = 1 and the fp32 Horner
+// evaluation adds a few 1e-7 at most (the largest partial terms are ~4).
+// No square root or trigonometric call is needed on the aggregation path.
+__host__ __device__ constexpr double cos_pi_sqrt_coef(int k) {
+    double c = 1.0;
+    for (int m = 1; m <= k; ++m) c *= -9.8696044010893586188 / ((2.0 * m - 1.0) * (2.0 * m));
+    return c;
+}
+
+__device__ __forceinline__ float cutoff_u(float u) {
+    float p = (float)cos_pi_sqrt_coef(10);
+    p = fmaf(p, u, (float)cos_pi_sqrt_coef(9));
+    p = fmaf(p, u, (float)cos_pi_sqrt_coef(8));
+    p = fmaf(p, u, (float)cos_pi_sqrt_coef(7));
+    p = fmaf(p, u, (float)cos_pi_sqrt_coef(6));
+    p = fmaf(p, u, (float)cos_pi_sqrt_coef(5));
+    p = fmaf(p, u, (float)cos_pi_sqrt_coef(4));
+    p = fmaf(p, u, (float)cos_pi_sqrt_coef(3));
+    p = fmaf(p, u, (float)cos_pi_sqrt_coef(2));
+    p = fmaf(p, u, (float)cos_pi_sqrt_coef(1));
+    p = fmaf(p, u, 1.0f);
+    return 0.5f * (p + 1.0f);
 }
 
 constexpr int EDGE_WARPS = 8;
@@ -119,9 +146,11 @@ __global__ __launch_bounds__(EDGE_WARPS * 32) void edge_kernel(EdgeArgs A) {
                     const float dx = min_image_f(pj.x - pi.x, A.L.x);
                     const float dy = min_image_f(pj.y - pi.y, A.L.y);
                     const float dz = min_image_f(pj.z - pi.z, A.L.z);
-                    const float r = sqrtf(fmaf(dz, dz, fmaf(dy, dy, dx * dx)));
-                    fc = r < A.rc ? 0.5f * (cospif(r * A.inv_rc) + 1.0f) : 0.0f;
+                    const float r2 = fmaf(dz, dz, fmaf(dy, dy, dx * dx));
+                    const float u = r2 * A.inv_rc2;
+                    fc = u < 1.0f ? cutoff_u(u) : 0.0f;
                     if (fc0 == 0 && edges) {
+                        const float r = sqrtf(r2);
                         const float inv_r = r > 0.f ? 1.0f / r : 0.f;
                         if (A.edge_vec) A.edge_vec[e] = make_float4(dx, dy, dz, r);
                         if (A.edge_fc) A.edge_fc[e] = fc;
@@ -163,7 +192,7 @@ __global__ __launch_bounds__(EDGE_WARPS * 32) void edge_kernel(EdgeArgs A) {
 constexpr int EV_WARPS = 8;
 constexpr int EV_MAXCAP = 512;       // live edges of one row staged in shared memory
 constexpr int EV_GEO_UNROLL = 4;     // neighbor/position loads in flight per lane
-constexpr int EV_ACC_UNROLL = 4;     // feature rows in flight per lane group
+constexpr int EV_ACC_UNROLL = 8;     // feature rows in flight per lane group
 
 // Features as float4 (F % 4 == 0, F <= 128): LPE = F/4 lanes share one edge,
 // so a warp reads 32/LPE neighbor feature rows per instruction with 16-byte
@@ -172,7 +201,7 @@ constexpr int EV_ACC_UNROLL = 4;     // feature rows in flight per lane group
 // memory; phase 2 accumulates f_c * h_j with several rows in flight; the lane
 // groups are then summed with shuffles.
 template <int LPE>
-__global__ __launch_bounds__(EV_WARPS * 32) void edge_vec4_kernel(EdgeArgs A) {
+__global__ __launch_bounds__(EV_WARPS * 32, 2) void edge_vec4_kernel(EdgeArgs A) {
     constexpr int EPI = 32 / LPE;
     __shared__ int2 s_edge[EV_WARPS][EV_MAXCAP];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -207,10 +236,12 @@ __global__ __launch_bounds__(EV_WARPS * 32) void edge_vec4_kernel(EdgeArgs A) {
                     const float dx = min_image_f(pj[u].x - pi.x, A.L.x);
                     const float dy = min_image_f(pj[u].y - pi.y, A.L.y);
                     const float dz = min_image_f(pj[u].z - pi.z, A.L.z);
-                    const float r = sqrtf(fmaf(dz, dz, fmaf(dy, dy, dx * dx)));
-                    fc = r < A.rc ? 0.5f * (cospif(r * A.inv_rc) + 1.0f) : 0.0f;
+                    const float r2 = fmaf(dz, dz, fmaf(dy, dy, dx * dx));
+                    const float u = r2 * A.inv_rc2;
+                    fc = u < 1.0f ? cutoff_u(u) : 0.0f;
                     if (edges) {
                         const size_t e = (size_t)i * A.cap + s;
+                        const float r = sqrtf(r2);
                         const float inv_r = r > 0.f ? 1.0f / r : 0.f;
                         if (A.edge_vec) A.edge_vec[e] = make_float4(dx, dy, dz, r);
                         if (A.edge_fc) A.edge_fc[e] = fc;
@@ -289,7 +320,7 @@ tess_status edge_aggregate(const float* pos, int n, tess_box box, float rc, cons
     A.F = F;
     A.L = make_float3(box.lx, box.ly, box.lz);
     A.rc = rc;
-    A.inv_rc = 1.0f / rc;
+    A.inv_rc2 = 1.0f / (rc * rc);
     StageScope sc(ST_EDGE, s);
     const long long rows_blocks = ((long long)n + EDGE_WARPS - 1) / EDGE_WARPS;
     const int blocks = (int)std::min<long long>(rows_blocks, (long long)sms * 64);
