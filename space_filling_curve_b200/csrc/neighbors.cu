@@ -215,7 +215,7 @@ constexpr int PS_MAXSEG = 64;        // cell-row segments per table batch
 constexpr int PS_UNROLL = 4;         // candidate loads in flight per lane
 constexpr int PS_BUF = 32;           // per-lane staging of accepted indices (linear)
 constexpr int PS_GROUP = 8;          // accepted indices leave in aligned groups of 8 (32 bytes)
-constexpr int PS_TEST_UNROLL = 8;    // candidate pairs tested between fullness votes
+constexpr int PS_TEST_UNROLL = 4;    // candidate pairs tested between fullness votes
 
 struct PairArgs {
     const float4* pos;
@@ -322,7 +322,9 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
         hix = fminf(hix, 2.f * A.L.x); hiy = fminf(hiy, 2.f * A.L.y); hiz = fminf(hiz, 2.f * A.L.z);
 
         int done = 0;      // accepted indices already written to the row (a multiple of 8 until the end)
-        int* wp = buf;     // next free slot of this lane's buffer
+        // next free slot of this lane's buffer, as a 32-bit shared-memory address
+        const unsigned buf_sa = (unsigned)__cvta_generic_to_shared(buf);
+        unsigned wsa = buf_sa;
         int ncand = 0;     // staged candidates (warp-uniform)
         const unsigned long long px2 = pk(p.x, p.x), py2 = pk(p.y, p.y), pz2 = pk(p.z, p.z);
 
@@ -330,7 +332,7 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
         // `all`, the remainder too.  The remainder of a partial drain moves
         // to the front of the buffer.
         auto drain = [&](bool all) {
-            const int pend = (int)(wp - buf);
+            const int pend = (int)((wsa - buf_sa) >> 2);
             const int groups = pend / PS_GROUP;
             for (int gi = 0; gi < groups; ++gi) {
                 const int* src = buf + gi * PS_GROUP;
@@ -350,10 +352,10 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
                 for (int e = 0; e < rest; ++e)
                     if (done + e < cap) row[done + e] = buf[groups * PS_GROUP + e];
                 done += rest;
-                wp = buf;
+                wsa = buf_sa;
             } else {
                 for (int e = 0; e < rest; ++e) buf[e] = buf[groups * PS_GROUP + e];
-                wp = buf + rest;
+                wsa = buf_sa + 4u * (unsigned)rest;
             }
         };
 
@@ -370,22 +372,27 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
             const int npair = ncand >> 1;
             for (int c = 0; c < npair; c += PS_TEST_UNROLL) {
                 // room for 2 * PS_TEST_UNROLL more in every lane's buffer?
-                if (__any_sync(FULL, (int)(wp - buf) > PS_BUF - 2 * PS_TEST_UNROLL)) drain(false);
+                if (__any_sync(FULL, (int)((wsa - buf_sa) >> 2) > PS_BUF - 2 * PS_TEST_UNROLL)) drain(false);
+                float4 a[PS_TEST_UNROLL], b[PS_TEST_UNROLL];
 #pragma unroll
                 for (int u = 0; u < PS_TEST_UNROLL; ++u) {
-                    if (c + u < npair) {
-                        const float4 a = W.ca[c + u];
-                        const float4 b = W.cb[c + u];
-                        const unsigned long long dx = f2_sub(pk(a.x, a.y), px2);
-                        const unsigned long long dy = f2_sub(pk(a.z, a.w), py2);
-                        const unsigned long long dz = f2_sub(pk(b.x, b.y), pz2);
-                        const unsigned long long r2 = f2_fma(dz, dz, f2_fma(dy, dy, f2_mul(dx, dx)));
-                        const int j0 = __float_as_int(b.z), j1 = __float_as_int(b.w);
-                        *wp = j0;
-                        wp += (pk_lo(r2) < A.rs2 && j0 != i) ? 1 : 0;
-                        *wp = j1;
-                        wp += (pk_hi(r2) < A.rs2 && j1 != i) ? 1 : 0;
-                    }
+                    // pairs past the end hold stale data; their index is forced to i (never accepted)
+                    const int k = min(c + u, PS_CHUNK / 2 - 1);
+                    a[u] = W.ca[k];
+                    b[u] = W.cb[k];
+                    if (c + u >= npair) b[u].z = b[u].w = __int_as_float(i);
+                }
+#pragma unroll
+                for (int u = 0; u < PS_TEST_UNROLL; ++u) {
+                    const unsigned long long dx = f2_sub(pk(a[u].x, a[u].y), px2);
+                    const unsigned long long dy = f2_sub(pk(a[u].z, a[u].w), py2);
+                    const unsigned long long dz = f2_sub(pk(b[u].x, b[u].y), pz2);
+                    const unsigned long long r2 = f2_fma(dz, dz, f2_fma(dy, dy, f2_mul(dx, dx)));
+                    const int j0 = __float_as_int(b[u].z), j1 = __float_as_int(b[u].w);
+                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(wsa), "r"(j0) : "memory");
+                    wsa += (pk_lo(r2) < A.rs2 && j0 != i) ? 4u : 0u;
+                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(wsa), "r"(j1) : "memory");
+                    wsa += (pk_hi(r2) < A.rs2 && j1 != i) ? 4u : 0u;
                 }
             }
             ncand = 0;

@@ -192,7 +192,7 @@ __global__ __launch_bounds__(EDGE_WARPS * 32) void edge_kernel(EdgeArgs A) {
 constexpr int EV_WARPS = 8;
 constexpr int EV_MAXCAP = 512;       // live edges of one row staged in shared memory
 constexpr int EV_GEO_UNROLL = 4;     // neighbor/position loads in flight per lane
-constexpr int EV_ACC_UNROLL = 8;     // feature rows in flight per lane group
+constexpr int EV_ACC_UNROLL = 4;     // feature rows in flight per lane group
 
 // Features as float4 (F % 4 == 0, F <= 128): LPE = F/4 lanes share one edge,
 // so a warp reads 32/LPE neighbor feature rows per instruction with 16-byte
@@ -201,7 +201,7 @@ constexpr int EV_ACC_UNROLL = 8;     // feature rows in flight per lane group
 // memory; phase 2 accumulates f_c * h_j with several rows in flight; the lane
 // groups are then summed with shuffles.
 template <int LPE>
-__global__ __launch_bounds__(EV_WARPS * 32, 2) void edge_vec4_kernel(EdgeArgs A) {
+__global__ __launch_bounds__(EV_WARPS * 32, 3) void edge_vec4_kernel(EdgeArgs A) {
     constexpr int EPI = 32 / LPE;
     __shared__ int2 s_edge[EV_WARPS][EV_MAXCAP];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
