@@ -287,7 +287,9 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
     __shared__ PairWarpSmem smem_w[PS_WARPS];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     PairWarpSmem& W = smem_w[warp];
-    int* const buf = W.buf + lane * PS_BUF;
+    // slot s of this lane's buffer is W.buf[s * 32 + lane]: lanes interleaved
+    // across the 32 banks, so the appends of a warp never conflict
+    int* const buf = W.buf + lane;
     const int cap = A.cap;
     const long long ntiles = ((long long)A.n + 31) / 32;
     const float nanf_ = __int_as_float(0x7fc00000);
@@ -332,30 +334,30 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
         // `all`, the remainder too.  The remainder of a partial drain moves
         // to the front of the buffer.
         auto drain = [&](bool all) {
-            const int pend = (int)((wsa - buf_sa) >> 2);
+            const int pend = (int)((wsa - buf_sa) >> 7);
             const int groups = pend / PS_GROUP;
             for (int gi = 0; gi < groups; ++gi) {
-                const int* src = buf + gi * PS_GROUP;
+                const int* src = buf + gi * PS_GROUP * 32;
                 if (done + PS_GROUP <= cap && A.vec_rows) {
-                    const int4 a = *reinterpret_cast<const int4*>(src);
-                    const int4 b = *reinterpret_cast<const int4*>(src + 4);
+                    const int4 a = make_int4(src[0], src[32], src[64], src[96]);
+                    const int4 b = make_int4(src[128], src[160], src[192], src[224]);
                     *reinterpret_cast<int4*>(row + done) = a;
                     *reinterpret_cast<int4*>(row + done + 4) = b;
                 } else {
                     for (int e = 0; e < PS_GROUP; ++e)
-                        if (done + e < cap) row[done + e] = src[e];
+                        if (done + e < cap) row[done + e] = src[e * 32];
                 }
                 done += PS_GROUP;
             }
             const int rest = pend - groups * PS_GROUP;
             if (all) {
                 for (int e = 0; e < rest; ++e)
-                    if (done + e < cap) row[done + e] = buf[groups * PS_GROUP + e];
+                    if (done + e < cap) row[done + e] = buf[(groups * PS_GROUP + e) * 32];
                 done += rest;
                 wsa = buf_sa;
             } else {
-                for (int e = 0; e < rest; ++e) buf[e] = buf[groups * PS_GROUP + e];
-                wsa = buf_sa + 4u * (unsigned)rest;
+                for (int e = 0; e < rest; ++e) buf[e * 32] = buf[(groups * PS_GROUP + e) * 32];
+                wsa = buf_sa + 128u * (unsigned)rest;
             }
         };
 
@@ -372,7 +374,7 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
             const int npair = ncand >> 1;
             for (int c = 0; c < npair; c += PS_TEST_UNROLL) {
                 // room for 2 * PS_TEST_UNROLL more in every lane's buffer?
-                if (__any_sync(FULL, (int)((wsa - buf_sa) >> 2) > PS_BUF - 2 * PS_TEST_UNROLL)) drain(false);
+                if (__any_sync(FULL, (int)((wsa - buf_sa) >> 7) > PS_BUF - 2 * PS_TEST_UNROLL)) drain(false);
                 float4 a[PS_TEST_UNROLL], b[PS_TEST_UNROLL];
 #pragma unroll
                 for (int u = 0; u < PS_TEST_UNROLL; ++u) {
@@ -390,9 +392,9 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
                     const unsigned long long r2 = f2_fma(dz, dz, f2_fma(dy, dy, f2_mul(dx, dx)));
                     const int j0 = __float_as_int(b[u].z), j1 = __float_as_int(b[u].w);
                     asm volatile("st.shared.b32 [%0], %1;" ::"r"(wsa), "r"(j0) : "memory");
-                    wsa += (pk_lo(r2) < A.rs2 && j0 != i) ? 4u : 0u;
+                    wsa += (pk_lo(r2) < A.rs2 && j0 != i) ? 128u : 0u;
                     asm volatile("st.shared.b32 [%0], %1;" ::"r"(wsa), "r"(j1) : "memory");
-                    wsa += (pk_hi(r2) < A.rs2 && j1 != i) ? 4u : 0u;
+                    wsa += (pk_hi(r2) < A.rs2 && j1 != i) ? 128u : 0u;
                 }
             }
             ncand = 0;

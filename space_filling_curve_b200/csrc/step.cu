@@ -194,13 +194,14 @@ constexpr int EV_MAXCAP = 512;       // live edges of one row staged in shared m
 constexpr int EV_GEO_UNROLL = 4;     // neighbor/position loads in flight per lane
 constexpr int EV_ACC_UNROLL = 4;     // feature rows in flight per lane group
 
-// Features as float4 (F % 4 == 0, F <= 128): LPE = F/4 lanes share one edge,
-// so a warp reads 32/LPE neighbor feature rows per instruction with 16-byte
-// loads.  Phase 1 computes the geometry of the whole row (one edge per lane,
-// several loads in flight) and compacts the live (j, f_c) pairs into shared
-// memory; phase 2 accumulates f_c * h_j with several rows in flight; the lane
-// groups are then summed with shuffles.
-template <int LPE>
+// Features as float4 (F % 4 == 0, F <= 256): LPE lanes share one edge and
+// each lane owns VPL float4 of the feature row (F = 4 * LPE * VPL), so a warp
+// reads 32/LPE neighbor feature rows per step with 16-byte loads.  Phase 1
+// computes the geometry of the whole row (one edge per lane, several loads in
+// flight) and compacts the live (j, f_c) pairs into shared memory; phase 2
+// accumulates f_c * h_j with several rows in flight; the lane groups are then
+// summed with shuffles.
+template <int LPE, int VPL>
 __global__ __launch_bounds__(EV_WARPS * 32, 3) void edge_vec4_kernel(EdgeArgs A) {
     constexpr int EPI = 32 / LPE;
     __shared__ int2 s_edge[EV_WARPS][EV_MAXCAP];
@@ -237,8 +238,8 @@ __global__ __launch_bounds__(EV_WARPS * 32, 3) void edge_vec4_kernel(EdgeArgs A)
                     const float dy = min_image_f(pj[u].y - pi.y, A.L.y);
                     const float dz = min_image_f(pj[u].z - pi.z, A.L.z);
                     const float r2 = fmaf(dz, dz, fmaf(dy, dy, dx * dx));
-                    const float u = r2 * A.inv_rc2;
-                    fc = u < 1.0f ? cutoff_u(u) : 0.0f;
+                    const float u2 = r2 * A.inv_rc2;
+                    fc = u2 < 1.0f ? cutoff_u(u2) : 0.0f;
                     if (edges) {
                         const size_t e = (size_t)i * A.cap + s;
                         const float r = sqrtf(r2);
@@ -259,37 +260,51 @@ __global__ __launch_bounds__(EV_WARPS * 32, 3) void edge_vec4_kernel(EdgeArgs A)
             }
         }
         __syncwarp();
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float4 acc[VPL];
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4* fbase = feat4 + fl * VPL;
         for (int e0 = 0; e0 < nlive; e0 += EPI * EV_ACC_UNROLL) {
             int2 ed[EV_ACC_UNROLL];
-            float4 h[EV_ACC_UNROLL];
+            float4 h[EV_ACC_UNROLL][VPL];
 #pragma unroll
             for (int u = 0; u < EV_ACC_UNROLL; ++u) {
                 const int e = e0 + u * EPI + g;
                 ed[u] = (e < nlive) ? live_e[e] : make_int2(-1, 0);
             }
 #pragma unroll
-            for (int u = 0; u < EV_ACC_UNROLL; ++u)
-                if (ed[u].x >= 0) h[u] = feat4[(size_t)ed[u].x * F4 + fl];
+            for (int u = 0; u < EV_ACC_UNROLL; ++u) {
+                const float4* src = fbase + (size_t)max(ed[u].x, 0) * F4;
+#pragma unroll
+                for (int v = 0; v < VPL; ++v) h[u][v] = src[v];
+            }
 #pragma unroll
             for (int u = 0; u < EV_ACC_UNROLL; ++u) {
-                if (ed[u].x >= 0) {
-                    const float w = __int_as_float(ed[u].y);
-                    acc.x = fmaf(w, h[u].x, acc.x);
-                    acc.y = fmaf(w, h[u].y, acc.y);
-                    acc.z = fmaf(w, h[u].z, acc.z);
-                    acc.w = fmaf(w, h[u].w, acc.w);
+                if (ed[u].x < 0) continue;     // past the last live edge
+                const float w = __int_as_float(ed[u].y);
+#pragma unroll
+                for (int v = 0; v < VPL; ++v) {
+                    acc[v].x = fmaf(w, h[u][v].x, acc[v].x);
+                    acc[v].y = fmaf(w, h[u][v].y, acc[v].y);
+                    acc[v].z = fmaf(w, h[u][v].z, acc[v].z);
+                    acc[v].w = fmaf(w, h[u][v].w, acc[v].w);
                 }
             }
         }
 #pragma unroll
         for (int o = LPE; o < 32; o <<= 1) {
-            acc.x += __shfl_xor_sync(FULL, acc.x, o);
-            acc.y += __shfl_xor_sync(FULL, acc.y, o);
-            acc.z += __shfl_xor_sync(FULL, acc.z, o);
-            acc.w += __shfl_xor_sync(FULL, acc.w, o);
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) {
+                acc[v].x += __shfl_xor_sync(FULL, acc[v].x, o);
+                acc[v].y += __shfl_xor_sync(FULL, acc[v].y, o);
+                acc[v].z += __shfl_xor_sync(FULL, acc[v].z, o);
+                acc[v].w += __shfl_xor_sync(FULL, acc[v].w, o);
+            }
         }
-        if (g == 0) out4[(size_t)i * F4 + fl] = acc;
+        if (g == 0) {
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) out4[(size_t)i * F4 + fl * VPL + v] = acc[v];
+        }
         __syncwarp();
     }
 }
@@ -324,22 +339,25 @@ tess_status edge_aggregate(const float* pos, int n, tess_box box, float rc, cons
     StageScope sc(ST_EDGE, s);
     const long long rows_blocks = ((long long)n + EDGE_WARPS - 1) / EDGE_WARPS;
     const int blocks = (int)std::min<long long>(rows_blocks, (long long)sms * 64);
-    const bool vec4 = (F % 4 == 0) && F <= 128 && aligned(feat, 16) && aligned(out, 16) && cap <= EV_MAXCAP;
+    const bool vec4 = (F % 4 == 0) && F <= 256 && aligned(feat, 16) && aligned(out, 16) && cap <= EV_MAXCAP;
+    const int vblocks = (int)std::min<long long>(((long long)n + EV_WARPS - 1) / EV_WARPS, (long long)sms * 32);
+    bool launched = false;
     if (vec4) {
-        const int vblocks = (int)std::min<long long>(((long long)n + EV_WARPS - 1) / EV_WARPS, (long long)sms * 32);
+        launched = true;
         switch (F / 4) {
-            case 1: edge_vec4_kernel<1><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
-            case 2: edge_vec4_kernel<2><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
-            case 4: edge_vec4_kernel<4><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
-            case 8: edge_vec4_kernel<8><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
-            case 16: edge_vec4_kernel<16><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
-            case 32: edge_vec4_kernel<32><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
-            default: edge_kernel<1><<<blocks, EDGE_WARPS * 32, 0, s>>>(A); break;
+            case 1: edge_vec4_kernel<1, 1><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
+            case 2: edge_vec4_kernel<2, 1><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
+            case 4: edge_vec4_kernel<2, 2><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
+            case 8: edge_vec4_kernel<4, 2><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
+            case 16: edge_vec4_kernel<8, 2><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
+            case 32: edge_vec4_kernel<16, 2><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
+            case 64: edge_vec4_kernel<32, 2><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
+            default: launched = false; break;
         }
-    } else if ((F % 2 == 0) && aligned(feat, 8) && F >= 64) {
-        edge_kernel<2><<<blocks, EDGE_WARPS * 32, 0, s>>>(A);
-    } else {
-        edge_kernel<1><<<blocks, EDGE_WARPS * 32, 0, s>>>(A);
+    }
+    if (!launched) {
+        if ((F % 2 == 0) && aligned(feat, 8) && F >= 64) edge_kernel<2><<<blocks, EDGE_WARPS * 32, 0, s>>>(A);
+        else edge_kernel<1><<<blocks, EDGE_WARPS * 32, 0, s>>>(A);
     }
     count_launch();
     return launch_status();
