@@ -62,6 +62,7 @@ typedef struct {
 
 /* tess_build_neighbors flags */
 #define TESS_NO_PAD_FILL    1   /* leave slots >= min(count, max_neighbors) unwritten */
+#define TESS_TILE_SEARCH    2   /* use the warp-shared tile search instead of the per-lane search */
 
 /* Human-readable name of a status code (static string). */
 const char* tess_status_string(tess_status s);
@@ -116,7 +117,8 @@ tess_status tess_hilbert_sort(const float* pos, int n, tess_box box, int bits,
  *   pos            [n,4] float (x, y, z, ignored), 16-byte aligned
  *   rc, skin       cutoff and skin (rc > 0, skin >= 0); rs = rc + skin in fp32
  *   max_neighbors  row capacity cap >= 1
- *   flags          0 or TESS_NO_PAD_FILL
+ *   flags          0, or'ed TESS_NO_PAD_FILL, TESS_TILE_SEARCH (same lists, other
+ *                  search order; boxes shorter than 2 rs + 2e-3 always use it)
  *   ws, ws_bytes   scratch of at least tess_build_neighbors_workspace(...)
  *   nbr            [n, cap] int32 out: row i in nbr[i*cap .. i*cap+cap);
  *                  the first min(counts[i], cap) slots hold neighbors, the

@@ -504,6 +504,149 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
     }
 }
 
+// ---------------------------------------------------------------- per-lane search
+
+// One warp per 32 consecutive atoms, but every lane walks its own stencil:
+// the 5 x 5 cell rows (cells of width >= rs/2, so +-2 rows cover rs) around
+// its own cell, each clipped to the x-window of its own sphere: for a row at
+// y/z distance (dy, dz) from the atom the window is x +- sqrt(reach^2 - dy^2 -
+// dz^2), and only the cells overlapping it are read.  Candidates are gathered
+// per lane (16-byte loads, L1-resident for a compact tile), tested in fp32,
+// and accepted indices go through the same bank-interleaved append buffer.
+// Loops are warp-uniform (bounded by the warp's longest window) so that the
+// buffer vote can run inside them.
+constexpr int PL_WARPS = 4;
+constexpr int PL_CHUNK = 8;          // candidates per lane between buffer votes
+
+__global__ __launch_bounds__(PL_WARPS * 32, 6) void pair_search_lane_kernel(PairArgs A) {
+    __shared__ int s_buf[PL_WARPS][32 * PS_BUF];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int* const buf = &s_buf[warp][lane];
+    const unsigned buf_sa = (unsigned)__cvta_generic_to_shared(buf);
+    const int cap = A.cap;
+    const long long ntiles = ((long long)A.n + 31) / 32;
+    const float wy = (float)A.L.y / (float)A.nc.y, wz = (float)A.L.z / (float)A.nc.z;
+    const float reach2 = A.reach * A.reach;
+
+    for (long long tile = (long long)blockIdx.x * PL_WARPS + warp; tile < ntiles;
+         tile += (long long)gridDim.x * PL_WARPS) {
+        const int i = (int)(tile * 32) + lane;
+        const bool valid = i < A.n;
+        float4 p = valid ? A.pos[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        // finite coordinates for the window arithmetic (invalid input is flagged by the binning)
+        p.x = fminf(fmaxf(p.x, 0.f), A.L.x);
+        p.y = fminf(fmaxf(p.y, 0.f), A.L.y);
+        p.z = fminf(fmaxf(p.z, 0.f), A.L.z);
+        const float4 p0 = valid ? A.pos[i] : p;
+        int* row = A.nbr + (size_t)(valid ? i : 0) * cap;
+        const int cy = cell_coord(p.y, A.inv_w.y, A.nc.y);
+        const int cz = cell_coord(p.z, A.inv_w.z, A.nc.z);
+
+        int done = 0;
+        unsigned wsa = buf_sa;
+        auto drain = [&](bool all) {
+            const int pend = (int)((wsa - buf_sa) >> 7);
+            const int groups = pend / PS_GROUP;
+            for (int gi = 0; gi < groups; ++gi) {
+                const int* src = buf + gi * PS_GROUP * 32;
+                if (done + PS_GROUP <= cap && A.vec_rows) {
+                    const int4 a = make_int4(src[0], src[32], src[64], src[96]);
+                    const int4 b = make_int4(src[128], src[160], src[192], src[224]);
+                    *reinterpret_cast<int4*>(row + done) = a;
+                    *reinterpret_cast<int4*>(row + done + 4) = b;
+                } else {
+                    for (int e = 0; e < PS_GROUP; ++e)
+                        if (done + e < cap) row[done + e] = src[e * 32];
+                }
+                done += PS_GROUP;
+            }
+            const int rest = pend - groups * PS_GROUP;
+            if (all) {
+                for (int e = 0; e < rest; ++e)
+                    if (done + e < cap) row[done + e] = buf[(groups * PS_GROUP + e) * 32];
+                done += rest;
+                wsa = buf_sa;
+            } else {
+                for (int e = 0; e < rest; ++e) buf[e * 32] = buf[(groups * PS_GROUP + e) * 32];
+                wsa = buf_sa + 128u * (unsigned)rest;
+            }
+        };
+
+        for (int t = 0; t < 25; ++t) {
+            const int uy = cy + (t % 5) - 2, uz = cz + (t / 5) - 2;
+            // distance from the atom to the row's y and z extents
+            const float ylo = (float)uy * wy, zlo = (float)uz * wz;
+            const float ddy = fmaxf(fmaxf(ylo - p.y, p.y - (ylo + wy)), 0.f);
+            const float ddz = fmaxf(fmaxf(zlo - p.z, p.z - (zlo + wz)), 0.f);
+            const float ch2 = reach2 - ddy * ddy - ddz * ddz;
+            int beg[2] = {0, 0}, len[2] = {0, 0};
+            float sx[2] = {0.f, 0.f};
+            float sy = 0.f, sz = 0.f;
+            if (valid && ch2 > 0.f) {
+                const float chord = sqrtf(ch2);
+                const int ky = floor_div(uy, A.nc.y), kz = floor_div(uz, A.nc.z);
+                sy = (float)ky * A.L.y;
+                sz = (float)kz * A.L.z;
+                const int rowbase = ((uz - kz * A.nc.z) * A.nc.y + (uy - ky * A.nc.y)) * A.nc.x;
+                int ua = (int)floorf((p.x - chord) * A.inv_w.x);
+                const int ub = (int)floorf((p.x + chord) * A.inv_w.x);
+                // with L >= 2 reach the window covers at most nc.x + 1 cells, so
+                // it wraps at most once: two pieces, each a contiguous range
+#pragma unroll
+                for (int pc = 0; pc < 2; ++pc) {
+                    if (ua <= ub) {
+                        const int kx = floor_div(ua, A.nc.x);
+                        const int e = min(ub, (kx + 1) * A.nc.x - 1);
+                        const int xa = ua - kx * A.nc.x, xb = e - kx * A.nc.x;
+                        beg[pc] = A.cell_start[rowbase + xa];
+                        len[pc] = A.cell_start[rowbase + xb + 1] - beg[pc];
+                        sx[pc] = (float)kx * A.L.x;
+                        ua = e + 1;
+                    }
+                }
+            }
+#pragma unroll
+            for (int pc = 0; pc < 2; ++pc) {
+                int maxlen = __reduce_max_sync(FULL, (unsigned)len[pc]);
+                for (int k0 = 0; k0 < maxlen; k0 += PL_CHUNK) {
+                    if (__any_sync(FULL, (int)((wsa - buf_sa) >> 7) > PS_BUF - PL_CHUNK)) drain(false);
+                    float4 c[PL_CHUNK];
+#pragma unroll
+                    for (int u = 0; u < PL_CHUNK; ++u)
+                        if (k0 + u < len[pc]) c[u] = A.pos_cell[beg[pc] + k0 + u];
+#pragma unroll
+                    for (int u = 0; u < PL_CHUNK; ++u) {
+                        if (k0 + u < len[pc]) {
+                            const float dx = (c[u].x + sx[pc]) - p0.x;
+                            const float dy = (c[u].y + sy) - p0.y;
+                            const float dz = (c[u].z + sz) - p0.z;
+                            const float r2 = fmaf(dz, dz, fmaf(dy, dy, dx * dx));
+                            const int j = __float_as_int(c[u].w);
+                            asm volatile("st.shared.b32 [%0], %1;" ::"r"(wsa), "r"(j) : "memory");
+                            wsa += (r2 < A.rs2 && j != i) ? 128u : 0u;
+                        }
+                    }
+                }
+            }
+        }
+        drain(true);
+        const int cnt = done;
+        if (valid) {
+            A.counts[i] = cnt;
+            if (A.pad_fill) {
+                int e = min(cnt, cap);
+                if (A.vec_rows) {
+                    for (; e < cap && (e & 3); ++e) row[e] = -1;
+                    for (; e + 4 <= cap; e += 4) *reinterpret_cast<int4*>(row + e) = make_int4(-1, -1, -1, -1);
+                }
+                for (; e < cap; ++e) row[e] = -1;
+            }
+        }
+        const unsigned ov = __ballot_sync(FULL, valid && cnt > cap);
+        if (ov && lane == 0) atomicOr(A.status, TESS_DEV_OVERFLOW);
+    }
+}
+
 // ---------------------------------------------------------------- host
 
 struct NbrLayout {
@@ -546,7 +689,7 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
     if (n <= 0 || !pos || !ws || !nbr || !counts || !overflow || cap < 1) return TESS_ERR_INVALID_ARG;
     if (!box_ok(box) || !(rc > 0.f) || !(skin >= 0.f) || !std::isfinite(rc) || !std::isfinite(skin))
         return TESS_ERR_INVALID_ARG;
-    if ((flags & ~TESS_NO_PAD_FILL) != 0) return TESS_ERR_INVALID_ARG;
+    if ((flags & ~(TESS_NO_PAD_FILL | TESS_TILE_SEARCH)) != 0) return TESS_ERR_INVALID_ARG;
     if (!aligned(pos, 16) || !aligned(ws, 256) || !aligned(nbr, 4) || !aligned(counts, 4)) return TESS_ERR_INVALID_ARG;
     const float rs = rc + skin;
     if (box.lx < 2.f * rs || box.ly < 2.f * rs || box.lz < 2.f * rs) return TESS_ERR_BOX_TOO_SMALL;
@@ -597,8 +740,16 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
         A.counts = counts;
         A.status = overflow;
         const long long ntiles = ((long long)n + 31) / 32;
-        const long long blocks = (ntiles + PS_WARPS - 1) / PS_WARPS;
-        pair_search_kernel<<<(unsigned)std::min<long long>(blocks, 1LL << 30), PS_WARPS * 32, 0, s>>>(A);
+        // the per-lane search needs every box length >= 2 reach (a window
+        // then wraps at most once); otherwise the tile search handles it
+        const bool lane_ok = box.lx >= 2.f * A.reach && box.ly >= 2.f * A.reach && box.lz >= 2.f * A.reach;
+        if ((flags & TESS_TILE_SEARCH) || !lane_ok) {
+            const long long blocks = (ntiles + PS_WARPS - 1) / PS_WARPS;
+            pair_search_kernel<<<(unsigned)std::min<long long>(blocks, 1LL << 30), PS_WARPS * 32, 0, s>>>(A);
+        } else {
+            const long long blocks = (ntiles + PL_WARPS - 1) / PL_WARPS;
+            pair_search_lane_kernel<<<(unsigned)std::min<long long>(blocks, 1LL << 30), PL_WARPS * 32, 0, s>>>(A);
+        }
         count_launch();
     }
     return launch_status();

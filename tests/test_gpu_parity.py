@@ -94,15 +94,15 @@ def test_sort_configs(cfg):
 # ------------------------------------------------------------------ neighbors
 
 
-def _gpu_list(pos4, box, rc, skin, cap, pad_fill=True):
+def _gpu_list(pos4, box, rc, skin, cap, pad_fill=True, tile=False):
     tess = _tess()
-    nbr, cnt, ov = tess.build_neighbors(_dev(pos4), box, rc, skin, cap, pad_fill=pad_fill)
+    nbr, cnt, ov = tess.build_neighbors(_dev(pos4), box, rc, skin, cap, pad_fill=pad_fill, tile_search=tile)
     torch_cuda().cuda.synchronize()
     return nbr, cnt, int(ov.item())
 
 
-def _check_list(pos4, box, rc, skin, cap, pad_fill=True, method="cells"):
-    nbr_d, cnt_d, ov = _gpu_list(pos4, box, rc, skin, cap, pad_fill)
+def _check_list(pos4, box, rc, skin, cap, pad_fill=True, method="cells", tile=False):
+    nbr_d, cnt_d, ov = _gpu_list(pos4, box, rc, skin, cap, pad_fill, tile)
     fn = oracle.neighbors_cells if method == "cells" else oracle.neighbors_brute
     onbr, ocnt, oov = fn(pos4, box, rc, skin, cap)
     cnt = cnt_d.cpu().numpy()
@@ -125,12 +125,13 @@ def _check_list(pos4, box, rc, skin, cap, pad_fill=True, method="cells"):
     return nbr_d, cnt
 
 
+@pytest.mark.parametrize("tile", [False, True])
 @pytest.mark.parametrize("cfg", [1, 2])
-def test_neighbors_configs_sorted_order(cfg):
+def test_neighbors_configs_sorted_order(cfg, tile):
     s = synth.system(cfg)
     perm, _ = oracle.hilbert_sort(s.pos, s.box, 10)
     p4 = s.pos4()[perm]
-    _check_list(p4, s.box, s.rc, s.skin, s.cap)
+    _check_list(p4, s.box, s.rc, s.skin, s.cap, tile=tile)
 
 
 def test_neighbors_config3():
@@ -139,45 +140,62 @@ def test_neighbors_config3():
     _check_list(s.pos4()[perm], s.box, s.rc, s.skin, s.cap)
 
 
-def test_neighbors_unsorted_input_gives_the_same_sets():
+@pytest.mark.parametrize("tile", [False, True])
+def test_neighbors_unsorted_input_gives_the_same_sets(tile):
     s = synth.system(1)
-    _check_list(s.pos4(), s.box, s.rc, s.skin, s.cap, method="brute")
+    _check_list(s.pos4(), s.box, s.rc, s.skin, s.cap, method="brute", tile=tile)
 
 
+@pytest.mark.parametrize("tile", [False, True])
 @pytest.mark.parametrize("n", [1, 2, 31, 32, 33, 97, 1000])
-def test_neighbors_ragged(n):
+def test_neighbors_ragged(n, tile):
     rng = np.random.default_rng(100 + n)
     L = 30.0
     p = np.zeros((n, 4), np.float32)
     p[:, :3] = rng.uniform(0, L, (n, 3))
-    _check_list(p, (L, L, L), 4.0, 0.5, 64, method="brute")
+    _check_list(p, (L, L, L), 4.0, 0.5, 64, method="brute", tile=tile)
 
 
-def test_neighbors_no_pad_fill_and_overflow():
+@pytest.mark.parametrize("tile", [False, True])
+def test_neighbors_no_pad_fill_and_overflow(tile):
     s = synth.system(1)
     perm, _ = oracle.hilbert_sort(s.pos, s.box, 10)
     p4 = s.pos4()[perm]
-    _check_list(p4, s.box, s.rc, s.skin, s.cap, pad_fill=False)
-    _check_list(p4, s.box, s.rc, s.skin, 40)                 # overflow: flag, true counts
-    _check_list(p4, s.box, s.rc, s.skin, 40, pad_fill=False)
+    _check_list(p4, s.box, s.rc, s.skin, s.cap, pad_fill=False, tile=tile)
+    _check_list(p4, s.box, s.rc, s.skin, 40, tile=tile)                 # overflow: flag, true counts
+    _check_list(p4, s.box, s.rc, s.skin, 40, pad_fill=False, tile=tile)
+    _check_list(p4, s.box, s.rc, s.skin, 37, tile=tile)                 # cap not a multiple of 4
 
 
-@pytest.mark.parametrize("L,rc", [(13.0, 6.0), (19.6, 6.0), (25.0, 5.75)])
-def test_neighbors_small_boxes(L, rc):
-    # boxes of 2 to 4 list radii: the cell range of a tile wraps onto itself
+@pytest.mark.parametrize("tile", [False, True])
+@pytest.mark.parametrize("L,rc", [(13.0, 6.0), (13.1, 6.0), (19.6, 6.0), (25.0, 5.75)])
+def test_neighbors_small_boxes(L, rc, tile):
+    # boxes of 2 to 4 list radii: cell ranges and windows wrap onto themselves
     rng = np.random.default_rng(int(L * 10))
     n = int(0.1 * L ** 3)
     p = np.zeros((n, 4), np.float32)
     p[:, :3] = rng.uniform(0, L, (n, 3))
     p = p[oracle.hilbert_sort(p, (L, L, L), 10)[0]]
-    _check_list(p, (L, L, L), rc, 0.5, 256, method="brute")
+    _check_list(p, (L, L, L), rc, 0.5, 256, method="brute", tile=tile)
 
 
-def test_neighbors_large_cap_global_rows():
-    # a cap too large for shared-memory rows takes the global-row path
+@pytest.mark.parametrize("tile", [False, True])
+def test_neighbors_large_cap(tile):
     s = synth.system(1)
     perm, _ = oracle.hilbert_sort(s.pos, s.box, 10)
-    _check_list(s.pos4()[perm], s.box, s.rc, s.skin, 1024)
+    _check_list(s.pos4()[perm], s.box, s.rc, s.skin, 1024, tile=tile)
+
+
+def test_neighbors_dense_rows_drain_the_buffer():
+    # a dense cluster: rows far longer than the per-lane staging buffer
+    rng = np.random.default_rng(5)
+    L = 40.0
+    n = 4000
+    p = np.zeros((n, 4), np.float32)
+    p[:, :3] = rng.uniform(0, 1, (n, 3)) * np.array([L, L, 6.0]) + np.array([0, 0, 10.0])
+    p = p[oracle.hilbert_sort(p, (L, L, L), 10)[0]]
+    for tile in (False, True):
+        _check_list(p, (L, L, L), 5.0, 0.5, 512, method="brute", tile=tile)
 
 
 def test_neighbors_box_errors():
