@@ -47,7 +47,8 @@ typedef enum {
     TESS_ERR_INVALID_ARG = 1,        /* n <= 0, null pointer, bad parameter, misalignment */
     TESS_ERR_BOX_TOO_SMALL = 2,      /* some box length below 2 (rc + skin) */
     TESS_ERR_WORKSPACE_TOO_SMALL = 3,/* ws_bytes below the workspace query */
-    TESS_ERR_CUDA = 4                /* a kernel launch failed */
+    TESS_ERR_CUDA = 4,               /* a kernel launch failed */
+    TESS_ERR_TOO_LARGE = 5           /* n above the capacity of tess_hilbert_sort_static */
 } tess_status;
 
 /* Orthorhombic periodic box lengths (Angstrom, or any unit used throughout). */
@@ -103,6 +104,34 @@ tess_status tess_hilbert_sort(const float* pos, int n, tess_box box, int bits,
                               void* ws, size_t ws_bytes,
                               int32_t* perm, uint32_t* keys_sorted, float* pos_sorted,
                               int32_t* dev_status, tess_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Allocation-free Hilbert sort.  The paper has no counterpart: this is a
+ * library convenience.
+ *
+ * Same computation, arguments and outputs as tess_hilbert_sort, but without a
+ * workspace argument: the scratch memory is an array inside the library
+ * (device memory, about 19 MiB, held by every GPU that loads the library until
+ * the process exits).  It is meant for callers that cannot allocate device
+ * memory -- for example a plugin whose host program owns all device buffers,
+ * or a time-step loop that must not call cudaMalloc because it synchronises
+ * the device -- and that have no buffer to lend as a workspace.
+ *
+ *   n  1 .. TESS_HILBERT_SORT_STATIC_MAX_N; larger n returns
+ *      TESS_ERR_TOO_LARGE (use tess_hilbert_sort with a workspace instead)
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current); make that first call before any stream capture.  All calls
+ * on a device share the array: calls that overlap on the GPU (different
+ * streams, or unordered host threads) race on it and corrupt each other's
+ * results, so order them on one stream.  Each call clears what must start at
+ * zero; nothing else carries over between calls.
+ * Errors: those of tess_hilbert_sort, plus TOO_LARGE.
+ * ------------------------------------------------------------------------- */
+#define TESS_HILBERT_SORT_STATIC_MAX_N (1 << 20)
+tess_status tess_hilbert_sort_static(const float* pos, int n, tess_box box, int bits,
+                                     int32_t* perm, uint32_t* keys_sorted, float* pos_sorted,
+                                     int32_t* dev_status, tess_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Verlet neighbor list at rs = rc + skin -- "fixes workload shapes between

@@ -22,7 +22,7 @@ import os
 __all__ = [
     "TessError", "lib", "library_path", "Box",
     "tess_status_string", "tess_version", "tess_kernel_launch_count",
-    "tess_hilbert_sort_workspace", "tess_hilbert_sort",
+    "tess_hilbert_sort_workspace", "tess_hilbert_sort", "tess_hilbert_sort_static", "HILBERT_SORT_STATIC_MAX_N",
     "tess_build_neighbors_workspace", "tess_build_neighbors",
     "tess_skin_check", "tess_edge_aggregate", "tess_stage_timing", "tess_stage_times",
     "hilbert_sort", "build_neighbors", "skin_check", "edge_aggregate",
@@ -38,7 +38,9 @@ TESS_DEV_TIMEOUT = 4
 TESS_NO_PAD_FILL = 1
 TESS_TILE_SEARCH = 2
 STAGES = ("hilbert_keys", "key_sort", "cell_binning", "pair_search", "skin_check", "edge_aggregate")
-_STATUS = {0: "ok", 1: "invalid argument", 2: "box too small", 3: "workspace too small", 4: "CUDA launch error"}
+_STATUS = {0: "ok", 1: "invalid argument", 2: "box too small", 3: "workspace too small", 4: "CUDA launch error",
+           5: "n above the static scratch capacity"}
+HILBERT_SORT_STATIC_MAX_N = 1 << 20
 
 
 class TessError(RuntimeError):
@@ -74,6 +76,8 @@ def lib() -> ctypes.CDLL:
     L.tess_hilbert_sort_workspace.restype = sz
     L.tess_hilbert_sort.argtypes = [P, i32, Box, i32, P, sz, P, P, P, P, P]
     L.tess_hilbert_sort.restype = i32
+    L.tess_hilbert_sort_static.argtypes = [P, i32, Box, i32, P, P, P, P, P]
+    L.tess_hilbert_sort_static.restype = i32
     L.tess_build_neighbors_workspace.argtypes = [i32, Box, f32, f32]
     L.tess_build_neighbors_workspace.restype = sz
     L.tess_build_neighbors.argtypes = [P, i32, Box, f32, f32, i32, i32, P, sz, P, P, P, P]
@@ -118,6 +122,14 @@ def tess_hilbert_sort_workspace(n: int) -> int:
 def tess_hilbert_sort(pos, n, box, bits, ws, ws_bytes, perm, keys_sorted, pos_sorted, dev_status, stream) -> int:
     return int(lib().tess_hilbert_sort(pos, n, _box(box), bits, ws, ws_bytes, perm, keys_sorted, pos_sorted,
                                        dev_status, stream))
+
+
+def tess_hilbert_sort_static(pos, n, box, bits, perm, keys_sorted, pos_sorted, dev_status, stream) -> int:
+    """Allocation-free Hilbert sort: the scratch lives inside the library
+    (for up to HILBERT_SORT_STATIC_MAX_N atoms), for callers that cannot
+    allocate device memory or lend a workspace."""
+    return int(lib().tess_hilbert_sort_static(pos, n, _box(box), bits, perm, keys_sorted, pos_sorted, dev_status,
+                                              stream))
 
 
 def tess_build_neighbors_workspace(n, box, rc, skin) -> int:

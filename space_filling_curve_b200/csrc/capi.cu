@@ -69,6 +69,7 @@ const char* tess_status_string(tess_status s) {
         case TESS_ERR_BOX_TOO_SMALL: return "box too small: some length below twice the cutoff radius";
         case TESS_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
         case TESS_ERR_CUDA: return "CUDA launch error";
+        case TESS_ERR_TOO_LARGE: return "n above the capacity of the static scratch (TESS_HILBERT_SORT_STATIC_MAX_N)";
     }
     return "unknown status";
 }
