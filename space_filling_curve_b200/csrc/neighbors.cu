@@ -572,58 +572,66 @@ __global__ __launch_bounds__(PL_WARPS * 32, 6) void pair_search_lane_kernel(Pair
             }
         };
 
-        for (int t = 0; t < 25; ++t) {
-            const int uy = cy + (t % 5) - 2, uz = cz + (t / 5) - 2;
-            // distance from the atom to the row's y and z extents
-            const float ylo = (float)uy * wy, zlo = (float)uz * wz;
-            const float ddy = fmaxf(fmaxf(ylo - p.y, p.y - (ylo + wy)), 0.f);
+        for (int dz = -2; dz <= 2; ++dz) {
+            // row z: unwrapped index for the geometry, wrapped index and image shift for the data
+            int wz_i = cz + dz, kz = 0;
+            while (wz_i < 0) { wz_i += A.nc.z; --kz; }
+            while (wz_i >= A.nc.z) { wz_i -= A.nc.z; ++kz; }
+            const float zlo = (float)(cz + dz) * wz;
             const float ddz = fmaxf(fmaxf(zlo - p.z, p.z - (zlo + wz)), 0.f);
-            const float ch2 = reach2 - ddy * ddy - ddz * ddz;
-            int beg[2] = {0, 0}, len[2] = {0, 0};
-            float sx[2] = {0.f, 0.f};
-            float sy = 0.f, sz = 0.f;
-            if (valid && ch2 > 0.f) {
-                const float chord = sqrtf(ch2);
-                const int ky = floor_div(uy, A.nc.y), kz = floor_div(uz, A.nc.z);
-                sy = (float)ky * A.L.y;
-                sz = (float)kz * A.L.z;
-                const int rowbase = ((uz - kz * A.nc.z) * A.nc.y + (uy - ky * A.nc.y)) * A.nc.x;
-                int ua = (int)floorf((p.x - chord) * A.inv_w.x);
-                const int ub = (int)floorf((p.x + chord) * A.inv_w.x);
-                // with L >= 2 reach the window covers at most nc.x + 1 cells, so
-                // it wraps at most once: two pieces, each a contiguous range
-#pragma unroll
-                for (int pc = 0; pc < 2; ++pc) {
-                    if (ua <= ub) {
-                        const int kx = floor_div(ua, A.nc.x);
-                        const int e = min(ub, (kx + 1) * A.nc.x - 1);
-                        const int xa = ua - kx * A.nc.x, xb = e - kx * A.nc.x;
-                        beg[pc] = A.cell_start[rowbase + xa];
-                        len[pc] = A.cell_start[rowbase + xb + 1] - beg[pc];
-                        sx[pc] = (float)kx * A.L.x;
-                        ua = e + 1;
+            const float qz = p0.z - (float)kz * A.L.z;
+            for (int dy = -2; dy <= 2; ++dy) {
+                int wy_i = cy + dy, ky = 0;
+                while (wy_i < 0) { wy_i += A.nc.y; --ky; }
+                while (wy_i >= A.nc.y) { wy_i -= A.nc.y; ++ky; }
+                const float ylo = (float)(cy + dy) * wy;
+                const float ddy = fmaxf(fmaxf(ylo - p.y, p.y - (ylo + wy)), 0.f);
+                const float ch2 = reach2 - ddy * ddy - ddz * ddz;
+                const float qy = p0.y - (float)ky * A.L.y;
+                int beg[2] = {0, 0}, len[2] = {0, 0};
+                float qx[2] = {0.f, 0.f};
+                if (valid && ch2 > 0.f) {
+                    // x-chord of the sphere in this row (approximate root, widened)
+                    const float chord = fmaf(ch2 * rsqrtf(ch2), 1.0001f, 1e-4f);
+                    const int rowbase = (wz_i * A.nc.y + wy_i) * A.nc.x;
+                    int ua = (int)floorf((p.x - chord) * A.inv_w.x);
+                    int ub = (int)floorf((p.x + chord) * A.inv_w.x);
+                    int kx = 0;
+                    while (ua < 0) { ua += A.nc.x; ub += A.nc.x; --kx; }
+                    while (ua >= A.nc.x) { ua -= A.nc.x; ub -= A.nc.x; ++kx; }
+                    // with L >= 2 reach the window covers at most nc.x + 1
+                    // cells, so it wraps at most once: two contiguous pieces
+                    const int e0 = min(ub, A.nc.x - 1);
+                    beg[0] = A.cell_start[rowbase + ua];
+                    len[0] = A.cell_start[rowbase + e0 + 1] - beg[0];
+                    qx[0] = p0.x - (float)kx * A.L.x;
+                    if (ub >= A.nc.x) {
+                        const int e1 = min(ub - A.nc.x, A.nc.x - 1);
+                        beg[1] = A.cell_start[rowbase];
+                        len[1] = A.cell_start[rowbase + e1 + 1] - beg[1];
+                        qx[1] = p0.x - (float)(kx + 1) * A.L.x;
                     }
                 }
-            }
 #pragma unroll
-            for (int pc = 0; pc < 2; ++pc) {
-                int maxlen = __reduce_max_sync(FULL, (unsigned)len[pc]);
-                for (int k0 = 0; k0 < maxlen; k0 += PL_CHUNK) {
-                    if (__any_sync(FULL, (int)((wsa - buf_sa) >> 7) > PS_BUF - PL_CHUNK)) drain(false);
-                    float4 c[PL_CHUNK];
+                for (int pc = 0; pc < 2; ++pc) {
+                    const int maxlen = (int)__reduce_max_sync(FULL, (unsigned)len[pc]);
+                    for (int k0 = 0; k0 < maxlen; k0 += PL_CHUNK) {
+                        if (__any_sync(FULL, (int)((wsa - buf_sa) >> 7) > PS_BUF - PL_CHUNK)) drain(false);
+                        float4 c[PL_CHUNK];
 #pragma unroll
-                    for (int u = 0; u < PL_CHUNK; ++u)
-                        if (k0 + u < len[pc]) c[u] = A.pos_cell[beg[pc] + k0 + u];
+                        for (int u = 0; u < PL_CHUNK; ++u)
+                            if (k0 + u < len[pc]) c[u] = A.pos_cell[beg[pc] + k0 + u];
 #pragma unroll
-                    for (int u = 0; u < PL_CHUNK; ++u) {
-                        if (k0 + u < len[pc]) {
-                            const float dx = (c[u].x + sx[pc]) - p0.x;
-                            const float dy = (c[u].y + sy) - p0.y;
-                            const float dz = (c[u].z + sz) - p0.z;
-                            const float r2 = fmaf(dz, dz, fmaf(dy, dy, dx * dx));
-                            const int j = __float_as_int(c[u].w);
-                            asm volatile("st.shared.b32 [%0], %1;" ::"r"(wsa), "r"(j) : "memory");
-                            wsa += (r2 < A.rs2 && j != i) ? 128u : 0u;
+                        for (int u = 0; u < PL_CHUNK; ++u) {
+                            if (k0 + u < len[pc]) {
+                                const float dx = c[u].x - qx[pc];
+                                const float ddy2 = c[u].y - qy;
+                                const float ddz2 = c[u].z - qz;
+                                const float r2 = fmaf(ddz2, ddz2, fmaf(ddy2, ddy2, dx * dx));
+                                const int j = __float_as_int(c[u].w);
+                                asm volatile("st.shared.b32 [%0], %1;" ::"r"(wsa), "r"(j) : "memory");
+                                wsa += (r2 < A.rs2 && j != i) ? 128u : 0u;
+                            }
                         }
                     }
                 }
