@@ -527,6 +527,7 @@ __global__ __launch_bounds__(PL_WARPS * 32, 6) void pair_search_lane_kernel(Pair
     const long long ntiles = ((long long)A.n + 31) / 32;
     const float wy = (float)A.L.y / (float)A.nc.y, wz = (float)A.L.z / (float)A.nc.z;
     const float reach2 = A.reach * A.reach;
+    const float nanf_ = __int_as_float(0x7fc00000);
 
     for (long long tile = (long long)blockIdx.x * PL_WARPS + warp; tile < ntiles;
          tile += (long long)gridDim.x * PL_WARPS) {
@@ -617,21 +618,24 @@ __global__ __launch_bounds__(PL_WARPS * 32, 6) void pair_search_lane_kernel(Pair
                     const int maxlen = (int)__reduce_max_sync(FULL, (unsigned)len[pc]);
                     for (int k0 = 0; k0 < maxlen; k0 += PL_CHUNK) {
                         if (__any_sync(FULL, (int)((wsa - buf_sa) >> 7) > PS_BUF - PL_CHUNK)) drain(false);
+                        // slots past this lane's window read a NaN dummy that is
+                        // never accepted, so the test below needs no branch
                         float4 c[PL_CHUNK];
-#pragma unroll
-                        for (int u = 0; u < PL_CHUNK; ++u)
-                            if (k0 + u < len[pc]) c[u] = A.pos_cell[beg[pc] + k0 + u];
+                        const float4* src = A.pos_cell + beg[pc] + k0;
 #pragma unroll
                         for (int u = 0; u < PL_CHUNK; ++u) {
-                            if (k0 + u < len[pc]) {
-                                const float dx = c[u].x - qx[pc];
-                                const float ddy2 = c[u].y - qy;
-                                const float ddz2 = c[u].z - qz;
-                                const float r2 = fmaf(ddz2, ddz2, fmaf(ddy2, ddy2, dx * dx));
-                                const int j = __float_as_int(c[u].w);
-                                asm volatile("st.shared.b32 [%0], %1;" ::"r"(wsa), "r"(j) : "memory");
-                                wsa += (r2 < A.rs2 && j != i) ? 128u : 0u;
-                            }
+                            c[u] = make_float4(nanf_, nanf_, nanf_, 0.f);
+                            if (k0 + u < len[pc]) c[u] = src[u];
+                        }
+#pragma unroll
+                        for (int u = 0; u < PL_CHUNK; ++u) {
+                            const float dx = c[u].x - qx[pc];
+                            const float ddy2 = c[u].y - qy;
+                            const float ddz2 = c[u].z - qz;
+                            const float r2 = fmaf(ddz2, ddz2, fmaf(ddy2, ddy2, dx * dx));
+                            const int j = __float_as_int(c[u].w);
+                            asm volatile("st.shared.b32 [%0], %1;" ::"r"(wsa), "r"(j) : "memory");
+                            wsa += (r2 < A.rs2 && j != i) ? 128u : 0u;
                         }
                     }
                 }
