@@ -67,6 +67,8 @@ def lib():
         L.oracle_neighbors_of.argtypes = [P, i32, i64, P, f32, f32, i64, P, i64]
         L.oracle_neighbors_of.restype = i64
         L.oracle_pair_distances.argtypes = [P, i32, P, P, P, i64, P]
+        L.oracle_neighbors_rows.argtypes = [P, i32, i64, P, f32, f32, P, i64, i32, P, P]
+        L.oracle_edge_aggregate_rows.argtypes = [P, i32, i64, P, f32, P, P, i32, P, i32, P, i64, P, P]
         L.oracle_skin_check.argtypes = [P, P, i32, i64, P, f32, P]
         L.oracle_skin_check.restype = i32
         L.oracle_cutoff.argtypes = [ctypes.c_double, ctypes.c_double]
@@ -167,6 +169,35 @@ def neighbors_of(pos, box, rc, skin, i: int) -> np.ndarray:
         buf = np.empty(int(m), dtype=np.int32)
         m = lib().oracle_neighbors_of(_ptr(pos), stride, len(pos), _ptr(b), float(rc), float(skin), int(i), _ptr(buf), len(buf))
     return buf[: int(m)].copy()
+
+
+def neighbors_rows(pos, box, rc, skin, rows, cap):
+    """Rows `rows` of the list by brute force (C3): (nbr [m, cap], counts [m])."""
+    pos, stride = _pos(pos)
+    b = _box(box)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    nbr = np.empty((len(rows), cap), dtype=np.int32)
+    counts = np.empty(len(rows), dtype=np.int32)
+    lib().oracle_neighbors_rows(_ptr(pos), stride, len(pos), _ptr(b), float(rc), float(skin), _ptr(rows), len(rows),
+                                int(cap), _ptr(nbr), _ptr(counts))
+    return nbr, counts
+
+
+def edge_aggregate_rows(pos, box, rc, nbr, counts, feat, rows):
+    """Aggregate (C5) of rows `rows` only: dict with out and out_abs [m, F]."""
+    pos, stride = _pos(pos)
+    b = _box(box)
+    nbr = np.ascontiguousarray(nbr, dtype=np.int32)
+    counts = np.ascontiguousarray(counts, dtype=np.int32)
+    feat = np.ascontiguousarray(feat, dtype=np.float32)
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    n, cap = nbr.shape
+    F = feat.shape[1]
+    out = np.empty((len(rows), F), dtype=np.float64)
+    out_abs = np.empty((len(rows), F), dtype=np.float64)
+    lib().oracle_edge_aggregate_rows(_ptr(pos), stride, n, _ptr(b), float(rc), _ptr(nbr), _ptr(counts), int(cap),
+                                     _ptr(feat), int(F), _ptr(rows), len(rows), _ptr(out), _ptr(out_abs))
+    return {"out": out, "out_abs": out_abs}
 
 
 def pair_distances(pos, box, i, j) -> np.ndarray:

@@ -357,6 +357,34 @@ int64_t oracle_neighbors_of(const float* pos, int stride, int64_t n, const float
 }
 
 /*
+ * Rows rows[0..m) of the list by brute force over all n atoms (sampled
+ * checks on large systems), rows in parallel.  Same row contract as the
+ * full-list functions: ascending indices, -1 pads, true counts.
+ */
+void oracle_neighbors_rows(const float* pos, int stride, int64_t n, const float* L, float rc, float skin,
+                           const int64_t* rows, int64_t m, int cap, int32_t* nbr, int32_t* counts)
+{
+    const double Ld[3] = {(double)L[0], (double)L[1], (double)L[2]};
+    const double rs = (double)rc + (double)skin;
+    const double rs2 = rs * rs;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t k = 0; k < m; ++k) {
+        const int64_t i = rows[k];
+        int32_t* row = nbr + k * (int64_t)cap;
+        int32_t cnt = 0;
+        for (int c = 0; c < cap; ++c) row[c] = -1;
+        for (int64_t j = 0; j < n; ++j) {
+            if (j == i) continue;
+            if (pair_r2(pos + i * stride, pos + j * stride, Ld) < rs2) {
+                if (cnt < cap) row[cnt] = (int32_t)j;
+                ++cnt;
+            }
+        }
+        counts[k] = cnt;
+    }
+}
+
+/*
  * Pair distances in fp64 for a list of (i, j) pairs -- used by tests to find
  * pairs whose distance is within a band of rs, where an fp32 test may round
  * either way.
@@ -417,6 +445,40 @@ double oracle_cutoff(double r, double rc)
 {
     if (r < rc) return 0.5 * (cos(ORACLE_PI * r / rc) + 1.0);
     return 0.0;
+}
+
+double oracle_cutoff(double r, double rc);
+
+/* C5 for rows rows[0..m) only (sampled checks): out/out_abs are [m, F]. */
+void oracle_edge_aggregate_rows(const float* pos, int stride, int64_t n, const float* L, float rc,
+                                const int32_t* nbr, const int32_t* counts, int cap, const float* feat, int F,
+                                const int64_t* rows, int64_t m, double* out, double* out_abs)
+{
+    const double Ld[3] = {(double)L[0], (double)L[1], (double)L[2]};
+    #pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t k = 0; k < m; ++k) {
+        const int64_t i = rows[k];
+        double* o = out + k * (int64_t)F;
+        double* oa = out_abs + k * (int64_t)F;
+        for (int f = 0; f < F; ++f) { o[f] = 0.0; oa[f] = 0.0; }
+        int64_t mm = counts[i] < cap ? counts[i] : cap;
+        for (int64_t s = 0; s < mm; ++s) {
+            int32_t j = nbr[i * (int64_t)cap + s];
+            if (j < 0 || j >= n) continue;
+            const float* pi = pos + i * stride;
+            const float* pj = pos + (int64_t)j * stride;
+            double dx = min_image((double)pj[0] - (double)pi[0], Ld[0]);
+            double dy = min_image((double)pj[1] - (double)pi[1], Ld[1]);
+            double dz = min_image((double)pj[2] - (double)pi[2], Ld[2]);
+            double fc = oracle_cutoff(sqrt(dx * dx + dy * dy + dz * dz), (double)rc);
+            if (fc == 0.0) continue;
+            const float* h = feat + (int64_t)j * F;
+            for (int f = 0; f < F; ++f) {
+                o[f] += fc * (double)h[f];
+                oa[f] += fc * fabs((double)h[f]);
+            }
+        }
+    }
 }
 
 /*

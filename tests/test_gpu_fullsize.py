@@ -1,0 +1,108 @@
+"""Parity at the full sizes the benchmark runs: the 10.24M-atom salt solution
+and the 10.06M-atom shell-in-water system, through the same calls and launch
+configuration as bench.py.
+
+Outputs the oracle can compute one by one are compared on samples: the whole
+permutation and key array (the oracle sorts 10M keys in seconds), neighbor rows
+of 3,000 sampled atoms plus the first and last tiles (brute force over all
+atoms), the skin flags and maximum displacements of a 6-step trajectory with
+rebuilds (exact, fp64), and aggregated features of sampled rows.  Properties
+that hold at any size are checked on the whole list: pads, counts >= 0, total
+pair count even, symmetry of sampled rows.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_util import agg_error, torch_cuda
+
+pytestmark = pytest.mark.gpu
+
+AGG_TOL = 1e-5
+
+
+@pytest.fixture(scope="module", params=[4, 5])
+def system(request):
+    return synth.system(request.param)
+
+
+def _sample_rows(n, k=3000, seed=0):
+    rng = np.random.default_rng(seed)
+    s = set(rng.choice(n, size=k, replace=False).tolist())
+    s.update(range(0, 32))
+    s.update(range(n - 32, n))
+    return np.array(sorted(s), dtype=np.int64)
+
+
+def test_fullsize_pipeline_against_oracle(system):
+    torch = torch_cuda()
+    import space_filling_curve_b200 as tess
+    s = system
+    dev = torch.device("cuda", 0)
+    pos = torch.from_numpy(s.pos).to(dev)
+
+    # A1-A3: whole permutation and keys
+    perm, keys, ps, st = tess.hilbert_sort(pos, s.box)
+    operm, okeys = oracle.hilbert_sort(s.pos, s.box, 10)
+    assert int(st.item()) == 0
+    assert np.array_equal(perm.cpu().numpy(), operm)
+    assert np.array_equal(keys.cpu().numpy().view(np.uint32), okeys)
+    p4 = s.pos4()[operm]
+    assert np.array_equal(ps.cpu().numpy(), p4)
+
+    # A4-A5: sampled rows, bit-exact sets and counts
+    nbr, cnt, ov = tess.build_neighbors(ps, s.box, s.rc, s.skin, s.cap)
+    torch.cuda.synchronize()
+    rows = _sample_rows(s.n)
+    onbr, ocnt = oracle.neighbors_rows(p4, s.box, s.rc, s.skin, rows, s.cap)
+    g = nbr[torch.from_numpy(rows).to(dev)].cpu().numpy()
+    gc = cnt.cpu().numpy()
+    assert np.array_equal(gc[rows], ocnt)
+    assert int(ov.item()) == int((gc > s.cap).any())
+    for k in range(len(rows)):
+        m = min(ocnt[k], s.cap)
+        assert np.array_equal(np.sort(g[k, :m]), onbr[k, :m]), "row %d differs" % rows[k]
+        assert np.all(g[k, m:] == -1)
+    # properties of the whole list
+    assert int(cnt.min().item()) >= 0 and int(cnt.sum().item()) % 2 == 0
+    slot = torch.arange(s.cap, device=dev)[None, :]
+    m_all = torch.clamp(cnt, max=s.cap)[:, None]
+    assert bool((nbr[slot.expand(s.n, -1) >= m_all] == -1).all().item())
+    # symmetry on the sample: j in row i => i in row j
+    for k in range(0, len(rows), 10):
+        i = int(rows[k])
+        for j in g[k, : min(ocnt[k], s.cap)]:
+            rj = nbr[int(j)].cpu().numpy()
+            assert i in rj[: min(int(gc[j]), s.cap)]
+
+    # A7: aggregation of sampled rows
+    feat = torch.from_numpy(s.features()).to(dev)[perm.long()].contiguous()
+    out = tess.edge_aggregate(ps, s.box, s.rc, nbr, cnt, feat)
+    torch.cuda.synchronize()
+    nb_host = nbr.cpu().numpy()
+    ref = oracle.edge_aggregate_rows(p4, s.box, s.rc, nb_host, gc, feat.cpu().numpy(), rows)
+    err, _ = agg_error(out[torch.from_numpy(rows).to(dev)].cpu().numpy(), ref)
+    assert err <= AGG_TOL
+
+    # A6: skin flags of a short trajectory with rebuilds, exact in fp64
+    ref4 = ps
+    cur_perm = perm
+    o_ref = p4
+    o_perm = operm
+    flags = []
+    for t, frame in s.trajectory(6, condition=False):
+        cur = torch.zeros_like(ref4)
+        cur[:, :3] = torch.from_numpy(frame).to(dev)[cur_perm.long()]
+        rb, md = tess.skin_check(cur, ref4, s.box, s.skin)
+        oc = np.zeros_like(o_ref)
+        oc[:, :3] = frame[o_perm]
+        f, m = oracle.skin_check(oc, o_ref, s.box, s.skin)
+        assert int(rb.item()) == f and float(md.item()) == m
+        flags.append(f)
+        if f:
+            cur_perm, _, ref4, _ = tess.hilbert_sort(torch.from_numpy(frame).to(dev), s.box)
+            o_perm, _ = oracle.hilbert_sort(frame, s.box, 10)
+            assert np.array_equal(cur_perm.cpu().numpy(), o_perm)
+            o_ref = np.zeros_like(o_ref)
+            o_ref[:, :3] = frame[o_perm]

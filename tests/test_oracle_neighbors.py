@@ -215,3 +215,16 @@ def test_aggregate_identities():
         d = s.pos[j].astype(np.float64) - s.pos[i].astype(np.float64)
         d -= np.asarray(s.box) * np.round(d / np.asarray(s.box))
         assert np.allclose(ev[i, slot, :3], d, atol=1e-12)
+
+
+def test_sampled_row_helpers_match_the_full_oracle():
+    s = synth.system(1)
+    nbr, cnt, _ = oracle.neighbors_brute(s.pos, s.box, s.rc, s.skin, s.cap)
+    rows = np.array([0, 5, 17, 2999])
+    r, rc = oracle.neighbors_rows(s.pos, s.box, s.rc, s.skin, rows, s.cap)
+    assert np.array_equal(r, nbr[rows]) and np.array_equal(rc, cnt[rows])
+    f = s.features()
+    full = oracle.edge_aggregate(s.pos, s.box, s.rc, nbr, cnt, f)
+    part = oracle.edge_aggregate_rows(s.pos, s.box, s.rc, nbr, cnt, f, rows)
+    assert np.array_equal(full["out"][rows], part["out"])
+    assert np.array_equal(full["out_abs"][rows], part["out_abs"])
