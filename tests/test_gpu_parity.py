@@ -322,3 +322,40 @@ def test_edge_aggregate_constant_features_sum_fc():
     ones = _dev(np.ones((s.n, 1), np.float32) * np.float32(3.0))
     out, ev, ef, eu = tess.edge_aggregate(_dev(p4), s.box, s.rc, nbr_d, cnt_d, ones, edges=True)
     assert np.allclose(out.cpu().numpy()[:, 0], 3.0 * ef.cpu().numpy().astype(np.float64).sum(1), rtol=1e-5)
+
+
+@pytest.mark.parametrize("cfg", [1, 2])
+def test_edge_aggregate_grouped_rows(cfg):
+    # no edge arrays, F a multiple of 32: the grouped-row union kernel
+    tess = _tess()
+    s = synth.system(cfg)
+    perm, _ = oracle.hilbert_sort(s.pos, s.box, 10)
+    p4 = s.pos4()[perm]
+    F = 32 if s.F < 32 else s.F
+    feat = np.random.default_rng(3).standard_normal((s.n, F)).astype(np.float32)
+    nbr_d, cnt_d, _ = tess.build_neighbors(_dev(p4), s.box, s.rc, s.skin, s.cap)
+    out1 = tess.edge_aggregate(_dev(p4), s.box, s.rc, nbr_d, cnt_d, _dev(feat)).cpu().numpy()
+    out2 = tess.edge_aggregate(_dev(p4), s.box, s.rc, nbr_d, cnt_d, _dev(feat)).cpu().numpy()
+    ref = oracle.edge_aggregate(p4, s.box, s.rc, nbr_d.cpu().numpy(), cnt_d.cpu().numpy(), feat)
+    err, _ = agg_error(out1, ref)
+    assert err <= AGG_TOL
+    assert np.array_equal(out1, out2), "repeated calls should give identical sums"
+
+
+@pytest.mark.parametrize("F", [32, 64, 128])
+def test_edge_aggregate_dense_groups_fall_back(F):
+    # ~300 neighbors per row: the union of 8 rows overflows the shared table
+    tess = _tess()
+    rng = np.random.default_rng(F)
+    L = 30.0
+    n = 6000
+    p = np.zeros((n, 4), np.float32)
+    p[:, :3] = rng.uniform(0, L, (n, 3))
+    p = p[oracle.hilbert_sort(p, (L, L, L), 10)[0]]
+    feat = rng.standard_normal((n, F)).astype(np.float32)
+    nbr_d, cnt_d, ov = tess.build_neighbors(_dev(p), (L, L, L), 5.0, 0.5, 512)
+    assert int(ov.item()) == 0
+    out = tess.edge_aggregate(_dev(p), (L, L, L), 5.0, nbr_d, cnt_d, _dev(feat)).cpu().numpy()
+    ref = oracle.edge_aggregate(p, (L, L, L), 5.0, nbr_d.cpu().numpy(), cnt_d.cpu().numpy(), feat)
+    err, _ = agg_error(out, ref)
+    assert err <= AGG_TOL
