@@ -309,212 +309,6 @@ __global__ __launch_bounds__(EV_WARPS * 32, 3) void edge_vec4_kernel(EdgeArgs A)
     }
 }
 
-// ---------------------------------------------------------------- aggregate over row groups
-
-// Consecutive (Hilbert-ordered) rows share most of their neighbors: eight rows
-// of the salt solution list ~86 live neighbors each but only ~25 distinct ones
-// per row between them.  This kernel gives each warp a group of AG_R rows,
-// builds the union of their live neighbors in a shared-memory hash (key j,
-// one f_c weight per row), then loads each union member's feature row once
-// and applies it to all AG_R accumulators: the feature gathers, which bound the
-// per-row kernel, shrink by the reuse factor.  FPL features per lane (F = 32
-// FPL).  A group whose union does not fit the table falls back to the per-row
-// sum in the same kernel.  Used when no edge arrays are requested.
-constexpr int AG_R = 8;
-constexpr int AG_TBL = 256;
-constexpr int AG_WARPS = 4;
-constexpr int AG_GEO_UNROLL = 4;
-constexpr int AG_ACC_UNROLL = 4;
-
-struct AggWarpSmem {
-    int key[AG_TBL];
-    float4 w[AG_TBL][AG_R / 4];
-    int list[AG_TBL];
-};
-
-template <int FPL> struct FVec;
-template <> struct FVec<1> { using T = float; };
-template <> struct FVec<2> { using T = float2; };
-template <> struct FVec<4> { using T = float4; };
-
-__device__ __forceinline__ void fv_fma(float& a, float w, float h) { a = fmaf(w, h, a); }
-template <int FPL>
-__device__ __forceinline__ void fv_acc(float* acc, float w, const typename FVec<FPL>::T& h) {
-    const float* hv = reinterpret_cast<const float*>(&h);
-#pragma unroll
-    for (int v = 0; v < FPL; ++v) acc[v] = fmaf(w, hv[v], acc[v]);
-}
-
-__device__ __forceinline__ unsigned agg_hash(int j) { return ((unsigned)j * 2654435761u) >> 24; }
-
-template <int FPL>
-__global__ __launch_bounds__(AG_WARPS * 32, 5) void edge_union_kernel(EdgeArgs A) {
-    using V = typename FVec<FPL>::T;
-    __shared__ AggWarpSmem smem_a[AG_WARPS];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    AggWarpSmem& T = smem_a[warp];
-    for (int k = lane; k < AG_TBL; k += 32) {
-        T.key[k] = -1;
-#pragma unroll
-        for (int q = 0; q < AG_R / 4; ++q) T.w[k][q] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    __syncwarp();
-    const V* feat = reinterpret_cast<const V*>(A.feat);
-    V* outv = reinterpret_cast<V*>(A.out);
-    const int FV = A.F / FPL;                 // V elements per feature row (= 32)
-    const long long ngroups = ((long long)A.n + AG_R - 1) / AG_R;
-
-    for (long long g = (long long)blockIdx.x * AG_WARPS + warp; g < ngroups; g += (long long)gridDim.x * AG_WARPS) {
-        const long long base = g * AG_R;
-        const int nrows = (int)min((long long)AG_R, (long long)A.n - base);
-        bool full = false;
-
-        // phase 1: geometry of every listed edge of the group's rows; live
-        // edges enter the table with their weight in the row's column
-        for (int r = 0; r < nrows; ++r) {
-            const long long i = base + r;
-            const float4 pi = A.pos[i];
-            const int m = max(min(A.counts[i], A.cap), 0);
-            for (int s0 = 0; s0 < m; s0 += 32 * AG_GEO_UNROLL) {
-                int j[AG_GEO_UNROLL];
-                float4 pj[AG_GEO_UNROLL];
-#pragma unroll
-                for (int u = 0; u < AG_GEO_UNROLL; ++u) {
-                    const int s = s0 + u * 32 + lane;
-                    j[u] = (s < m) ? A.nbr[(size_t)i * A.cap + s] : -1;
-                    if (j[u] >= A.n) j[u] = -1;
-                }
-#pragma unroll
-                for (int u = 0; u < AG_GEO_UNROLL; ++u)
-                    if (j[u] >= 0) pj[u] = A.pos[j[u]];
-#pragma unroll
-                for (int u = 0; u < AG_GEO_UNROLL; ++u) {
-                    if (j[u] < 0) continue;
-                    const float dx = min_image_f(pj[u].x - pi.x, A.L.x);
-                    const float dy = min_image_f(pj[u].y - pi.y, A.L.y);
-                    const float dz = min_image_f(pj[u].z - pi.z, A.L.z);
-                    const float u2 = fmaf(dz, dz, fmaf(dy, dy, dx * dx)) * A.inv_rc2;
-                    if (!(u2 < 1.0f)) continue;
-                    const float fc = cutoff_u(u2);
-                    unsigned slot = agg_hash(j[u]);
-                    int probes = 0;
-                    for (; probes < AG_TBL; ++probes) {
-                        const int old = atomicCAS(&T.key[slot], -1, j[u]);
-                        if (old == -1 || old == j[u]) break;
-                        slot = (slot + 1) & (AG_TBL - 1);
-                    }
-                    if (probes == AG_TBL) full = true;
-                    else reinterpret_cast<float*>(&T.w[slot][0])[r] = fc;
-                }
-            }
-        }
-        const bool group_full = __any_sync(FULL, full);
-        __syncwarp();
-
-        // phase 2: compact the occupied slots
-        int nu = 0;
-        for (int k0 = 0; k0 < AG_TBL; k0 += 32) {
-            const bool occ = T.key[k0 + lane] != -1;
-            const unsigned bm = __ballot_sync(FULL, occ);
-            if (occ) T.list[nu + __popc(bm & lanemask_lt())] = k0 + lane;
-            nu += __popc(bm);
-        }
-        __syncwarp();
-
-        float acc[AG_R][FPL];
-#pragma unroll
-        for (int r = 0; r < AG_R; ++r)
-#pragma unroll
-            for (int v = 0; v < FPL; ++v) acc[r][v] = 0.f;
-
-        if (!group_full) {
-            // phase 3: one feature load per union member, AG_R FMAs per feature
-            for (int e0 = 0; e0 < nu; e0 += AG_ACC_UNROLL) {
-                int slot[AG_ACC_UNROLL];
-                V h[AG_ACC_UNROLL];
-#pragma unroll
-                for (int u = 0; u < AG_ACC_UNROLL; ++u) {
-                    slot[u] = T.list[min(e0 + u, nu - 1)];
-                    h[u] = feat[(size_t)T.key[slot[u]] * FV + lane];
-                }
-#pragma unroll
-                for (int u = 0; u < AG_ACC_UNROLL; ++u) {
-                    if (e0 + u >= nu) break;
-                    const float4 wa = T.w[slot[u]][0];
-                    const float4 wb = T.w[slot[u]][1];
-                    fv_acc<FPL>(acc[0], wa.x, h[u]);
-                    fv_acc<FPL>(acc[1], wa.y, h[u]);
-                    fv_acc<FPL>(acc[2], wa.z, h[u]);
-                    fv_acc<FPL>(acc[3], wa.w, h[u]);
-                    fv_acc<FPL>(acc[4], wb.x, h[u]);
-                    fv_acc<FPL>(acc[5], wb.y, h[u]);
-                    fv_acc<FPL>(acc[6], wb.z, h[u]);
-                    fv_acc<FPL>(acc[7], wb.w, h[u]);
-                }
-            }
-        } else {
-            // the union did not fit: sum row by row, edges broadcast by shuffles
-            for (int r = 0; r < nrows; ++r) {
-                const long long i = base + r;
-                const float4 pi = A.pos[i];
-                const int m = max(min(A.counts[i], A.cap), 0);
-                for (int s0 = 0; s0 < m; s0 += 32) {
-                    const int s = s0 + lane;
-                    int j = (s < m) ? A.nbr[(size_t)i * A.cap + s] : -1;
-                    if (j >= A.n) j = -1;
-                    float fc = 0.f;
-                    if (j >= 0) {
-                        const float4 pj = A.pos[j];
-                        const float dx = min_image_f(pj.x - pi.x, A.L.x);
-                        const float dy = min_image_f(pj.y - pi.y, A.L.y);
-                        const float dz = min_image_f(pj.z - pi.z, A.L.z);
-                        const float u2 = fmaf(dz, dz, fmaf(dy, dy, dx * dx)) * A.inv_rc2;
-                        fc = u2 < 1.0f ? cutoff_u(u2) : 0.0f;
-                    }
-                    unsigned live = __ballot_sync(FULL, fc != 0.f);
-                    while (live) {
-                        const int l = __ffs(live) - 1;
-                        live &= live - 1;
-                        const int jj = __shfl_sync(FULL, j, l);
-                        const float w = __shfl_sync(FULL, fc, l);
-                        const V hv = feat[(size_t)jj * FV + lane];
-#pragma unroll
-                        for (int rr = 0; rr < AG_R; ++rr)
-                            if (rr == r) fv_acc<FPL>(acc[rr], w, hv);
-                    }
-                }
-            }
-        }
-
-        // write the group's rows (coalesced), then clear the used slots
-#pragma unroll
-        for (int r = 0; r < AG_R; ++r) {
-            if (r < nrows) {
-                V o;
-                float* ov = reinterpret_cast<float*>(&o);
-#pragma unroll
-                for (int v = 0; v < FPL; ++v) ov[v] = acc[r][v];
-                outv[(size_t)(base + r) * FV + lane] = o;
-            }
-        }
-        if (group_full) {
-            for (int k = lane; k < AG_TBL; k += 32) {
-                T.key[k] = -1;
-#pragma unroll
-                for (int q = 0; q < AG_R / 4; ++q) T.w[k][q] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-        } else {
-            for (int e = lane; e < nu; e += 32) {
-                const int sl = T.list[e];
-                T.key[sl] = -1;
-#pragma unroll
-                for (int q = 0; q < AG_R / 4; ++q) T.w[sl][q] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-        }
-        __syncwarp();
-    }
-}
-
 tess_status edge_aggregate(const float* pos, int n, tess_box box, float rc, const int32_t* nbr, const int32_t* counts,
                            int cap, const float* feat, int F, float* out, float* edge_vec, float* edge_fc,
                            float* edge_unit, cudaStream_t s) {
@@ -545,17 +339,6 @@ tess_status edge_aggregate(const float* pos, int n, tess_box box, float rc, cons
     StageScope sc(ST_EDGE, s);
     const long long rows_blocks = ((long long)n + EDGE_WARPS - 1) / EDGE_WARPS;
     const int blocks = (int)std::min<long long>(rows_blocks, (long long)sms * 64);
-    const bool edges = edge_vec || edge_fc || edge_unit;
-    const int fpl = F / 32;
-    if (!edges && F % 32 == 0 && (fpl == 1 || fpl == 2 || fpl == 4) && aligned(feat, 4 * fpl) && aligned(out, 4 * fpl)) {
-        const int ublocks = (int)std::min<long long>(((long long)n + AG_R * AG_WARPS - 1) / (AG_R * AG_WARPS),
-                                                     (long long)sms * 40);
-        if (fpl == 1) edge_union_kernel<1><<<ublocks, AG_WARPS * 32, 0, s>>>(A);
-        else if (fpl == 2) edge_union_kernel<2><<<ublocks, AG_WARPS * 32, 0, s>>>(A);
-        else edge_union_kernel<4><<<ublocks, AG_WARPS * 32, 0, s>>>(A);
-        count_launch();
-        return launch_status();
-    }
     const bool vec4 = (F % 4 == 0) && F <= 256 && aligned(feat, 16) && aligned(out, 16) && cap <= EV_MAXCAP;
     const int vblocks = (int)std::min<long long>(((long long)n + EV_WARPS - 1) / EV_WARPS, (long long)sms * 32);
     bool launched = false;

@@ -325,8 +325,7 @@ def test_edge_aggregate_constant_features_sum_fc():
 
 
 @pytest.mark.parametrize("cfg", [1, 2])
-def test_edge_aggregate_grouped_rows(cfg):
-    # no edge arrays, F a multiple of 32: the grouped-row union kernel
+def test_edge_aggregate_without_edge_arrays(cfg):
     tess = _tess()
     s = synth.system(cfg)
     perm, _ = oracle.hilbert_sort(s.pos, s.box, 10)
@@ -343,8 +342,8 @@ def test_edge_aggregate_grouped_rows(cfg):
 
 
 @pytest.mark.parametrize("F", [32, 64, 128])
-def test_edge_aggregate_dense_groups_fall_back(F):
-    # ~300 neighbors per row: the union of 8 rows overflows the shared table
+def test_edge_aggregate_dense_rows(F):
+    # ~300 neighbors per row
     tess = _tess()
     rng = np.random.default_rng(F)
     L = 30.0
