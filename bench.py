@@ -123,7 +123,7 @@ def sum_over_ranks(value: float, world: int, device=None) -> float:
 class Step:
     """All device buffers of one replica and the step itself, through the C ABI."""
 
-    def __init__(self, s, device, pad_fill=True):
+    def __init__(self, s, device, pad_fill=True, tile_search=False):
         import torch
         import space_filling_curve_b200 as tess
         self.tess = tess
@@ -151,6 +151,7 @@ class Step:
         self.feat = torch.randn((n, F), generator=g, device=device, dtype=torch.float32)
         self.out = torch.empty((n, F), dtype=torch.float32, device=device)
         self.pad_fill = pad_fill
+        self.tile_search = tile_search
         # the next frame of the trajectory, in the sorted order of frame 0
         t1 = next(iter(s.trajectory(1, condition=False)))[1]
         self.frame1 = torch.from_numpy(t1).to(device)
@@ -172,7 +173,8 @@ class Step:
                                    P(self.perm), P(self.keys), P(self.pos_sorted), P(self.status), st)
         assert c == 0, c
         c = tess.tess_build_neighbors(P(self.pos_sorted), self.n, s.box, s.rc, s.skin, s.cap,
-                                      0 if self.pad_fill else tess.TESS_NO_PAD_FILL, P(self.ws_nbr),
+                                      (0 if self.pad_fill else tess.TESS_NO_PAD_FILL)
+                                      | (tess.TESS_TILE_SEARCH if self.tile_search else 0), P(self.ws_nbr),
                                       self.ws_nbr.numel(), P(self.nbr), P(self.counts), P(self.overflow), st)
         assert c == 0, c
         c = tess.tess_skin_check(P(self.pos_next), P(self.pos_sorted), self.n, s.box, s.skin, P(self.rebuild),
@@ -207,7 +209,7 @@ def run_cuda(args, world, rank, local):
     import synth
     import space_filling_curve_b200 as tess
     s = synth.system(args.config)
-    step = Step(s, dev, pad_fill=not args.no_pad_fill)
+    step = Step(s, dev, pad_fill=not args.no_pad_fill, tile_search=args.tile_search)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
         flush.zero_()
@@ -293,6 +295,7 @@ def run_cuda(args, world, rank, local):
                             % (s.n, s.box[0], s.rc, s.skin, s.cap, s.F),
                 "atoms": s.n,
                 "pad_fill": not args.no_pad_fill,
+                "pair_search": "tile" if args.tile_search else "per-lane",
                 "l2": "flushed between timed steps (256 MB write); each step also moves ~9 GB",
                 "parallelism": "replicas (no collective in the data path)",
                 "mean_neighbors": mean_count,
@@ -423,6 +426,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["tess", "reference"], default="tess")
     ap.add_argument("--config", type=int, default=WORKLOAD_CFG)
     ap.add_argument("--no-pad-fill", action="store_true")
+    ap.add_argument("--tile-search", action="store_true", help="use the warp-shared tile pair search")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     world, rank, local = _dist_setup(args)

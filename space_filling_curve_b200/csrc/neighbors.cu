@@ -366,31 +366,32 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
         // (stores for rejected candidates are overwritten by the next one).
         auto test_chunk = [&]() {
             __syncwarp();
-            if (ncand & 1) {
-                if (lane == 0) put_cand(W, ncand, make_float4(nanf_, nanf_, nanf_, __int_as_float(-1)));
-                ++ncand;
-                __syncwarp();
-            }
-            const int npair = ncand >> 1;
-            for (int c = 0; c < npair; c += PS_TEST_UNROLL) {
+            // pad to a whole number of unrolled steps with candidates that are
+            // never accepted (NaN position), so the loop needs no bounds tests
+            const int padded = (ncand + 2 * PS_TEST_UNROLL - 1) & ~(2 * PS_TEST_UNROLL - 1);
+            if (lane < padded - ncand)
+                put_cand(W, ncand + lane, make_float4(nanf_, nanf_, nanf_, __int_as_float(-1)));
+            __syncwarp();
+            const unsigned ca_sa = (unsigned)__cvta_generic_to_shared(&W.ca[0]);
+            const unsigned cb_sa = (unsigned)__cvta_generic_to_shared(&W.cb[0]);
+            for (int c = 0; c < (padded >> 1); c += PS_TEST_UNROLL) {
                 // room for 2 * PS_TEST_UNROLL more in every lane's buffer?
                 if (__any_sync(FULL, (int)((wsa - buf_sa) >> 7) > PS_BUF - 2 * PS_TEST_UNROLL)) drain(false);
-                float4 a[PS_TEST_UNROLL], b[PS_TEST_UNROLL];
+                unsigned long long xx[PS_TEST_UNROLL], yy[PS_TEST_UNROLL], zz[PS_TEST_UNROLL], jj[PS_TEST_UNROLL];
 #pragma unroll
                 for (int u = 0; u < PS_TEST_UNROLL; ++u) {
-                    // pairs past the end hold stale data; their index is forced to i (never accepted)
-                    const int k = min(c + u, PS_CHUNK / 2 - 1);
-                    a[u] = W.ca[k];
-                    b[u] = W.cb[k];
-                    if (c + u >= npair) b[u].z = b[u].w = __int_as_float(i);
+                    asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];"
+                                 : "=l"(xx[u]), "=l"(yy[u]) : "r"(ca_sa + 16u * (unsigned)(c + u)));
+                    asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];"
+                                 : "=l"(zz[u]), "=l"(jj[u]) : "r"(cb_sa + 16u * (unsigned)(c + u)));
                 }
 #pragma unroll
                 for (int u = 0; u < PS_TEST_UNROLL; ++u) {
-                    const unsigned long long dx = f2_sub(pk(a[u].x, a[u].y), px2);
-                    const unsigned long long dy = f2_sub(pk(a[u].z, a[u].w), py2);
-                    const unsigned long long dz = f2_sub(pk(b[u].x, b[u].y), pz2);
+                    const unsigned long long dx = f2_sub(xx[u], px2);
+                    const unsigned long long dy = f2_sub(yy[u], py2);
+                    const unsigned long long dz = f2_sub(zz[u], pz2);
                     const unsigned long long r2 = f2_fma(dz, dz, f2_fma(dy, dy, f2_mul(dx, dx)));
-                    const int j0 = __float_as_int(b[u].z), j1 = __float_as_int(b[u].w);
+                    const int j0 = (int)(unsigned)jj[u], j1 = (int)(unsigned)(jj[u] >> 32);
                     asm volatile("st.shared.b32 [%0], %1;" ::"r"(wsa), "r"(j0) : "memory");
                     wsa += (pk_lo(r2) < A.rs2 && j0 != i) ? 128u : 0u;
                     asm volatile("st.shared.b32 [%0], %1;" ::"r"(wsa), "r"(j1) : "memory");
@@ -454,7 +455,7 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
 
             int sc = 0;   // this lane's segment cursor
             for (int t0 = 0; t0 < total; t0 += 32 * PS_UNROLL) {
-                if (ncand > PS_CHUNK - 1 - 32 * PS_UNROLL) test_chunk();
+                if (ncand > PS_CHUNK - 2 * PS_TEST_UNROLL - 32 * PS_UNROLL) test_chunk();
                 float4 q[PS_UNROLL];
                 bool ok[PS_UNROLL];
 #pragma unroll
