@@ -215,7 +215,7 @@ constexpr int PS_MAXSEG = 64;        // cell-row segments per table batch
 constexpr int PS_UNROLL = 4;         // candidate loads in flight per lane
 constexpr int PS_BUF = 32;           // per-lane staging of accepted indices (linear)
 constexpr int PS_GROUP = 8;          // accepted indices leave in aligned groups of 8 (32 bytes)
-constexpr int PS_TEST_UNROLL = 4;    // candidate pairs tested between fullness votes
+constexpr int PS_TEST_UNROLL = 4;    // candidate pairs tested between fullness votes (the loop is written for 4)
 
 struct PairArgs {
     const float4* pos;
@@ -273,6 +273,27 @@ __device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsig
     return d;
 }
 
+// Two 8-byte words from shared memory at base + OFF (OFF an immediate).
+template <int OFF>
+__device__ __forceinline__ void ld_pair(unsigned base, unsigned long long& a, unsigned long long& b) {
+    asm volatile("ld.shared.v2.u64 {%0, %1}, [%2+%3];" : "=l"(a), "=l"(b) : "r"(base), "n"(OFF));
+}
+
+// Append candidate j at the buffer slot *wsa and advance the slot by one
+// lane-interleaved step (128 bytes) if r2 < rs2 and j is not the atom itself.
+// The store happens either way; a rejected index is overwritten by the next.
+__device__ __forceinline__ void append_if(unsigned& wsa, float r2, float rs2, int j, int self) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.lt.f32 p, %1, %2;\n\t"
+        "setp.ne.and.s32 p, %3, %4, p;\n\t"
+        "st.shared.b32 [%0], %3;\n\t"
+        "@p add.u32 %0, %0, 128;\n\t}"
+        : "+r"(wsa)
+        : "f"(r2), "f"(rs2), "r"(j), "r"(self)
+        : "memory");
+}
+
 // Store one accepted index into slot `slot` of a candidate pair array.
 __device__ __forceinline__ void put_cand(PairWarpSmem& W, int slot, float4 q) {
     float* a = reinterpret_cast<float*>(&W.ca[slot >> 1]) + (slot & 1);
@@ -286,6 +307,7 @@ __device__ __forceinline__ void put_cand(PairWarpSmem& W, int slot, float4 q) {
 __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs A) {
     __shared__ PairWarpSmem smem_w[PS_WARPS];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const unsigned lt_mask = lanemask_lt();
     PairWarpSmem& W = smem_w[warp];
     // slot s of this lane's buffer is W.buf[s * 32 + lane]: lanes interleaved
     // across the 32 banks, so the appends of a warp never conflict
@@ -377,25 +399,24 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
             for (int c = 0; c < (padded >> 1); c += PS_TEST_UNROLL) {
                 // room for 2 * PS_TEST_UNROLL more in every lane's buffer?
                 if (__any_sync(FULL, (int)((wsa - buf_sa) >> 7) > PS_BUF - 2 * PS_TEST_UNROLL)) drain(false);
-                unsigned long long xx[PS_TEST_UNROLL], yy[PS_TEST_UNROLL], zz[PS_TEST_UNROLL], jj[PS_TEST_UNROLL];
+                unsigned long long xx[4], yy[4], zz[4], jj[4];
+                const unsigned ab = ca_sa + 16u * (unsigned)c, bb = cb_sa + 16u * (unsigned)c;
+                ld_pair<0>(ab, xx[0], yy[0]);
+                ld_pair<0>(bb, zz[0], jj[0]);
+                ld_pair<16>(ab, xx[1], yy[1]);
+                ld_pair<16>(bb, zz[1], jj[1]);
+                ld_pair<32>(ab, xx[2], yy[2]);
+                ld_pair<32>(bb, zz[2], jj[2]);
+                ld_pair<48>(ab, xx[3], yy[3]);
+                ld_pair<48>(bb, zz[3], jj[3]);
 #pragma unroll
-                for (int u = 0; u < PS_TEST_UNROLL; ++u) {
-                    asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];"
-                                 : "=l"(xx[u]), "=l"(yy[u]) : "r"(ca_sa + 16u * (unsigned)(c + u)));
-                    asm volatile("ld.shared.v2.u64 {%0, %1}, [%2];"
-                                 : "=l"(zz[u]), "=l"(jj[u]) : "r"(cb_sa + 16u * (unsigned)(c + u)));
-                }
-#pragma unroll
-                for (int u = 0; u < PS_TEST_UNROLL; ++u) {
+                for (int u = 0; u < 4; ++u) {
                     const unsigned long long dx = f2_sub(xx[u], px2);
                     const unsigned long long dy = f2_sub(yy[u], py2);
                     const unsigned long long dz = f2_sub(zz[u], pz2);
                     const unsigned long long r2 = f2_fma(dz, dz, f2_fma(dy, dy, f2_mul(dx, dx)));
-                    const int j0 = (int)(unsigned)jj[u], j1 = (int)(unsigned)(jj[u] >> 32);
-                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(wsa), "r"(j0) : "memory");
-                    wsa += (pk_lo(r2) < A.rs2 && j0 != i) ? 128u : 0u;
-                    asm volatile("st.shared.b32 [%0], %1;" ::"r"(wsa), "r"(j1) : "memory");
-                    wsa += (pk_hi(r2) < A.rs2 && j1 != i) ? 128u : 0u;
+                    append_if(wsa, pk_lo(r2), A.rs2, (int)(unsigned)jj[u], i);
+                    append_if(wsa, pk_hi(r2), A.rs2, (int)(unsigned)(jj[u] >> 32), i);
                 }
             }
             ncand = 0;
@@ -479,7 +500,7 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
                         keep = fmaf(ez, ez, fmaf(ey, ey, ex * ex)) < reach2;
                     }
                     const unsigned bm = __ballot_sync(FULL, keep);
-                    if (keep) put_cand(W, ncand + __popc(bm & lanemask_lt()), q[u]);
+                    if (keep) put_cand(W, ncand + __popc(bm & lt_mask), q[u]);
                     ncand += __popc(bm);
                 }
             }
@@ -634,9 +655,7 @@ __global__ __launch_bounds__(PL_WARPS * 32, 6) void pair_search_lane_kernel(Pair
                             const float ddy2 = c[u].y - qy;
                             const float ddz2 = c[u].z - qz;
                             const float r2 = fmaf(ddz2, ddz2, fmaf(ddy2, ddy2, dx * dx));
-                            const int j = __float_as_int(c[u].w);
-                            asm volatile("st.shared.b32 [%0], %1;" ::"r"(wsa), "r"(j) : "memory");
-                            wsa += (r2 < A.rs2 && j != i) ? 128u : 0u;
+                            append_if(wsa, r2, A.rs2, __float_as_int(c[u].w), i);
                         }
                     }
                 }
