@@ -294,6 +294,36 @@ __device__ __forceinline__ void append_if(unsigned& wsa, float r2, float rs2, in
         : "memory");
 }
 
+// Test one candidate pair (x0,x1), (y0,y1), (z0,z1), (j0,j1) against the atom
+// at (px, py, pz) (each duplicated into both halves) with packed f32x2
+// arithmetic, and append the accepted indices at *wsa (see append_if).  One
+// PTX block, so the halves are never moved out of their register pairs.
+__device__ __forceinline__ void test_pair(unsigned& wsa, unsigned long long xx, unsigned long long yy,
+                                          unsigned long long zz, unsigned long long jj, unsigned long long px2,
+                                          unsigned long long py2, unsigned long long pz2, float rs2, int self) {
+    asm volatile(
+        "{\n\t.reg .b64 dx, dy, dz, r2;\n\t.reg .f32 r0, r1;\n\t.reg .b32 j0, j1;\n\t.reg .pred p, q;\n\t"
+        "sub.rn.f32x2 dx, %1, %5;\n\t"
+        "sub.rn.f32x2 dy, %2, %6;\n\t"
+        "sub.rn.f32x2 dz, %3, %7;\n\t"
+        "mul.rn.f32x2 r2, dx, dx;\n\t"
+        "fma.rn.f32x2 r2, dy, dy, r2;\n\t"
+        "fma.rn.f32x2 r2, dz, dz, r2;\n\t"
+        "mov.b64 {r0, r1}, r2;\n\t"
+        "mov.b64 {j0, j1}, %4;\n\t"
+        "setp.lt.f32 p, r0, %8;\n\t"
+        "setp.ne.and.s32 p, j0, %9, p;\n\t"
+        "st.shared.b32 [%0], j0;\n\t"
+        "@p add.u32 %0, %0, 128;\n\t"
+        "setp.lt.f32 q, r1, %8;\n\t"
+        "setp.ne.and.s32 q, j1, %9, q;\n\t"
+        "st.shared.b32 [%0], j1;\n\t"
+        "@q add.u32 %0, %0, 128;\n\t}"
+        : "+r"(wsa)
+        : "l"(xx), "l"(yy), "l"(zz), "l"(jj), "l"(px2), "l"(py2), "l"(pz2), "f"(rs2), "r"(self)
+        : "memory");
+}
+
 // Store one accepted index into slot `slot` of a candidate pair array.
 __device__ __forceinline__ void put_cand(PairWarpSmem& W, int slot, float4 q) {
     float* a = reinterpret_cast<float*>(&W.ca[slot >> 1]) + (slot & 1);
@@ -351,6 +381,7 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
         unsigned wsa = buf_sa;
         int ncand = 0;     // staged candidates (warp-uniform)
         const unsigned long long px2 = pk(p.x, p.x), py2 = pk(p.y, p.y), pz2 = pk(p.z, p.z);
+        const float rs2 = A.rs2;
 
         // write the complete groups of 8 buffered indices to the row; with
         // `all`, the remainder too.  The remainder of a partial drain moves
@@ -410,14 +441,7 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
                 ld_pair<48>(ab, xx[3], yy[3]);
                 ld_pair<48>(bb, zz[3], jj[3]);
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const unsigned long long dx = f2_sub(xx[u], px2);
-                    const unsigned long long dy = f2_sub(yy[u], py2);
-                    const unsigned long long dz = f2_sub(zz[u], pz2);
-                    const unsigned long long r2 = f2_fma(dz, dz, f2_fma(dy, dy, f2_mul(dx, dx)));
-                    append_if(wsa, pk_lo(r2), A.rs2, (int)(unsigned)jj[u], i);
-                    append_if(wsa, pk_hi(r2), A.rs2, (int)(unsigned)(jj[u] >> 32), i);
-                }
+                for (int u = 0; u < 4; ++u) test_pair(wsa, xx[u], yy[u], zz[u], jj[u], px2, py2, pz2, rs2, i);
             }
             ncand = 0;
             __syncwarp();
