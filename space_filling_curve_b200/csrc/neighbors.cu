@@ -24,18 +24,22 @@ namespace tess {
 
 // ---------------------------------------------------------------- grid
 
+// Cells are at least rs / CELL_DIV wide, so +-CELL_DIV cell rows cover rs.
+constexpr int CELL_DIV = 3;
+
 struct Grid {
     int nc[3];
     float inv_w[3];
     long long ncell;
 };
 
-// Cells of width about rs/2 (the pair search adapts to any width), coarsened
-// when that would give more than ~2 cells per atom.
+// Cells of width about rs/CELL_DIV (the tile search adapts to any width; the
+// per-lane stencil relies on width >= rs/CELL_DIV, which coarsening keeps),
+// coarsened when that would give more than ~2 cells per atom.
 static Grid make_grid(int n, tess_box box, float rs) {
     Grid g{};
     const float L[3] = {box.lx, box.ly, box.lz};
-    double w = (double)rs * 1.0001 / 2.0;
+    double w = (double)rs * 1.0001 / (double)CELL_DIV;
     for (int it = 0; it < 64; ++it) {
         long long tot = 1;
         for (int d = 0; d < 3; ++d) {
@@ -553,7 +557,8 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
 // ---------------------------------------------------------------- per-lane search
 
 // One warp per 32 consecutive atoms, but every lane walks its own stencil:
-// the 5 x 5 cell rows (cells of width >= rs/2, so +-2 rows cover rs) around
+// the (2 CELL_DIV + 1)^2 cell rows (cells of width >= rs/CELL_DIV, so +-CELL_DIV
+// rows cover rs) around
 // its own cell, each clipped to the x-window of its own sphere: for a row at
 // y/z distance (dy, dz) from the atom the window is x +- sqrt(reach^2 - dy^2 -
 // dz^2), and only the cells overlapping it are read.  Candidates are gathered
@@ -619,7 +624,7 @@ __global__ __launch_bounds__(PL_WARPS * 32, 6) void pair_search_lane_kernel(Pair
             }
         };
 
-        for (int dz = -2; dz <= 2; ++dz) {
+        for (int dz = -CELL_DIV; dz <= CELL_DIV; ++dz) {
             // row z: unwrapped index for the geometry, wrapped index and image shift for the data
             int wz_i = cz + dz, kz = 0;
             while (wz_i < 0) { wz_i += A.nc.z; --kz; }
@@ -627,7 +632,7 @@ __global__ __launch_bounds__(PL_WARPS * 32, 6) void pair_search_lane_kernel(Pair
             const float zlo = (float)(cz + dz) * wz;
             const float ddz = fmaxf(fmaxf(zlo - p.z, p.z - (zlo + wz)), 0.f);
             const float qz = p0.z - (float)kz * A.L.z;
-            for (int dy = -2; dy <= 2; ++dy) {
+            for (int dy = -CELL_DIV; dy <= CELL_DIV; ++dy) {
                 int wy_i = cy + dy, ky = 0;
                 while (wy_i < 0) { wy_i += A.nc.y; --ky; }
                 while (wy_i >= A.nc.y) { wy_i -= A.nc.y; ++ky; }
