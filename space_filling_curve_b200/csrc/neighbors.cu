@@ -25,7 +25,7 @@ namespace tess {
 // ---------------------------------------------------------------- grid
 
 // Cells are at least rs / CELL_DIV wide, so +-CELL_DIV cell rows cover rs.
-constexpr int CELL_DIV = 2;
+constexpr int CELL_DIV = 3;
 
 struct Grid {
     int nc[3];
@@ -591,18 +591,8 @@ __global__ __launch_bounds__(PL_WARPS * 32, 6) void pair_search_lane_kernel(Pair
         p.z = fminf(fmaxf(p.z, 0.f), A.L.z);
         const float4 p0 = valid ? A.pos[i] : p;
         int* row = A.nbr + (size_t)(valid ? i : 0) * cap;
-        // the warp's cell rows: every row within reach of the tile's y/z extent
-        float loy = valid ? p.y : INFINITY, loz = valid ? p.z : INFINITY;
-        float hiy = valid ? p.y : -INFINITY, hiz = valid ? p.z : -INFINITY;
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) {
-            loy = fminf(loy, __shfl_xor_sync(FULL, loy, o));
-            loz = fminf(loz, __shfl_xor_sync(FULL, loz, o));
-            hiy = fmaxf(hiy, __shfl_xor_sync(FULL, hiy, o));
-            hiz = fmaxf(hiz, __shfl_xor_sync(FULL, hiz, o));
-        }
-        const int uy0 = (int)floorf((loy - A.reach) * A.inv_w.y), uy1 = (int)floorf((hiy + A.reach) * A.inv_w.y);
-        const int uz0 = (int)floorf((loz - A.reach) * A.inv_w.z), uz1 = (int)floorf((hiz + A.reach) * A.inv_w.z);
+        const int cy = cell_coord(p.y, A.inv_w.y, A.nc.y);
+        const int cz = cell_coord(p.z, A.inv_w.z, A.nc.z);
 
         int done = 0;
         unsigned wsa = buf_sa;
@@ -634,19 +624,19 @@ __global__ __launch_bounds__(PL_WARPS * 32, 6) void pair_search_lane_kernel(Pair
             }
         };
 
-        for (int uz = uz0; uz <= uz1; ++uz) {
+        for (int dz = -CELL_DIV; dz <= CELL_DIV; ++dz) {
             // row z: unwrapped index for the geometry, wrapped index and image shift for the data
-            int wz_i = uz, kz = 0;
+            int wz_i = cz + dz, kz = 0;
             while (wz_i < 0) { wz_i += A.nc.z; --kz; }
             while (wz_i >= A.nc.z) { wz_i -= A.nc.z; ++kz; }
-            const float zlo = (float)uz * wz;
+            const float zlo = (float)(cz + dz) * wz;
             const float ddz = fmaxf(fmaxf(zlo - p.z, p.z - (zlo + wz)), 0.f);
             const float qz = p0.z - (float)kz * A.L.z;
-            for (int uy = uy0; uy <= uy1; ++uy) {
-                int wy_i = uy, ky = 0;
+            for (int dy = -CELL_DIV; dy <= CELL_DIV; ++dy) {
+                int wy_i = cy + dy, ky = 0;
                 while (wy_i < 0) { wy_i += A.nc.y; --ky; }
                 while (wy_i >= A.nc.y) { wy_i -= A.nc.y; ++ky; }
-                const float ylo = (float)uy * wy;
+                const float ylo = (float)(cy + dy) * wy;
                 const float ddy = fmaxf(fmaxf(ylo - p.y, p.y - (ylo + wy)), 0.f);
                 const float ch2 = reach2 - ddy * ddy - ddz * ddz;
                 const float qy = p0.y - (float)ky * A.L.y;
