@@ -25,7 +25,7 @@ namespace tess {
 // ---------------------------------------------------------------- grid
 
 // Cells are at least rs / CELL_DIV wide, so +-CELL_DIV cell rows cover rs.
-constexpr int CELL_DIV = 3;
+constexpr int CELL_DIV = 2;
 
 struct Grid {
     int nc[3];
@@ -556,7 +556,7 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
 
 // ---------------------------------------------------------------- per-lane search
 
-// One warp per 32 consecutive atoms, but every lane walks its own stencil:
+// One warp per 32 atoms consecutive in cell order; every lane walks its own stencil:
 // the (2 CELL_DIV + 1)^2 cell rows (cells of width >= rs/CELL_DIV, so +-CELL_DIV
 // rows cover rs) around
 // its own cell, each clipped to the x-window of its own sphere: for a row at
@@ -582,14 +582,19 @@ __global__ __launch_bounds__(PL_WARPS * 32, 6) void pair_search_lane_kernel(Pair
 
     for (long long tile = (long long)blockIdx.x * PL_WARPS + warp; tile < ntiles;
          tile += (long long)gridDim.x * PL_WARPS) {
-        const int i = (int)(tile * 32) + lane;
-        const bool valid = i < A.n;
-        float4 p = valid ? A.pos[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        // lanes take 32 consecutive atoms in cell order (the binning's copy,
+        // atom index in w): they share a cell row, so their stencils coincide
+        // and their gathers fall on few lines
+        const int slot = (int)(tile * 32) + lane;
+        const bool valid = slot < A.n;
+        const float4 pc = valid ? A.pos_cell[slot] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const int i = valid ? __float_as_int(pc.w) : -1;
+        float4 p = pc;
         // finite coordinates for the window arithmetic (invalid input is flagged by the binning)
         p.x = fminf(fmaxf(p.x, 0.f), A.L.x);
         p.y = fminf(fmaxf(p.y, 0.f), A.L.y);
         p.z = fminf(fmaxf(p.z, 0.f), A.L.z);
-        const float4 p0 = valid ? A.pos[i] : p;
+        const float4 p0 = valid ? pc : p;
         int* row = A.nbr + (size_t)(valid ? i : 0) * cap;
         const int cy = cell_coord(p.y, A.inv_w.y, A.nc.y);
         const int cz = cell_coord(p.z, A.inv_w.z, A.nc.z);
