@@ -148,7 +148,7 @@ struct SortShared {
 };
 
 template <bool FINAL>
-__global__ __launch_bounds__(SORT_THREADS) void onesweep_pass(const unsigned long long* __restrict__ in,
+__global__ __launch_bounds__(SORT_THREADS, 3) void onesweep_pass(const unsigned long long* __restrict__ in,
                                                               unsigned long long* __restrict__ out, int n, int shift,
                                                               const unsigned* __restrict__ hist,
                                                               unsigned long long* states, unsigned* tile_counter,

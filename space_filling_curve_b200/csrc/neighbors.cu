@@ -66,7 +66,8 @@ __device__ __forceinline__ int cell_coord(float x, float inv_w, int nc) {
 // ---------------------------------------------------------------- binning
 
 __global__ void cell_count_kernel(const float4* __restrict__ pos, int n, int3 nc, float3 inv_w, float3 L,
-                                  int* __restrict__ cell_id, int* __restrict__ cnt, int32_t* status) {
+                                  int* __restrict__ cell_id, int* __restrict__ cell_rank, int* __restrict__ cnt,
+                                  int32_t* status) {
     bool bad = false;
     const int stride = gridDim.x * blockDim.x;
     for (int base = blockIdx.x * blockDim.x; base < n; base += stride) {
@@ -84,8 +85,14 @@ __global__ void cell_count_kernel(const float4* __restrict__ pos, int n, int3 nc
         }
         const unsigned act = __ballot_sync(FULL, valid);
         if (valid) {
+            // one atomic per group of lanes in the same cell; each lane keeps its
+            // slot among the cell's atoms (any order: cell_order fixes it)
             const unsigned peers = __match_any_sync(act, c);
-            if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&cnt[c], __popc(peers));
+            const int lane = threadIdx.x & 31, leader = __ffs(peers) - 1;
+            int b0 = 0;
+            if (lane == leader) b0 = atomicAdd(&cnt[c], __popc(peers));
+            b0 = __shfl_sync(peers, b0, leader);
+            cell_rank[i] = b0 + __popc(peers & lanemask_lt());
         }
     }
     if (__any_sync(FULL, bad) && (threadIdx.x & 31) == 0 && status) atomicOr(status, TESS_DEV_BAD_INPUT);
@@ -175,23 +182,11 @@ __global__ __launch_bounds__(SCAN_THREADS) void scan_apply_kernel(int* __restric
     if (b < m && b + SCAN_ITEMS >= m) cell_start[m] = run;   // the thread holding the last cell
 }
 
-__global__ void cell_scatter_kernel(const int* __restrict__ cell_id, int n, const int* __restrict__ cell_start,
-                                    int* __restrict__ cursor, int* __restrict__ slot_atom) {
+__global__ void cell_scatter_kernel(const int* __restrict__ cell_id, const int* __restrict__ cell_rank, int n,
+                                    const int* __restrict__ cell_start, int* __restrict__ slot_atom) {
     const int stride = gridDim.x * blockDim.x;
-    for (int base = blockIdx.x * blockDim.x; base < n; base += stride) {
-        const int i = base + threadIdx.x;
-        const bool valid = i < n;
-        const int c = valid ? cell_id[i] : -1;
-        const unsigned act = __ballot_sync(FULL, valid);
-        if (valid) {
-            const unsigned peers = __match_any_sync(act, c);
-            const int lane = threadIdx.x & 31, leader = __ffs(peers) - 1;
-            int b0 = 0;
-            if (lane == leader) b0 = atomicAdd(&cursor[c], __popc(peers));
-            b0 = __shfl_sync(peers, b0, leader);
-            slot_atom[cell_start[c] + b0 + __popc(peers & lanemask_lt())] = i;
-        }
-    }
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
+        slot_atom[cell_start[cell_id[i]] + cell_rank[i]] = i;
 }
 
 // Deterministic order inside each cell: the slot of atom i is the cell start
@@ -717,6 +712,7 @@ __global__ __launch_bounds__(PL_WARPS * 32, 6) void pair_search_lane_kernel(Pair
 
 struct NbrLayout {
     int* cell_id;
+    int* cell_rank;
     int* cnt;
     int* cell_start;
     int* sums;
@@ -731,6 +727,7 @@ static NbrLayout nbr_layout(void* ws, int n, const Grid& g) {
     NbrLayout L{};
     const long long m = g.ncell;
     L.cell_id = c.take<int>((size_t)n);
+    L.cell_rank = c.take<int>((size_t)n);
     L.cnt = c.take<int>((size_t)m);
     L.cell_start = c.take<int>((size_t)m + 1);
     L.sums = c.take<int>((size_t)((m + SCAN_TILE - 1) / SCAN_TILE) + 1);
@@ -778,11 +775,11 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
         StageScope sc(ST_CELLS, s);
         cudaMemsetAsync(L.cnt, 0, sizeof(int) * (size_t)m, s);
         const int blocks = (int)std::min<long long>(((long long)n + 255) / 256, (long long)sms * 16);
-        cell_count_kernel<<<blocks, 256, 0, s>>>(pos4, n, nc, inv_w, Lb, L.cell_id, L.cnt, overflow);
+        cell_count_kernel<<<blocks, 256, 0, s>>>(pos4, n, nc, inv_w, Lb, L.cell_id, L.cell_rank, L.cnt, overflow);
         scan_reduce_kernel<<<(unsigned)scan_tiles, SCAN_THREADS, 0, s>>>(L.cnt, m, L.sums);
         scan_sums_kernel<<<1, SCAN_THREADS, 0, s>>>(L.sums, scan_tiles);
         scan_apply_kernel<<<(unsigned)scan_tiles, SCAN_THREADS, 0, s>>>(L.cnt, m, L.sums, L.cell_start);
-        cell_scatter_kernel<<<blocks, 256, 0, s>>>(L.cell_id, n, L.cell_start, L.cnt, L.slot_atom);
+        cell_scatter_kernel<<<blocks, 256, 0, s>>>(L.cell_id, L.cell_rank, n, L.cell_start, L.slot_atom);
         cell_order_kernel<<<blocks, 256, 0, s>>>(L.slot_atom, n, L.cell_id, L.cell_start, pos4, L.pos_cell);
         count_launch(6);
     }
