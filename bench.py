@@ -123,7 +123,7 @@ def sum_over_ranks(value: float, world: int, device=None) -> float:
 class Step:
     """All device buffers of one replica and the step itself, through the C ABI."""
 
-    def __init__(self, s, device, pad_fill=True, tile_search=False):
+    def __init__(self, s, device, pad_fill=True, tile_search=False, curve="hilbert"):
         import torch
         import space_filling_curve_b200 as tess
         self.tess = tess
@@ -152,6 +152,7 @@ class Step:
         self.out = torch.empty((n, F), dtype=torch.float32, device=device)
         self.pad_fill = pad_fill
         self.tile_search = tile_search
+        self.sort_fn = tess.tess_hilbert_sort if curve == "hilbert" else tess.tess_morton_sort
         # the next frame of the trajectory, in the sorted order of frame 0
         t1 = next(iter(s.trajectory(1, condition=False)))[1]
         self.frame1 = torch.from_numpy(t1).to(device)
@@ -169,7 +170,7 @@ class Step:
         import torch
         st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
         s = self.s
-        c = tess.tess_hilbert_sort(P(self.pos3), self.n, s.box, 10, P(self.ws_sort), self.ws_sort.numel(),
+        c = self.sort_fn(P(self.pos3), self.n, s.box, 10, P(self.ws_sort), self.ws_sort.numel(),
                                    P(self.perm), P(self.keys), P(self.pos_sorted), P(self.status), st)
         assert c == 0, c
         c = tess.tess_build_neighbors(P(self.pos_sorted), self.n, s.box, s.rc, s.skin, s.cap,
@@ -209,7 +210,7 @@ def run_cuda(args, world, rank, local):
     import synth
     import space_filling_curve_b200 as tess
     s = synth.system(args.config)
-    step = Step(s, dev, pad_fill=not args.no_pad_fill, tile_search=args.tile_search)
+    step = Step(s, dev, pad_fill=not args.no_pad_fill, tile_search=args.tile_search, curve=args.curve)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
         flush.zero_()
@@ -243,6 +244,34 @@ def run_cuda(args, world, rank, local):
     ms_max = max_over_ranks(ms, world, dev)
     n_total = sum_over_ranks(float(s.n * args.steps), world, dev)
     value = n_total / (ms_max / 1e3)
+
+    graph = None
+    if args.graph:
+        # the same step captured once as a CUDA graph and replayed
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            step.run()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g):
+            step.run()
+        for _ in range(args.warmup):
+            flush.zero_()
+            g.replay()
+        gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        torch.cuda.synchronize()
+        for k in range(args.steps):
+            flush.zero_()
+            gev[k][0].record()
+            g.replay()
+            gev[k][1].record()
+        torch.cuda.synchronize()
+        gms = max_over_ranks(sum(a.elapsed_time(b) for a, b in gev), world, dev)
+        graph = {"ms_per_step": gms / args.steps, "eager_ms_per_step": ms_max / args.steps,
+                 "speedup": ms_max / gms}
+        del g
 
     # e2e: through the C ABI with host buffers (pinned), copies inside the timed region
     host_pos = torch.from_numpy(s.pos).pin_memory()
@@ -296,6 +325,7 @@ def run_cuda(args, world, rank, local):
                 "atoms": s.n,
                 "pad_fill": not args.no_pad_fill,
                 "pair_search": "tile" if args.tile_search else "per-lane",
+                "curve": args.curve,
                 "l2": "flushed between timed steps (256 MB write); each step also moves ~9 GB",
                 "parallelism": "replicas (no collective in the data path)",
                 "mean_neighbors": mean_count,
@@ -321,6 +351,7 @@ def run_cuda(args, world, rank, local):
             "e2e": {"value": e2e_val, "unit": "atoms/s", "steps": e2e_steps, "h2d_bytes_per_step": s.n * 12,
                     "d2h_bytes_per_step": s.n * 8 + 8},
             "gpu_launches": launches,
+            "graph": graph,
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -427,7 +458,10 @@ def main(argv=None):
     ap.add_argument("--config", type=int, default=WORKLOAD_CFG)
     ap.add_argument("--no-pad-fill", action="store_true")
     ap.add_argument("--tile-search", action="store_true", help="use the warp-shared tile pair search")
+    ap.add_argument("--curve", choices=["hilbert", "morton"], default="hilbert",
+                    help="space-filling curve of the sort (morton: the comparison curve)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true", help="also time the step captured as one CUDA graph")
     args = ap.parse_args(argv)
     world, rank, local = _dist_setup(args)
     if args.impl == "reference":

@@ -58,6 +58,10 @@ def lib():
         L.oracle_hilbert_index.argtypes = [ctypes.c_uint32] * 3 + [i32]
         L.oracle_hilbert_index.restype = ctypes.c_uint32
         L.oracle_hilbert_index_many.argtypes = [P, i64, i32, P]
+        L.oracle_morton_index.argtypes = [ctypes.c_uint32] * 3 + [i32]
+        L.oracle_morton_index.restype = ctypes.c_uint32
+        L.oracle_morton_index_many.argtypes = [P, i64, i32, P]
+        L.oracle_morton_sort.argtypes = [P, i32, i64, P, i32, P, P]
         L.oracle_hilbert_keys.argtypes = [P, i32, i64, P, i32, P]
         L.oracle_hilbert_sort.argtypes = [P, i32, i64, P, i32, P, P]
         for name in ("oracle_neighbors_brute", "oracle_neighbors_cells"):
@@ -118,6 +122,29 @@ def hilbert_index_grid(q: np.ndarray, bits: int) -> np.ndarray:
     out = np.empty(len(q), dtype=np.uint32)
     lib().oracle_hilbert_index_many(_ptr(q), len(q), int(bits), _ptr(out))
     return out
+
+
+def morton_index(q0: int, q1: int, q2: int, bits: int) -> int:
+    """Morton (Z-order) index of one grid point."""
+    return int(lib().oracle_morton_index(int(q0), int(q1), int(q2), int(bits)))
+
+
+def morton_index_grid(q: np.ndarray, bits: int) -> np.ndarray:
+    q = np.ascontiguousarray(q, dtype=np.uint32).reshape(-1, 3)
+    out = np.empty(len(q), dtype=np.uint32)
+    lib().oracle_morton_index_many(_ptr(q), len(q), int(bits), _ptr(out))
+    return out
+
+
+def morton_sort(pos, box, bits: int = 10):
+    """(perm, keys_sorted) along the Morton curve, ties by input index."""
+    pos, stride = _pos(pos)
+    b = _box(box)
+    n = len(pos)
+    perm = np.empty(n, dtype=np.int32)
+    keys = np.empty(n, dtype=np.uint32)
+    lib().oracle_morton_sort(_ptr(pos), stride, n, _ptr(b), int(bits), _ptr(perm), _ptr(keys))
+    return perm, keys
 
 
 def hilbert_keys(pos, box, bits: int = 10) -> np.ndarray:

@@ -23,6 +23,7 @@ __all__ = [
     "TessError", "lib", "library_path", "Box",
     "tess_status_string", "tess_version", "tess_kernel_launch_count",
     "tess_hilbert_sort_workspace", "tess_hilbert_sort", "tess_hilbert_sort_static", "HILBERT_SORT_STATIC_MAX_N",
+    "tess_morton_sort", "morton_sort",
     "tess_build_neighbors_workspace", "tess_build_neighbors",
     "tess_skin_check", "tess_edge_aggregate", "tess_stage_timing", "tess_stage_times",
     "hilbert_sort", "build_neighbors", "skin_check", "edge_aggregate",
@@ -76,6 +77,8 @@ def lib() -> ctypes.CDLL:
     L.tess_hilbert_sort_workspace.restype = sz
     L.tess_hilbert_sort.argtypes = [P, i32, Box, i32, P, sz, P, P, P, P, P]
     L.tess_hilbert_sort.restype = i32
+    L.tess_morton_sort.argtypes = [P, i32, Box, i32, P, sz, P, P, P, P, P]
+    L.tess_morton_sort.restype = i32
     L.tess_hilbert_sort_static.argtypes = [P, i32, Box, i32, P, P, P, P, P]
     L.tess_hilbert_sort_static.restype = i32
     L.tess_build_neighbors_workspace.argtypes = [i32, Box, f32, f32]
@@ -122,6 +125,11 @@ def tess_hilbert_sort_workspace(n: int) -> int:
 def tess_hilbert_sort(pos, n, box, bits, ws, ws_bytes, perm, keys_sorted, pos_sorted, dev_status, stream) -> int:
     return int(lib().tess_hilbert_sort(pos, n, _box(box), bits, ws, ws_bytes, perm, keys_sorted, pos_sorted,
                                        dev_status, stream))
+
+
+def tess_morton_sort(pos, n, box, bits, ws, ws_bytes, perm, keys_sorted, pos_sorted, dev_status, stream) -> int:
+    return int(lib().tess_morton_sort(pos, n, _box(box), bits, ws, ws_bytes, perm, keys_sorted, pos_sorted,
+                                      dev_status, stream))
 
 
 def tess_hilbert_sort_static(pos, n, box, bits, perm, keys_sorted, pos_sorted, dev_status, stream) -> int:
@@ -207,7 +215,7 @@ def _workspace(nbytes, device, ws=None):
 
 
 def hilbert_sort(pos, box, bits: int = 10, *, ws=None, perm=None, keys_sorted=None, pos_sorted=None,
-                 dev_status=None, want_keys: bool = True, want_pos: bool = True, stream=None):
+                 dev_status=None, want_keys: bool = True, want_pos: bool = True, stream=None, curve: str = "hilbert"):
     """Order atoms along the 3-D Hilbert curve.  ``pos``: float32 [n, 3]
     CUDA tensor.  Returns (perm int32 [n], keys uint32->int32 view [n] or
     None, pos_sorted float32 [n, 4] or None, dev_status int32 [1])."""
@@ -222,10 +230,16 @@ def hilbert_sort(pos, box, bits: int = 10, *, ws=None, perm=None, keys_sorted=No
     if want_pos and pos_sorted is None:
         pos_sorted = torch.empty((n, 4), dtype=torch.float32, device=dev)
     dev_status = torch.empty(1, dtype=torch.int32, device=dev) if dev_status is None else dev_status
-    code = tess_hilbert_sort(_ptr(pos), n, box, bits, _ptr(ws), ws.numel() * ws.element_size(), _ptr(perm),
-                             _ptr(keys_sorted), _ptr(pos_sorted), _ptr(dev_status), _stream(stream))
-    _check("tess_hilbert_sort", code)
+    fn = tess_hilbert_sort if curve == "hilbert" else tess_morton_sort
+    code = fn(_ptr(pos), n, box, bits, _ptr(ws), ws.numel() * ws.element_size(), _ptr(perm), _ptr(keys_sorted),
+              _ptr(pos_sorted), _ptr(dev_status), _stream(stream))
+    _check(fn.__name__, code)
     return perm, keys_sorted, pos_sorted, dev_status
+
+
+def morton_sort(pos, box, bits: int = 10, **kw):
+    """Order atoms along the Morton (Z-order) curve; same outputs as hilbert_sort."""
+    return hilbert_sort(pos, box, bits, curve="morton", **kw)
 
 
 def build_neighbors(pos4, box, rc: float, skin: float, max_neighbors: int, *, pad_fill: bool = True,

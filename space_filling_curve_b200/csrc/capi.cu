@@ -11,6 +11,8 @@ std::atomic<long long> g_launches{0};
 size_t hilbert_sort_workspace(int n);
 tess_status hilbert_sort(const float* pos, int n, tess_box box, int bits, void* ws, size_t ws_bytes, int32_t* perm,
                          uint32_t* keys_sorted, float* pos_sorted, int32_t* dev_status, cudaStream_t s);
+tess_status morton_sort(const float* pos, int n, tess_box box, int bits, void* ws, size_t ws_bytes, int32_t* perm,
+                        uint32_t* keys_sorted, float* pos_sorted, int32_t* dev_status, cudaStream_t s);
 size_t build_neighbors_workspace(int n, tess_box box, float rc, float skin);
 tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, float skin, int cap, int flags,
                             void* ws, size_t ws_bytes, int32_t* nbr, int32_t* counts, int32_t* overflow,
@@ -85,6 +87,13 @@ tess_status tess_hilbert_sort(const float* pos, int n, tess_box box, int bits, v
                               tess_stream_t stream) {
     return hilbert_sort(pos, n, box, bits, ws, ws_bytes, perm, keys_sorted, pos_sorted, dev_status,
                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+tess_status tess_morton_sort(const float* pos, int n, tess_box box, int bits, void* ws, size_t ws_bytes,
+                             int32_t* perm, uint32_t* keys_sorted, float* pos_sorted, int32_t* dev_status,
+                             tess_stream_t stream) {
+    return morton_sort(pos, n, box, bits, ws, ws_bytes, perm, keys_sorted, pos_sorted, dev_status,
+                       reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t tess_build_neighbors_workspace(int n, tess_box box, float rc, float skin) {

@@ -75,6 +75,12 @@ constexpr int KEYS_THREADS = 256;
 constexpr int RADIX = 256;
 constexpr int MAX_PASSES = 4;
 
+// Morton (Z-order) index: the three words interleaved with no transform.
+__device__ __forceinline__ uint32_t morton_key(uint32_t x, uint32_t y, uint32_t z) {
+    return (spread3(x) << 2) | (spread3(y) << 1) | spread3(z);
+}
+
+template <int CURVE>   // 0 Hilbert, 1 Morton
 __global__ __launch_bounds__(KEYS_THREADS) void keys_kernel(const float* __restrict__ pos, int n, float3 scale,
                                                             float3 L, int bits, int npass,
                                                             unsigned long long* __restrict__ elems,
@@ -87,8 +93,8 @@ __global__ __launch_bounds__(KEYS_THREADS) void keys_kernel(const float* __restr
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
         const float x = pos[3 * (size_t)i], y = pos[3 * (size_t)i + 1], z = pos[3 * (size_t)i + 2];
         bad |= !(x >= 0.0f && x < L.x && y >= 0.0f && y < L.y && z >= 0.0f && z < L.z);
-        const uint32_t key = hilbert_key(quantize(x, scale.x, top), quantize(y, scale.y, top),
-                                         quantize(z, scale.z, top), bits);
+        const uint32_t qx = quantize(x, scale.x, top), qy = quantize(y, scale.y, top), qz = quantize(z, scale.z, top);
+        const uint32_t key = CURVE == 0 ? hilbert_key(qx, qy, qz, bits) : morton_key(qx, qy, qz);
         elems[i] = ((unsigned long long)key << 32) | (unsigned)i;
         for (int p = 0; p < npass; ++p) atomicAdd(&sh[p][(key >> (8 * p)) & 0xffu], 1u);
     }
@@ -302,8 +308,8 @@ size_t hilbert_sort_workspace(int n) {
     return sort_layout(nullptr, n).total;
 }
 
-tess_status hilbert_sort(const float* pos, int n, tess_box box, int bits, void* ws, size_t ws_bytes, int32_t* perm,
-                         uint32_t* keys_sorted, float* pos_sorted, int32_t* dev_status, cudaStream_t s) {
+tess_status sfc_sort(const float* pos, int n, tess_box box, int bits, int curve, void* ws, size_t ws_bytes,
+                     int32_t* perm, uint32_t* keys_sorted, float* pos_sorted, int32_t* dev_status, cudaStream_t s) {
     if (n <= 0 || !pos || !perm || !ws || bits < 1 || bits > 10) return TESS_ERR_INVALID_ARG;
     if (!finite_pos(box.lx) || !finite_pos(box.ly) || !finite_pos(box.lz)) return TESS_ERR_INVALID_ARG;
     if (pos_sorted && !aligned(pos_sorted, 16)) return TESS_ERR_INVALID_ARG;
@@ -324,8 +330,12 @@ tess_status hilbert_sort(const float* pos, int n, tess_box box, int bits, void* 
     {
         StageScope sc(ST_KEYS, s);
         const int blocks = (int)std::min<long long>(((long long)n + KEYS_THREADS - 1) / KEYS_THREADS, (long long)sms * 8);
-        keys_kernel<<<blocks, KEYS_THREADS, 0, s>>>(pos, n, scale, make_float3(box.lx, box.ly, box.lz), bits, npass,
-                                                    L.a, L.hist, status);
+        if (curve == 0)
+            keys_kernel<0><<<blocks, KEYS_THREADS, 0, s>>>(pos, n, scale, make_float3(box.lx, box.ly, box.lz), bits,
+                                                           npass, L.a, L.hist, status);
+        else
+            keys_kernel<1><<<blocks, KEYS_THREADS, 0, s>>>(pos, n, scale, make_float3(box.lx, box.ly, box.lz), bits,
+                                                           npass, L.a, L.hist, status);
         count_launch();
     }
     {
@@ -351,6 +361,16 @@ tess_status hilbert_sort(const float* pos, int n, tess_box box, int bits, void* 
         }
     }
     return launch_status();
+}
+
+tess_status hilbert_sort(const float* pos, int n, tess_box box, int bits, void* ws, size_t ws_bytes, int32_t* perm,
+                         uint32_t* keys_sorted, float* pos_sorted, int32_t* dev_status, cudaStream_t s) {
+    return sfc_sort(pos, n, box, bits, 0, ws, ws_bytes, perm, keys_sorted, pos_sorted, dev_status, s);
+}
+
+tess_status morton_sort(const float* pos, int n, tess_box box, int bits, void* ws, size_t ws_bytes, int32_t* perm,
+                        uint32_t* keys_sorted, float* pos_sorted, int32_t* dev_status, cudaStream_t s) {
+    return sfc_sort(pos, n, box, bits, 1, ws, ws_bytes, perm, keys_sorted, pos_sorted, dev_status, s);
 }
 
 }  // namespace tess

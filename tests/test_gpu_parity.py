@@ -358,3 +358,40 @@ def test_edge_aggregate_dense_rows(F):
     ref = oracle.edge_aggregate(p, (L, L, L), 5.0, nbr_d.cpu().numpy(), cnt_d.cpu().numpy(), feat)
     err, _ = agg_error(out, ref)
     assert err <= AGG_TOL
+
+
+# ------------------------------------------------------------------ Morton order (comparison curve)
+
+
+@pytest.mark.parametrize("bits", [1, 3, 8, 10])
+@pytest.mark.parametrize("n", [1, 33, 4097, 20000])
+def test_morton_sort_against_oracle(n, bits):
+    tess = _tess()
+    rng = np.random.default_rng(n + bits)
+    box = (31.0, 45.0, 60.0)
+    pos = (rng.uniform(0, 1, (n, 3)) * np.array(box)).astype(np.float32)
+    perm, keys, ps, st = tess.morton_sort(_dev(pos), box, bits)
+    torch_cuda().cuda.synchronize()
+    operm, okeys = oracle.morton_sort(pos, box, bits)
+    assert int(st.item()) == 0
+    assert np.array_equal(keys.cpu().numpy().view(np.uint32), okeys)
+    assert np.array_equal(perm.cpu().numpy(), operm)
+    assert np.array_equal(ps.cpu().numpy()[:, :3], pos[operm])
+
+
+def test_morton_order_lists_match_hilbert_order_lists():
+    # the list is the same set of pairs in any index order: relabel and compare
+    tess = _tess()
+    s = synth.system(2)
+    hp, _ = oracle.hilbert_sort(s.pos, s.box, 10)
+    mp, _ = oracle.morton_sort(s.pos, s.box, 10)
+    nh, ch, _ = tess.build_neighbors(_dev(s.pos4()[hp]), s.box, s.rc, s.skin, s.cap)
+    nm, cm, _ = tess.build_neighbors(_dev(s.pos4()[mp]), s.box, s.rc, s.skin, s.cap)
+    nh, ch, nm, cm = nh.cpu().numpy(), ch.cpu().numpy(), nm.cpu().numpy(), cm.cpu().numpy()
+    # original index of each row and of each entry
+    rows_h = {int(hp[i]): set(hp[nh[i, :ch[i]]].tolist()) for i in range(0, s.n, 37)}
+    inv_m = np.empty(s.n, np.int64)
+    inv_m[mp] = np.arange(s.n)
+    for a, ref in rows_h.items():
+        k = inv_m[a]
+        assert set(mp[nm[k, :cm[k]]].tolist()) == ref

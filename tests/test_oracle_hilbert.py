@@ -116,3 +116,44 @@ def test_sort_is_stable_total_order():
     assert np.all(np.diff(perm)[same] > 0)                  # ties by ascending index
     # and agrees with numpy's stable sort of the same keys
     assert np.array_equal(perm, np.argsort(k_all, kind="stable"))
+
+
+# ---------------------------------------------------------------- Morton (comparison curve)
+
+
+def test_morton_hand_values():
+    # the interleave read MSB-first, x's bit first: (1,0,0) at 1 bit is 0b100
+    assert oracle.morton_index(1, 0, 0, 1) == 4
+    assert oracle.morton_index(0, 1, 1, 1) == 3
+    assert oracle.morton_index(3, 0, 0, 2) == 0b100100
+    assert oracle.morton_index(0, 0, 3, 2) == 0b001001
+    assert oracle.morton_index(1023, 1023, 1023, 10) == (1 << 30) - 1
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5])
+def test_morton_bijection_nesting_and_jumps(bits):
+    q = _grid(bits)
+    keys = oracle.morton_index_grid(q, bits).astype(np.int64)
+    assert len(np.unique(keys)) == len(keys) == 1 << (3 * bits)
+    for k in range(1, bits):
+        cube = (q >> k).astype(np.int64)
+        cid = (cube[:, 0] << 20) | (cube[:, 1] << 10) | cube[:, 2]
+        pairs = np.unique(np.stack([cid, keys >> (3 * k)], axis=1), axis=0)
+        assert len(pairs) == len(np.unique(cid))
+    # unlike the Hilbert curve, the Z-order curve jumps: consecutive keys can
+    # be far apart (from the top of one octant to the next)
+    inv = np.empty((1 << (3 * bits), 3), dtype=np.int64)
+    inv[keys] = q
+    steps = np.abs(np.diff(inv, axis=0)).sum(axis=1)
+    if bits >= 2:
+        assert steps.max() > 1
+
+
+def test_morton_sort_is_stable():
+    rng = np.random.default_rng(5)
+    pos = rng.uniform(0, 20, (4000, 3)).astype(np.float32)
+    perm, keys = oracle.morton_sort(pos, (20, 20, 20), bits=2)
+    q = np.stack([np.array([oracle.quantize(x, 20.0, 2) for x in pos[:, d]]) for d in range(3)], 1)
+    k_all = oracle.morton_index_grid(q, 2)
+    assert np.array_equal(perm, np.argsort(k_all, kind="stable"))
+    assert np.array_equal(keys, k_all[perm])
