@@ -624,6 +624,9 @@ __global__ __launch_bounds__(PL_WARPS * 32, 6) void pair_search_lane_kernel(Pair
             }
         };
 
+        float4 c[PL_CHUNK];
+#pragma unroll
+        for (int u = 0; u < PL_CHUNK; ++u) c[u] = make_float4(0.f, 0.f, 0.f, 0.f);
         for (int dz = -CELL_DIV; dz <= CELL_DIV; ++dz) {
             // row z: unwrapped index for the geometry, wrapped index and image shift for the data
             int wz_i = cz + dz, kz = 0;
@@ -669,22 +672,20 @@ __global__ __launch_bounds__(PL_WARPS * 32, 6) void pair_search_lane_kernel(Pair
                     const int maxlen = (int)__reduce_max_sync(FULL, (unsigned)len[pc]);
                     for (int k0 = 0; k0 < maxlen; k0 += PL_CHUNK) {
                         if (__any_sync(FULL, (int)((wsa - buf_sa) >> 7) > PS_BUF - PL_CHUNK)) drain(false);
-                        // slots past this lane's window read a NaN dummy that is
-                        // never accepted, so the test below needs no branch
-                        float4 c[PL_CHUNK];
+                        // slots past this lane's window keep stale data; their
+                        // index becomes the atom's own, which the test rejects, so
+                        // the test below needs no branch
                         const float4* src = A.pos_cell + beg[pc] + k0;
 #pragma unroll
-                        for (int u = 0; u < PL_CHUNK; ++u) {
-                            c[u] = make_float4(nanf_, nanf_, nanf_, 0.f);
+                        for (int u = 0; u < PL_CHUNK; ++u)
                             if (k0 + u < len[pc]) c[u] = src[u];
-                        }
 #pragma unroll
                         for (int u = 0; u < PL_CHUNK; ++u) {
                             const float dx = c[u].x - qx[pc];
                             const float ddy2 = c[u].y - qy;
                             const float ddz2 = c[u].z - qz;
                             const float r2 = fmaf(ddz2, ddz2, fmaf(ddy2, ddy2, dx * dx));
-                            append_if(wsa, r2, A.rs2, __float_as_int(c[u].w), i);
+                            append_if(wsa, r2, A.rs2, (k0 + u < len[pc]) ? __float_as_int(c[u].w) : i, i);
                         }
                     }
                 }
