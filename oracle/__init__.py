@@ -78,6 +78,9 @@ def lib():
         L.oracle_cutoff.argtypes = [ctypes.c_double, ctypes.c_double]
         L.oracle_cutoff.restype = ctypes.c_double
         L.oracle_edge_aggregate.argtypes = [P, i32, i64, P, f32, P, P, i32, P, i32, P, P, P, P, P]
+        L.oracle_cutoff_deriv.argtypes = [ctypes.c_double, ctypes.c_double]
+        L.oracle_cutoff_deriv.restype = ctypes.c_double
+        L.oracle_edge_backward.argtypes = [P, i32, i64, P, f32, P, P, i32, P, P, i32, P, P]
         _lib = L
     return _lib
 
@@ -295,3 +298,26 @@ def rebuild(pos3, box, rc, skin, cap, bits: int = 10, method: str = "cells"):
     fn = neighbors_cells if method == "cells" else neighbors_brute
     nbr, counts, ov = fn(ps, box, rc, skin, cap)
     return perm, keys, ps, nbr, counts, ov
+
+
+def cutoff_deriv(r: float, rc: float) -> float:
+    """d f_c / d r."""
+    return float(lib().oracle_cutoff_deriv(float(r), float(rc)))
+
+
+def edge_backward(pos, box, rc, nbr, counts, feat, grad_out):
+    """VJP of the aggregation: (grad_feat [n, F], grad_pos [n, 3]) in fp64."""
+    pos, stride = _pos(pos)
+    b = _box(box)
+    nbr = np.ascontiguousarray(nbr, dtype=np.int32)
+    counts = np.ascontiguousarray(counts, dtype=np.int32)
+    feat = np.ascontiguousarray(feat, dtype=np.float32)
+    g = np.ascontiguousarray(grad_out, dtype=np.float32)
+    n, cap = nbr.shape
+    F = feat.shape[1]
+    gf = np.empty((n, F), dtype=np.float64)
+    gp = np.empty((n, 3), dtype=np.float64)
+    lib().oracle_edge_backward(_ptr(pos), stride, n, _ptr(b), float(rc), _ptr(nbr), _ptr(counts), int(cap),
+                               _ptr(feat), _ptr(g), int(F), _ptr(gf), _ptr(gp))
+    return gf, gp
+

@@ -575,3 +575,66 @@ void oracle_edge_aggregate(const float* pos, int stride, int64_t n, const float*
         }
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Backward of C5 (force path)                                               */
+/* ------------------------------------------------------------------------ */
+
+/* d f_c / d r of the Behler cutoff: -(pi / (2 rc)) sin(pi r / rc) for r < rc. */
+double oracle_cutoff_deriv(double r, double rc)
+{
+    if (r < rc) return -0.5 * ORACLE_PI / rc * sin(ORACLE_PI * r / rc);
+    return 0.0;
+}
+
+/*
+ * Vector-Jacobian product of out_i = sum_{j in row i} f_c(|r_ij|) h_j with
+ * respect to the features and the positions, given g = dL/d out ([n, F]).
+ * "force backpropagation repeats the exchange" (Tessera, abstract); the
+ * review of arXiv 2505.06711 describes the same VJP over one-hop edges.
+ * Plain chain rule over the listed edges, accumulated serially in fp64:
+ *   grad_feat[j] += f_c(r_ij) g_i                       for each listed (i, j)
+ *   s = f_c'(r_ij) (g_i . h_j);  grad_pos[i] -= s u_ij;  grad_pos[j] += s u_ij
+ * with u_ij = r_ij / |r_ij| (0 when |r_ij| = 0).  grad_feat [n, F] and
+ * grad_pos [n, 3] are overwritten.
+ */
+void oracle_edge_backward(const float* pos, int stride, int64_t n, const float* L, float rc,
+                          const int32_t* nbr, const int32_t* counts, int cap, const float* feat,
+                          const float* grad_out, int F, double* grad_feat, double* grad_pos)
+{
+    const double Ld[3] = {(double)L[0], (double)L[1], (double)L[2]};
+    for (int64_t k = 0; k < n * (int64_t)F; ++k) grad_feat[k] = 0.0;
+    for (int64_t k = 0; k < n * 3; ++k) grad_pos[k] = 0.0;
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t m = counts[i] < cap ? counts[i] : cap;
+        for (int64_t s = 0; s < m; ++s) {
+            int32_t j = nbr[i * (int64_t)cap + s];
+            if (j < 0 || j >= n) continue;
+            const float* pi = pos + i * stride;
+            const float* pj = pos + (int64_t)j * stride;
+            double d[3];
+            d[0] = min_image((double)pj[0] - (double)pi[0], Ld[0]);
+            d[1] = min_image((double)pj[1] - (double)pi[1], Ld[1]);
+            d[2] = min_image((double)pj[2] - (double)pi[2], Ld[2]);
+            double r = sqrt(d[0] * d[0] + d[1] * d[1] + d[2] * d[2]);
+            double fc = oracle_cutoff(r, (double)rc);
+            double dfc = oracle_cutoff_deriv(r, (double)rc);
+            if (fc == 0.0 && dfc == 0.0) continue;
+            const float* gi = grad_out + i * (int64_t)F;
+            const float* hj = feat + (int64_t)j * F;
+            double dot = 0.0;
+            for (int f = 0; f < F; ++f) {
+                grad_feat[(int64_t)j * F + f] += fc * (double)gi[f];
+                dot += (double)gi[f] * (double)hj[f];
+            }
+            if (r > 0.0) {
+                double sc = dfc * dot / r;
+                for (int a = 0; a < 3; ++a) {
+                    grad_pos[i * 3 + a] -= sc * d[a];
+                    grad_pos[(int64_t)j * 3 + a] += sc * d[a];
+                }
+            }
+        }
+    }
+}
+
