@@ -245,6 +245,31 @@ def run_cuda(args, world, rank, local):
     n_total = sum_over_ranks(float(s.n * args.steps), world, dev)
     value = n_total / (ms_max / 1e3)
 
+    backward = None
+    if args.backward:
+        # the aggregation's backward (force path) on the same list, timed alone
+        gout = torch.randn((s.n, s.F), generator=torch.Generator(device=dev).manual_seed(2), device=dev)
+        gfeat = torch.empty_like(gout)
+        gpos = torch.empty((s.n, 3), dtype=torch.float32, device=dev)
+        import ctypes
+        P = lambda t: ctypes.c_void_p(t.data_ptr())
+        stc = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        call = lambda: tess.tess_edge_aggregate_backward(P(step.pos_sorted), s.n, s.box, s.rc, P(step.nbr),
+                                                         P(step.counts), s.cap, P(step.feat), P(gout), s.F,
+                                                         P(gfeat), P(gpos), stc)
+        for _ in range(args.warmup):
+            assert call() == 0
+        bev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for k in range(args.steps):
+            flush.zero_()
+            bev[k][0].record()
+            call()
+            bev[k][1].record()
+        torch.cuda.synchronize()
+        bms = sum(a.elapsed_time(b) for a, b in bev) / args.steps
+        bbytes = s.n * (3 * 4 * s.F + 16 + 4 * mean_count + 4 + 12)
+        backward = {"ms": bms, "algorithmic_bytes": bbytes, "achieved_gbs": bbytes / (bms / 1e3) / 1e9}
+
     graph = None
     if args.graph:
         # the same step captured once as a CUDA graph and replayed
@@ -352,6 +377,7 @@ def run_cuda(args, world, rank, local):
                     "d2h_bytes_per_step": s.n * 8 + 8},
             "gpu_launches": launches,
             "graph": graph,
+            "backward": backward,
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -462,6 +488,7 @@ def main(argv=None):
                     help="space-filling curve of the sort (morton: the comparison curve)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph", action="store_true", help="also time the step captured as one CUDA graph")
+    ap.add_argument("--backward", action="store_true", help="also time the aggregation's backward on the same list")
     args = ap.parse_args(argv)
     world, rank, local = _dist_setup(args)
     if args.impl == "reference":

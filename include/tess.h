@@ -225,11 +225,38 @@ tess_status tess_edge_aggregate(const float* pos, int n, tess_box box, float rc,
                                 tess_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Backward of the aggregation -- "force backpropagation repeats the
+ * exchange" (Tessera, abstract); the review of arXiv 2505.06711 describes
+ * the same vector-Jacobian product over one-hop edges.
+ *
+ * Given g = dL/d out ([n, F]), writes
+ *   grad_feat[i] = dL/d feat[i] = sum_{j in row i} f_c(r_ij) g_j
+ *   grad_pos[i]  = dL/d r_i     = -sum_{j in row i} f_c'(r_ij) (g_i . h_j + g_j . h_i) r_ij / |r_ij|
+ * (f_c' = d f_c / d r; edges with r >= rc contribute nothing).  These are
+ * the chain rule of tess_edge_aggregate for a FULL SYMMETRIC list without
+ * overflow (j in row i exactly when i in row j), which is what
+ * tess_build_neighbors writes when its overflow word is 0; the symmetry
+ * lets every row gather its own gradients.  The forces of a model layer are
+ * -grad_pos.
+ *
+ *   feat, grad_out  [n, F] float, 16-byte aligned, F = 4 * 2^k (4 ... 256)
+ *   grad_feat       [n, F] float out, 16-byte aligned
+ *   grad_pos        [n, 3] float out
+ *   max_neighbors   <= 512
+ * Errors: INVALID_ARG (as tess_edge_aggregate, plus F or cap outside the
+ * supported set, misaligned feature arrays), BOX_TOO_SMALL, CUDA.
+ * ------------------------------------------------------------------------- */
+tess_status tess_edge_aggregate_backward(const float* pos, int n, tess_box box, float rc,
+                                         const int32_t* nbr, const int32_t* counts, int max_neighbors,
+                                         const float* feat, const float* grad_out, int F,
+                                         float* grad_feat, float* grad_pos, tess_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Stage timing (diagnostic).  When enabled, each entry point records CUDA
  * events on its stream around its kernels; tess_stage_times adds the elapsed
  * times of all recorded calls per stage (this synchronises on the events)
- * and clears them.  Stages: 0 hilbert keys, 1 key sort, 2 cell binning,
- * 3 pair search, 4 skin check, 5 edge aggregate.  Returns the number of
+ * and clears them.  Stages: 0 space-filling-curve keys, 1 key sort, 2 cell
+ * binning, 3 pair search, 4 skin check, 5 edge aggregate, 6 aggregate backward.  Returns the number of
  * stages written (<= max_stages).  ms_out[k] = total milliseconds,
  * calls_out[k] (nullable) = number of timed calls.
  * ------------------------------------------------------------------------- */

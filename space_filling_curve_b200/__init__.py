@@ -27,6 +27,7 @@ __all__ = [
     "tess_build_neighbors_workspace", "tess_build_neighbors",
     "tess_skin_check", "tess_edge_aggregate", "tess_stage_timing", "tess_stage_times",
     "hilbert_sort", "build_neighbors", "skin_check", "edge_aggregate",
+    "tess_edge_aggregate_backward", "edge_aggregate_backward",
     "TESS_DEV_OVERFLOW", "TESS_DEV_BAD_INPUT", "TESS_DEV_TIMEOUT", "TESS_NO_PAD_FILL", "TESS_TILE_SEARCH", "STAGES",
 ]
 
@@ -38,7 +39,7 @@ TESS_DEV_BAD_INPUT = 2
 TESS_DEV_TIMEOUT = 4
 TESS_NO_PAD_FILL = 1
 TESS_TILE_SEARCH = 2
-STAGES = ("hilbert_keys", "key_sort", "cell_binning", "pair_search", "skin_check", "edge_aggregate")
+STAGES = ("hilbert_keys", "key_sort", "cell_binning", "pair_search", "skin_check", "edge_aggregate", "edge_backward")
 _STATUS = {0: "ok", 1: "invalid argument", 2: "box too small", 3: "workspace too small", 4: "CUDA launch error",
            5: "n above the static scratch capacity"}
 HILBERT_SORT_STATIC_MAX_N = 1 << 20
@@ -89,6 +90,8 @@ def lib() -> ctypes.CDLL:
     L.tess_skin_check.restype = i32
     L.tess_edge_aggregate.argtypes = [P, i32, Box, f32, P, P, i32, P, i32, P, P, P, P, P]
     L.tess_edge_aggregate.restype = i32
+    L.tess_edge_aggregate_backward.argtypes = [P, i32, Box, f32, P, P, i32, P, P, i32, P, P, P]
+    L.tess_edge_aggregate_backward.restype = i32
     L.tess_stage_timing.argtypes = [i32]
     L.tess_stage_times.argtypes = [P, P, i32]
     L.tess_stage_times.restype = i32
@@ -158,6 +161,12 @@ def tess_edge_aggregate(pos, n, box, rc, nbr, counts, max_neighbors, feat, F, ou
                         stream) -> int:
     return int(lib().tess_edge_aggregate(pos, n, _box(box), rc, nbr, counts, max_neighbors, feat, F, out, edge_vec,
                                          edge_fc, edge_unit, stream))
+
+
+def tess_edge_aggregate_backward(pos, n, box, rc, nbr, counts, max_neighbors, feat, grad_out, F, grad_feat, grad_pos,
+                                 stream) -> int:
+    return int(lib().tess_edge_aggregate_backward(pos, n, _box(box), rc, nbr, counts, max_neighbors, feat, grad_out,
+                                                  F, grad_feat, grad_pos, stream))
 
 
 def tess_stage_timing(enable: bool) -> None:
@@ -301,3 +310,25 @@ def edge_aggregate(pos4, box, rc: float, nbr, counts, feat, *, out=None, edges: 
     if edges:
         return out, ev, ef, eu
     return out
+
+
+def edge_aggregate_backward(pos4, box, rc: float, nbr, counts, feat, grad_out, *, grad_feat=None, grad_pos=None,
+                            stream=None):
+    """(dL/dfeat [n, F], dL/dpos [n, 3]) given dL/dout, for a full symmetric
+    list without overflow (the output of build_neighbors)."""
+    torch = _torch()
+    _need_cuda("pos4", pos4, torch.float32, 4)
+    _need_cuda("nbr", nbr, torch.int32)
+    _need_cuda("counts", counts, torch.int32)
+    _need_cuda("feat", feat, torch.float32)
+    _need_cuda("grad_out", grad_out, torch.float32)
+    n, cap = nbr.shape
+    F = feat.shape[1]
+    dev = pos4.device
+    grad_feat = torch.empty((n, F), dtype=torch.float32, device=dev) if grad_feat is None else grad_feat
+    grad_pos = torch.empty((n, 3), dtype=torch.float32, device=dev) if grad_pos is None else grad_pos
+    code = tess_edge_aggregate_backward(_ptr(pos4), n, box, float(rc), _ptr(nbr), _ptr(counts), cap, _ptr(feat),
+                                        _ptr(grad_out), F, _ptr(grad_feat), _ptr(grad_pos), _stream(stream))
+    _check("tess_edge_aggregate_backward", code)
+    return grad_feat, grad_pos
+

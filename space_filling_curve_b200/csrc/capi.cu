@@ -23,6 +23,10 @@ tess_status edge_aggregate(const float* pos, int n, tess_box box, float rc, cons
                            int cap, const float* feat, int F, float* out, float* edge_vec, float* edge_fc,
                            float* edge_unit, cudaStream_t s);
 
+tess_status edge_backward(const float* pos, int n, tess_box box, float rc, const int32_t* nbr, const int32_t* counts,
+                          int cap, const float* feat, const float* grad_out, int F, float* grad_feat,
+                          float* grad_pos, cudaStream_t s);
+
 // ---------------------------------------------------------------- stage timing
 
 namespace {
@@ -117,6 +121,14 @@ tess_status tess_edge_aggregate(const float* pos, int n, tess_box box, float rc,
                                 float* edge_vec, float* edge_fc, float* edge_unit, tess_stream_t stream) {
     return edge_aggregate(pos, n, box, rc, nbr, counts, max_neighbors, feat, F, out, edge_vec, edge_fc, edge_unit,
                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+tess_status tess_edge_aggregate_backward(const float* pos, int n, tess_box box, float rc, const int32_t* nbr,
+                                         const int32_t* counts, int max_neighbors, const float* feat,
+                                         const float* grad_out, int F, float* grad_feat, float* grad_pos,
+                                         tess_stream_t stream) {
+    return edge_backward(pos, n, box, rc, nbr, counts, max_neighbors, feat, grad_out, F, grad_feat, grad_pos,
+                         reinterpret_cast<cudaStream_t>(stream));
 }
 
 void tess_stage_timing(int enable) {

@@ -309,6 +309,205 @@ __global__ __launch_bounds__(EV_WARPS * 32, 3) void edge_vec4_kernel(EdgeArgs A)
     }
 }
 
+// ---------------------------------------------------------------- backward (force path)
+
+// sin(pi sqrt(u)) / (pi sqrt(u)) as the Taylor series sum_k (-pi^2 u)^k /
+// (2k+1)!, eleven terms (truncation below 2e-10 at u = 1), so that
+// d f_c / d r divided by r is -(pi^2 / (2 rc^2)) times this, with no root.
+__host__ __device__ constexpr double sinc_pi_sqrt_coef(int k) {
+    double c = 1.0;
+    for (int m = 1; m <= k; ++m) c *= -9.8696044010893586188 / ((2.0 * m) * (2.0 * m + 1.0));
+    return c;
+}
+
+__device__ __forceinline__ float sinc_u(float u) {
+    float p = (float)sinc_pi_sqrt_coef(10);
+    p = fmaf(p, u, (float)sinc_pi_sqrt_coef(9));
+    p = fmaf(p, u, (float)sinc_pi_sqrt_coef(8));
+    p = fmaf(p, u, (float)sinc_pi_sqrt_coef(7));
+    p = fmaf(p, u, (float)sinc_pi_sqrt_coef(6));
+    p = fmaf(p, u, (float)sinc_pi_sqrt_coef(5));
+    p = fmaf(p, u, (float)sinc_pi_sqrt_coef(4));
+    p = fmaf(p, u, (float)sinc_pi_sqrt_coef(3));
+    p = fmaf(p, u, (float)sinc_pi_sqrt_coef(2));
+    p = fmaf(p, u, (float)sinc_pi_sqrt_coef(1));
+    return fmaf(p, u, 1.0f);
+}
+
+struct BackArgs {
+    const float4* pos;
+    const int* nbr;
+    const int* counts;
+    const float* feat;
+    const float* grad_out;
+    float* grad_feat;
+    float* grad_pos;
+    int n, cap, F;
+    float3 L;
+    float inv_rc2;
+    float dfc_scale;     // -(pi^2 / (2 rc^2)): (d f_c / d r) / r = dfc_scale * sinc_u(u)
+};
+
+// Vector-Jacobian product of the aggregation over a full symmetric list
+// (j in row i exactly when i in row j, as tess_build_neighbors writes it):
+//   grad_feat[i] = sum_{j in row i} f_c(r_ij) g_j
+//   grad_pos[i]  = -sum_{j in row i} f_c'(r_ij) (g_i . h_j + g_j . h_i) r_ij / |r_ij|
+// The symmetry turns the scatter of the chain rule into a per-row gather, so
+// no atomics.  Same layout as edge_vec4_kernel: phase 1 geometry and live-edge
+// compaction, phase 2 LPE lanes per edge with VPL float4 of h_j and g_j each;
+// the edge's dot product is reduced within its lane group.
+constexpr int BK_WARPS = 4;
+constexpr int BK_MAXCAP = 512;
+
+template <int LPE, int VPL>
+__global__ __launch_bounds__(BK_WARPS * 32, 4) void edge_backward_kernel(BackArgs A) {
+    constexpr int EPI = 32 / LPE;
+    __shared__ int s_j[BK_WARPS][BK_MAXCAP];
+    __shared__ float4 s_w[BK_WARPS][BK_MAXCAP];    // (f_c, v.x, v.y, v.z) with v = (f_c'/r) r_ij
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane / LPE, fl = lane % LPE;
+    const int F4 = A.F / 4;
+    const float4* h4 = reinterpret_cast<const float4*>(A.feat);
+    const float4* g4 = reinterpret_cast<const float4*>(A.grad_out);
+    float4* gf4 = reinterpret_cast<float4*>(A.grad_feat);
+    for (long long i = (long long)blockIdx.x * BK_WARPS + warp; i < A.n; i += (long long)gridDim.x * BK_WARPS) {
+        const float4 pi = A.pos[i];
+        const int m = max(min(A.counts[i], A.cap), 0);
+        int nlive = 0;
+        for (int s0 = 0; s0 < m; s0 += 32) {
+            const int s = s0 + lane;
+            int j = (s < m) ? A.nbr[(size_t)i * A.cap + s] : -1;
+            if (j >= A.n) j = -1;
+            float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+            bool live = false;
+            if (j >= 0) {
+                const float4 pj = A.pos[j];
+                const float dx = min_image_f(pj.x - pi.x, A.L.x);
+                const float dy = min_image_f(pj.y - pi.y, A.L.y);
+                const float dz = min_image_f(pj.z - pi.z, A.L.z);
+                const float u2 = fmaf(dz, dz, fmaf(dy, dy, dx * dx)) * A.inv_rc2;
+                if (u2 < 1.0f) {
+                    const float dr = A.dfc_scale * sinc_u(u2);
+                    w = make_float4(cutoff_u(u2), dr * dx, dr * dy, dr * dz);
+                    live = true;
+                }
+            }
+            const unsigned bm = __ballot_sync(FULL, live);
+            if (live) {
+                const int k = nlive + __popc(bm & lanemask_lt());
+                s_j[warp][k] = j;
+                s_w[warp][k] = w;
+            }
+            nlive += __popc(bm);
+        }
+        __syncwarp();
+        float4 gi[VPL], hi[VPL], acc[VPL];
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) {
+            gi[v] = g4[(size_t)i * F4 + fl * VPL + v];
+            hi[v] = h4[(size_t)i * F4 + fl * VPL + v];
+            acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        float fx = 0.f, fy = 0.f, fz = 0.f;
+        for (int e0 = 0; e0 < nlive; e0 += EPI) {
+            const int e = e0 + g;
+            const bool ok = e < nlive;
+            const int j = ok ? s_j[warp][e] : (int)i;
+            const float4 w = ok ? s_w[warp][e] : make_float4(0.f, 0.f, 0.f, 0.f);
+            float dot = 0.f;
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) {
+                const float4 hj = h4[(size_t)j * F4 + fl * VPL + v];
+                const float4 gj = g4[(size_t)j * F4 + fl * VPL + v];
+                acc[v].x = fmaf(w.x, gj.x, acc[v].x);
+                acc[v].y = fmaf(w.x, gj.y, acc[v].y);
+                acc[v].z = fmaf(w.x, gj.z, acc[v].z);
+                acc[v].w = fmaf(w.x, gj.w, acc[v].w);
+                dot = fmaf(gi[v].x, hj.x, fmaf(gj.x, hi[v].x, dot));
+                dot = fmaf(gi[v].y, hj.y, fmaf(gj.y, hi[v].y, dot));
+                dot = fmaf(gi[v].z, hj.z, fmaf(gj.z, hi[v].z, dot));
+                dot = fmaf(gi[v].w, hj.w, fmaf(gj.w, hi[v].w, dot));
+            }
+#pragma unroll
+            for (int o = 1; o < LPE; o <<= 1) dot += __shfl_xor_sync(FULL, dot, o);
+            if (ok) {
+                fx = fmaf(dot, w.y, fx);
+                fy = fmaf(dot, w.z, fy);
+                fz = fmaf(dot, w.w, fz);
+            }
+        }
+        // lane groups hold disjoint edges (sum them); within a group every
+        // lane holds the same force but different features
+#pragma unroll
+        for (int o = LPE; o < 32; o <<= 1) {
+            fx += __shfl_xor_sync(FULL, fx, o);
+            fy += __shfl_xor_sync(FULL, fy, o);
+            fz += __shfl_xor_sync(FULL, fz, o);
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) {
+                acc[v].x += __shfl_xor_sync(FULL, acc[v].x, o);
+                acc[v].y += __shfl_xor_sync(FULL, acc[v].y, o);
+                acc[v].z += __shfl_xor_sync(FULL, acc[v].z, o);
+                acc[v].w += __shfl_xor_sync(FULL, acc[v].w, o);
+            }
+        }
+        if (g == 0) {
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) gf4[(size_t)i * F4 + fl * VPL + v] = acc[v];
+        }
+        if (lane == 0) {
+            A.grad_pos[3 * (size_t)i] = -fx;
+            A.grad_pos[3 * (size_t)i + 1] = -fy;
+            A.grad_pos[3 * (size_t)i + 2] = -fz;
+        }
+        __syncwarp();
+    }
+}
+
+tess_status edge_backward(const float* pos, int n, tess_box box, float rc, const int32_t* nbr, const int32_t* counts,
+                          int cap, const float* feat, const float* grad_out, int F, float* grad_feat,
+                          float* grad_pos, cudaStream_t s) {
+    if (n <= 0 || !pos || !nbr || !counts || !feat || !grad_out || !grad_feat || !grad_pos || cap < 1 || F < 1)
+        return TESS_ERR_INVALID_ARG;
+    if (!(rc > 0.f) || !std::isfinite(rc)) return TESS_ERR_INVALID_ARG;
+    if (!finite_pos(box.lx) || !finite_pos(box.ly) || !finite_pos(box.lz)) return TESS_ERR_INVALID_ARG;
+    if (F % 4 != 0 || F > 256 || cap > BK_MAXCAP || !aligned(pos, 16) || !aligned(feat, 16) ||
+        !aligned(grad_out, 16) || !aligned(grad_feat, 16))
+        return TESS_ERR_INVALID_ARG;
+    if (box.lx < 2.f * rc || box.ly < 2.f * rc || box.lz < 2.f * rc) return TESS_ERR_BOX_TOO_SMALL;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    BackArgs A;
+    A.pos = reinterpret_cast<const float4*>(pos);
+    A.nbr = nbr;
+    A.counts = counts;
+    A.feat = feat;
+    A.grad_out = grad_out;
+    A.grad_feat = grad_feat;
+    A.grad_pos = grad_pos;
+    A.n = n;
+    A.cap = cap;
+    A.F = F;
+    A.L = make_float3(box.lx, box.ly, box.lz);
+    A.inv_rc2 = 1.0f / (rc * rc);
+    A.dfc_scale = (float)(-9.8696044010893586188 / (2.0 * (double)rc * (double)rc));
+    StageScope sc(ST_BACKWARD, s);
+    const int blocks = (int)std::min<long long>(((long long)n + BK_WARPS - 1) / BK_WARPS, (long long)sms * 32);
+    switch (F / 4) {
+        case 1: edge_backward_kernel<1, 1><<<blocks, BK_WARPS * 32, 0, s>>>(A); break;
+        case 2: edge_backward_kernel<2, 1><<<blocks, BK_WARPS * 32, 0, s>>>(A); break;
+        case 4: edge_backward_kernel<2, 2><<<blocks, BK_WARPS * 32, 0, s>>>(A); break;
+        case 8: edge_backward_kernel<4, 2><<<blocks, BK_WARPS * 32, 0, s>>>(A); break;
+        case 16: edge_backward_kernel<8, 2><<<blocks, BK_WARPS * 32, 0, s>>>(A); break;
+        case 32: edge_backward_kernel<16, 2><<<blocks, BK_WARPS * 32, 0, s>>>(A); break;
+        case 64: edge_backward_kernel<32, 2><<<blocks, BK_WARPS * 32, 0, s>>>(A); break;
+        default: return TESS_ERR_INVALID_ARG;    // F a multiple of 4 that is not 4 * 2^k
+    }
+    count_launch();
+    return launch_status();
+}
+
 tess_status edge_aggregate(const float* pos, int n, tess_box box, float rc, const int32_t* nbr, const int32_t* counts,
                            int cap, const float* feat, int F, float* out, float* edge_vec, float* edge_fc,
                            float* edge_unit, cudaStream_t s) {
