@@ -195,8 +195,10 @@ constexpr int EV_GEO_UNROLL = 4;     // neighbor/position loads in flight per la
 constexpr int EV_ACC_UNROLL = 4;     // feature rows in flight per lane group
 
 // Features as float4 (F % 4 == 0, F <= 256): LPE lanes share one edge and
-// each lane owns VPL float4 of the feature row (F = 4 * LPE * VPL), so a warp
-// reads 32/LPE neighbor feature rows per step with 16-byte loads.  Phase 1
+// each lane owns VPL float4 of the feature row (F = 4 * LPE * VPL), float4
+// number v * LPE + fl for lane fl, so that one load instruction of a lane
+// group reads LPE * 16 contiguous bytes (whole sectors, one cache line per
+// edge at LPE = 8) and a warp reads 32/LPE neighbor feature rows per step.  Phase 1
 // computes the geometry of the whole row (one edge per lane, several loads in
 // flight) and compacts the live (j, f_c) pairs into shared memory; phase 2
 // accumulates f_c * h_j with several rows in flight; the lane groups are then
@@ -263,7 +265,7 @@ __global__ __launch_bounds__(EV_WARPS * 32, 3) void edge_vec4_kernel(EdgeArgs A)
         float4 acc[VPL];
 #pragma unroll
         for (int v = 0; v < VPL; ++v) acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4* fbase = feat4 + fl * VPL;
+        const float4* fbase = feat4 + fl;
         for (int e0 = 0; e0 < nlive; e0 += EPI * EV_ACC_UNROLL) {
             int2 ed[EV_ACC_UNROLL];
             float4 h[EV_ACC_UNROLL][VPL];
@@ -276,7 +278,7 @@ __global__ __launch_bounds__(EV_WARPS * 32, 3) void edge_vec4_kernel(EdgeArgs A)
             for (int u = 0; u < EV_ACC_UNROLL; ++u) {
                 const float4* src = fbase + (size_t)max(ed[u].x, 0) * F4;
 #pragma unroll
-                for (int v = 0; v < VPL; ++v) h[u][v] = src[v];
+                for (int v = 0; v < VPL; ++v) h[u][v] = src[v * LPE];
             }
 #pragma unroll
             for (int u = 0; u < EV_ACC_UNROLL; ++u) {
@@ -303,7 +305,7 @@ __global__ __launch_bounds__(EV_WARPS * 32, 3) void edge_vec4_kernel(EdgeArgs A)
         }
         if (g == 0) {
 #pragma unroll
-            for (int v = 0; v < VPL; ++v) out4[(size_t)i * F4 + fl * VPL + v] = acc[v];
+            for (int v = 0; v < VPL; ++v) out4[(size_t)i * F4 + v * LPE + fl] = acc[v];
         }
         __syncwarp();
     }
@@ -404,8 +406,8 @@ __global__ __launch_bounds__(BK_WARPS * 32, 4) void edge_backward_kernel(BackArg
         float4 gi[VPL], hi[VPL], acc[VPL];
 #pragma unroll
         for (int v = 0; v < VPL; ++v) {
-            gi[v] = g4[(size_t)i * F4 + fl * VPL + v];
-            hi[v] = h4[(size_t)i * F4 + fl * VPL + v];
+            gi[v] = g4[(size_t)i * F4 + v * LPE + fl];
+            hi[v] = h4[(size_t)i * F4 + v * LPE + fl];
             acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
         float fx = 0.f, fy = 0.f, fz = 0.f;
@@ -417,8 +419,8 @@ __global__ __launch_bounds__(BK_WARPS * 32, 4) void edge_backward_kernel(BackArg
             float dot = 0.f;
 #pragma unroll
             for (int v = 0; v < VPL; ++v) {
-                const float4 hj = h4[(size_t)j * F4 + fl * VPL + v];
-                const float4 gj = g4[(size_t)j * F4 + fl * VPL + v];
+                const float4 hj = h4[(size_t)j * F4 + v * LPE + fl];
+                const float4 gj = g4[(size_t)j * F4 + v * LPE + fl];
                 acc[v].x = fmaf(w.x, gj.x, acc[v].x);
                 acc[v].y = fmaf(w.x, gj.y, acc[v].y);
                 acc[v].z = fmaf(w.x, gj.z, acc[v].z);
@@ -453,7 +455,7 @@ __global__ __launch_bounds__(BK_WARPS * 32, 4) void edge_backward_kernel(BackArg
         }
         if (g == 0) {
 #pragma unroll
-            for (int v = 0; v < VPL; ++v) gf4[(size_t)i * F4 + fl * VPL + v] = acc[v];
+            for (int v = 0; v < VPL; ++v) gf4[(size_t)i * F4 + v * LPE + fl] = acc[v];
         }
         if (lane == 0) {
             A.grad_pos[3 * (size_t)i] = -fx;
