@@ -76,8 +76,8 @@ const char* tess_version(void);
 long long tess_kernel_launch_count(void);
 
 /* ---------------------------------------------------------------------------
- * Hilbert sort -- "sorts atoms along a space-filling curve" (Tessera,
- * abstract).
+ * Hilbert sort -- Tessera orders the atoms along a space-filling curve
+ * before cutting them into shards (Tessera, abstract).
  *
  * Each coordinate is quantised on a grid of 2^bits cells per axis: the scale
  * s = 2^bits / L is one fp32 division, the cell is floor(x * s) with x * s a
@@ -106,8 +106,9 @@ tess_status tess_hilbert_sort(const float* pos, int n, tess_box box, int bits,
                               int32_t* dev_status, tess_stream_t stream);
 
 /* ---------------------------------------------------------------------------
- * Morton (Z-order) sort -- the comparison curve of the Tessera abstract
- * ("neighbor-search cost grows 1.7x, versus 3.0x for Morton order").
+ * Morton (Z-order) sort -- the curve the Tessera abstract compares against:
+ * it reports neighbor-search cost growing 1.7x along its curve and 3.0x
+ * along the Morton order.
  *
  * Same quantisation, arguments, outputs, workspace and errors as
  * tess_hilbert_sort; the key is the plain bit interleave of the three grid
@@ -149,8 +150,9 @@ tess_status tess_hilbert_sort_static(const float* pos, int n, tess_box box, int 
                                      int32_t* dev_status, tess_stream_t stream);
 
 /* ---------------------------------------------------------------------------
- * Verlet neighbor list at rs = rc + skin -- "fixes workload shapes between
- * rebuilds", "three-level neighbor search" (Tessera, abstract).
+ * Verlet neighbor list at rs = rc + skin -- Tessera keeps every per-atom
+ * shape constant from one rebuild to the next and names a neighbor search
+ * in three levels (Tessera, abstract).
  *
  * Row i lists every j != i whose minimum-image distance to i is below rs
  * (strictly), computed in fp32.  The list is full (j in row i iff i in row
@@ -182,8 +184,8 @@ tess_status tess_build_neighbors(const float* pos, int n, tess_box box, float rc
                                  tess_stream_t stream);
 
 /* ---------------------------------------------------------------------------
- * Skin check -- "a conservative neighbor skin preserves topology across
- * updates" (Tessera, abstract).  Rebuild when some atom has moved more than
+ * Skin check -- Tessera's conservative skin keeps the neighbor graph valid
+ * while atoms move between rebuilds (Tessera, abstract).  Rebuild when some atom has moved more than
  * skin/2 since the reference frame: max_i |minimg(r_i - r_i^ref)|^2 >
  * (skin/2)^2.  Displacements, squares and the threshold are fp64 (each
  * operation one IEEE rounding: (dx*dx + dy*dy) + dz*dz), so the flag and
@@ -200,8 +202,8 @@ tess_status tess_skin_check(const float* pos, const float* pos_ref, int n, tess_
 /* ---------------------------------------------------------------------------
  * Edge geometry and one-hop aggregation -- each message-passing layer
  * aggregates one-hop neighbor features within the cutoff (review of arXiv
- * 2505.06711, "load-bearing attack" paragraph); "Fused kernels" (Tessera,
- * abstract).
+ * 2505.06711, "load-bearing attack" paragraph); Tessera fuses such kernels
+ * (Tessera, abstract).
  *
  * For row i and each of its first min(counts[i], cap) listed j (entries < 0
  * skipped): r_ij = minimg(r_j - r_i), r = |r_ij|, f_c(r) = (cos(pi r / rc) +
@@ -225,9 +227,10 @@ tess_status tess_edge_aggregate(const float* pos, int n, tess_box box, float rc,
                                 tess_stream_t stream);
 
 /* ---------------------------------------------------------------------------
- * Backward of the aggregation -- "force backpropagation repeats the
- * exchange" (Tessera, abstract); the review of arXiv 2505.06711 describes
- * the same vector-Jacobian product over one-hop edges.
+ * Backward of the aggregation -- in Tessera the backward pass that yields
+ * the forces goes through the same neighbor exchange again (Tessera,
+ * abstract); the review of arXiv 2505.06711 describes the same
+ * vector-Jacobian product over one-hop edges.
  *
  * Given g = dL/d out ([n, F]), writes
  *   grad_feat[i] = dL/d feat[i] = sum_{j in row i} f_c(r_ij) g_j

@@ -147,8 +147,8 @@ static int cmp_u64(const void* a, const void* b)
  * Morton (Z-order) index of grid point (q0, q1, q2): the bits of the three
  * coordinates interleaved most-significant level first, axis 0's bit first
  * within each level -- the same read-out as the Hilbert index without the
- * transform.  This is the comparison curve of the Tessera abstract ("versus
- * 3.0x for Morton order").
+ * transform.  The Tessera abstract compares its curve against this order
+ * (neighbor-search cost grows 3.0x along it, 1.7x along its own curve).
  */
 uint32_t oracle_morton_index(uint32_t q0, uint32_t q1, uint32_t q2, int bits)
 {
@@ -590,8 +590,8 @@ double oracle_cutoff_deriv(double r, double rc)
 /*
  * Vector-Jacobian product of out_i = sum_{j in row i} f_c(|r_ij|) h_j with
  * respect to the features and the positions, given g = dL/d out ([n, F]).
- * "force backpropagation repeats the exchange" (Tessera, abstract); the
- * review of arXiv 2505.06711 describes the same VJP over one-hop edges.
+ * The backward pass that yields the forces repeats the neighbor exchange
+ * (Tessera, abstract); the review of arXiv 2505.06711 describes the same VJP over one-hop edges.
  * Plain chain rule over the listed edges, accumulated serially in fp64:
  *   grad_feat[j] += f_c(r_ij) g_i                       for each listed (i, j)
  *   s = f_c'(r_ij) (g_i . h_j);  grad_pos[i] -= s u_ij;  grad_pos[j] += s u_ij

@@ -1,5 +1,5 @@
 // hilbert_sort.cu -- Hilbert keys and the device radix sort that orders atoms
-// along the curve ("sorts atoms along a space-filling curve", Tessera,
+// along the curve (Tessera orders atoms along a space-filling curve; Tessera,
 // abstract).
 //
 // Pipeline (one stream, no host sync):

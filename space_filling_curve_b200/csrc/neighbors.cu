@@ -1,6 +1,6 @@
-// neighbors.cu -- fixed-capacity Verlet list at rs = rc + skin ("fixes
-// workload shapes between rebuilds", "three-level neighbor search",
-// Tessera, abstract).
+// neighbors.cu -- fixed-capacity Verlet list at rs = rc + skin (shapes held
+// constant between rebuilds, a neighbor search in three levels; Tessera,
+// abstract).
 //
 // Level 0 (binning, deterministic):
 //   cell_count     cell id per atom, warp-aggregated histogram

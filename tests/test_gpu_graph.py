@@ -1,5 +1,5 @@
-"""The per-step path replayed as one CUDA graph ("enabling each rebuild
-interval to replay as one CUDA Graph", Tessera, abstract): every entry point
+"""The per-step path replayed as one CUDA graph (Tessera replays each
+interval between rebuilds as a single CUDA graph; Tessera, abstract): every entry point
 is stream-ordered, allocates nothing and never synchronises the host, so a
 whole step -- sort, list, skin check, aggregation -- can be captured once and
 replayed.  Replays must reproduce the eager results exactly (the kernels are

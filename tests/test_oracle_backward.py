@@ -1,9 +1,10 @@
 """Pins of the oracle's backward (VJP) of the aggregation against finite
 differences of the forward oracle and against identities of the full list.
 
-"force backpropagation repeats the exchange" ("Ab Initio Accuracy Beyond the
-Cutoff" (Tessera), abstract): forces are -dE/dr through every layer; this is
-the one-hop aggregation's share of that chain rule.
+The forces come from a backward pass through every layer, which repeats the
+neighbor exchange ("Ab Initio Accuracy Beyond the Cutoff" (Tessera),
+abstract): forces are -dE/dr; this is the one-hop aggregation's share of that
+chain rule.
 """
 import numpy as np
 import pytest
