@@ -326,7 +326,7 @@ def run_cuda(args, world, rank, local):
     stage_ms = {k: (v[0] / max(v[1], 1)) for k, v in stages.items() if v[1] > 0}
     dom = max(stage_ms, key=stage_ms.get)
     achieved = nbytes[dom] / (stage_ms[dom] / 1e3) / 1e9
-    traffic = _traffic_from_profile(dom)
+    traffic = _traffic_from_profile(dom, s.n)
     clocks = clk.summary()
 
     if rank == 0:
@@ -344,9 +344,9 @@ def run_cuda(args, world, rank, local):
             "dtype": "f32",
             "data": "synthetic (seeded salt-solution generator; no dataset)",
             "config": {
-                "workload": "salt-10.24M: %d atoms, box %.3f A cubic, rc %.2f, skin %.2f, cap %d, F %d; step = "
+                "workload": "%s: %d atoms, box %.3f x %.3f x %.3f A, rc %.2f, skin %.2f, cap %d, F %d; step = "
                             "hilbert_sort + build_neighbors (pad-filled) + skin_check + edge_aggregate"
-                            % (s.n, s.box[0], s.rc, s.skin, s.cap, s.F),
+                            % (s.name, s.n, s.box[0], s.box[1], s.box[2], s.rc, s.skin, s.cap, s.F),
                 "atoms": s.n,
                 "pad_fill": not args.no_pad_fill,
                 "pair_search": "tile" if args.tile_search else "per-lane",
@@ -394,14 +394,20 @@ def _rebuild_roofline(n, mean_count, stage_ms, peak):
             "frac": (b / (t / 1e3) / 1e9) / peak if t else None}
 
 
-def _traffic_from_profile(kernel_stage):
-    """DRAM bytes per launch of the dominant kernel from the committed ncu
-    summary (profiles/<stage>_traffic.json), or None."""
+def _traffic_from_profile(kernel_stage, n):
+    """DRAM bytes per launch of the dominant kernel at n atoms, from the
+    committed ncu summary (profiles/<stage>_traffic.json: bytes per atom of
+    one capture), or None when there is none or when the kernel's source
+    file has changed since the counters were taken."""
+    import hashlib
     path = os.path.join(ROOT, "profiles", "%s_traffic.json" % kernel_stage)
     try:
         with open(path) as f:
             d = json.load(f)
-        return d.get("bytes_per_launch_full_size")
+        with open(os.path.join(ROOT, d["source_file"]), "rb") as f:
+            if hashlib.sha1(f.read()).hexdigest() != d["source_sha1"]:
+                return None
+        return d["dram_bytes_per_atom"] * n
     except Exception:
         return None
 

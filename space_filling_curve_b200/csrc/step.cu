@@ -1,9 +1,12 @@
-// step.cu -- the per-step kernels: the skin check ("a conservative neighbor
-// skin preserves topology across updates", Tessera, abstract) and the fused
+// step.cu -- the per-step kernels: the skin check (a conservative skin keeps
+// the neighbor graph valid between rebuilds; Tessera, abstract) and the fused
 // edge-geometry + one-hop aggregation that each message-passing layer
 // consumes (review of arXiv 2505.06711, "load-bearing attack" paragraph:
 // each layer aggregates one-hop neighbor features within the cutoff).
 #include "common.cuh"
+
+#include <initializer_list>
+#include <type_traits>
 
 namespace tess {
 
@@ -191,30 +194,109 @@ __global__ __launch_bounds__(EDGE_WARPS * 32) void edge_kernel(EdgeArgs A) {
 
 constexpr int EV_WARPS = 8;
 constexpr int EV_MAXCAP = 512;       // live edges of one row staged in shared memory
+#ifndef TESS_EV_MINB
+#define TESS_EV_MINB 3               // resident blocks per SM the register budget aims at
+#endif
+#ifndef TESS_EV_CHUNK
+#define TESS_EV_CHUNK 256
+#endif
+#ifndef TESS_EV_W
+#define TESS_EV_W 4                  // floats per feature load when F allows (4 or 8)
+#endif
+// Rows are taken in chunks of consecutive rows per block (chunks dealt to
+// blocks round robin), so that the neighbor feature rows one row pulls into
+// L1 serve the next rows too: rows adjacent in the sorted order are adjacent
+// in space and share most of their neighbors.  All blocks together sweep a
+// front of gridDim * chunk rows, which bounds the L2 working set.
+constexpr int EV_CHUNK = TESS_EV_CHUNK;
 constexpr int EV_GEO_UNROLL = 4;     // neighbor/position loads in flight per lane
 constexpr int EV_ACC_UNROLL = 4;     // feature rows in flight per lane group
 
-// Features as float4 (F % 4 == 0, F <= 256): LPE lanes share one edge and
-// each lane owns VPL float4 of the feature row (F = 4 * LPE * VPL), float4
-// number v * LPE + fl for lane fl, so that one load instruction of a lane
-// group reads LPE * 16 contiguous bytes (whole sectors, one cache line per
-// edge at LPE = 8) and a warp reads 32/LPE neighbor feature rows per step.  Phase 1
-// computes the geometry of the whole row (one edge per lane, several loads in
-// flight) and compacts the live (j, f_c) pairs into shared memory; phase 2
-// accumulates f_c * h_j with several rows in flight; the lane groups are then
-// summed with shuffles.
-template <int LPE, int VPL>
-__global__ __launch_bounds__(EV_WARPS * 32, 3) void edge_vec4_kernel(EdgeArgs A) {
+// W consecutive floats of a feature row (W = 4: one 16-byte load; W = 8: one
+// 32-byte load, which sm_100 issues as a single instruction).
+template <int W>
+struct FVec {
+    float4 q[W / 4];
+    __device__ __forceinline__ void zero() {
+#pragma unroll
+        for (int k = 0; k < W / 4; ++k) q[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __device__ __forceinline__ void fma(float w, const FVec& h) {
+#pragma unroll
+        for (int k = 0; k < W / 4; ++k) {
+            q[k].x = fmaf(w, h.q[k].x, q[k].x);
+            q[k].y = fmaf(w, h.q[k].y, q[k].y);
+            q[k].z = fmaf(w, h.q[k].z, q[k].z);
+            q[k].w = fmaf(w, h.q[k].w, q[k].w);
+        }
+    }
+    // acc + sum_k a_k b_k
+    __device__ __forceinline__ static float dot(const FVec& a, const FVec& b, float acc) {
+#pragma unroll
+        for (int k = 0; k < W / 4; ++k) {
+            acc = fmaf(a.q[k].x, b.q[k].x, acc);
+            acc = fmaf(a.q[k].y, b.q[k].y, acc);
+            acc = fmaf(a.q[k].z, b.q[k].z, acc);
+            acc = fmaf(a.q[k].w, b.q[k].w, acc);
+        }
+        return acc;
+    }
+    __device__ __forceinline__ void shfl_add(int o) {
+#pragma unroll
+        for (int k = 0; k < W / 4; ++k) {
+            q[k].x += __shfl_xor_sync(FULL, q[k].x, o);
+            q[k].y += __shfl_xor_sync(FULL, q[k].y, o);
+            q[k].z += __shfl_xor_sync(FULL, q[k].z, o);
+            q[k].w += __shfl_xor_sync(FULL, q[k].w, o);
+        }
+    }
+    __device__ __forceinline__ void store(float* p) const {
+#pragma unroll
+        for (int k = 0; k < W / 4; ++k) reinterpret_cast<float4*>(p)[k] = q[k];
+    }
+};
+
+template <int W>
+__device__ __forceinline__ FVec<W> ld_vec(const float* p);
+
+template <>
+__device__ __forceinline__ FVec<4> ld_vec<4>(const float* p) {
+    FVec<4> r;
+    r.q[0] = *reinterpret_cast<const float4*>(p);
+    return r;
+}
+
+// 32-byte load (p 32-byte aligned); the features are read-only for the
+// kernel's duration, so the load has no ordering constraint.
+template <>
+__device__ __forceinline__ FVec<8> ld_vec<8>(const float* p) {
+    FVec<8> r;
+    asm("ld.global.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+        : "=f"(r.q[0].x), "=f"(r.q[0].y), "=f"(r.q[0].z), "=f"(r.q[0].w), "=f"(r.q[1].x), "=f"(r.q[1].y),
+          "=f"(r.q[1].z), "=f"(r.q[1].w)
+        : "l"(p));
+    return r;
+}
+
+// Features in vectors of W floats (F = W * LPE * VPL, F <= 256): LPE lanes
+// share one edge and lane fl owns vectors v * LPE + fl (v < VPL) of the row,
+// so one load instruction of a lane group reads LPE * W * 4 contiguous bytes
+// (whole sectors) and a warp reads 32/LPE neighbor feature rows per step.
+// Phase 1 computes the geometry of the whole row (one edge per lane, several
+// loads in flight) and compacts the live (j, f_c) pairs into shared memory;
+// phase 2 accumulates f_c * h_j with several rows in flight; the lane groups
+// are then summed with shuffles.  Shared memory: EV_WARPS * cap int2
+// (dynamic, so that what a small cap leaves over serves as L1).
+template <int W, int LPE, int VPL>
+__global__ __launch_bounds__(EV_WARPS * 32, TESS_EV_MINB) void edge_vec_kernel(EdgeArgs A) {
     constexpr int EPI = 32 / LPE;
-    __shared__ int2 s_edge[EV_WARPS][EV_MAXCAP];
+    extern __shared__ int2 s_edge[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    int2* live_e = s_edge[warp];
+    int2* live_e = s_edge + (size_t)warp * A.cap;
     const int g = lane / LPE, fl = lane % LPE;
-    const int F4 = A.F / 4;
-    const float4* feat4 = reinterpret_cast<const float4*>(A.feat);
-    float4* out4 = reinterpret_cast<float4*>(A.out);
     const bool edges = A.edge_vec || A.edge_fc || A.edge_unit;
-    for (long long i = (long long)blockIdx.x * EV_WARPS + warp; i < A.n; i += (long long)gridDim.x * EV_WARPS) {
+    for (long long c0 = (long long)blockIdx.x * EV_CHUNK; c0 < A.n; c0 += (long long)gridDim.x * EV_CHUNK)
+    for (long long i = c0 + warp, c1 = min((long long)A.n, c0 + EV_CHUNK); i < c1; i += EV_WARPS) {
         const float4 pi = A.pos[i];
         const int m = max(min(A.counts[i], A.cap), 0);
         const int limit = edges ? A.cap : m;
@@ -262,13 +344,13 @@ __global__ __launch_bounds__(EV_WARPS * 32, 3) void edge_vec4_kernel(EdgeArgs A)
             }
         }
         __syncwarp();
-        float4 acc[VPL];
+        FVec<W> acc[VPL];
 #pragma unroll
-        for (int v = 0; v < VPL; ++v) acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4* fbase = feat4 + fl;
+        for (int v = 0; v < VPL; ++v) acc[v].zero();
+        const float* fbase = A.feat + fl * W;
         for (int e0 = 0; e0 < nlive; e0 += EPI * EV_ACC_UNROLL) {
             int2 ed[EV_ACC_UNROLL];
-            float4 h[EV_ACC_UNROLL][VPL];
+            FVec<W> h[EV_ACC_UNROLL][VPL];
 #pragma unroll
             for (int u = 0; u < EV_ACC_UNROLL; ++u) {
                 const int e = e0 + u * EPI + g;
@@ -276,36 +358,26 @@ __global__ __launch_bounds__(EV_WARPS * 32, 3) void edge_vec4_kernel(EdgeArgs A)
             }
 #pragma unroll
             for (int u = 0; u < EV_ACC_UNROLL; ++u) {
-                const float4* src = fbase + (size_t)max(ed[u].x, 0) * F4;
+                const float* src = fbase + (size_t)max(ed[u].x, 0) * A.F;
 #pragma unroll
-                for (int v = 0; v < VPL; ++v) h[u][v] = src[v * LPE];
+                for (int v = 0; v < VPL; ++v) h[u][v] = ld_vec<W>(src + v * LPE * W);
             }
 #pragma unroll
             for (int u = 0; u < EV_ACC_UNROLL; ++u) {
                 if (ed[u].x < 0) continue;     // past the last live edge
                 const float w = __int_as_float(ed[u].y);
 #pragma unroll
-                for (int v = 0; v < VPL; ++v) {
-                    acc[v].x = fmaf(w, h[u][v].x, acc[v].x);
-                    acc[v].y = fmaf(w, h[u][v].y, acc[v].y);
-                    acc[v].z = fmaf(w, h[u][v].z, acc[v].z);
-                    acc[v].w = fmaf(w, h[u][v].w, acc[v].w);
-                }
+                for (int v = 0; v < VPL; ++v) acc[v].fma(w, h[u][v]);
             }
         }
 #pragma unroll
         for (int o = LPE; o < 32; o <<= 1) {
 #pragma unroll
-            for (int v = 0; v < VPL; ++v) {
-                acc[v].x += __shfl_xor_sync(FULL, acc[v].x, o);
-                acc[v].y += __shfl_xor_sync(FULL, acc[v].y, o);
-                acc[v].z += __shfl_xor_sync(FULL, acc[v].z, o);
-                acc[v].w += __shfl_xor_sync(FULL, acc[v].w, o);
-            }
+            for (int v = 0; v < VPL; ++v) acc[v].shfl_add(o);
         }
         if (g == 0) {
 #pragma unroll
-            for (int v = 0; v < VPL; ++v) out4[(size_t)i * F4 + v * LPE + fl] = acc[v];
+            for (int v = 0; v < VPL; ++v) acc[v].store(A.out + (size_t)i * A.F + (v * LPE + fl) * W);
         }
         __syncwarp();
     }
@@ -355,24 +427,33 @@ struct BackArgs {
 //   grad_feat[i] = sum_{j in row i} f_c(r_ij) g_j
 //   grad_pos[i]  = -sum_{j in row i} f_c'(r_ij) (g_i . h_j + g_j . h_i) r_ij / |r_ij|
 // The symmetry turns the scatter of the chain rule into a per-row gather, so
-// no atomics.  Same layout as edge_vec4_kernel: phase 1 geometry and live-edge
-// compaction, phase 2 LPE lanes per edge with VPL float4 of h_j and g_j each;
-// the edge's dot product is reduced within its lane group.
+// no atomics.  Same layout as edge_vec_kernel: phase 1 geometry and live-edge
+// compaction, phase 2 LPE lanes per edge with VPL vectors of h_j and g_j
+// each.  Each lane keeps its own share of the force, sum over edges of (its
+// part of the dot product) times (f_c'/r) r_ij, which is linear in the parts,
+// so the lanes are summed once per row instead of once per edge.
 constexpr int BK_WARPS = 4;
 constexpr int BK_MAXCAP = 512;
+#ifndef TESS_BK_CHUNK
+#define TESS_BK_CHUNK 256
+#endif
+#ifndef TESS_BK_MINB
+#define TESS_BK_MINB 4
+#endif
+constexpr int BK_CHUNK = TESS_BK_CHUNK;
 
-template <int LPE, int VPL>
-__global__ __launch_bounds__(BK_WARPS * 32, 4) void edge_backward_kernel(BackArgs A) {
+template <int W, int LPE, int VPL>
+__global__ __launch_bounds__(BK_WARPS * 32, TESS_BK_MINB) void edge_backward_kernel(BackArgs A) {
     constexpr int EPI = 32 / LPE;
-    __shared__ int s_j[BK_WARPS][BK_MAXCAP];
-    __shared__ float4 s_w[BK_WARPS][BK_MAXCAP];    // (f_c, v.x, v.y, v.z) with v = (f_c'/r) r_ij
+    // dynamic: BK_WARPS * cap float4 (f_c, v.x, v.y, v.z) with v = (f_c'/r) r_ij,
+    // then BK_WARPS * cap int (j)
+    extern __shared__ float4 s_dyn[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float4* s_w = s_dyn + (size_t)warp * A.cap;
+    int* s_j = reinterpret_cast<int*>(s_dyn + (size_t)BK_WARPS * A.cap) + (size_t)warp * A.cap;
     const int g = lane / LPE, fl = lane % LPE;
-    const int F4 = A.F / 4;
-    const float4* h4 = reinterpret_cast<const float4*>(A.feat);
-    const float4* g4 = reinterpret_cast<const float4*>(A.grad_out);
-    float4* gf4 = reinterpret_cast<float4*>(A.grad_feat);
-    for (long long i = (long long)blockIdx.x * BK_WARPS + warp; i < A.n; i += (long long)gridDim.x * BK_WARPS) {
+    for (long long c0 = (long long)blockIdx.x * BK_CHUNK; c0 < A.n; c0 += (long long)gridDim.x * BK_CHUNK)
+    for (long long i = c0 + warp, c1 = min((long long)A.n, c0 + BK_CHUNK); i < c1; i += BK_WARPS) {
         const float4 pi = A.pos[i];
         const int m = max(min(A.counts[i], A.cap), 0);
         int nlive = 0;
@@ -397,65 +478,62 @@ __global__ __launch_bounds__(BK_WARPS * 32, 4) void edge_backward_kernel(BackArg
             const unsigned bm = __ballot_sync(FULL, live);
             if (live) {
                 const int k = nlive + __popc(bm & lanemask_lt());
-                s_j[warp][k] = j;
-                s_w[warp][k] = w;
+                s_j[k] = j;
+                s_w[k] = w;
             }
             nlive += __popc(bm);
         }
         __syncwarp();
-        float4 gi[VPL], hi[VPL], acc[VPL];
+        const size_t own = (size_t)i * A.F + fl * W;
+        FVec<W> gi[VPL], hi[VPL], acc[VPL];
 #pragma unroll
         for (int v = 0; v < VPL; ++v) {
-            gi[v] = g4[(size_t)i * F4 + v * LPE + fl];
-            hi[v] = h4[(size_t)i * F4 + v * LPE + fl];
-            acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+            gi[v] = ld_vec<W>(A.grad_out + own + v * LPE * W);
+            hi[v] = ld_vec<W>(A.feat + own + v * LPE * W);
+            acc[v].zero();
         }
         float fx = 0.f, fy = 0.f, fz = 0.f;
         for (int e0 = 0; e0 < nlive; e0 += EPI) {
             const int e = e0 + g;
             const bool ok = e < nlive;
-            const int j = ok ? s_j[warp][e] : (int)i;
-            const float4 w = ok ? s_w[warp][e] : make_float4(0.f, 0.f, 0.f, 0.f);
-            float dot = 0.f;
+            const int j = ok ? s_j[e] : (int)i;
+            const float4 w = ok ? s_w[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+            const size_t base = (size_t)j * A.F + fl * W;
+            FVec<W> hj[VPL], gj[VPL];
 #pragma unroll
             for (int v = 0; v < VPL; ++v) {
-                const float4 hj = h4[(size_t)j * F4 + v * LPE + fl];
-                const float4 gj = g4[(size_t)j * F4 + v * LPE + fl];
-                acc[v].x = fmaf(w.x, gj.x, acc[v].x);
-                acc[v].y = fmaf(w.x, gj.y, acc[v].y);
-                acc[v].z = fmaf(w.x, gj.z, acc[v].z);
-                acc[v].w = fmaf(w.x, gj.w, acc[v].w);
-                dot = fmaf(gi[v].x, hj.x, fmaf(gj.x, hi[v].x, dot));
-                dot = fmaf(gi[v].y, hj.y, fmaf(gj.y, hi[v].y, dot));
-                dot = fmaf(gi[v].z, hj.z, fmaf(gj.z, hi[v].z, dot));
-                dot = fmaf(gi[v].w, hj.w, fmaf(gj.w, hi[v].w, dot));
+                hj[v] = ld_vec<W>(A.feat + base + v * LPE * W);
+                gj[v] = ld_vec<W>(A.grad_out + base + v * LPE * W);
             }
-#pragma unroll
-            for (int o = 1; o < LPE; o <<= 1) dot += __shfl_xor_sync(FULL, dot, o);
             if (ok) {
+                float dot = 0.f;
+#pragma unroll
+                for (int v = 0; v < VPL; ++v) {
+                    acc[v].fma(w.x, gj[v]);
+                    dot = FVec<W>::dot(gi[v], hj[v], dot);
+                    dot = FVec<W>::dot(gj[v], hi[v], dot);
+                }
                 fx = fmaf(dot, w.y, fx);
                 fy = fmaf(dot, w.z, fy);
                 fz = fmaf(dot, w.w, fz);
             }
         }
-        // lane groups hold disjoint edges (sum them); within a group every
-        // lane holds the same force but different features
+        // feature gradient: lane groups hold disjoint edges of the same
+        // features; force: every lane holds a share
 #pragma unroll
-        for (int o = LPE; o < 32; o <<= 1) {
+        for (int o = 1; o < 32; o <<= 1) {
             fx += __shfl_xor_sync(FULL, fx, o);
             fy += __shfl_xor_sync(FULL, fy, o);
             fz += __shfl_xor_sync(FULL, fz, o);
+        }
 #pragma unroll
-            for (int v = 0; v < VPL; ++v) {
-                acc[v].x += __shfl_xor_sync(FULL, acc[v].x, o);
-                acc[v].y += __shfl_xor_sync(FULL, acc[v].y, o);
-                acc[v].z += __shfl_xor_sync(FULL, acc[v].z, o);
-                acc[v].w += __shfl_xor_sync(FULL, acc[v].w, o);
-            }
+        for (int o = LPE; o < 32; o <<= 1) {
+#pragma unroll
+            for (int v = 0; v < VPL; ++v) acc[v].shfl_add(o);
         }
         if (g == 0) {
 #pragma unroll
-            for (int v = 0; v < VPL; ++v) gf4[(size_t)i * F4 + v * LPE + fl] = acc[v];
+            for (int v = 0; v < VPL; ++v) acc[v].store(A.grad_feat + own + v * LPE * W);
         }
         if (lane == 0) {
             A.grad_pos[3 * (size_t)i] = -fx;
@@ -464,6 +542,68 @@ __global__ __launch_bounds__(BK_WARPS * 32, 4) void edge_backward_kernel(BackArg
         }
         __syncwarp();
     }
+}
+
+// Grid of a chunked row walk for `kernel` (`threads` per block, `smem`
+// dynamic bytes): one resident wave, as many blocks per SM as registers and
+// shared memory allow, never more blocks than chunks.  Also sets the kernel's
+// shared-memory carveout hint to what that wave needs, so that the rest of
+// the SM's 256 KB serves as L1 for the feature gathers (the driver may
+// otherwise keep a larger carveout than the launch needs).
+template <class K>
+int chunk_grid(K* kernel, int threads, size_t smem, int n, int sms, int chunk) {
+    int dev = 0, max_sm = 0, per_sm = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&max_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess || per_sm < 1)
+        per_sm = 1;
+    if (max_sm > 0) {
+        const size_t need = (size_t)per_sm * (smem + 1024);
+        const int pct = (int)std::min<size_t>(100, (need * 100 + max_sm - 1) / max_sm);
+        cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, pct);
+    }
+    const long long chunks = ((long long)n + chunk - 1) / chunk;
+    return (int)std::max<long long>(1, std::min<long long>(chunks, (long long)sms * per_sm));
+}
+
+template <int V>
+using ic = std::integral_constant<int, V>;
+
+// Launch shape for q = F / W vectors per row (q a power of two): calls
+// launch(W, LPE, VPL) as integral constants; false when q is not covered.
+template <int W, class Launch>
+bool by_shape(int q, Launch&& launch) {
+    if (W == 4) {
+        switch (q) {
+            case 1: launch(ic<W>{}, ic<1>{}, ic<1>{}); return true;
+            case 2: launch(ic<W>{}, ic<2>{}, ic<1>{}); return true;
+            case 4: launch(ic<W>{}, ic<2>{}, ic<2>{}); return true;
+            case 8: launch(ic<W>{}, ic<4>{}, ic<2>{}); return true;
+            case 16: launch(ic<W>{}, ic<8>{}, ic<2>{}); return true;
+            case 32: launch(ic<W>{}, ic<16>{}, ic<2>{}); return true;
+            case 64: launch(ic<W>{}, ic<32>{}, ic<2>{}); return true;
+            default: return false;
+        }
+    }
+    switch (q) {
+        case 1: launch(ic<W>{}, ic<1>{}, ic<1>{}); return true;
+        case 2: launch(ic<W>{}, ic<2>{}, ic<1>{}); return true;
+        case 4: launch(ic<W>{}, ic<4>{}, ic<1>{}); return true;
+        case 8: launch(ic<W>{}, ic<8>{}, ic<1>{}); return true;
+        case 16: launch(ic<W>{}, ic<8>{}, ic<2>{}); return true;
+        case 32: launch(ic<W>{}, ic<16>{}, ic<2>{}); return true;
+        default: return false;
+    }
+}
+
+// Vector width for feature rows of F floats whose arrays are `ptrs`: 8 when
+// F is a multiple of 8 and every array is 32-byte aligned, else 4 (the
+// callers require 16-byte alignment and F % 4 == 0 for either).
+inline int pick_width(int F, std::initializer_list<const void*> ptrs) {
+    if (TESS_EV_W != 8 || F % 8 != 0) return 4;
+    for (const void* p : ptrs)
+        if (!aligned(p, 32)) return 4;
+    return 8;
 }
 
 tess_status edge_backward(const float* pos, int n, tess_box box, float rc, const int32_t* nbr, const int32_t* counts,
@@ -495,17 +635,14 @@ tess_status edge_backward(const float* pos, int n, tess_box box, float rc, const
     A.inv_rc2 = 1.0f / (rc * rc);
     A.dfc_scale = (float)(-9.8696044010893586188 / (2.0 * (double)rc * (double)rc));
     StageScope sc(ST_BACKWARD, s);
-    const int blocks = (int)std::min<long long>(((long long)n + BK_WARPS - 1) / BK_WARPS, (long long)sms * 32);
-    switch (F / 4) {
-        case 1: edge_backward_kernel<1, 1><<<blocks, BK_WARPS * 32, 0, s>>>(A); break;
-        case 2: edge_backward_kernel<2, 1><<<blocks, BK_WARPS * 32, 0, s>>>(A); break;
-        case 4: edge_backward_kernel<2, 2><<<blocks, BK_WARPS * 32, 0, s>>>(A); break;
-        case 8: edge_backward_kernel<4, 2><<<blocks, BK_WARPS * 32, 0, s>>>(A); break;
-        case 16: edge_backward_kernel<8, 2><<<blocks, BK_WARPS * 32, 0, s>>>(A); break;
-        case 32: edge_backward_kernel<16, 2><<<blocks, BK_WARPS * 32, 0, s>>>(A); break;
-        case 64: edge_backward_kernel<32, 2><<<blocks, BK_WARPS * 32, 0, s>>>(A); break;
-        default: return TESS_ERR_INVALID_ARG;    // F a multiple of 4 that is not 4 * 2^k
-    }
+    const size_t smem = (size_t)BK_WARPS * cap * (sizeof(float4) + sizeof(int));
+    auto launch = [&](auto w, auto lpe, auto vpl) {
+        auto* k = edge_backward_kernel<decltype(w)::value, decltype(lpe)::value, decltype(vpl)::value>;
+        k<<<chunk_grid(k, BK_WARPS * 32, smem, n, sms, BK_CHUNK), BK_WARPS * 32, smem, s>>>(A);
+    };
+    const int W = pick_width(F, {feat, grad_out, grad_feat});
+    const bool ok = W == 8 ? by_shape<8>(F / 8, launch) : by_shape<4>(F / 4, launch);
+    if (!ok) return TESS_ERR_INVALID_ARG;    // F a multiple of 4 that is not 4 * 2^k
     count_launch();
     return launch_status();
 }
@@ -540,21 +677,16 @@ tess_status edge_aggregate(const float* pos, int n, tess_box box, float rc, cons
     StageScope sc(ST_EDGE, s);
     const long long rows_blocks = ((long long)n + EDGE_WARPS - 1) / EDGE_WARPS;
     const int blocks = (int)std::min<long long>(rows_blocks, (long long)sms * 64);
-    const bool vec4 = (F % 4 == 0) && F <= 256 && aligned(feat, 16) && aligned(out, 16) && cap <= EV_MAXCAP;
-    const int vblocks = (int)std::min<long long>(((long long)n + EV_WARPS - 1) / EV_WARPS, (long long)sms * 32);
+    const bool vec = (F % 4 == 0) && F <= 256 && aligned(feat, 16) && aligned(out, 16) && cap <= EV_MAXCAP;
+    const size_t vsmem = (size_t)EV_WARPS * cap * sizeof(int2);
     bool launched = false;
-    if (vec4) {
-        launched = true;
-        switch (F / 4) {
-            case 1: edge_vec4_kernel<1, 1><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
-            case 2: edge_vec4_kernel<2, 1><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
-            case 4: edge_vec4_kernel<2, 2><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
-            case 8: edge_vec4_kernel<4, 2><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
-            case 16: edge_vec4_kernel<8, 2><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
-            case 32: edge_vec4_kernel<16, 2><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
-            case 64: edge_vec4_kernel<32, 2><<<vblocks, EV_WARPS * 32, 0, s>>>(A); break;
-            default: launched = false; break;
-        }
+    if (vec) {
+        auto launch = [&](auto w, auto lpe, auto vpl) {
+            auto* k = edge_vec_kernel<decltype(w)::value, decltype(lpe)::value, decltype(vpl)::value>;
+            k<<<chunk_grid(k, EV_WARPS * 32, vsmem, n, sms, EV_CHUNK), EV_WARPS * 32, vsmem, s>>>(A);
+        };
+        const int W = pick_width(F, {feat, out});
+        launched = W == 8 ? by_shape<8>(F / 8, launch) : by_shape<4>(F / 4, launch);
     }
     if (!launched) {
         if ((F % 2 == 0) && aligned(feat, 8) && F >= 64) edge_kernel<2><<<blocks, EDGE_WARPS * 32, 0, s>>>(A);
