@@ -270,6 +270,46 @@ def run_cuda(args, world, rank, local):
         bbytes = s.n * (3 * 4 * s.F + 16 + 4 * mean_count + 4 + 12)
         backward = {"ms": bms, "algorithmic_bytes": bbytes, "achieved_gbs": bbytes / (bms / 1e3) / 1e9}
 
+    resort = None
+    if args.resort:
+        # the re-sort at the next rebuild: every atom moved by a rebuild
+        # interval of the trajectory's random walk (20 steps of sigma per axis)
+        L = torch.tensor(s.box, dtype=torch.float64, device=dev)
+        x = step.pos3.double() + torch.randn(step.pos3.shape, generator=torch.Generator(device=dev).manual_seed(4),
+                                             device=dev, dtype=torch.float64) * (s.sigma * 20 ** 0.5)
+        pos1 = (x - L * torch.floor(x / L)).float()
+        pos1 = torch.where(pos1 >= L.float(), torch.zeros_like(pos1), pos1).contiguous()
+        perm0, keys0 = step.perm.clone(), step.keys.clone()
+        ws_rs = torch.empty(tess.tess_hilbert_resort_workspace(s.n), dtype=torch.uint8, device=dev)
+        perm1 = torch.empty_like(perm0)
+        keys1 = torch.empty_like(keys0)
+        ps1 = torch.empty((s.n, 4), dtype=torch.float32, device=dev)
+        st1 = torch.empty(1, dtype=torch.int32, device=dev)
+        import ctypes
+        P = lambda t: ctypes.c_void_p(t.data_ptr())
+        stc = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        calls = {
+            "full_sort": lambda: tess.tess_hilbert_sort(P(pos1), s.n, s.box, 10, P(step.ws_sort), step.ws_sort.numel(),
+                                                        P(perm1), P(keys1), P(ps1), P(st1), stc),
+            "resort": lambda: tess.tess_hilbert_resort(P(pos1), s.n, s.box, 10, P(perm0), P(keys0), P(ws_rs),
+                                                       ws_rs.numel(), P(perm1), P(keys1), P(ps1), P(st1), stc),
+        }
+        resort = {"sigma_total": s.sigma * 20 ** 0.5}
+        for name, call in calls.items():
+            for _ in range(args.warmup):
+                assert call() == 0
+            rev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            for k in range(args.steps):
+                flush.zero_()
+                rev[k][0].record()
+                call()
+                rev[k][1].record()
+            torch.cuda.synchronize()
+            resort[name + "_ms"] = sum(a.elapsed_time(b) for a, b in rev) / args.steps
+            if name == "resort":
+                resort["incremental_path"] = not (int(st1.item()) & tess.TESS_DEV_FULL_SORT)
+
     graph = None
     if args.graph:
         # the same step captured once as a CUDA graph and replayed
@@ -378,6 +418,7 @@ def run_cuda(args, world, rank, local):
             "gpu_launches": launches,
             "graph": graph,
             "backward": backward,
+            "resort": resort,
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -495,6 +536,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph", action="store_true", help="also time the step captured as one CUDA graph")
     ap.add_argument("--backward", action="store_true", help="also time the aggregation's backward on the same list")
+    ap.add_argument("--resort", action="store_true",
+                    help="also time the incremental re-sort against the full sort a rebuild interval later")
     args = ap.parse_args(argv)
     world, rank, local = _dist_setup(args)
     if args.impl == "reference":

@@ -60,6 +60,7 @@ typedef struct {
 #define TESS_DEV_OVERFLOW   1   /* some neighbor count exceeded max_neighbors */
 #define TESS_DEV_BAD_INPUT  2   /* some position outside [0, L) or not finite (clamped into the grid) */
 #define TESS_DEV_TIMEOUT    4   /* an inter-block wait gave up; outputs of that call are invalid */
+#define TESS_DEV_FULL_SORT  8   /* tess_hilbert_resort ran the full sort (its fast path did not apply) */
 
 /* tess_build_neighbors flags */
 #define TESS_NO_PAD_FILL    1   /* leave slots >= min(count, max_neighbors) unwritten */
@@ -104,6 +105,40 @@ tess_status tess_hilbert_sort(const float* pos, int n, tess_box box, int bits,
                               void* ws, size_t ws_bytes,
                               int32_t* perm, uint32_t* keys_sorted, float* pos_sorted,
                               int32_t* dev_status, tess_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Incremental Hilbert re-sort -- the re-sort at a rebuild, after the atoms
+ * have moved a little since the previous sort (Tessera re-sorts along its
+ * curve at every rebuild; Tessera, abstract).
+ *
+ * Output: exactly what tess_hilbert_sort(pos, n, box, bits, ...) writes for
+ * the same positions (perm, keys_sorted, pos_sorted, dev_status bits), for
+ * any perm_prev / keys_prev.  It runs faster when they are the perm and
+ * keys_sorted of an earlier sort of the same n atoms whose positions moved
+ * little since: the call then starts from that order, fixes the atoms whose
+ * key stayed within their old neighbors' keys with local block sorts, radix
+ * sorts the few others and merges the two.  Its checks run on the device;
+ * when one fails (perm_prev not a permutation, more than n/8 + 1024 atoms
+ * far from their old place, a local run out of order) the call runs the full
+ * sort instead and sets TESS_DEV_FULL_SORT in *dev_status.  No host
+ * synchronisation either way.
+ *
+ *   pos        [n, 3] float, device, CURRENT positions in the original
+ *              (unsorted) index order -- the same input as tess_hilbert_sort
+ *   perm_prev  [n] int32, device: the earlier sort's perm
+ *   keys_prev  [n] uint32, device: the earlier sort's keys_sorted
+ *   perm, keys_sorted, pos_sorted, dev_status: as tess_hilbert_sort; they
+ *              must not overlap perm_prev / keys_prev
+ *   ws         tess_hilbert_resort_workspace(n) bytes, 256-byte aligned
+ *              (about 19 n bytes plus small tables)
+ * Errors: as tess_hilbert_sort, plus INVALID_ARG if perm_prev or keys_prev
+ * is NULL.
+ * ------------------------------------------------------------------------- */
+size_t tess_hilbert_resort_workspace(int n);
+tess_status tess_hilbert_resort(const float* pos, int n, tess_box box, int bits, const int32_t* perm_prev,
+                                const uint32_t* keys_prev, void* ws, size_t ws_bytes, int32_t* perm,
+                                uint32_t* keys_sorted, float* pos_sorted, int32_t* dev_status,
+                                tess_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Morton (Z-order) sort -- the curve the Tessera abstract compares against:
@@ -259,7 +294,8 @@ tess_status tess_edge_aggregate_backward(const float* pos, int n, tess_box box, 
  * events on its stream around its kernels; tess_stage_times adds the elapsed
  * times of all recorded calls per stage (this synchronises on the events)
  * and clears them.  Stages: 0 space-filling-curve keys, 1 key sort, 2 cell
- * binning, 3 pair search, 4 skin check, 5 edge aggregate, 6 aggregate backward.  Returns the number of
+ * binning, 3 pair search, 4 skin check, 5 edge aggregate, 6 aggregate backward,
+ * 7 incremental re-sort (its fallback full sort records under 0 and 1).  Returns the number of
  * stages written (<= max_stages).  ms_out[k] = total milliseconds,
  * calls_out[k] (nullable) = number of timed calls.
  * ------------------------------------------------------------------------- */

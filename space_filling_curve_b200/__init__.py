@@ -23,6 +23,7 @@ __all__ = [
     "TessError", "lib", "library_path", "Box",
     "tess_status_string", "tess_version", "tess_kernel_launch_count",
     "tess_hilbert_sort_workspace", "tess_hilbert_sort", "tess_hilbert_sort_static", "HILBERT_SORT_STATIC_MAX_N",
+    "tess_hilbert_resort_workspace", "tess_hilbert_resort", "hilbert_resort", "TESS_DEV_FULL_SORT",
     "tess_morton_sort", "morton_sort",
     "tess_build_neighbors_workspace", "tess_build_neighbors",
     "tess_skin_check", "tess_edge_aggregate", "tess_stage_timing", "tess_stage_times",
@@ -35,11 +36,13 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libtess.so")
 
 TESS_DEV_OVERFLOW = 1
+TESS_DEV_FULL_SORT = 8
 TESS_DEV_BAD_INPUT = 2
 TESS_DEV_TIMEOUT = 4
 TESS_NO_PAD_FILL = 1
 TESS_TILE_SEARCH = 2
-STAGES = ("hilbert_keys", "key_sort", "cell_binning", "pair_search", "skin_check", "edge_aggregate", "edge_backward")
+STAGES = ("hilbert_keys", "key_sort", "cell_binning", "pair_search", "skin_check", "edge_aggregate", "edge_backward",
+          "resort")
 _STATUS = {0: "ok", 1: "invalid argument", 2: "box too small", 3: "workspace too small", 4: "CUDA launch error",
            5: "n above the static scratch capacity"}
 HILBERT_SORT_STATIC_MAX_N = 1 << 20
@@ -78,6 +81,10 @@ def lib() -> ctypes.CDLL:
     L.tess_hilbert_sort_workspace.restype = sz
     L.tess_hilbert_sort.argtypes = [P, i32, Box, i32, P, sz, P, P, P, P, P]
     L.tess_hilbert_sort.restype = i32
+    L.tess_hilbert_resort_workspace.argtypes = [i32]
+    L.tess_hilbert_resort_workspace.restype = sz
+    L.tess_hilbert_resort.argtypes = [P, i32, Box, i32, P, P, P, sz, P, P, P, P, P]
+    L.tess_hilbert_resort.restype = i32
     L.tess_morton_sort.argtypes = [P, i32, Box, i32, P, sz, P, P, P, P, P]
     L.tess_morton_sort.restype = i32
     L.tess_hilbert_sort_static.argtypes = [P, i32, Box, i32, P, P, P, P, P]
@@ -123,6 +130,16 @@ def tess_kernel_launch_count() -> int:
 
 def tess_hilbert_sort_workspace(n: int) -> int:
     return int(lib().tess_hilbert_sort_workspace(int(n)))
+
+
+def tess_hilbert_resort_workspace(n: int) -> int:
+    return int(lib().tess_hilbert_resort_workspace(int(n)))
+
+
+def tess_hilbert_resort(pos, n, box, bits, perm_prev, keys_prev, ws, ws_bytes, perm, keys_sorted, pos_sorted,
+                        dev_status, stream) -> int:
+    return int(lib().tess_hilbert_resort(pos, n, _box(box), bits, perm_prev, keys_prev, ws, ws_bytes, perm,
+                                         keys_sorted, pos_sorted, dev_status, stream))
 
 
 def tess_hilbert_sort(pos, n, box, bits, ws, ws_bytes, perm, keys_sorted, pos_sorted, dev_status, stream) -> int:
@@ -243,6 +260,31 @@ def hilbert_sort(pos, box, bits: int = 10, *, ws=None, perm=None, keys_sorted=No
     code = fn(_ptr(pos), n, box, bits, _ptr(ws), ws.numel() * ws.element_size(), _ptr(perm), _ptr(keys_sorted),
               _ptr(pos_sorted), _ptr(dev_status), _stream(stream))
     _check(fn.__name__, code)
+    return perm, keys_sorted, pos_sorted, dev_status
+
+
+def hilbert_resort(pos, box, perm_prev, keys_prev, bits: int = 10, *, ws=None, perm=None, keys_sorted=None,
+                   pos_sorted=None, dev_status=None, want_pos: bool = True, stream=None):
+    """Re-sort after the atoms moved, starting from an earlier sort's (perm,
+    keys).  Same outputs as hilbert_sort for the same ``pos``; dev_status
+    carries TESS_DEV_FULL_SORT when the full sort ran instead of the
+    incremental one."""
+    torch = _torch()
+    _need_cuda("pos", pos, torch.float32, 3)
+    _need_cuda("perm_prev", perm_prev, torch.int32)
+    _need_cuda("keys_prev", keys_prev, torch.int32)
+    n = pos.shape[0]
+    dev = pos.device
+    ws = _workspace(tess_hilbert_resort_workspace(n), dev, ws)
+    perm = torch.empty(n, dtype=torch.int32, device=dev) if perm is None else perm
+    keys_sorted = torch.empty(n, dtype=torch.int32, device=dev) if keys_sorted is None else keys_sorted
+    if want_pos and pos_sorted is None:
+        pos_sorted = torch.empty((n, 4), dtype=torch.float32, device=dev)
+    dev_status = torch.empty(1, dtype=torch.int32, device=dev) if dev_status is None else dev_status
+    code = tess_hilbert_resort(_ptr(pos), n, box, bits, _ptr(perm_prev), _ptr(keys_prev), _ptr(ws),
+                               ws.numel() * ws.element_size(), _ptr(perm), _ptr(keys_sorted), _ptr(pos_sorted),
+                               _ptr(dev_status), _stream(stream))
+    _check("tess_hilbert_resort", code)
     return perm, keys_sorted, pos_sorted, dev_status
 
 

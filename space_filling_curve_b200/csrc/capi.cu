@@ -9,6 +9,10 @@ namespace tess {
 std::atomic<long long> g_launches{0};
 
 size_t hilbert_sort_workspace(int n);
+size_t hilbert_resort_workspace(int n);
+tess_status hilbert_resort(const float* pos, int n, tess_box box, int bits, const int32_t* perm_prev,
+                           const uint32_t* keys_prev, void* ws, size_t ws_bytes, int32_t* perm,
+                           uint32_t* keys_sorted, float* pos_sorted, int32_t* dev_status, cudaStream_t s);
 tess_status hilbert_sort(const float* pos, int n, tess_box box, int bits, void* ws, size_t ws_bytes, int32_t* perm,
                          uint32_t* keys_sorted, float* pos_sorted, int32_t* dev_status, cudaStream_t s);
 tess_status morton_sort(const float* pos, int n, tess_box box, int bits, void* ws, size_t ws_bytes, int32_t* perm,
@@ -91,6 +95,16 @@ tess_status tess_hilbert_sort(const float* pos, int n, tess_box box, int bits, v
                               tess_stream_t stream) {
     return hilbert_sort(pos, n, box, bits, ws, ws_bytes, perm, keys_sorted, pos_sorted, dev_status,
                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t tess_hilbert_resort_workspace(int n) { return hilbert_resort_workspace(n); }
+
+tess_status tess_hilbert_resort(const float* pos, int n, tess_box box, int bits, const int32_t* perm_prev,
+                                const uint32_t* keys_prev, void* ws, size_t ws_bytes, int32_t* perm,
+                                uint32_t* keys_sorted, float* pos_sorted, int32_t* dev_status,
+                                tess_stream_t stream) {
+    return hilbert_resort(pos, n, box, bits, perm_prev, keys_prev, ws, ws_bytes, perm, keys_sorted, pos_sorted,
+                          dev_status, reinterpret_cast<cudaStream_t>(stream));
 }
 
 tess_status tess_morton_sort(const float* pos, int n, tess_box box, int bits, void* ws, size_t ws_bytes,

@@ -84,7 +84,10 @@ template <int CURVE>   // 0 Hilbert, 1 Morton
 __global__ __launch_bounds__(KEYS_THREADS) void keys_kernel(const float* __restrict__ pos, int n, float3 scale,
                                                             float3 L, int bits, int npass,
                                                             unsigned long long* __restrict__ elems,
-                                                            unsigned* __restrict__ hist, int32_t* status) {
+                                                            unsigned* __restrict__ hist, int32_t* status,
+                                                            const int32_t* gate, int want) {
+    // gate: when given, the kernel runs only if *gate == want
+    if (gate && *gate != want) return;
     __shared__ unsigned sh[MAX_PASSES][RADIX];
     for (int k = threadIdx.x; k < MAX_PASSES * RADIX; k += blockDim.x) (&sh[0][0])[k] = 0u;
     __syncthreads();
@@ -144,16 +147,22 @@ __device__ __forceinline__ unsigned block_excl_scan256(unsigned v, unsigned* s_w
     return wpre + x - v;
 }
 
-struct SortShared {
-    unsigned long long elems[SORT_TILE];
+template <int ITEMS>
+struct SortSharedT {
+    unsigned long long elems[SORT_THREADS * ITEMS];
     unsigned wcnt[SORT_WARPS][RADIX];
     unsigned lbase[RADIX];
     unsigned long long gbase[RADIX];
     unsigned scan_tmp[SORT_WARPS];
     int tile;
 };
+using SortShared = SortSharedT<SORT_ITEMS>;
 
-template <bool FINAL>
+// One counting pass of the LSD sort over 64-bit elements: digit =
+// (element >> shift) & 0xff.  n_dev, when given, holds the element count
+// (the grid may then have more tiles than needed: tiles past the end return);
+// gate, when given, runs the pass only if *gate == want.
+template <bool FINAL, int ITEMS = SORT_ITEMS>
 __global__ __launch_bounds__(SORT_THREADS, 3) void onesweep_pass(const unsigned long long* __restrict__ in,
                                                               unsigned long long* __restrict__ out, int n, int shift,
                                                               const unsigned* __restrict__ hist,
@@ -161,29 +170,34 @@ __global__ __launch_bounds__(SORT_THREADS, 3) void onesweep_pass(const unsigned 
                                                               int32_t* status, int32_t* __restrict__ perm,
                                                               uint32_t* __restrict__ keys_out,
                                                               float4* __restrict__ pos_sorted,
-                                                              const float* __restrict__ pos3) {
+                                                              const float* __restrict__ pos3, const int* n_dev,
+                                                              const int32_t* gate, int want) {
+    constexpr int TILE = SORT_THREADS * ITEMS;
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    SortShared& S = *reinterpret_cast<SortShared*>(smem_raw);
+    SortSharedT<ITEMS>& S = *reinterpret_cast<SortSharedT<ITEMS>*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    if (gate && *gate != want) return;
+    if (n_dev) n = *n_dev;
 
     if (tid == 0) S.tile = (int)atomicAdd(tile_counter, 1u);
     for (int k = tid; k < SORT_WARPS * RADIX; k += SORT_THREADS) (&S.wcnt[0][0])[k] = 0u;
     __syncthreads();
     const int tile = S.tile;
-    const long long base = (long long)tile * SORT_TILE;
-    const long long wbase = base + (long long)warp * SORT_ITEMS * 32;
+    const long long base = (long long)tile * TILE;
+    if (base >= n) return;     // a spare tile of a device-sized launch
+    const long long wbase = base + (long long)warp * ITEMS * 32;
 
-    unsigned long long e[SORT_ITEMS];
-    unsigned rank[SORT_ITEMS];
+    unsigned long long e[ITEMS];
+    unsigned rank[ITEMS];
 #pragma unroll
-    for (int k = 0; k < SORT_ITEMS; ++k) {
+    for (int k = 0; k < ITEMS; ++k) {
         const long long idx = wbase + k * 32 + lane;
         e[k] = idx < n ? in[idx] : ~0ull;
     }
 #pragma unroll
-    for (int k = 0; k < SORT_ITEMS; ++k) {
+    for (int k = 0; k < ITEMS; ++k) {
         const bool valid = (wbase + k * 32 + lane) < n;
-        const unsigned d = (unsigned)(e[k] >> (32 + shift)) & 0xffu;
+        const unsigned d = (unsigned)(e[k] >> shift) & 0xffu;
         const unsigned act = __ballot_sync(FULL, valid);
         rank[k] = 0;
         if (valid) {
@@ -244,18 +258,18 @@ __global__ __launch_bounds__(SORT_THREADS, 3) void onesweep_pass(const unsigned 
 
     // digit-sorted copy of the tile in shared memory
 #pragma unroll
-    for (int k = 0; k < SORT_ITEMS; ++k) {
+    for (int k = 0; k < ITEMS; ++k) {
         if ((wbase + k * 32 + lane) < n) {
-            const unsigned d = (unsigned)(e[k] >> (32 + shift)) & 0xffu;
+            const unsigned d = (unsigned)(e[k] >> shift) & 0xffu;
             S.elems[S.lbase[d] + S.wcnt[warp][d] + rank[k]] = e[k];
         }
     }
     __syncthreads();
 
-    const int tile_n = (int)min((long long)SORT_TILE, (long long)n - base);
+    const int tile_n = (int)min((long long)TILE, (long long)n - base);
     for (int s = tid; s < tile_n; s += SORT_THREADS) {
         const unsigned long long v = S.elems[s];
-        const unsigned d = (unsigned)(v >> (32 + shift)) & 0xffu;
+        const unsigned d = (unsigned)(v >> shift) & 0xffu;
         const unsigned long long g = S.gbase[d] + (unsigned long long)(s - (int)S.lbase[d]);
         if (FINAL) {
             const unsigned idx = (unsigned)v;
@@ -308,34 +322,35 @@ size_t hilbert_sort_workspace(int n) {
     return sort_layout(nullptr, n).total;
 }
 
-tess_status sfc_sort(const float* pos, int n, tess_box box, int bits, int curve, void* ws, size_t ws_bytes,
-                     int32_t* perm, uint32_t* keys_sorted, float* pos_sorted, int32_t* dev_status, cudaStream_t s) {
-    if (n <= 0 || !pos || !perm || !ws || bits < 1 || bits > 10) return TESS_ERR_INVALID_ARG;
-    if (!finite_pos(box.lx) || !finite_pos(box.ly) || !finite_pos(box.lz)) return TESS_ERR_INVALID_ARG;
-    if (pos_sorted && !aligned(pos_sorted, 16)) return TESS_ERR_INVALID_ARG;
-    if (!aligned(ws, 256)) return TESS_ERR_INVALID_ARG;
-    SortLayout L = sort_layout(ws, n);
-    if (ws_bytes < L.total) return TESS_ERR_WORKSPACE_TOO_SMALL;
-    int32_t* status = dev_status ? dev_status : L.status;
-
-    cudaMemsetAsync(static_cast<char*>(ws) + L.zero_begin, 0, L.zero_bytes, s);
-    if (dev_status) cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s);
-
+static float3 grid_scale(tess_box box, int bits) {
     const float g = (float)(1u << bits);
-    const float3 scale = make_float3(g / box.lx, g / box.ly, g / box.lz);   // fp32 IEEE divisions
-    const int npass = passes_for(bits);
+    return make_float3(g / box.lx, g / box.ly, g / box.lz);   // fp32 IEEE divisions
+}
+
+static int sm_count() {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
+// The full sort's launches over a zeroed layout L; with a gate, every kernel
+// runs only if *gate == want.
+static void sfc_sort_launch(const float* pos, int n, tess_box box, int bits, int curve, const SortLayout& L,
+                            int32_t* perm, uint32_t* keys_sorted, float* pos_sorted, int32_t* status,
+                            const int32_t* gate, int want, cudaStream_t s) {
+    const float3 scale = grid_scale(box, bits);
+    const int npass = passes_for(bits);
+    const int sms = sm_count();
     {
         StageScope sc(ST_KEYS, s);
         const int blocks = (int)std::min<long long>(((long long)n + KEYS_THREADS - 1) / KEYS_THREADS, (long long)sms * 8);
         if (curve == 0)
             keys_kernel<0><<<blocks, KEYS_THREADS, 0, s>>>(pos, n, scale, make_float3(box.lx, box.ly, box.lz), bits,
-                                                           npass, L.a, L.hist, status);
+                                                           npass, L.a, L.hist, status, gate, want);
         else
             keys_kernel<1><<<blocks, KEYS_THREADS, 0, s>>>(pos, n, scale, make_float3(box.lx, box.ly, box.lz), bits,
-                                                           npass, L.a, L.hist, status);
+                                                           npass, L.a, L.hist, status, gate, want);
         count_launch();
     }
     {
@@ -349,17 +364,32 @@ tess_status sfc_sort(const float* pos, int n, tess_box box, int bits, int curve,
             unsigned long long* states = L.states + (size_t)p * tiles * RADIX;
             if (p == npass - 1) {
                 onesweep_pass<true><<<(unsigned)tiles, SORT_THREADS, smem, s>>>(
-                    src, nullptr, n, 8 * p, L.hist + p * RADIX, states, L.counters + p, status, perm, keys_sorted,
-                    reinterpret_cast<float4*>(pos_sorted), pos);
+                    src, nullptr, n, 32 + 8 * p, L.hist + p * RADIX, states, L.counters + p, status, perm,
+                    keys_sorted, reinterpret_cast<float4*>(pos_sorted), pos, nullptr, gate, want);
             } else {
                 onesweep_pass<false><<<(unsigned)tiles, SORT_THREADS, smem, s>>>(
-                    src, dst, n, 8 * p, L.hist + p * RADIX, states, L.counters + p, status, nullptr, nullptr,
-                    nullptr, nullptr);
+                    src, dst, n, 32 + 8 * p, L.hist + p * RADIX, states, L.counters + p, status, nullptr, nullptr,
+                    nullptr, nullptr, nullptr, gate, want);
             }
             count_launch();
             std::swap(src, dst);
         }
     }
+}
+
+tess_status sfc_sort(const float* pos, int n, tess_box box, int bits, int curve, void* ws, size_t ws_bytes,
+                     int32_t* perm, uint32_t* keys_sorted, float* pos_sorted, int32_t* dev_status, cudaStream_t s) {
+    if (n <= 0 || !pos || !perm || !ws || bits < 1 || bits > 10) return TESS_ERR_INVALID_ARG;
+    if (!finite_pos(box.lx) || !finite_pos(box.ly) || !finite_pos(box.lz)) return TESS_ERR_INVALID_ARG;
+    if (pos_sorted && !aligned(pos_sorted, 16)) return TESS_ERR_INVALID_ARG;
+    if (!aligned(ws, 256)) return TESS_ERR_INVALID_ARG;
+    SortLayout L = sort_layout(ws, n);
+    if (ws_bytes < L.total) return TESS_ERR_WORKSPACE_TOO_SMALL;
+    int32_t* status = dev_status ? dev_status : L.status;
+
+    cudaMemsetAsync(static_cast<char*>(ws) + L.zero_begin, 0, L.zero_bytes, s);
+    if (dev_status) cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s);
+    sfc_sort_launch(pos, n, box, bits, curve, L, perm, keys_sorted, pos_sorted, status, nullptr, 0, s);
     return launch_status();
 }
 
@@ -371,6 +401,525 @@ tess_status hilbert_sort(const float* pos, int n, tess_box box, int bits, void* 
 tess_status morton_sort(const float* pos, int n, tess_box box, int bits, void* ws, size_t ws_bytes, int32_t* perm,
                         uint32_t* keys_sorted, float* pos_sorted, int32_t* dev_status, cudaStream_t s) {
     return sfc_sort(pos, n, box, bits, 1, ws, ws_bytes, perm, keys_sorted, pos_sorted, dev_status, s);
+}
+
+// ---------------------------------------------------------------- incremental resort
+//
+// Re-sorts atoms that have moved since an earlier sort, starting from that
+// sort's order (perm_prev, keys_prev).  Each atom's composite element
+// (key << 32 | index) is unique, so the sorted order is unique and any exact
+// method reproduces the full sort.  Between rebuilds most atoms move by a
+// fraction of a grid cell, so their new key stays inside the range of old
+// keys of their old neighbors in the order: such "local" atoms (S) can only
+// be out of order with atoms at most 2 * RS_W old ranks away and are sorted
+// by two rounds of block sorts of RS_BLK elements (the second offset by half
+// a block).  The others (O, atoms whose key jumped along the curve: the
+// curve's neighboring cells can be far apart in key) are few; they are radix
+// sorted by the full 64-bit element and merged in by binary search.  Every
+// assumption is checked on the device: perm_prev must be a permutation, O
+// must fit its buffer and S must come out strictly increasing; otherwise a
+// device flag switches to the full sort, whose kernels are launched gated on
+// that flag (no host synchronisation either way).
+
+constexpr int RS_W = 64;                 // old-rank window of the key range
+constexpr int RS_D = 2 * RS_W;           // displacement bound of local atoms
+constexpr int RS_BLK = 2 * RS_D;         // 256 elements per block sort (one warp, 8 per lane)
+constexpr int RS_THREADS = 256;
+constexpr int RS_TILE = 1024;            // elements per classify / compact block
+
+struct ResortCtl {
+    int32_t fallback;    // 1: the fast path's assumptions failed, run the full sort
+    int32_t m_local;     // |S|
+    int32_t m_out;       // |O|
+    int32_t pad;
+};
+
+__device__ __forceinline__ int block_sum256(int v, int* s_red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+    if (lane == 0) s_red[warp] = v;
+    __syncthreads();
+    int t = 0;
+#pragma unroll
+    for (int w = 0; w < RS_THREADS / 32; ++w) t += s_red[w];
+    __syncthreads();
+    return t;
+}
+
+// Composite elements in the previous order, local flags, per-tile local
+// counts.  An index of perm_prev outside [0, n) switches to the full sort;
+// a repeated index is caught later (two equal elements meet in the runs'
+// order checks or in the merge), so perm_prev is a permutation whenever
+// the fast path completes.
+__global__ __launch_bounds__(RS_THREADS) void resort_classify(const float* __restrict__ pos, int n, float3 scale,
+                                                              float3 L, int bits,
+                                                              const int32_t* __restrict__ perm_prev,
+                                                              const uint32_t* __restrict__ keys_prev,
+                                                              unsigned long long* __restrict__ elems,
+                                                              uint8_t* __restrict__ local,
+                                                              int* __restrict__ tile_cnt, ResortCtl* ctl,
+                                                              int32_t* status) {
+    __shared__ int s_red[RS_THREADS / 32];
+    const long long base = (long long)blockIdx.x * RS_TILE;
+    const uint32_t top = (1u << bits) - 1u;
+    constexpr int U = RS_TILE / RS_THREADS;
+    int cnt = 0;
+    bool bad = false, broken = false;
+    int idx[U];
+    float px[U], py[U], pz[U];
+    uint32_t lo[U], hi[U];
+    // all loads of the thread's elements first, so that their latencies overlap
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const long long k = base + u * RS_THREADS + threadIdx.x;
+        idx[u] = k < n ? perm_prev[k] : 0;
+        if (idx[u] < 0 || idx[u] >= n) {
+            broken = true;
+            idx[u] = 0;
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const long long k = base + u * RS_THREADS + threadIdx.x;
+        const long long kk = k < n ? k : n - 1;
+        px[u] = pos[3 * (size_t)idx[u]];
+        py[u] = pos[3 * (size_t)idx[u] + 1];
+        pz[u] = pos[3 * (size_t)idx[u] + 2];
+        lo[u] = keys_prev[kk >= RS_W ? kk - RS_W : 0];
+        hi[u] = keys_prev[kk + RS_W < n ? kk + RS_W : n - 1];
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const long long k = base + u * RS_THREADS + threadIdx.x;
+        if (k >= n) break;
+        const float x = px[u], y = py[u], z = pz[u];
+        bad |= !(x >= 0.0f && x < L.x && y >= 0.0f && y < L.y && z >= 0.0f && z < L.z);
+        const uint32_t key =
+            hilbert_key(quantize(x, scale.x, top), quantize(y, scale.y, top), quantize(z, scale.z, top), bits);
+        elems[k] = ((unsigned long long)key << 32) | (unsigned)idx[u];
+        const bool loc = key >= lo[u] && key <= hi[u];
+        local[k] = loc ? 1 : 0;
+        cnt += loc ? 1 : 0;
+    }
+    if (__any_sync(FULL, bad) && (threadIdx.x & 31) == 0 && status) atomicOr(status, TESS_DEV_BAD_INPUT);
+    if (broken) atomicExch(&ctl->fallback, 1);
+    const int total = block_sum256(cnt, s_red);
+    if (threadIdx.x == 0) tile_cnt[blockIdx.x] = total;
+}
+
+// Exclusive scan of the per-tile local counts (one block of 1024 threads);
+// sizes of S and O; O larger than its buffer switches to the full sort.
+__global__ __launch_bounds__(1024) void resort_scan(int* tile_cnt, int ntiles, int n, int cap_out, ResortCtl* ctl) {
+    __shared__ int s_warp[32];
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int per = (ntiles + 1023) / 1024;
+    const int b0 = min(t * per, ntiles), b1 = min(b0 + per, ntiles);
+    int sum = 0;
+    for (int b = b0; b < b1; ++b) sum += tile_cnt[b];
+    int x = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(FULL, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) s_warp[warp] = x;
+    __syncthreads();
+    int wpre = 0;
+    for (int w = 0; w < warp; ++w) wpre += s_warp[w];
+    int run = wpre + x - sum;
+    for (int b = b0; b < b1; ++b) {
+        const int c = tile_cnt[b];
+        tile_cnt[b] = run;
+        run += c;
+    }
+    if (t == 1023) {
+        const int m_local = wpre + x;
+        ctl->m_local = m_local;
+        ctl->m_out = n - m_local;
+        if (n - m_local > cap_out) atomicExch(&ctl->fallback, 1);
+    }
+}
+
+// O is radix sorted by its key bytes (stable, in O's own order); equal keys
+// whose indices come out descending are caught in the merge.
+// Splits the elements into S and O in order (per-tile offsets from
+// resort_scan) and builds O's digit histograms.
+__global__ __launch_bounds__(RS_THREADS) void resort_compact(const unsigned long long* __restrict__ elems,
+                                                             const uint8_t* __restrict__ local, int n,
+                                                             const int* __restrict__ tile_off,
+                                                             unsigned long long* __restrict__ S,
+                                                             unsigned long long* __restrict__ O, int npass,
+                                                             unsigned* ohist, const ResortCtl* ctl) {
+    __shared__ int s_warp[RS_THREADS / 32];
+    __shared__ unsigned sh[2 * MAX_PASSES][RADIX];
+    if (ctl->fallback) return;
+    for (int k = threadIdx.x; k < 2 * MAX_PASSES * RADIX; k += RS_THREADS) (&sh[0][0])[k] = 0u;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const long long base = (long long)blockIdx.x * RS_TILE;
+    constexpr int PER = RS_TILE / RS_THREADS;     // consecutive elements per thread
+    const long long k0 = base + (long long)t * PER;
+    int f[PER];
+    int c = 0;
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        f[u] = (k0 + u < n) ? local[k0 + u] : 0;
+        c += f[u];
+    }
+    int x = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(FULL, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) s_warp[warp] = x;
+    __syncthreads();
+    int wpre = 0;
+#pragma unroll
+    for (int w = 0; w < RS_THREADS / 32; ++w) wpre += (w < warp) ? s_warp[w] : 0;
+    const int pre_local = wpre + x - c;                          // local atoms of this tile before thread t
+    const long long valid_before = min((long long)t * PER, max(0ll, (long long)n - base));
+    long long si = (long long)tile_off[blockIdx.x] + pre_local;
+    long long oi = (base - tile_off[blockIdx.x]) + (valid_before - pre_local);
+#pragma unroll
+    for (int u = 0; u < PER; ++u) {
+        if (k0 + u >= n) break;
+        const unsigned long long v = elems[k0 + u];
+        if (f[u]) {
+            S[si++] = v;
+        } else {
+            O[oi++] = v;
+            for (int p = 0; p < npass; ++p) atomicAdd(&sh[p][(unsigned)(v >> (32 + 8 * p)) & 0xffu], 1u);
+        }
+    }
+    __syncthreads();
+    for (int k = threadIdx.x; k < npass * RADIX; k += RS_THREADS) {
+        const unsigned v = (&sh[0][0])[k];
+        if (v) atomicAdd(&ohist[k], v);
+    }
+}
+
+__device__ __forceinline__ unsigned long long shfl_xor_u64(unsigned long long v, int m) {
+    const unsigned lo = __shfl_xor_sync(FULL, (unsigned)v, m);
+    const unsigned hi = __shfl_xor_sync(FULL, (unsigned)(v >> 32), m);
+    return ((unsigned long long)hi << 32) | lo;
+}
+
+// Sorts blocks of S in place, one warp per block of RS_BLK elements held in
+// registers (lane l holds positions 8l .. 8l+7), with a bitonic network.
+// Round 0: blocks at multiples of RS_BLK; round 1: the same shifted by RS_D
+// (the first block is [0, RS_D)).  Missing elements are padded with the
+// largest value, so they sort last and are not written back.  Global memory
+// is read and written in coalesced stripes (lane l: positions l + 32r) and
+// transposed through shared memory, skewed by one slot per 8 against bank
+// conflicts.
+__device__ __forceinline__ int rs_skew(int p) { return p + (p >> 3); }
+
+template <int ROUND>
+__global__ __launch_bounds__(RS_THREADS) void resort_block_sort(unsigned long long* __restrict__ S,
+                                                                const ResortCtl* ctl) {
+    __shared__ unsigned long long sx[RS_THREADS / 32][RS_BLK + RS_BLK / 8];
+    if (ctl->fallback) return;
+    const int m = ctl->m_local;
+    const int lane = threadIdx.x & 31;
+    unsigned long long* t = sx[threadIdx.x >> 5];
+    const long long wg = (long long)blockIdx.x * (RS_THREADS / 32) + (threadIdx.x >> 5);
+    // round 1: block w >= 1 starts at RS_D + (w - 1) * RS_BLK; its halves are
+    // the sorted second half of one round-0 block and the sorted first half
+    // of the next (the first RS_D elements are a sorted half already)
+    if (ROUND == 1 && wg == 0) return;
+    const long long start = ROUND == 0 ? wg * RS_BLK : RS_D + (wg - 1) * RS_BLK;
+    if (start >= m) return;
+    const long long len = min((long long)RS_BLK, (long long)m - start);
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const int p = 32 * r + lane;
+        t[rs_skew(p)] = p < len ? S[start + p] : ~0ull;
+    }
+    __syncwarp();
+    unsigned long long x[8];
+    if (ROUND == 0) {
+#pragma unroll
+        for (int r = 0; r < 8; ++r) x[r] = t[rs_skew(8 * lane + r)];
+    } else {
+        // second half reversed: the block becomes one bitonic sequence
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const int p = 8 * lane + r;
+            x[r] = t[rs_skew(p < RS_D ? p : 3 * RS_D - 1 - p)];
+        }
+    }
+#pragma unroll
+    for (int k = ROUND == 0 ? 2 : RS_BLK; k <= RS_BLK; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            if (j >= 8) {
+#pragma unroll
+                for (int r = 0; r < 8; ++r) {
+                    const int p = 8 * lane + r;
+                    const unsigned long long y = shfl_xor_u64(x[r], j >> 3);
+                    const bool lower = (p & j) == 0, asc = (p & k) == 0;
+                    x[r] = (lower == asc) ? (x[r] < y ? x[r] : y) : (x[r] < y ? y : x[r]);
+                }
+            } else {
+#pragma unroll
+                for (int r = 0; r < 8; ++r) {
+                    const int q = r ^ j;
+                    if (q > r) {
+                        const bool asc = ((8 * lane + r) & k) == 0;
+                        const unsigned long long a = x[r], b = x[q];
+                        const bool sw = asc ? (a > b) : (a < b);
+                        x[r] = sw ? b : a;
+                        x[q] = sw ? a : b;
+                    }
+                }
+            }
+        }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int r = 0; r < 8; ++r) t[rs_skew(8 * lane + r)] = x[r];
+    __syncwarp();
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const int p = 32 * r + lane;
+        if (p < len) S[start + p] = t[rs_skew(p)];
+    }
+}
+
+// S must be strictly increasing after the block sorts; otherwise fall back.
+__global__ __launch_bounds__(RS_THREADS) void resort_check(const unsigned long long* __restrict__ S, ResortCtl* ctl) {
+    if (ctl->fallback) return;
+    const long long m = ctl->m_local;
+    bool bad = false;
+    for (long long k = (long long)blockIdx.x * RS_THREADS + threadIdx.x; k + 1 < m; k += (long long)gridDim.x * RS_THREADS)
+        bad |= !(S[k] < S[k + 1]);
+    if (__any_sync(FULL, bad) && (threadIdx.x & 31) == 0) atomicExch(&ctl->fallback, 1);
+}
+
+// Number of elements of a[0..m) below v (a strictly increasing).
+__device__ __forceinline__ long long count_below(const unsigned long long* __restrict__ a, long long m,
+                                                 unsigned long long v) {
+    long long lo = 0, hi = m;
+    while (lo < hi) {
+        const long long mid = (lo + hi) >> 1;
+        if (a[mid] < v) lo = mid + 1;
+        else hi = mid;
+    }
+    return lo;
+}
+
+// Number of entries of c[0..m) that are <= t (c non-decreasing).
+template <class T>
+__device__ __forceinline__ int count_le(const T* c, int m, long long t) {
+    int lo = 0, hi = m;
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if ((long long)c[mid] <= t) lo = mid + 1;
+        else hi = mid;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ void write_sorted(long long g, unsigned long long v, const float* __restrict__ pos3,
+                                             int32_t* __restrict__ perm, uint32_t* __restrict__ keys_out,
+                                             float4* __restrict__ pos_sorted) {
+    const unsigned idx = (unsigned)v;
+    perm[g] = (int32_t)idx;
+    if (keys_out) keys_out[g] = (uint32_t)(v >> 32);
+    if (pos_sorted) {
+        const float* p = pos3 + 3 * (size_t)idx;
+        pos_sorted[g] = make_float4(p[0], p[1], p[2], 0.0f);
+    }
+}
+
+// Merge, part 1: each element of O (rank r) counts the elements of S below
+// it, c[r], and lands in slot r + c[r].  c is non-decreasing in r.  O must
+// be strictly increasing (equal keys in index order, no repeated element)
+// and share no element with S; otherwise the full sort runs (it rewrites
+// every output slot, and every slot written here is below n).
+__global__ __launch_bounds__(RS_THREADS) void resort_merge_out(const unsigned long long* __restrict__ S,
+                                                               const unsigned long long* __restrict__ Os,
+                                                               int* __restrict__ c_out, const ResortCtl* ctl,
+                                                               const float* __restrict__ pos3,
+                                                               int32_t* __restrict__ perm,
+                                                               uint32_t* __restrict__ keys_out,
+                                                               float4* __restrict__ pos_sorted, ResortCtl* ctl_w) {
+    if (ctl->fallback) return;
+    const long long ms = ctl->m_local, mo = ctl->m_out;
+    bool bad = false;
+    for (long long r = (long long)blockIdx.x * RS_THREADS + threadIdx.x; r < mo; r += (long long)gridDim.x * RS_THREADS) {
+        const unsigned long long v = Os[r];
+        const long long c = count_below(S, ms, v);
+        bad |= (c < ms && S[c] == v) || (r + 1 < mo && !(v < Os[r + 1]));
+        c_out[r] = (int)c;
+        write_sorted(r + c, v, pos3, perm, keys_out, pos_sorted);
+    }
+    if (__any_sync(FULL, bad) && (threadIdx.x & 31) == 0) atomicExch(&ctl_w->fallback, 1);
+}
+
+constexpr int RS_MERGE_SPAN = 4096;      // S elements per block in merge part 2
+constexpr int RS_MERGE_STAGE = 1024;     // O counts staged in shared memory per block
+
+// Merge, part 2: element t of S lands in slot t + #{r : c[r] <= t}.  A block
+// owns S[t0, t0 + RS_MERGE_SPAN); the c[r] that fall in that span are
+// staged in shared memory (searched in global memory if there are more).
+__global__ __launch_bounds__(RS_THREADS) void resort_merge_local(const unsigned long long* __restrict__ S,
+                                                                 const int* __restrict__ c_out, const ResortCtl* ctl,
+                                                                 const float* __restrict__ pos3,
+                                                                 int32_t* __restrict__ perm,
+                                                                 uint32_t* __restrict__ keys_out,
+                                                                 float4* __restrict__ pos_sorted, int32_t* status) {
+    __shared__ int s_c[RS_MERGE_STAGE];
+    __shared__ int s_lo, s_hi;
+    if (ctl->fallback) {
+        if (blockIdx.x == 0 && threadIdx.x == 0 && status) atomicOr(status, TESS_DEV_FULL_SORT);
+        return;
+    }
+    const long long ms = ctl->m_local;
+    const int mo = ctl->m_out;
+    for (long long t0 = (long long)blockIdx.x * RS_MERGE_SPAN; t0 < ms; t0 += (long long)gridDim.x * RS_MERGE_SPAN) {
+        const long long t1 = min(ms, t0 + RS_MERGE_SPAN);
+        if (threadIdx.x == 0) {
+            s_lo = count_le(c_out, mo, t0 - 1);        // O elements below S[t0]
+            s_hi = count_le(c_out, mo, t1 - 1);
+        }
+        __syncthreads();
+        const int lo = s_lo, cnt = s_hi - s_lo;
+        const bool staged = cnt <= RS_MERGE_STAGE;
+        if (staged)
+            for (int k = threadIdx.x; k < cnt; k += RS_THREADS) s_c[k] = c_out[lo + k];
+        __syncthreads();
+        constexpr int U = 4;
+        for (long long tb = t0 + threadIdx.x; tb < t1; tb += U * RS_THREADS) {
+            unsigned long long v[U];
+            float3 q[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const long long t = tb + u * RS_THREADS;
+                v[u] = t < t1 ? S[t] : 0ull;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const float* p = pos3 + 3 * (size_t)(unsigned)v[u];
+                q[u] = make_float3(p[0], p[1], p[2]);
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const long long t = tb + u * RS_THREADS;
+                if (t >= t1) break;
+                const int below = staged ? lo + count_le(s_c, cnt, t) : count_le(c_out, mo, t);
+                const long long g = t + below;
+                perm[g] = (int32_t)(unsigned)v[u];
+                if (keys_out) keys_out[g] = (uint32_t)(v[u] >> 32);
+                if (pos_sorted) pos_sorted[g] = make_float4(q[u].x, q[u].y, q[u].z, 0.0f);
+            }
+        }
+        __syncthreads();
+    }
+}
+
+struct ResortLayout {
+    SortLayout full;            // the full sort's buffers (fallback); full.a / full.b also hold elems / S
+    unsigned long long* o0;
+    unsigned long long* o1;
+    int* c_out;                 // [cap_out] S elements below each O element
+    uint8_t* local;
+    int* tile_cnt;
+    unsigned* ohist;            // [2 * MAX_PASSES][RADIX]
+    unsigned* ocounters;        // [2 * MAX_PASSES]
+    unsigned long long* ostates;  // [2 * MAX_PASSES][out tiles][RADIX]
+    ResortCtl* ctl;
+    size_t zero_begin, zero_bytes, total;
+    int cap_out;
+};
+
+static int resort_cap_out(int n) { return n / 8 + 1024; }
+
+static ResortLayout resort_layout(void* ws, int n) {
+    ResortLayout R{};
+    R.full = sort_layout(ws, n);
+    Carve c(ws);
+    c.off = R.full.total;
+    R.cap_out = resort_cap_out(n);
+    R.o0 = c.take<unsigned long long>((size_t)R.cap_out);
+    R.o1 = c.take<unsigned long long>((size_t)R.cap_out);
+    R.c_out = c.take<int>((size_t)R.cap_out);
+    R.local = c.take<uint8_t>((size_t)n);
+    const long long ntiles = ((long long)n + RS_TILE - 1) / RS_TILE;
+    R.tile_cnt = c.take<int>((size_t)ntiles);
+    c.off = align_up(c.off, 256);
+    R.zero_begin = c.off;
+    R.ohist = c.take<unsigned>(2 * MAX_PASSES * RADIX);
+    R.ocounters = c.take<unsigned>(2 * MAX_PASSES);
+    R.ctl = c.take<ResortCtl>(1);
+    R.ostates = c.take<unsigned long long>((size_t)2 * MAX_PASSES * (((size_t)R.cap_out + 1023) / 1024) * RADIX);
+    R.zero_bytes = c.off - R.zero_begin;
+    R.total = align_up(c.off, 256);
+    return R;
+}
+
+size_t hilbert_resort_workspace(int n) {
+    if (n <= 0) return 0;
+    return resort_layout(nullptr, n).total;
+}
+
+tess_status hilbert_resort(const float* pos, int n, tess_box box, int bits, const int32_t* perm_prev,
+                           const uint32_t* keys_prev, void* ws, size_t ws_bytes, int32_t* perm,
+                           uint32_t* keys_sorted, float* pos_sorted, int32_t* dev_status, cudaStream_t s) {
+    if (n <= 0 || !pos || !perm || !perm_prev || !keys_prev || !ws || bits < 1 || bits > 10)
+        return TESS_ERR_INVALID_ARG;
+    if (!finite_pos(box.lx) || !finite_pos(box.ly) || !finite_pos(box.lz)) return TESS_ERR_INVALID_ARG;
+    if (pos_sorted && !aligned(pos_sorted, 16)) return TESS_ERR_INVALID_ARG;
+    if (!aligned(ws, 256)) return TESS_ERR_INVALID_ARG;
+    ResortLayout R = resort_layout(ws, n);
+    if (ws_bytes < R.total) return TESS_ERR_WORKSPACE_TOO_SMALL;
+    int32_t* status = dev_status ? dev_status : R.full.status;
+    char* w = static_cast<char*>(ws);
+    cudaMemsetAsync(w + R.full.zero_begin, 0, R.full.zero_bytes, s);
+    cudaMemsetAsync(w + R.zero_begin, 0, R.zero_bytes, s);
+    if (dev_status) cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s);
+
+    const int sms = sm_count();
+    const int ntiles = (int)(((long long)n + RS_TILE - 1) / RS_TILE);
+    const int npass = passes_for(bits);
+    unsigned long long* elems = R.full.a;
+    unsigned long long* S = R.full.b;
+    {
+        StageScope sc(ST_RESORT, s);
+        resort_classify<<<ntiles, RS_THREADS, 0, s>>>(pos, n, grid_scale(box, bits),
+                                                      make_float3(box.lx, box.ly, box.lz), bits, perm_prev,
+                                                      keys_prev, elems, R.local, R.tile_cnt, R.ctl, status);
+        resort_scan<<<1, 1024, 0, s>>>(R.tile_cnt, ntiles, n, R.cap_out, R.ctl);
+        resort_compact<<<ntiles, RS_THREADS, 0, s>>>(elems, R.local, n, R.tile_cnt, S, R.o0, npass, R.ohist, R.ctl);
+        const long long warps1 = ((long long)n + RS_BLK - 1) / RS_BLK + 1;
+        const int bs_blocks = (int)((warps1 + RS_THREADS / 32 - 1) / (RS_THREADS / 32));
+        resort_block_sort<0><<<bs_blocks, RS_THREADS, 0, s>>>(S, R.ctl);
+        resort_block_sort<1><<<bs_blocks, RS_THREADS, 0, s>>>(S, R.ctl);
+        resort_check<<<sms * 4, RS_THREADS, 0, s>>>(S, R.ctl);
+        count_launch(6);
+        // O: LSD radix sort by key, gated on the fast path
+        constexpr int O_ITEMS = 4;     // small tiles: O is short, so more tiles run side by side
+        const long long otiles = ((long long)R.cap_out + SORT_THREADS * O_ITEMS - 1) / (SORT_THREADS * O_ITEMS);
+        unsigned long long* src = R.o0;
+        unsigned long long* dst = R.o1;
+        for (int p = 0; p < npass; ++p) {
+            onesweep_pass<false, O_ITEMS><<<(unsigned)otiles, SORT_THREADS, sizeof(SortSharedT<O_ITEMS>), s>>>(
+                src, dst, R.cap_out, 32 + 8 * p, R.ohist + p * RADIX,
+                R.ostates + (size_t)p * otiles * RADIX, R.ocounters + p, status, nullptr, nullptr, nullptr, nullptr,
+                &R.ctl->m_out, &R.ctl->fallback, 0);
+            std::swap(src, dst);
+        }
+        count_launch(npass);
+        resort_merge_out<<<sms * 2, RS_THREADS, 0, s>>>(S, src, R.c_out, R.ctl, pos, perm, keys_sorted,
+                                                        reinterpret_cast<float4*>(pos_sorted), R.ctl);
+        resort_merge_local<<<sms * 8, RS_THREADS, 0, s>>>(S, R.c_out, R.ctl, pos, perm, keys_sorted,
+                                                          reinterpret_cast<float4*>(pos_sorted), status);
+        count_launch(2);
+    }
+    // the full sort, run only when the fast path's checks failed
+    sfc_sort_launch(pos, n, box, bits, 0, R.full, perm, keys_sorted, pos_sorted, status, &R.ctl->fallback, 1, s);
+    return launch_status();
 }
 
 }  // namespace tess
