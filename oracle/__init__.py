@@ -81,6 +81,7 @@ def lib():
         L.oracle_cutoff_deriv.argtypes = [ctypes.c_double, ctypes.c_double]
         L.oracle_cutoff_deriv.restype = ctypes.c_double
         L.oracle_edge_backward.argtypes = [P, i32, i64, P, f32, P, P, i32, P, P, i32, P, P]
+        L.oracle_min_pair.argtypes = [P, i32, i64, P, P, P, i32, P, P, P]
         _lib = L
     return _lib
 
@@ -320,4 +321,19 @@ def edge_backward(pos, box, rc, nbr, counts, feat, grad_out):
     lib().oracle_edge_backward(_ptr(pos), stride, n, _ptr(b), float(rc), _ptr(nbr), _ptr(counts), int(cap),
                                _ptr(feat), _ptr(g), int(F), _ptr(gf), _ptr(gp))
     return gf, gp
+
+
+def min_pair(pos, box, nbr, counts):
+    """Closest listed pair: (r2 fp64, i, j); (inf, -1, -1) when nothing is listed."""
+    pos, stride = _pos(pos)
+    b = _box(box)
+    nbr = np.ascontiguousarray(nbr, dtype=np.int32)
+    counts = np.ascontiguousarray(counts, dtype=np.int32)
+    n, cap = nbr.shape
+    r2 = ctypes.c_double(0.0)
+    i = ctypes.c_int32(0)
+    j = ctypes.c_int32(0)
+    lib().oracle_min_pair(_ptr(pos), stride, n, _ptr(b), _ptr(nbr), _ptr(counts), int(cap), ctypes.byref(r2),
+                          ctypes.byref(i), ctypes.byref(j))
+    return float(r2.value), int(i.value), int(j.value)
 

@@ -638,3 +638,42 @@ void oracle_edge_backward(const float* pos, int stride, int64_t n, const float* 
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* Closest listed pair (a structural check: Tessera's runs are checked for   */
+/* atoms that come anomalously close; Tessera, abstract)                     */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Over every listed (i, j) -- the first min(counts[i], cap) entries of row
+ * i, entries < 0 or >= n skipped -- the smallest squared minimum-image
+ * distance, computed as the list computes it (pair_r2, fp64 from the fp32
+ * coordinates), and the pair that has it: ties go to the smallest i, then
+ * the smallest j.  No listed pair: *r2 = +infinity, *pi = *pj = -1.
+ * READING: the pages only say that close pairs were looked for; the
+ * closest listed pair is the plainest quantity that says whether there is
+ * one.
+ */
+void oracle_min_pair(const float* pos, int stride, int64_t n, const float* L, const int32_t* nbr,
+                     const int32_t* counts, int cap, double* r2, int32_t* pi, int32_t* pj)
+{
+    const double Ld[3] = {L[0], L[1], L[2]};
+    double best = 1.0 / 0.0;
+    int32_t bi = -1, bj = -1;
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t m = counts[i] < cap ? counts[i] : cap;
+        for (int64_t s = 0; s < m; ++s) {
+            int32_t j = nbr[i * cap + s];
+            if (j < 0 || j >= n) continue;
+            double d = pair_r2(pos + i * stride, pos + (int64_t)j * stride, Ld);
+            if (d < best || (d == best && (i < bi || (i == bi && j < bj)))) {
+                best = d;
+                bi = (int32_t)i;
+                bj = j;
+            }
+        }
+    }
+    *r2 = best;
+    *pi = bi;
+    *pj = bj;
+}
+
