@@ -310,6 +310,30 @@ def run_cuda(args, world, rank, local):
             if name == "resort":
                 resort["incremental_path"] = not (int(st1.item()) & tess.TESS_DEV_FULL_SORT)
 
+    monitor = None
+    if args.monitor:
+        # the closest listed pair on the step's list
+        mws = torch.empty(tess.tess_min_pair_distance_workspace(), dtype=torch.uint8, device=dev)
+        r2m = torch.empty(1, dtype=torch.float64, device=dev)
+        pairm = torch.empty(2, dtype=torch.int32, device=dev)
+        import ctypes
+        P = lambda t: ctypes.c_void_p(t.data_ptr())
+        stc = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        call = lambda: tess.tess_min_pair_distance(P(step.pos_sorted), s.n, s.box, P(step.nbr), P(step.counts), s.cap,
+                                                   P(mws), mws.numel(), P(r2m), P(pairm), stc)
+        for _ in range(args.warmup):
+            assert call() == 0
+        mev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for k in range(args.steps):
+            flush.zero_()
+            mev[k][0].record()
+            call()
+            mev[k][1].record()
+        torch.cuda.synchronize()
+        mms = sum(a.elapsed_time(b) for a, b in mev) / args.steps
+        monitor = {"ms": mms, "min_distance": float(r2m.item()) ** 0.5, "pair": [int(v) for v in pairm.cpu()],
+                   "list_bytes_read_gbs": pairs * 4 / (mms / 1e3) / 1e9}
+
     graph = None
     if args.graph:
         # the same step captured once as a CUDA graph and replayed
@@ -419,6 +443,7 @@ def run_cuda(args, world, rank, local):
             "graph": graph,
             "backward": backward,
             "resort": resort,
+            "min_pair": monitor,
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -536,6 +561,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph", action="store_true", help="also time the step captured as one CUDA graph")
     ap.add_argument("--backward", action="store_true", help="also time the aggregation's backward on the same list")
+    ap.add_argument("--monitor", action="store_true", help="also time the closest-listed-pair check on the step's list")
     ap.add_argument("--resort", action="store_true",
                     help="also time the incremental re-sort against the full sort a rebuild interval later")
     args = ap.parse_args(argv)

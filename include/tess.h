@@ -290,12 +290,37 @@ tess_status tess_edge_aggregate_backward(const float* pos, int n, tess_box box, 
                                          float* grad_feat, float* grad_pos, tess_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Closest listed pair -- a structural check for atoms that come anomalously
+ * close (Tessera's runs were checked for such pairs; Tessera, abstract).
+ *
+ * Over every listed (i, j) -- the first min(counts[i], max_neighbors)
+ * entries of row i, entries < 0 or >= n skipped -- the smallest squared
+ * minimum-image distance and the pair that has it.  Distances are computed
+ * as tess_skin_check computes displacements: fp64 from the fp32
+ * coordinates, one IEEE rounding per product and sum, (dx^2 + dy^2) + dz^2.
+ * Ties go to the smallest i, then the smallest j.  Reads the list once
+ * (about 4 bytes per listed pair), so it is meant for occasional checks.
+ *
+ *   pos      [n, 4] float (sorted index space, as the list), 16-byte aligned
+ *   ws       tess_min_pair_distance_workspace() bytes, 16-byte aligned,
+ *            nothing needs to be zeroed
+ *   min_r2   [1] double out: the smallest r^2, +infinity if nothing is listed
+ *   min_pair [2] int32 out: (i, j), or (-1, -1) if nothing is listed
+ * Errors: INVALID_ARG, WORKSPACE_TOO_SMALL, CUDA.
+ * ------------------------------------------------------------------------- */
+size_t tess_min_pair_distance_workspace(void);
+tess_status tess_min_pair_distance(const float* pos, int n, tess_box box, const int32_t* nbr,
+                                   const int32_t* counts, int max_neighbors, void* ws, size_t ws_bytes,
+                                   double* min_r2, int32_t* min_pair, tess_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Stage timing (diagnostic).  When enabled, each entry point records CUDA
  * events on its stream around its kernels; tess_stage_times adds the elapsed
  * times of all recorded calls per stage (this synchronises on the events)
  * and clears them.  Stages: 0 space-filling-curve keys, 1 key sort, 2 cell
  * binning, 3 pair search, 4 skin check, 5 edge aggregate, 6 aggregate backward,
- * 7 incremental re-sort (its fallback full sort records under 0 and 1).  Returns the number of
+ * 7 incremental re-sort (its fallback full sort records under 0 and 1),
+ * 8 closest listed pair.  Returns the number of
  * stages written (<= max_stages).  ms_out[k] = total milliseconds,
  * calls_out[k] (nullable) = number of timed calls.
  * ------------------------------------------------------------------------- */

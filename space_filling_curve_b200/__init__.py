@@ -24,6 +24,7 @@ __all__ = [
     "tess_status_string", "tess_version", "tess_kernel_launch_count",
     "tess_hilbert_sort_workspace", "tess_hilbert_sort", "tess_hilbert_sort_static", "HILBERT_SORT_STATIC_MAX_N",
     "tess_hilbert_resort_workspace", "tess_hilbert_resort", "hilbert_resort", "TESS_DEV_FULL_SORT",
+    "tess_min_pair_distance_workspace", "tess_min_pair_distance", "min_pair_distance",
     "tess_morton_sort", "morton_sort",
     "tess_build_neighbors_workspace", "tess_build_neighbors",
     "tess_skin_check", "tess_edge_aggregate", "tess_stage_timing", "tess_stage_times",
@@ -42,7 +43,7 @@ TESS_DEV_TIMEOUT = 4
 TESS_NO_PAD_FILL = 1
 TESS_TILE_SEARCH = 2
 STAGES = ("hilbert_keys", "key_sort", "cell_binning", "pair_search", "skin_check", "edge_aggregate", "edge_backward",
-          "resort")
+          "resort", "min_pair")
 _STATUS = {0: "ok", 1: "invalid argument", 2: "box too small", 3: "workspace too small", 4: "CUDA launch error",
            5: "n above the static scratch capacity"}
 HILBERT_SORT_STATIC_MAX_N = 1 << 20
@@ -81,6 +82,10 @@ def lib() -> ctypes.CDLL:
     L.tess_hilbert_sort_workspace.restype = sz
     L.tess_hilbert_sort.argtypes = [P, i32, Box, i32, P, sz, P, P, P, P, P]
     L.tess_hilbert_sort.restype = i32
+    L.tess_min_pair_distance_workspace.argtypes = []
+    L.tess_min_pair_distance_workspace.restype = sz
+    L.tess_min_pair_distance.argtypes = [P, i32, Box, P, P, i32, P, sz, P, P, P]
+    L.tess_min_pair_distance.restype = i32
     L.tess_hilbert_resort_workspace.argtypes = [i32]
     L.tess_hilbert_resort_workspace.restype = sz
     L.tess_hilbert_resort.argtypes = [P, i32, Box, i32, P, P, P, sz, P, P, P, P, P]
@@ -130,6 +135,15 @@ def tess_kernel_launch_count() -> int:
 
 def tess_hilbert_sort_workspace(n: int) -> int:
     return int(lib().tess_hilbert_sort_workspace(int(n)))
+
+
+def tess_min_pair_distance_workspace() -> int:
+    return int(lib().tess_min_pair_distance_workspace())
+
+
+def tess_min_pair_distance(pos, n, box, nbr, counts, max_neighbors, ws, ws_bytes, min_r2, min_pair, stream) -> int:
+    return int(lib().tess_min_pair_distance(pos, n, _box(box), nbr, counts, max_neighbors, ws, ws_bytes, min_r2,
+                                            min_pair, stream))
 
 
 def tess_hilbert_resort_workspace(n: int) -> int:
@@ -373,4 +387,22 @@ def edge_aggregate_backward(pos4, box, rc: float, nbr, counts, feat, grad_out, *
                                         _ptr(grad_out), F, _ptr(grad_feat), _ptr(grad_pos), _stream(stream))
     _check("tess_edge_aggregate_backward", code)
     return grad_feat, grad_pos
+
+
+def min_pair_distance(pos4, box, nbr, counts, *, ws=None, stream=None):
+    """Closest listed pair: (min_r2 float64 [1], pair int32 [2]) on the device;
+    (+inf, (-1, -1)) when nothing is listed."""
+    torch = _torch()
+    _need_cuda("pos4", pos4, torch.float32, 4)
+    _need_cuda("nbr", nbr, torch.int32)
+    _need_cuda("counts", counts, torch.int32)
+    n, cap = nbr.shape
+    dev = pos4.device
+    ws = _workspace(tess_min_pair_distance_workspace(), dev, ws)
+    r2 = torch.empty(1, dtype=torch.float64, device=dev)
+    pair = torch.empty(2, dtype=torch.int32, device=dev)
+    code = tess_min_pair_distance(_ptr(pos4), n, box, _ptr(nbr), _ptr(counts), cap, _ptr(ws),
+                                  ws.numel() * ws.element_size(), _ptr(r2), _ptr(pair), _stream(stream))
+    _check("tess_min_pair_distance", code)
+    return r2, pair
 

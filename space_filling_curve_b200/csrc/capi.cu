@@ -10,6 +10,10 @@ std::atomic<long long> g_launches{0};
 
 size_t hilbert_sort_workspace(int n);
 size_t hilbert_resort_workspace(int n);
+size_t min_pair_workspace();
+tess_status min_pair_distance(const float* pos, int n, tess_box box, const int32_t* nbr, const int32_t* counts,
+                              int cap, void* ws, size_t ws_bytes, double* min_r2, int32_t* min_pair,
+                              cudaStream_t s);
 tess_status hilbert_resort(const float* pos, int n, tess_box box, int bits, const int32_t* perm_prev,
                            const uint32_t* keys_prev, void* ws, size_t ws_bytes, int32_t* perm,
                            uint32_t* keys_sorted, float* pos_sorted, int32_t* dev_status, cudaStream_t s);
@@ -98,6 +102,15 @@ tess_status tess_hilbert_sort(const float* pos, int n, tess_box box, int bits, v
 }
 
 size_t tess_hilbert_resort_workspace(int n) { return hilbert_resort_workspace(n); }
+
+size_t tess_min_pair_distance_workspace(void) { return min_pair_workspace(); }
+
+tess_status tess_min_pair_distance(const float* pos, int n, tess_box box, const int32_t* nbr,
+                                   const int32_t* counts, int max_neighbors, void* ws, size_t ws_bytes,
+                                   double* min_r2, int32_t* min_pair, tess_stream_t stream) {
+    return min_pair_distance(pos, n, box, nbr, counts, max_neighbors, ws, ws_bytes, min_r2, min_pair,
+                             reinterpret_cast<cudaStream_t>(stream));
+}
 
 tess_status tess_hilbert_resort(const float* pos, int n, tess_box box, int bits, const int32_t* perm_prev,
                                 const uint32_t* keys_prev, void* ws, size_t ws_bytes, int32_t* perm,

@@ -18,7 +18,7 @@ extern std::atomic<long long> g_launches;
 inline void count_launch(long long k = 1) { g_launches.fetch_add(k, std::memory_order_relaxed); }
 
 // Stage ids for the optional event timing.
-enum Stage { ST_KEYS = 0, ST_SORT = 1, ST_CELLS = 2, ST_PAIRS = 3, ST_SKIN = 4, ST_EDGE = 5, ST_BACKWARD = 6, ST_RESORT = 7, ST_COUNT = 8 };
+enum Stage { ST_KEYS = 0, ST_SORT = 1, ST_CELLS = 2, ST_PAIRS = 3, ST_SKIN = 4, ST_EDGE = 5, ST_BACKWARD = 6, ST_RESORT = 7, ST_MONITOR = 8, ST_COUNT = 9 };
 
 // Records an event pair around a stage when stage timing is enabled.
 struct StageScope {

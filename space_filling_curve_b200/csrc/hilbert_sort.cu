@@ -113,7 +113,13 @@ __global__ __launch_bounds__(KEYS_THREADS) void keys_kernel(const float* __restr
 
 constexpr int SORT_THREADS = 256;
 constexpr int SORT_WARPS = SORT_THREADS / 32;
-constexpr int SORT_ITEMS = 16;
+#ifndef TESS_SORT_ITEMS
+#define TESS_SORT_ITEMS 16
+#endif
+#ifndef TESS_SORT_MINB
+#define TESS_SORT_MINB 3
+#endif
+constexpr int SORT_ITEMS = TESS_SORT_ITEMS;     // elements per thread in one sort tile
 constexpr int SORT_TILE = SORT_THREADS * SORT_ITEMS;
 constexpr unsigned long long ST_AGG = 1ull << 62;
 constexpr unsigned long long ST_INC = 2ull << 62;
@@ -163,7 +169,7 @@ using SortShared = SortSharedT<SORT_ITEMS>;
 // (the grid may then have more tiles than needed: tiles past the end return);
 // gate, when given, runs the pass only if *gate == want.
 template <bool FINAL, int ITEMS = SORT_ITEMS>
-__global__ __launch_bounds__(SORT_THREADS, 3) void onesweep_pass(const unsigned long long* __restrict__ in,
+__global__ __launch_bounds__(SORT_THREADS, TESS_SORT_MINB) void onesweep_pass(const unsigned long long* __restrict__ in,
                                                               unsigned long long* __restrict__ out, int n, int shift,
                                                               const unsigned* __restrict__ hist,
                                                               unsigned long long* states, unsigned* tile_counter,

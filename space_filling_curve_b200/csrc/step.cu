@@ -192,7 +192,16 @@ __global__ __launch_bounds__(EDGE_WARPS * 32) void edge_kernel(EdgeArgs A) {
     }
 }
 
-constexpr int EV_WARPS = 8;
+#ifndef TESS_EV_WARPS
+#define TESS_EV_WARPS 8
+#endif
+#ifndef TESS_EV_GEO_UNROLL
+#define TESS_EV_GEO_UNROLL 4
+#endif
+#ifndef TESS_EV_ACC_UNROLL
+#define TESS_EV_ACC_UNROLL 4
+#endif
+constexpr int EV_WARPS = TESS_EV_WARPS;
 constexpr int EV_MAXCAP = 512;       // live edges of one row staged in shared memory
 #ifndef TESS_EV_MINB
 #define TESS_EV_MINB 3               // resident blocks per SM the register budget aims at
@@ -209,8 +218,8 @@ constexpr int EV_MAXCAP = 512;       // live edges of one row staged in shared m
 // in space and share most of their neighbors.  All blocks together sweep a
 // front of gridDim * chunk rows, which bounds the L2 working set.
 constexpr int EV_CHUNK = TESS_EV_CHUNK;
-constexpr int EV_GEO_UNROLL = 4;     // neighbor/position loads in flight per lane
-constexpr int EV_ACC_UNROLL = 4;     // feature rows in flight per lane group
+constexpr int EV_GEO_UNROLL = TESS_EV_GEO_UNROLL;     // neighbor/position loads in flight per lane
+constexpr int EV_ACC_UNROLL = TESS_EV_ACC_UNROLL;     // feature rows in flight per lane group
 
 // W consecutive floats of a feature row (W = 4: one 16-byte load; W = 8: one
 // 32-byte load, which sm_100 issues as a single instruction).
@@ -693,6 +702,153 @@ tess_status edge_aggregate(const float* pos, int n, tess_box box, float rc, cons
         else edge_kernel<1><<<blocks, EDGE_WARPS * 32, 0, s>>>(A);
     }
     count_launch();
+    return launch_status();
+}
+
+// ---------------------------------------------------------------- closest listed pair
+
+// The closest pair the list holds -- a structural check for atoms that come
+// anomalously close (Tessera runs are checked for such pairs; Tessera,
+// abstract).  Squared distances as the skin check computes them: fp64 from
+// the fp32 coordinates, one IEEE rounding per product and sum, no
+// contraction.  Order: (r2, i, j) lexicographic, so ties go to the smallest
+// pair.  One warp per row; per-block minima go to the workspace and one
+// block reduces them.
+constexpr int MP_THREADS = 256;
+constexpr int MP_MAX_BLOCKS = 1024;
+
+struct MinPairCand {
+    unsigned long long r2;    // bits of the fp64 r2 (non-negative: ordered as integers)
+    unsigned long long ij;    // (i << 32) | j
+};
+
+__device__ __forceinline__ bool mp_less(unsigned long long ar, unsigned long long aij, unsigned long long br,
+                                        unsigned long long bij) {
+    return ar < br || (ar == br && aij < bij);
+}
+
+__device__ __forceinline__ unsigned long long shfl_xor_u64s(unsigned long long v, int m) {
+    const unsigned lo = __shfl_xor_sync(FULL, (unsigned)v, m);
+    const unsigned hi = __shfl_xor_sync(FULL, (unsigned)(v >> 32), m);
+    return ((unsigned long long)hi << 32) | lo;
+}
+
+__device__ __forceinline__ void mp_warp_min(unsigned long long& r, unsigned long long& ij) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long orr = shfl_xor_u64s(r, o), oij = shfl_xor_u64s(ij, o);
+        if (mp_less(orr, oij, r, ij)) {
+            r = orr;
+            ij = oij;
+        }
+    }
+}
+
+__global__ __launch_bounds__(MP_THREADS) void min_pair_kernel(const float4* __restrict__ pos, int n, double3 L,
+                                                              const int* __restrict__ nbr,
+                                                              const int* __restrict__ counts, int cap,
+                                                              MinPairCand* __restrict__ cand) {
+    __shared__ unsigned long long s_r[MP_THREADS / 32], s_ij[MP_THREADS / 32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned long long br = ~0ull, bij = ~0ull;
+    // chunks of consecutive rows per block, as in the aggregation: the rows'
+    // neighbors overlap, so their positions stay in L1
+    for (long long c0 = (long long)blockIdx.x * EV_CHUNK; c0 < n; c0 += (long long)gridDim.x * EV_CHUNK)
+    for (long long i = c0 + warp, c1 = min((long long)n, c0 + EV_CHUNK); i < c1; i += MP_THREADS / 32) {
+        const float4 pi = pos[i];
+        const int m = max(min(counts[i], cap), 0);
+        constexpr int U = 4;     // list entries in flight per lane
+        for (int s0 = 0; s0 < m; s0 += 32 * U) {
+            int j[U];
+            float4 pj[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int s = s0 + 32 * u + lane;
+                j[u] = s < m ? nbr[(size_t)i * cap + s] : -1;
+                if (j[u] >= n) j[u] = -1;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                if (j[u] >= 0) pj[u] = pos[j[u]];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (j[u] < 0) continue;
+                const double dx = min_image_d((double)pj[u].x - (double)pi.x, L.x);
+                const double dy = min_image_d((double)pj[u].y - (double)pi.y, L.y);
+                const double dz = min_image_d((double)pj[u].z - (double)pi.z, L.z);
+                const double r2 = __dadd_rn(__dadd_rn(__dmul_rn(dx, dx), __dmul_rn(dy, dy)), __dmul_rn(dz, dz));
+                const unsigned long long rb = (unsigned long long)__double_as_longlong(r2);
+                const unsigned long long ij = ((unsigned long long)i << 32) | (unsigned)j[u];
+                if (mp_less(rb, ij, br, bij)) {
+                    br = rb;
+                    bij = ij;
+                }
+            }
+        }
+    }
+    mp_warp_min(br, bij);
+    if (lane == 0) {
+        s_r[warp] = br;
+        s_ij[warp] = bij;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        br = lane < MP_THREADS / 32 ? s_r[lane] : ~0ull;
+        bij = lane < MP_THREADS / 32 ? s_ij[lane] : ~0ull;
+        mp_warp_min(br, bij);
+        if (lane == 0) cand[blockIdx.x] = MinPairCand{br, bij};
+    }
+}
+
+__global__ __launch_bounds__(1024) void min_pair_reduce(const MinPairCand* __restrict__ cand, int nc,
+                                                        double* __restrict__ r2_out, int32_t* __restrict__ pair_out) {
+    __shared__ unsigned long long s_r[32], s_ij[32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned long long br = ~0ull, bij = ~0ull;
+    for (int k = threadIdx.x; k < nc; k += blockDim.x)
+        if (mp_less(cand[k].r2, cand[k].ij, br, bij)) {
+            br = cand[k].r2;
+            bij = cand[k].ij;
+        }
+    mp_warp_min(br, bij);
+    if (lane == 0) {
+        s_r[warp] = br;
+        s_ij[warp] = bij;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        br = s_r[lane];
+        bij = s_ij[lane];
+        mp_warp_min(br, bij);
+        if (lane == 0) {
+            const bool none = bij == ~0ull;
+            r2_out[0] = none ? __longlong_as_double(0x7ff0000000000000ll) : __longlong_as_double((long long)br);
+            pair_out[0] = none ? -1 : (int32_t)(bij >> 32);
+            pair_out[1] = none ? -1 : (int32_t)(unsigned)bij;
+        }
+    }
+}
+
+size_t min_pair_workspace() { return MP_MAX_BLOCKS * sizeof(MinPairCand); }
+
+tess_status min_pair_distance(const float* pos, int n, tess_box box, const int32_t* nbr, const int32_t* counts,
+                              int cap, void* ws, size_t ws_bytes, double* min_r2, int32_t* min_pair,
+                              cudaStream_t s) {
+    if (n <= 0 || !pos || !nbr || !counts || !ws || !min_r2 || !min_pair || cap < 1) return TESS_ERR_INVALID_ARG;
+    if (!finite_pos(box.lx) || !finite_pos(box.ly) || !finite_pos(box.lz)) return TESS_ERR_INVALID_ARG;
+    if (!aligned(pos, 16) || !aligned(ws, 16)) return TESS_ERR_INVALID_ARG;
+    if (ws_bytes < min_pair_workspace()) return TESS_ERR_WORKSPACE_TOO_SMALL;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // one resident wave (no more blocks than the workspace holds)
+    const int blocks = std::min(chunk_grid(min_pair_kernel, MP_THREADS, 0, n, sms, EV_CHUNK), MP_MAX_BLOCKS);
+    MinPairCand* cand = static_cast<MinPairCand*>(ws);
+    StageScope sc(ST_MONITOR, s);
+    min_pair_kernel<<<blocks, MP_THREADS, 0, s>>>(reinterpret_cast<const float4*>(pos), n,
+                                                  make_double3(box.lx, box.ly, box.lz), nbr, counts, cap, cand);
+    min_pair_reduce<<<1, 1024, 0, s>>>(cand, blocks, min_r2, min_pair);
+    count_launch(2);
     return launch_status();
 }
 
