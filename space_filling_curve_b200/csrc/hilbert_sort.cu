@@ -114,10 +114,10 @@ __global__ __launch_bounds__(KEYS_THREADS) void keys_kernel(const float* __restr
 constexpr int SORT_THREADS = 256;
 constexpr int SORT_WARPS = SORT_THREADS / 32;
 #ifndef TESS_SORT_ITEMS
-#define TESS_SORT_ITEMS 16
+#define TESS_SORT_ITEMS 8
 #endif
 #ifndef TESS_SORT_MINB
-#define TESS_SORT_MINB 3
+#define TESS_SORT_MINB 6
 #endif
 constexpr int SORT_ITEMS = TESS_SORT_ITEMS;     // elements per thread in one sort tile
 constexpr int SORT_TILE = SORT_THREADS * SORT_ITEMS;

@@ -554,25 +554,50 @@ __global__ __launch_bounds__(BK_WARPS * 32, TESS_BK_MINB) void edge_backward_ker
 }
 
 // Grid of a chunked row walk for `kernel` (`threads` per block, `smem`
-// dynamic bytes): one resident wave, as many blocks per SM as registers and
-// shared memory allow, never more blocks than chunks.  Also sets the kernel's
-// shared-memory carveout hint to what that wave needs, so that the rest of
-// the SM's 256 KB serves as L1 for the feature gathers (the driver may
-// otherwise keep a larger carveout than the launch needs).
+// dynamic bytes, `chunk` rows per chunk): CHUNK_WAVES times the blocks that
+// are resident at once, never more blocks than chunks.  With a single
+// resident wave the slowest block sets the kernel time and its time varies
+// from launch to launch (measured at 10.24M atoms, 40 launches: aggregation
+// median 15.7 ms, max 16.9); with four waves the hardware scheduler starts a
+// new block wherever one finishes (median 13.7 ms, max 14.2).  Blocks per SM come from the kernel's registers and
+// thread count alone; the shared-memory carveout is then set to the smallest
+// configuration that holds that many blocks, so that the rest of the SM's
+// 256 KB serves as L1 for the gathers (the driver may otherwise keep a
+// larger carveout than the launch needs).  Deriving the block count from the
+// carveout instead would feed back: a carveout rounded down lowers the
+// count, which lowers the next carveout.
+constexpr int CHUNK_WAVES = 4;
+
 template <class K>
 int chunk_grid(K* kernel, int threads, size_t smem, int n, int sms, int chunk) {
-    int dev = 0, max_sm = 0, per_sm = 0;
+    static const int configs_kb[] = {0, 8, 16, 32, 64, 100, 132, 164, 196, 228};
+    int dev = 0, max_sm = 0, regs_sm = 65536, thr_sm = 2048;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&max_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess || per_sm < 1)
-        per_sm = 1;
+    cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
+    cudaDeviceGetAttribute(&thr_sm, cudaDevAttrMaxThreadsPerMultiProcessor, dev);
+    cudaFuncAttributes fa{};
+    int per_sm = 1;
+    if (cudaFuncGetAttributes(&fa, kernel) == cudaSuccess && fa.numRegs > 0) {
+        const int regs_block = ((fa.numRegs * 32 + 255) / 256 * 256) * (threads / 32);    // per-warp allocation unit
+        per_sm = std::max(1, std::min(regs_sm / regs_block, thr_sm / threads));
+    }
     if (max_sm > 0) {
-        const size_t need = (size_t)per_sm * (smem + 1024);
-        const int pct = (int)std::min<size_t>(100, (need * 100 + max_sm - 1) / max_sm);
+        const size_t need = (size_t)per_sm * (smem + fa.sharedSizeBytes + 1024);
+        int kb = configs_kb[sizeof(configs_kb) / sizeof(int) - 1];
+        for (int c : configs_kb)
+            if ((size_t)c * 1024 >= need) {
+                kb = c;
+                break;
+            }
+        const int pct = std::min(100, (kb * 1024 * 100 + max_sm - 1) / max_sm);
         cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, pct);
     }
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, threads, smem) == cudaSuccess && occ > 0)
+        per_sm = std::min(per_sm, occ);
     const long long chunks = ((long long)n + chunk - 1) / chunk;
-    return (int)std::max<long long>(1, std::min<long long>(chunks, (long long)sms * per_sm));
+    return (int)std::max<long long>(1, std::min<long long>(chunks, (long long)sms * per_sm * CHUNK_WAVES));
 }
 
 template <int V>
@@ -715,7 +740,7 @@ tess_status edge_aggregate(const float* pos, int n, tess_box box, float rc, cons
 // pair.  One warp per row; per-block minima go to the workspace and one
 // block reduces them.
 constexpr int MP_THREADS = 256;
-constexpr int MP_MAX_BLOCKS = 1024;
+constexpr int MP_MAX_BLOCKS = 4096;
 
 struct MinPairCand {
     unsigned long long r2;    // bits of the fp64 r2 (non-negative: ordered as integers)
