@@ -162,8 +162,9 @@ tess_status tess_morton_sort(const float* pos, int n, tess_box box, int bits,
  *
  * Same computation, arguments and outputs as tess_hilbert_sort, but without a
  * workspace argument: the scratch memory is an array inside the library
- * (device memory, about 19 MiB, held by every GPU that loads the library until
- * the process exits).  It is meant for callers that cannot allocate device
+ * (device memory, TESS_HILBERT_SORT_STATIC_BYTES = 21 MiB, held by every GPU
+ * that loads the library until the process exits).  It is meant for callers
+ * that cannot allocate device
  * memory -- for example a plugin whose host program owns all device buffers,
  * or a time-step loop that must not call cudaMalloc because it synchronises
  * the device -- and that have no buffer to lend as a workspace.
@@ -180,6 +181,7 @@ tess_status tess_morton_sort(const float* pos, int n, tess_box box, int bits,
  * Errors: those of tess_hilbert_sort, plus TOO_LARGE.
  * ------------------------------------------------------------------------- */
 #define TESS_HILBERT_SORT_STATIC_MAX_N (1 << 20)
+#define TESS_HILBERT_SORT_STATIC_BYTES (21u << 20)   /* >= tess_hilbert_sort_workspace(MAX_N) */
 tess_status tess_hilbert_sort_static(const float* pos, int n, tess_box box, int bits,
                                      int32_t* perm, uint32_t* keys_sorted, float* pos_sorted,
                                      int32_t* dev_status, tess_stream_t stream);

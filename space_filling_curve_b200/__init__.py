@@ -23,6 +23,7 @@ __all__ = [
     "TessError", "lib", "library_path", "Box",
     "tess_status_string", "tess_version", "tess_kernel_launch_count",
     "tess_hilbert_sort_workspace", "tess_hilbert_sort", "tess_hilbert_sort_static", "HILBERT_SORT_STATIC_MAX_N",
+    "HILBERT_SORT_STATIC_BYTES",
     "tess_hilbert_resort_workspace", "tess_hilbert_resort", "hilbert_resort", "TESS_DEV_FULL_SORT",
     "tess_min_pair_distance_workspace", "tess_min_pair_distance", "min_pair_distance",
     "tess_morton_sort", "morton_sort",
@@ -47,6 +48,7 @@ STAGES = ("hilbert_keys", "key_sort", "cell_binning", "pair_search", "skin_check
 _STATUS = {0: "ok", 1: "invalid argument", 2: "box too small", 3: "workspace too small", 4: "CUDA launch error",
            5: "n above the static scratch capacity"}
 HILBERT_SORT_STATIC_MAX_N = 1 << 20
+HILBERT_SORT_STATIC_BYTES = 21 << 20
 
 
 class TessError(RuntimeError):

@@ -8,7 +8,7 @@
 // has no spare buffer to lend as a workspace.  For them this entry point runs
 // the same sort kernels on a scratch area that the library carries itself: a
 // fixed array in device memory, sized for TESS_HILBERT_SORT_STATIC_MAX_N atoms
-// (about 19 MiB).  Every GPU that loads the library holds that array until
+// (TESS_HILBERT_SORT_STATIC_BYTES, 21 MiB).  Every GPU that loads the library holds that array until
 // the process exits.
 //
 // The array is shared by every call on a device and keeps what the previous
@@ -27,7 +27,7 @@ size_t hilbert_sort_workspace(int n);
 tess_status hilbert_sort(const float* pos, int n, tess_box box, int bits, void* ws, size_t ws_bytes, int32_t* perm,
                          uint32_t* keys_sorted, float* pos_sorted, int32_t* dev_status, cudaStream_t s);
 
-constexpr size_t STATIC_SORT_SCRATCH_BYTES = (size_t)19 << 20;
+constexpr size_t STATIC_SORT_SCRATCH_BYTES = TESS_HILBERT_SORT_STATIC_BYTES;
 
 // The scratch area.  Host code must not pass the name itself to a kernel (on
 // the host it is a stand-in, not a device address); its device address comes

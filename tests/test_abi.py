@@ -67,3 +67,15 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert tess.tess_build_neighbors(p, 10, box, 6.0, 0.5, 16, 8, p, 1 << 30, p, p, p, null) == 1
     assert tess.tess_skin_check(p, p, 10, box, -0.5, p, null, null) == 1
     assert tess.tess_edge_aggregate(p, 10, box, 6.0, p, p, 16, p, 0, p, null, null, null, null) == 1
+
+
+def test_static_sort_scratch_holds_the_largest_sort(lib):
+    """The allocation-free sort's scratch array (its size in the header)
+    holds the sort's workspace at the largest n it accepts."""
+    src = open(os.path.join(ROOT, "include", "tess.h")).read()
+    max_n = int(re.search(r"#define TESS_HILBERT_SORT_STATIC_MAX_N \(1 << (\d+)\)", src).group(1))
+    nbytes = int(re.search(r"#define TESS_HILBERT_SORT_STATIC_BYTES \((\d+)u << 20\)", src).group(1)) << 20
+    assert tess.HILBERT_SORT_STATIC_MAX_N == 1 << max_n
+    assert tess.HILBERT_SORT_STATIC_BYTES == nbytes
+    assert tess.tess_hilbert_sort_workspace(1 << max_n) <= nbytes
+
