@@ -334,6 +334,79 @@ def run_cuda(args, world, rank, local):
         monitor = {"ms": mms, "min_distance": float(r2m.item()) ** 0.5, "pair": [int(v) for v in pairm.cpu()],
                    "list_bytes_read_gbs": pairs * 4 / (mms / 1e3) / 1e9}
 
+    step_graph = None
+    if args.step_graph:
+        # a time-step loop over a random walk (sigma per axis per step): the
+        # step graph decides rebuilds on the device; the eager loop reads the
+        # skin check's flag back every step and calls the rebuild itself
+        nsteps = 30
+        gen = torch.Generator(device=dev).manual_seed(5)
+        L = torch.tensor(s.box, dtype=torch.float32, device=dev)
+        walk = [step.pos3.clone()]
+        for _ in range(nsteps):
+            x = walk[-1] + torch.randn(walk[-1].shape, generator=gen, device=dev) * s.sigma
+            walk.append(torch.remainder(x, L).contiguous())
+        sg = tess.StepGraph(walk[0], s.box, s.rc, s.skin, s.cap, step.feat)
+        try:
+            def run_graph():
+                for t in range(nsteps):
+                    sg.pos.copy_(walk[t])
+                    sg.launch()
+            with torch.cuda.stream(sg.stream):
+                run_graph()                                    # warm-up (and first rebuild)
+                sg.request_rebuild()
+            before = sg.rebuilds
+            with torch.cuda.stream(sg.stream):
+                a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a_ev.record()
+                run_graph()
+                b_ev.record()
+            sg.stream.synchronize()
+            g_ms = a_ev.elapsed_time(b_ev) / nsteps
+            g_rebuilds = sg.rebuilds - before
+        finally:
+            sg.close()
+        # the same loop driven from the host
+        ref4 = torch.empty((s.n, 4), dtype=torch.float32, device=dev)
+        cur4 = torch.zeros((s.n, 4), dtype=torch.float32, device=dev)
+        flag = torch.empty(1, dtype=torch.int32, device=dev)
+        md2 = torch.empty(1, dtype=torch.float64, device=dev)
+        import ctypes
+        P = lambda t_: ctypes.c_void_p(t_.data_ptr())
+        stc = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+        def run_eager():
+            rebuilds = 0
+            for t in range(nsteps):
+                pos = walk[t]
+                if t == 0:
+                    r = 1
+                else:
+                    cur4[:, :3] = pos[step.perm.long()]
+                    assert tess.tess_skin_check(P(cur4), P(ref4), s.n, s.box, s.skin, P(flag), P(md2), stc) == 0
+                    r = int(flag.item())                     # the host round trip of a host-driven loop
+                if r:
+                    rebuilds += 1
+                    assert step.sort_fn(P(pos), s.n, s.box, 10, P(step.ws_sort), step.ws_sort.numel(), P(step.perm),
+                                        P(step.keys), P(ref4), P(step.status), stc) == 0
+                    assert tess.tess_build_neighbors(P(ref4), s.n, s.box, s.rc, s.skin, s.cap, 0, P(step.ws_nbr),
+                                                     step.ws_nbr.numel(), P(step.nbr), P(step.counts),
+                                                     P(step.overflow), stc) == 0
+                    cur4.copy_(ref4)
+                assert tess.tess_edge_aggregate(P(cur4), s.n, s.box, s.rc, P(step.nbr), P(step.counts), s.cap,
+                                                P(step.feat), s.F, P(step.out), None, None, None, stc) == 0
+            return rebuilds
+        run_eager()
+        torch.cuda.synchronize()
+        a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_ev.record()
+        e_rebuilds = run_eager()
+        b_ev.record()
+        torch.cuda.synchronize()
+        e_ms = a_ev.elapsed_time(b_ev) / nsteps
+        step_graph = {"steps": nsteps, "sigma": s.sigma, "graph_ms_per_step": g_ms, "eager_ms_per_step": e_ms,
+                      "speedup": e_ms / g_ms, "graph_rebuilds": g_rebuilds, "eager_rebuilds": e_rebuilds}
+
     graph = None
     if args.graph:
         # the same step captured once as a CUDA graph and replayed
@@ -444,6 +517,7 @@ def run_cuda(args, world, rank, local):
             "backward": backward,
             "resort": resort,
             "min_pair": monitor,
+            "step_graph": step_graph,
             "clocks": clocks,
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -561,6 +635,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph", action="store_true", help="also time the step captured as one CUDA graph")
     ap.add_argument("--backward", action="store_true", help="also time the aggregation's backward on the same list")
+    ap.add_argument("--step-graph", action="store_true",
+                    help="also time a 30-step loop as the device-decided step graph against a host-driven loop")
     ap.add_argument("--monitor", action="store_true", help="also time the closest-listed-pair check on the step's list")
     ap.add_argument("--resort", action="store_true",
                     help="also time the incremental re-sort against the full sort a rebuild interval later")

@@ -316,6 +316,70 @@ tess_status tess_min_pair_distance(const float* pos, int n, tess_box box, const 
                                    double* min_r2, int32_t* min_pair, tess_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Step graph -- one time step as a CUDA graph whose rebuild branch is taken
+ * on the device.  Tessera replays each interval between rebuilds as one CUDA
+ * graph (Tessera, abstract); here the skin check's flag sets the condition
+ * of a conditional (IF) node, so a loop of launches needs no host round trip
+ * per step, rebuilds included.  One launch:
+ *   pos_cur = pos gathered into the order of the last rebuild (perm)
+ *   skin check of pos_cur against pos_sorted -> *rebuild, *max_disp2
+ *   rebuild = flag, or a pending request (control[0], then cleared);
+ *             control[1] counts rebuilds
+ *   IF rebuild: tess_hilbert_sort(pos) -> perm, keys, pos_sorted;
+ *               tess_build_neighbors(pos_sorted) -> nbr, counts, overflow;
+ *               pos_cur = pos_sorted
+ *   tess_edge_aggregate(pos_cur, nbr, counts, feat) -> out
+ * The caller writes the step's positions into `pos` (original index order)
+ * before each launch.  `feat` is read in the index order of the current
+ * sort: a caller whose features follow the atoms re-orders them after a
+ * launch whose *rebuild is 1 (perm gives the order).  Every buffer is
+ * device memory owned by the caller and must outlive the graph; sizes as for
+ * the entry points above.  The first launch after create always rebuilds.
+ * ------------------------------------------------------------------------- */
+typedef struct tess_step_buffers {
+    int n;                 /* atoms */
+    tess_box box;
+    float rc, skin;
+    int max_neighbors;     /* list capacity per row */
+    int bits;              /* Hilbert grid bits, 1..10 */
+    int F;                 /* features per atom */
+    int flags;             /* tess_build_neighbors flags */
+    const float* pos;      /* [n, 3] current positions, original order (written by the caller) */
+    const float* feat;     /* [n, F] */
+    void* ws_sort;         /* tess_hilbert_sort_workspace(n) bytes, 256-byte aligned */
+    size_t ws_sort_bytes;
+    void* ws_list;         /* tess_build_neighbors_workspace(...) bytes, 256-byte aligned */
+    size_t ws_list_bytes;
+    int32_t* perm;         /* [n] */
+    uint32_t* keys;        /* [n] */
+    float* pos_sorted;     /* [n, 4] positions at the last rebuild, sorted order */
+    float* pos_cur;        /* [n, 4] current positions, sorted order */
+    int32_t* nbr;          /* [n, max_neighbors] */
+    int32_t* counts;       /* [n] */
+    int32_t* overflow;     /* [1] */
+    int32_t* sort_status;  /* [1] */
+    int32_t* rebuild;      /* [1] out: 1 when the step rebuilt */
+    double* max_disp2;     /* [1] out */
+    int32_t* control;      /* [2] device words (see above) */
+    float* out;            /* [n, F] */
+} tess_step_buffers;
+
+typedef struct tess_step_graph tess_step_graph;
+
+/* Builds and instantiates the graph (stream capture on `stream`, which must
+ * not be the legacy default stream) and queues a rebuild request for the
+ * first launch.  Call outside any other capture, with stage timing off or on
+ * (timing is skipped while capturing).  Errors: INVALID_ARG,
+ * WORKSPACE_TOO_SMALL, BOX_TOO_SMALL, CUDA (e.g. a driver without
+ * conditional nodes); *out is NULL then. */
+tess_status tess_step_graph_create(const tess_step_buffers* b, tess_stream_t stream, tess_step_graph** out);
+/* One step: cudaGraphLaunch on `stream`. */
+tess_status tess_step_graph_launch(tess_step_graph* g, tess_stream_t stream);
+/* Makes the next launch rebuild whatever the skin check says (stream-ordered). */
+tess_status tess_step_graph_request_rebuild(const tess_step_buffers* b, tess_stream_t stream);
+void tess_step_graph_destroy(tess_step_graph* g);
+
+/* ---------------------------------------------------------------------------
  * Stage timing (diagnostic).  When enabled, each entry point records CUDA
  * events on its stream around its kernels; tess_stage_times adds the elapsed
  * times of all recorded calls per stage (this synchronises on the events)

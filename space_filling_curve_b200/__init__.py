@@ -26,6 +26,8 @@ __all__ = [
     "HILBERT_SORT_STATIC_BYTES",
     "tess_hilbert_resort_workspace", "tess_hilbert_resort", "hilbert_resort", "TESS_DEV_FULL_SORT",
     "tess_min_pair_distance_workspace", "tess_min_pair_distance", "min_pair_distance",
+    "tess_step_graph_create", "tess_step_graph_launch", "tess_step_graph_request_rebuild", "tess_step_graph_destroy",
+    "StepBuffers", "StepGraph",
     "tess_morton_sort", "morton_sort",
     "tess_build_neighbors_workspace", "tess_build_neighbors",
     "tess_skin_check", "tess_edge_aggregate", "tess_stage_timing", "tess_stage_times",
@@ -84,6 +86,14 @@ def lib() -> ctypes.CDLL:
     L.tess_hilbert_sort_workspace.restype = sz
     L.tess_hilbert_sort.argtypes = [P, i32, Box, i32, P, sz, P, P, P, P, P]
     L.tess_hilbert_sort.restype = i32
+    L.tess_step_graph_create.argtypes = [ctypes.POINTER(StepBuffers), P, ctypes.POINTER(P)]
+    L.tess_step_graph_create.restype = i32
+    L.tess_step_graph_launch.argtypes = [P, P]
+    L.tess_step_graph_launch.restype = i32
+    L.tess_step_graph_request_rebuild.argtypes = [ctypes.POINTER(StepBuffers), P]
+    L.tess_step_graph_request_rebuild.restype = i32
+    L.tess_step_graph_destroy.argtypes = [P]
+    L.tess_step_graph_destroy.restype = None
     L.tess_min_pair_distance_workspace.argtypes = []
     L.tess_min_pair_distance_workspace.restype = sz
     L.tess_min_pair_distance.argtypes = [P, i32, Box, P, P, i32, P, sz, P, P, P]
@@ -113,6 +123,18 @@ def lib() -> ctypes.CDLL:
     return L
 
 
+class StepBuffers(ctypes.Structure):
+    """Mirror of tess_step_buffers (include/tess.h)."""
+    _fields_ = [("n", ctypes.c_int), ("box", Box), ("rc", ctypes.c_float), ("skin", ctypes.c_float),
+                ("max_neighbors", ctypes.c_int), ("bits", ctypes.c_int), ("F", ctypes.c_int), ("flags", ctypes.c_int),
+                ("pos", ctypes.c_void_p), ("feat", ctypes.c_void_p), ("ws_sort", ctypes.c_void_p),
+                ("ws_sort_bytes", ctypes.c_size_t), ("ws_list", ctypes.c_void_p), ("ws_list_bytes", ctypes.c_size_t),
+                ("perm", ctypes.c_void_p), ("keys", ctypes.c_void_p), ("pos_sorted", ctypes.c_void_p),
+                ("pos_cur", ctypes.c_void_p), ("nbr", ctypes.c_void_p), ("counts", ctypes.c_void_p),
+                ("overflow", ctypes.c_void_p), ("sort_status", ctypes.c_void_p), ("rebuild", ctypes.c_void_p),
+                ("max_disp2", ctypes.c_void_p), ("control", ctypes.c_void_p), ("out", ctypes.c_void_p)]
+
+
 def _box(box) -> Box:
     if isinstance(box, Box):
         return box
@@ -137,6 +159,22 @@ def tess_kernel_launch_count() -> int:
 
 def tess_hilbert_sort_workspace(n: int) -> int:
     return int(lib().tess_hilbert_sort_workspace(int(n)))
+
+
+def tess_step_graph_create(buffers, stream, out) -> int:
+    return int(lib().tess_step_graph_create(buffers, stream, out))
+
+
+def tess_step_graph_launch(graph, stream) -> int:
+    return int(lib().tess_step_graph_launch(graph, stream))
+
+
+def tess_step_graph_request_rebuild(buffers, stream) -> int:
+    return int(lib().tess_step_graph_request_rebuild(buffers, stream))
+
+
+def tess_step_graph_destroy(graph) -> None:
+    lib().tess_step_graph_destroy(graph)
 
 
 def tess_min_pair_distance_workspace() -> int:
@@ -407,4 +445,70 @@ def min_pair_distance(pos4, box, nbr, counts, *, ws=None, stream=None):
                                   ws.numel() * ws.element_size(), _ptr(r2), _ptr(pair), _stream(stream))
     _check("tess_min_pair_distance", code)
     return r2, pair
+
+
+class StepGraph:
+    """One time step as a CUDA graph whose rebuild branch is decided on the
+    device (tess_step_graph_*).  Owns its buffers (torch tensors) and a
+    stream; write the step's positions into ``pos`` ([n, 3], original order)
+    before each ``launch``.  After a launch: ``rebuild`` (1 when the step
+    rebuilt), ``perm``, ``nbr``, ``counts``, ``out`` and the rest hold that
+    step's state; ``rebuilds`` reads the device's rebuild counter."""
+
+    def __init__(self, pos, box, rc: float, skin: float, max_neighbors: int, feat, *, bits: int = 10,
+                 pad_fill: bool = True, stream=None):
+        torch = _torch()
+        _need_cuda("pos", pos, torch.float32, 3)
+        _need_cuda("feat", feat, torch.float32)
+        n, F = pos.shape[0], feat.shape[1]
+        dev = pos.device
+        self.stream = torch.cuda.Stream(device=dev) if stream is None else stream
+        self.pos = pos.clone()
+        self.feat = feat
+        self.ws_sort = _workspace(tess_hilbert_sort_workspace(n), dev)
+        self.ws_list = _workspace(tess_build_neighbors_workspace(n, box, rc, skin), dev)
+        e = lambda *shape, dtype=torch.int32: torch.zeros(shape, dtype=dtype, device=dev)
+        self.perm, self.keys = e(n), e(n)
+        self.pos_sorted, self.pos_cur = e(n, 4, dtype=torch.float32), e(n, 4, dtype=torch.float32)
+        self.nbr, self.counts = e(n, max_neighbors), e(n)
+        self.overflow, self.sort_status, self.rebuild = e(1), e(1), e(1)
+        self.max_disp2 = e(1, dtype=torch.float64)
+        self.control = e(2)
+        self.out = e(n, F, dtype=torch.float32)
+        b = StepBuffers()
+        b.n, b.box, b.rc, b.skin = n, _box(box), float(rc), float(skin)
+        b.max_neighbors, b.bits, b.F, b.flags = max_neighbors, bits, F, 0 if pad_fill else TESS_NO_PAD_FILL
+        for name in ("pos", "feat", "ws_sort", "ws_list", "perm", "keys", "pos_sorted", "pos_cur", "nbr", "counts",
+                     "overflow", "sort_status", "rebuild", "max_disp2", "control", "out"):
+            setattr(b, name, getattr(self, name).data_ptr())
+        b.ws_sort_bytes = self.ws_sort.numel()
+        b.ws_list_bytes = self.ws_list.numel()
+        self._b = b
+        self._g = ctypes.c_void_p()
+        torch.cuda.synchronize(dev)
+        code = tess_step_graph_create(ctypes.byref(b), ctypes.c_void_p(self.stream.cuda_stream), ctypes.byref(self._g))
+        _check("tess_step_graph_create", code)
+
+    def launch(self):
+        _check("tess_step_graph_launch", tess_step_graph_launch(self._g, ctypes.c_void_p(self.stream.cuda_stream)))
+
+    def request_rebuild(self):
+        _check("tess_step_graph_request_rebuild",
+               tess_step_graph_request_rebuild(ctypes.byref(self._b), ctypes.c_void_p(self.stream.cuda_stream)))
+
+    @property
+    def rebuilds(self) -> int:
+        return int(self.control[1].item())
+
+    def close(self):
+        if self._g:
+            self.stream.synchronize()
+            tess_step_graph_destroy(self._g)
+            self._g = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 

@@ -10,7 +10,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libtess.so")
-SOURCES = ["capi.cu", "hilbert_sort.cu", "neighbors.cu", "step.cu", "static_scratch.cu"]
+SOURCES = ["capi.cu", "hilbert_sort.cu", "neighbors.cu", "step.cu", "static_scratch.cu", "step_graph.cu"]
 HEADERS = ["common.cuh"]
 
 NVCC_FLAGS = [

@@ -57,6 +57,10 @@ StageScope::StageScope(int stage_, cudaStream_t s_) : stage(stage_), s(s_) {
     Timing& t = timing();
     std::lock_guard<std::mutex> g(t.mu);
     if (!t.enabled) return;
+    // no timing inside a graph capture: event nodes are not allowed in every
+    // graph (conditional bodies), and a captured stage runs at replay time
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return;
     cudaEventCreate(&a);
     cudaEventCreate(&b);
     cudaEventRecord(a, s);
