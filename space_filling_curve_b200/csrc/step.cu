@@ -441,13 +441,16 @@ struct BackArgs {
 // each.  Each lane keeps its own share of the force, sum over edges of (its
 // part of the dot product) times (f_c'/r) r_ij, which is linear in the parts,
 // so the lanes are summed once per row instead of once per edge.
-constexpr int BK_WARPS = 4;
+#ifndef TESS_BK_WARPS
+#define TESS_BK_WARPS 8
+#endif
+constexpr int BK_WARPS = TESS_BK_WARPS;
 constexpr int BK_MAXCAP = 512;
 #ifndef TESS_BK_CHUNK
-#define TESS_BK_CHUNK 256
+#define TESS_BK_CHUNK 512
 #endif
 #ifndef TESS_BK_MINB
-#define TESS_BK_MINB 4
+#define TESS_BK_MINB 3
 #endif
 constexpr int BK_CHUNK = TESS_BK_CHUNK;
 
@@ -672,6 +675,7 @@ tess_status edge_backward(const float* pos, int n, tess_box box, float rc, const
     const size_t smem = (size_t)BK_WARPS * cap * (sizeof(float4) + sizeof(int));
     auto launch = [&](auto w, auto lpe, auto vpl) {
         auto* k = edge_backward_kernel<decltype(w)::value, decltype(lpe)::value, decltype(vpl)::value>;
+        if (smem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         k<<<chunk_grid(k, BK_WARPS * 32, smem, n, sms, BK_CHUNK), BK_WARPS * 32, smem, s>>>(A);
     };
     const int W = pick_width(F, {feat, grad_out, grad_feat});

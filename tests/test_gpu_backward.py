@@ -21,14 +21,15 @@ def _dev(a):
     return torch.from_numpy(np.ascontiguousarray(a)).cuda()
 
 
-def _case(s, F, seed):
+def _case(s, F, seed, cap=None):
     import space_filling_curve_b200 as tess
+    cap = s.cap if cap is None else cap
     perm, _ = oracle.hilbert_sort(s.pos, s.box, 10)
     p4 = s.pos4()[perm]
     rng = np.random.default_rng(seed)
     feat = rng.standard_normal((s.n, F)).astype(np.float32)
     g = rng.standard_normal((s.n, F)).astype(np.float32)
-    nbr_d, cnt_d, ov = tess.build_neighbors(_dev(p4), s.box, s.rc, s.skin, s.cap)
+    nbr_d, cnt_d, ov = tess.build_neighbors(_dev(p4), s.box, s.rc, s.skin, cap)
     assert int(ov.item()) == 0
     gf, gp = tess.edge_aggregate_backward(_dev(p4), s.box, s.rc, nbr_d, cnt_d, _dev(feat), _dev(g))
     nbr, cnt = nbr_d.cpu().numpy(), cnt_d.cpu().numpy()
@@ -41,8 +42,8 @@ def _case(s, F, seed):
     # position gradient: per-row magnitude scale of the sum
     e = oracle.edge_aggregate(p4, s.box, s.rc, nbr, cnt, np.ones((s.n, 1), np.float32), edges=True)
     r = e["edge_vec"][..., 3]
-    i_idx = np.repeat(np.arange(s.n), s.cap).reshape(s.n, s.cap)
-    live = (np.arange(s.cap)[None, :] < np.minimum(cnt, s.cap)[:, None]) & (r < s.rc) & (nbr >= 0)
+    i_idx = np.repeat(np.arange(s.n), cap).reshape(s.n, cap)
+    live = (np.arange(cap)[None, :] < np.minimum(cnt, cap)[:, None]) & (r < s.rc) & (nbr >= 0)
     ii, jj = i_idx[live], nbr[live]
     dfc = np.abs(-0.5 * np.pi / s.rc * np.sin(np.pi * r[live] / s.rc))
     gn = np.linalg.norm(g.astype(np.float64), axis=1)
@@ -62,6 +63,12 @@ def test_backward_uniform(F):
 
 def test_backward_salt():
     _case(synth.system(2), 64, 7)
+
+
+def test_backward_large_cap():
+    """cap 512: the staging buffers of a block exceed the default 48 KB of
+    dynamic shared memory."""
+    _case(synth.system(1), 32, 9, cap=512)
 
 
 def test_backward_rejects_unsupported_widths():
