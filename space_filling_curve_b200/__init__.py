@@ -498,6 +498,8 @@ class StepGraph:
 
     @property
     def rebuilds(self) -> int:
+        """Rebuilds since create (waits for the graph's stream)."""
+        self.stream.synchronize()
         return int(self.control[1].item())
 
     def close(self):

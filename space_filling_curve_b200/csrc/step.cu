@@ -193,7 +193,7 @@ __global__ __launch_bounds__(EDGE_WARPS * 32) void edge_kernel(EdgeArgs A) {
 }
 
 #ifndef TESS_EV_WARPS
-#define TESS_EV_WARPS 8
+#define TESS_EV_WARPS 24
 #endif
 #ifndef TESS_EV_GEO_UNROLL
 #define TESS_EV_GEO_UNROLL 4
@@ -204,10 +204,10 @@ __global__ __launch_bounds__(EDGE_WARPS * 32) void edge_kernel(EdgeArgs A) {
 constexpr int EV_WARPS = TESS_EV_WARPS;
 constexpr int EV_MAXCAP = 512;       // live edges of one row staged in shared memory
 #ifndef TESS_EV_MINB
-#define TESS_EV_MINB 3               // resident blocks per SM the register budget aims at
+#define TESS_EV_MINB 1               // resident blocks per SM the register budget aims at
 #endif
 #ifndef TESS_EV_CHUNK
-#define TESS_EV_CHUNK 256
+#define TESS_EV_CHUNK 768
 #endif
 #ifndef TESS_EV_W
 #define TESS_EV_W 4                  // floats per feature load when F allows (4 or 8)
@@ -721,6 +721,7 @@ tess_status edge_aggregate(const float* pos, int n, tess_box box, float rc, cons
     if (vec) {
         auto launch = [&](auto w, auto lpe, auto vpl) {
             auto* k = edge_vec_kernel<decltype(w)::value, decltype(lpe)::value, decltype(vpl)::value>;
+            if (vsmem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)vsmem);
             k<<<chunk_grid(k, EV_WARPS * 32, vsmem, n, sms, EV_CHUNK), EV_WARPS * 32, vsmem, s>>>(A);
         };
         const int W = pick_width(F, {feat, out});
