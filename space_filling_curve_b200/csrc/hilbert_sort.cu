@@ -418,7 +418,7 @@ tess_status morton_sort(const float* pos, int n, tess_box box, int bits, void* w
 // fraction of a grid cell, so their new key stays inside the range of old
 // keys of their old neighbors in the order: such "local" atoms (S) can only
 // be out of order with atoms at most 2 * RS_W old ranks away and are sorted
-// by two rounds of block sorts of RS_BLK elements (the second offset by half
+// by two phases of block sorts of RS_BLK elements (the second offset by half
 // a block).  The others (O, atoms whose key jumped along the curve: the
 // curve's neighboring cells can be far apart in key) are few; they are radix
 // sorted by the full 64-bit element and merged in by binary search.  Every
@@ -613,7 +613,7 @@ __device__ __forceinline__ unsigned long long shfl_xor_u64(unsigned long long v,
 
 // Sorts blocks of S in place, one warp per block of RS_BLK elements held in
 // registers (lane l holds positions 8l .. 8l+7), with a bitonic network.
-// Round 0: blocks at multiples of RS_BLK; round 1: the same shifted by RS_D
+// Phase 0: blocks at multiples of RS_BLK; phase 1: the same shifted by RS_D
 // (the first block is [0, RS_D)).  Missing elements are padded with the
 // largest value, so they sort last and are not written back.  Global memory
 // is read and written in coalesced stripes (lane l: positions l + 32r) and
@@ -621,7 +621,7 @@ __device__ __forceinline__ unsigned long long shfl_xor_u64(unsigned long long v,
 // conflicts.
 __device__ __forceinline__ int rs_skew(int p) { return p + (p >> 3); }
 
-template <int ROUND>
+template <int PHASE>
 __global__ __launch_bounds__(RS_THREADS) void resort_block_sort(unsigned long long* __restrict__ S,
                                                                 const ResortCtl* ctl) {
     __shared__ unsigned long long sx[RS_THREADS / 32][RS_BLK + RS_BLK / 8];
@@ -630,11 +630,11 @@ __global__ __launch_bounds__(RS_THREADS) void resort_block_sort(unsigned long lo
     const int lane = threadIdx.x & 31;
     unsigned long long* t = sx[threadIdx.x >> 5];
     const long long wg = (long long)blockIdx.x * (RS_THREADS / 32) + (threadIdx.x >> 5);
-    // round 1: block w >= 1 starts at RS_D + (w - 1) * RS_BLK; its halves are
-    // the sorted second half of one round-0 block and the sorted first half
+    // phase 1: block w >= 1 starts at RS_D + (w - 1) * RS_BLK; its halves are
+    // the sorted second half of one phase-0 block and the sorted first half
     // of the next (the first RS_D elements are a sorted half already)
-    if (ROUND == 1 && wg == 0) return;
-    const long long start = ROUND == 0 ? wg * RS_BLK : RS_D + (wg - 1) * RS_BLK;
+    if (PHASE == 1 && wg == 0) return;
+    const long long start = PHASE == 0 ? wg * RS_BLK : RS_D + (wg - 1) * RS_BLK;
     if (start >= m) return;
     const long long len = min((long long)RS_BLK, (long long)m - start);
 #pragma unroll
@@ -644,7 +644,7 @@ __global__ __launch_bounds__(RS_THREADS) void resort_block_sort(unsigned long lo
     }
     __syncwarp();
     unsigned long long x[8];
-    if (ROUND == 0) {
+    if (PHASE == 0) {
 #pragma unroll
         for (int r = 0; r < 8; ++r) x[r] = t[rs_skew(8 * lane + r)];
     } else {
@@ -656,7 +656,7 @@ __global__ __launch_bounds__(RS_THREADS) void resort_block_sort(unsigned long lo
         }
     }
 #pragma unroll
-    for (int k = ROUND == 0 ? 2 : RS_BLK; k <= RS_BLK; k <<= 1) {
+    for (int k = PHASE == 0 ? 2 : RS_BLK; k <= RS_BLK; k <<= 1) {
 #pragma unroll
         for (int j = k >> 1; j > 0; j >>= 1) {
             if (j >= 8) {

@@ -38,7 +38,7 @@ def canon_rows_gpu(nbr, counts):
 def agg_error(gpu_out: np.ndarray, ref: dict):
     """(worst condition-aware relative error, worst plain relative error over
     |ref| > 1e-3).  The condition-aware error divides by
-    max(|ref|, sum_j f_c |h_j|), so that sums that cancel are not judged
+    max(|ref|, sum_j f_c |h_j|), so that sums that cancel are not measured
     against their tiny result."""
     out = ref["out"]
     den = np.maximum(np.abs(out), ref["out_abs"])
