@@ -493,7 +493,7 @@ def run_cuda(args, world, rank, local):
     stage_ms = {k: (v[0] / max(v[1], 1)) for k, v in stages.items() if v[1] > 0}
     dom = max(stage_ms, key=stage_ms.get)
     achieved = nbytes[dom] / (stage_ms[dom] / 1e3) / 1e9
-    traffic = _traffic_from_profile(dom, s.n)
+    traffic = _traffic_from_profile(dom, s.n, s.name)
     clocks = clk.summary()
 
     if rank == 0:
@@ -564,11 +564,12 @@ def _rebuild_roofline(n, mean_count, stage_ms, peak):
             "frac": (b / (t / 1e3) / 1e9) / peak if t else None}
 
 
-def _traffic_from_profile(kernel_stage, n):
+def _traffic_from_profile(kernel_stage, n, workload=""):
     """DRAM bytes per launch of the dominant kernel at n atoms, from the
     committed ncu summary (profiles/<stage>_traffic.json: bytes per atom of
-    one capture), or None when there is none or when the kernel's source
-    file has changed since the counters were taken."""
+    one capture), or None when there is none, when the kernel's source file
+    has changed since the counters were taken, or when the workload is not
+    of the captured family (bytes per atom depend on the neighbor counts)."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "%s_traffic.json" % kernel_stage)
     try:
@@ -577,6 +578,8 @@ def _traffic_from_profile(kernel_stage, n):
         with open(os.path.join(ROOT, d["source_file"]), "rb") as f:
             if hashlib.sha1(f.read()).hexdigest() != d["source_sha1"]:
                 return None
+        if not workload.startswith(d.get("workload_family", "")):
+            return None
         return d["dram_bytes_per_atom"] * n
     except Exception:
         return None

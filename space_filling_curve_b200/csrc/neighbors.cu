@@ -562,7 +562,10 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
 // Loops are warp-uniform (bounded by the warp's longest window) so that the
 // buffer vote can run inside them.
 constexpr int PL_WARPS = 4;
-constexpr int PL_CHUNK = 8;          // candidates per lane between buffer votes
+#ifndef TESS_PL_CHUNK
+#define TESS_PL_CHUNK 4
+#endif
+constexpr int PL_CHUNK = TESS_PL_CHUNK;   // candidates per lane between buffer votes
 
 __global__ __launch_bounds__(PL_WARPS * 32, 6) void pair_search_lane_kernel(PairArgs A) {
     __shared__ int s_buf[PL_WARPS][32 * PS_BUF];
