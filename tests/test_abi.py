@@ -67,6 +67,28 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert tess.tess_build_neighbors(p, 10, box, 6.0, 0.5, 16, 8, p, 1 << 30, p, p, p, null) == 1
     assert tess.tess_skin_check(p, p, 10, box, -0.5, p, null, null) == 1
     assert tess.tess_edge_aggregate(p, 10, box, 6.0, p, p, 16, p, 0, p, null, null, null, null) == 1
+    # backward: F not a multiple of 4, cap above 512, box below 2 rc
+    assert tess.tess_edge_aggregate_backward(p, 10, box, 6.0, p, p, 16, p, p, 6, p, p, null) == 1
+    assert tess.tess_edge_aggregate_backward(p, 10, box, 6.0, p, p, 513, p, p, 64, p, p, null) == 1
+    assert tess.tess_edge_aggregate_backward(p, 10, (10.0, 30.0, 30.0), 6.0, p, p, 16, p, p, 64, p, p, null) == 2
+    # re-sort: no earlier order, workspace too small
+    assert tess.tess_hilbert_resort(p, 10, box, 10, null, p, p, 1 << 20, p, p, null, null, null) == 1
+    assert tess.tess_hilbert_resort(p, 10, box, 10, p, p, p, 16, p, p, null, null, null) == 3
+    # closest pair: no workspace, workspace too small
+    assert tess.tess_min_pair_distance(p, 10, box, p, p, 16, null, 0, p, p, null) == 1
+    assert tess.tess_min_pair_distance(p, 10, box, p, p, 16, p, 16, p, p, null) == 3
+    # step graph: missing buffers, small workspaces; nothing is created
+    out = ctypes.c_void_p()
+    assert tess.tess_step_graph_create(null, null, ctypes.byref(out)) == 1 and not out.value
+    b = tess.StepBuffers()
+    b.n, b.box, b.rc, b.skin, b.max_neighbors, b.bits, b.F = 10, tess._box(box), 6.0, 0.5, 16, 10, 8
+    for name in ("pos", "feat", "ws_sort", "ws_list", "perm", "keys", "pos_sorted", "pos_cur", "nbr", "counts",
+                 "overflow", "sort_status", "rebuild", "max_disp2", "control", "out"):
+        setattr(b, name, 256)
+    b.ws_sort_bytes, b.ws_list_bytes = 16, 16
+    assert tess.tess_step_graph_create(ctypes.byref(b), null, ctypes.byref(out)) == 3 and not out.value
+    b.control = None
+    assert tess.tess_step_graph_create(ctypes.byref(b), null, ctypes.byref(out)) == 1 and not out.value
 
 
 def test_static_sort_scratch_holds_the_largest_sort(lib):
