@@ -380,6 +380,21 @@ tess_status tess_step_graph_request_rebuild(const tess_step_buffers* b, tess_str
 void tess_step_graph_destroy(tess_step_graph* g);
 
 /* ---------------------------------------------------------------------------
+ * Look-back timeout probe (diagnostic, no counterpart in the paper).  The
+ * sort's counting passes wait on each other through a decoupled look-back
+ * whose wait is bounded: after a fixed number of polls it gives up, sets
+ * TESS_DEV_TIMEOUT in the status word and lets the kernel finish, so the
+ * GPU context stays usable.  This call makes that happen on purpose: one
+ * block runs the second tile of a pass whose first tile never runs.  It
+ * takes a few seconds, writes only inside `ws`, and its output means
+ * nothing; *dev_status ends with TESS_DEV_TIMEOUT set.
+ *   ws  tess_debug_lookback_timeout_workspace() bytes, 256-byte aligned
+ * Errors: INVALID_ARG, WORKSPACE_TOO_SMALL, CUDA.
+ * ------------------------------------------------------------------------- */
+size_t tess_debug_lookback_timeout_workspace(void);
+tess_status tess_debug_lookback_timeout(void* ws, size_t ws_bytes, int32_t* dev_status, tess_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * Stage timing (diagnostic).  When enabled, each entry point records CUDA
  * events on its stream around its kernels; tess_stage_times adds the elapsed
  * times of all recorded calls per stage (this synchronises on the events)

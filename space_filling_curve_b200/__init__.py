@@ -28,6 +28,7 @@ __all__ = [
     "tess_min_pair_distance_workspace", "tess_min_pair_distance", "min_pair_distance",
     "tess_step_graph_create", "tess_step_graph_launch", "tess_step_graph_request_rebuild", "tess_step_graph_destroy",
     "StepBuffers", "StepGraph",
+    "tess_debug_lookback_timeout_workspace", "tess_debug_lookback_timeout",
     "tess_morton_sort", "morton_sort",
     "tess_build_neighbors_workspace", "tess_build_neighbors",
     "tess_skin_check", "tess_edge_aggregate", "tess_stage_timing", "tess_stage_times",
@@ -94,6 +95,10 @@ def lib() -> ctypes.CDLL:
     L.tess_step_graph_request_rebuild.restype = i32
     L.tess_step_graph_destroy.argtypes = [P]
     L.tess_step_graph_destroy.restype = None
+    L.tess_debug_lookback_timeout_workspace.argtypes = []
+    L.tess_debug_lookback_timeout_workspace.restype = sz
+    L.tess_debug_lookback_timeout.argtypes = [P, sz, P, P]
+    L.tess_debug_lookback_timeout.restype = i32
     L.tess_min_pair_distance_workspace.argtypes = []
     L.tess_min_pair_distance_workspace.restype = sz
     L.tess_min_pair_distance.argtypes = [P, i32, Box, P, P, i32, P, sz, P, P, P]
@@ -175,6 +180,14 @@ def tess_step_graph_request_rebuild(buffers, stream) -> int:
 
 def tess_step_graph_destroy(graph) -> None:
     lib().tess_step_graph_destroy(graph)
+
+
+def tess_debug_lookback_timeout_workspace() -> int:
+    return int(lib().tess_debug_lookback_timeout_workspace())
+
+
+def tess_debug_lookback_timeout(ws, ws_bytes, dev_status, stream) -> int:
+    return int(lib().tess_debug_lookback_timeout(ws, ws_bytes, dev_status, stream))
 
 
 def tess_min_pair_distance_workspace() -> int:

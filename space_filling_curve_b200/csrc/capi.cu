@@ -10,6 +10,8 @@ std::atomic<long long> g_launches{0};
 
 size_t hilbert_sort_workspace(int n);
 size_t hilbert_resort_workspace(int n);
+size_t lookback_probe_workspace();
+tess_status lookback_timeout_probe(void* ws, size_t ws_bytes, int32_t* status, cudaStream_t s);
 size_t min_pair_workspace();
 tess_status min_pair_distance(const float* pos, int n, tess_box box, const int32_t* nbr, const int32_t* counts,
                               int cap, void* ws, size_t ws_bytes, double* min_r2, int32_t* min_pair,
@@ -106,6 +108,12 @@ tess_status tess_hilbert_sort(const float* pos, int n, tess_box box, int bits, v
 }
 
 size_t tess_hilbert_resort_workspace(int n) { return hilbert_resort_workspace(n); }
+
+size_t tess_debug_lookback_timeout_workspace(void) { return lookback_probe_workspace(); }
+
+tess_status tess_debug_lookback_timeout(void* ws, size_t ws_bytes, int32_t* dev_status, tess_stream_t stream) {
+    return lookback_timeout_probe(ws, ws_bytes, dev_status, reinterpret_cast<cudaStream_t>(stream));
+}
 
 size_t tess_min_pair_distance_workspace(void) { return min_pair_workspace(); }
 

@@ -928,4 +928,55 @@ tess_status hilbert_resort(const float* pos, int n, tess_box box, int bits, cons
     return launch_status();
 }
 
+// ---------------------------------------------------------------- look-back timeout probe
+//
+// Exercises the bounded wait of the counting pass: one block runs tile 1 of
+// a two-tile pass (the tile counter starts at 1) while tile 0 never runs, so
+// the look-back finds tile 0 unpublished, gives up after LOOKBACK_SPIN_LIMIT
+// polls and sets TESS_DEV_TIMEOUT; the pass then completes.  All keys are 0
+// and the digit histogram counts both tiles, so every write stays inside
+// the workspace.  For tests of the timeout path; its output means nothing.
+
+struct ProbeLayout {
+    unsigned long long* in;
+    unsigned long long* out;
+    unsigned* hist;
+    unsigned long long* states;
+    unsigned* counter;
+    size_t total;
+};
+
+static ProbeLayout probe_layout(void* ws) {
+    Carve c(ws);
+    ProbeLayout P{};
+    P.in = c.take<unsigned long long>(2 * SORT_TILE);
+    P.out = c.take<unsigned long long>(2 * SORT_TILE);
+    P.hist = c.take<unsigned>(RADIX);
+    P.states = c.take<unsigned long long>(2 * RADIX);
+    P.counter = c.take<unsigned>(1);
+    P.total = align_up(c.off, 256);
+    return P;
+}
+
+__global__ void probe_init(unsigned* hist, unsigned* counter, unsigned n) {
+    hist[0] = n;          // every key is 0: digit 0 holds all elements
+    *counter = 1;         // the only block takes tile 1
+}
+
+size_t lookback_probe_workspace() { return probe_layout(nullptr).total; }
+
+tess_status lookback_timeout_probe(void* ws, size_t ws_bytes, int32_t* status, cudaStream_t s) {
+    if (!ws || !status || !aligned(ws, 256)) return TESS_ERR_INVALID_ARG;
+    ProbeLayout P = probe_layout(ws);
+    if (ws_bytes < P.total) return TESS_ERR_WORKSPACE_TOO_SMALL;
+    cudaMemsetAsync(ws, 0, P.total, s);
+    cudaMemsetAsync(status, 0, sizeof(int32_t), s);
+    probe_init<<<1, 1, 0, s>>>(P.hist, P.counter, 2u * SORT_TILE);
+    onesweep_pass<false><<<1, SORT_THREADS, sizeof(SortShared), s>>>(
+        P.in, P.out, 2 * SORT_TILE, 32, P.hist, P.states, P.counter, status, nullptr, nullptr, nullptr, nullptr,
+        nullptr, nullptr, 0);
+    count_launch(2);
+    return launch_status();
+}
+
 }  // namespace tess
