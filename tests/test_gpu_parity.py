@@ -157,6 +157,35 @@ def test_neighbors_ragged(n, tile):
 
 
 @pytest.mark.parametrize("tile", [False, True])
+def test_neighbors_flag_invalid_positions(tile):
+    """A NaN atom and atoms outside [0, L) are flagged in the overflow word
+    (TESS_DEV_BAD_INPUT) without a fault; rows away from them are exact."""
+    tess = _tess()
+    rng = np.random.default_rng(77)
+    n, L, rc, skin = 2000, 30.0, 4.0, 0.5
+    p = np.zeros((n, 4), np.float32)
+    p[:, :3] = rng.uniform(0, L, (n, 3))
+    bad = [5, 9, 13]
+    p[5, 0] = np.nan
+    p[9, 0] = -0.5
+    p[13, 1] = L + 1.0
+    nbr_d, cnt_d, ov = tess.build_neighbors(_dev(p), (L, L, L), rc, skin, 128,
+                                            tile_search=tile)
+    assert int(ov.item()) & 2
+    onbr, ocnt, _ = oracle.neighbors_brute(p, (L, L, L), rc, skin, 128)
+    good = np.ones(n, bool)
+    for b in bad:
+        d = p[:, :3].astype(np.float64) - np.nan_to_num(p[b, :3]).astype(np.float64)
+        d -= L * np.round(d / L)
+        good &= np.sqrt((d ** 2).sum(1)) > rc + skin + 1.5
+    g = canon_rows(nbr_d.cpu().numpy(), cnt_d.cpu().numpy())
+    o = canon_rows(onbr, ocnt)
+    assert good.sum() > n // 2
+    assert np.array_equal(cnt_d.cpu().numpy()[good], ocnt[good])
+    assert np.array_equal(g[good], o[good])
+
+
+@pytest.mark.parametrize("tile", [False, True])
 def test_neighbors_no_pad_fill_and_overflow(tile):
     s = synth.system(1)
     perm, _ = oracle.hilbert_sort(s.pos, s.box, 10)
