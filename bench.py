@@ -1,12 +1,14 @@
 """Benchmark of the neighbor-rebuild hot path on B200.
 
-One step = one pass of the whole path over the 10.24M-atom salt solution
-(rc 5.75 A, skin 0.5 A, 160 neighbors per row, 64 features):
-    Hilbert sort -> neighbor list (padded) -> skin check -> edge aggregation
+One step = one full neighbor rebuild of the 10.24M-atom salt solution
+(rc 5.75 A, skin 0.5 A, 160 neighbors per row):
+    Hilbert sort -> padded neighbor list
 with every input resident in HBM when the timed region starts.  The value is
 atoms per second over all ranks (weak scaling: with --gpus N each rank runs
 an independent replica of the same workload, there is no collective in the
-data path).
+data path).  The line also carries the whole step (rebuild, skin check,
+aggregation of 64 features), the end-to-end rate with host copies, and with
+--all-configs the same figures for all five workloads.
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle
 instead (a deliberately plain program, on the host cores, on a bounded
@@ -121,9 +123,9 @@ def sum_over_ranks(value: float, world: int, device=None) -> float:
 
 
 class Step:
-    """All device buffers of one replica and the step itself, through the C ABI."""
+    """All device buffers of one replica, and the path through the C ABI."""
 
-    def __init__(self, s, device, pad_fill=True, tile_search=False, curve="hilbert"):
+    def __init__(self, s, device, pad_fill=True, lane_search=False, curve="hilbert"):
         import torch
         import space_filling_curve_b200 as tess
         self.tess = tess
@@ -143,15 +145,14 @@ class Step:
         self.nbr = torch.empty((n, cap), dtype=torch.int32, device=device)
         self.counts = torch.empty(n, dtype=torch.int32, device=device)
         self.overflow = torch.empty(1, dtype=torch.int32, device=device)
-        self.rebuild = torch.empty(1, dtype=torch.int32, device=device)
+        self.rebuild_flag = torch.empty(1, dtype=torch.int32, device=device)
         self.maxd = torch.empty(1, dtype=torch.float64, device=device)
         g = torch.Generator(device=device)
         g.manual_seed(s.seed)
         # features live in the sorted index space (produced there by the model)
         self.feat = torch.randn((n, F), generator=g, device=device, dtype=torch.float32)
         self.out = torch.empty((n, F), dtype=torch.float32, device=device)
-        self.pad_fill = pad_fill
-        self.tile_search = tile_search
+        self.flags = (0 if pad_fill else tess.TESS_NO_PAD_FILL) | (tess.TESS_LANE_SEARCH if lane_search else 0)
         self.sort_fn = tess.tess_hilbert_sort if curve == "hilbert" else tess.tess_morton_sort
         # the next frame of the trajectory, in the sorted order of frame 0
         t1 = next(iter(s.trajectory(1, condition=False)))[1]
@@ -163,41 +164,118 @@ class Step:
         self.pos_next[:, :3] = self.frame1[self.perm.long()]
         torch.cuda.synchronize()
 
-    def run(self, pos3=None):
+    @staticmethod
+    def _ptr(t):
         import ctypes
-        tess = self.tess
-        P = lambda t: ctypes.c_void_p(t.data_ptr())
+        return ctypes.c_void_p(t.data_ptr())
+
+    def _stream(self):
+        import ctypes
         import torch
-        st = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-        s = self.s
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+    def rebuild(self, pos3=None):
+        """The timed unit: Hilbert sort, then the padded neighbor list."""
+        tess, s, P, st = self.tess, self.s, self._ptr, self._stream()
         pos3 = self.pos3 if pos3 is None else pos3
         c = self.sort_fn(P(pos3), self.n, s.box, 10, P(self.ws_sort), self.ws_sort.numel(),
-                                   P(self.perm), P(self.keys), P(self.pos_sorted), P(self.status), st)
+                         P(self.perm), P(self.keys), P(self.pos_sorted), P(self.status), st)
         assert c == 0, c
-        c = tess.tess_build_neighbors(P(self.pos_sorted), self.n, s.box, s.rc, s.skin, s.cap,
-                                      (0 if self.pad_fill else tess.TESS_NO_PAD_FILL)
-                                      | (tess.TESS_TILE_SEARCH if self.tile_search else 0), P(self.ws_nbr),
-                                      self.ws_nbr.numel(), P(self.nbr), P(self.counts), P(self.overflow), st)
+        c = tess.tess_build_neighbors(P(self.pos_sorted), self.n, s.box, s.rc, s.skin, s.cap, self.flags,
+                                      P(self.ws_nbr), self.ws_nbr.numel(), P(self.nbr), P(self.counts),
+                                      P(self.overflow), st)
         assert c == 0, c
-        c = tess.tess_skin_check(P(self.pos_next), P(self.pos_sorted), self.n, s.box, s.skin, P(self.rebuild),
-                                 P(self.maxd), st)
+
+    def per_step(self):
+        """What every MD step runs between rebuilds: skin check, aggregation."""
+        tess, s, P, st = self.tess, self.s, self._ptr, self._stream()
+        c = tess.tess_skin_check(P(self.pos_next), P(self.pos_sorted), self.n, s.box, s.skin,
+                                 P(self.rebuild_flag), P(self.maxd), st)
         assert c == 0, c
         c = tess.tess_edge_aggregate(P(self.pos_sorted), self.n, s.box, s.rc, P(self.nbr), P(self.counts), s.cap,
                                      P(self.feat), s.F, P(self.out), None, None, None, st)
         assert c == 0, c
 
+    def run(self, pos3=None):
+        """The whole path once: rebuild, skin check, aggregation."""
+        self.rebuild(pos3)
+        self.per_step()
+
 
 def _algorithmic_bytes(n, mean_count, F):
-    """Minimum bytes each stage must move (per launch), from the per-atom
-    figures of the design notes."""
+    """Minimum bytes each stage must move per launch (the per-atom figures of
+    the design notes times n)."""
     return {
         "hilbert_keys": n * (16 + 8),
-        "key_sort": n * 12,
+        "key_sort": n * (12 + 36),          # the ideal single pass plus the fused gather of perm / positions
         "cell_binning": n * 28,
         "pair_search": n * (16 + 4 * mean_count + 4),
         "skin_check": n * 32,
         "edge_aggregate": n * (4 * F + 4 * F + 16 + 4 * mean_count + 4),
     }
+
+
+def rebuild_bytes(n, mean_count):
+    """Algorithmic bytes of one full rebuild: keys 24, sort 12, gather 36,
+    binning 28, pair search 16 + 4 * mean count + 4 (per atom)."""
+    return n * (24 + 12 + 36 + 28 + 16 + 4 * mean_count + 4)
+
+
+def _timed(fn, steps, flush):
+    """Per-call CUDA events on the current stream around fn(); the 256 MB
+    flush write runs before each call, outside its events.  Returns the list
+    of per-call milliseconds."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for k in range(steps):
+        flush.zero_()
+        evs[k][0].record()
+        fn()
+        evs[k][1].record()
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def _stage_ms(stages):
+    return {k: v[0] / v[1] for k, v in stages.items() if v[1] > 0}
+
+
+def _config_summary(step, steps, flush, peak):
+    """Rebuild, skin check and aggregation of one workload, each timed alone
+    (stage timing on; per-call means)."""
+    import torch
+    tess, s = step.tess, step.s
+    tess.tess_stage_times()
+    tess.tess_stage_timing(True)
+    reb = _timed(step.rebuild, steps, flush)
+    per = _timed(step.per_step, steps, flush)
+    tess.tess_stage_timing(False)
+    st = _stage_ms(tess.tess_stage_times())
+    counts = step.counts.double()
+    mean = float(counts.mean().item())
+    pairs = float(counts.sum().item())
+    n = s.n
+    rb = rebuild_bytes(n, mean)
+    ab = _algorithmic_bytes(n, mean, s.F)
+    reb_ms = sum(reb) / len(reb)
+    out = {
+        "workload": s.name, "atoms": n, "box": list(s.box), "rc": s.rc, "skin": s.skin, "cap": s.cap, "F": s.F,
+        "mean_neighbors": mean, "overflow": int(step.overflow.item()),
+        "rebuild_ms": reb_ms, "rebuild_atoms_per_s": n / (reb_ms / 1e3), "pairs_per_s": pairs / (reb_ms / 1e3),
+        "rebuild_frac_hbm": rb / (reb_ms / 1e3) / 1e9 / peak,
+        "stages_ms": {k: round(v, 4) for k, v in st.items()},
+    }
+    if "pair_search" in st:
+        out["pair_search_frac_hbm"] = ab["pair_search"] / (st["pair_search"] / 1e3) / 1e9 / peak
+    if "skin_check" in st:
+        out["skin_check_gbs"] = ab["skin_check"] / (st["skin_check"] / 1e3) / 1e9
+        out["skin_check_atoms_per_s"] = n / (st["skin_check"] / 1e3)
+    if "edge_aggregate" in st:
+        out["aggregate_gbs"] = ab["edge_aggregate"] / (st["edge_aggregate"] / 1e3) / 1e9
+        out["aggregate_frac_hbm"] = out["aggregate_gbs"] / peak
+        out["aggregate_pairs_per_s"] = pairs / (st["edge_aggregate"] / 1e3)
+    del torch
+    return out
 
 
 def run_cuda(args, world, rank, local):
@@ -211,67 +289,226 @@ def run_cuda(args, world, rank, local):
     import synth
     import space_filling_curve_b200 as tess
     s = synth.system(args.config)
-    step = Step(s, dev, pad_fill=not args.no_pad_fill, tile_search=args.tile_search, curve=args.curve)
+    step = Step(s, dev, pad_fill=not args.no_pad_fill, lane_search=args.lane_search, curve=args.curve)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    peak, peak_kind = _peaks()
+
+    # warm-up (W whole steps); stage timing on so that its event pool fills
+    tess.tess_stage_times()
+    tess.tess_stage_timing(True)
     for _ in range(args.warmup):
         flush.zero_()
         step.run()
     torch.cuda.synchronize()
+    tess.tess_stage_times()
     ov = int(step.overflow.item())
-    counts = step.counts
-    mean_count = float(counts.double().mean().item())
-    pairs = float(counts.double().sum().item())
+    counts = step.counts.double()
+    mean_count = float(counts.mean().item())
+    pairs = float(counts.sum().item())
 
+    # timed region: K rebuilds (sort + list), per-rebuild events on the
+    # launching stream, L2 flushed before each; the library's stage events
+    # (pooled, no event creation) give the per-kernel durations
     launches0 = tess.tess_kernel_launch_count()
-    tess.tess_stage_times()          # clear
-    tess.tess_stage_timing(True)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        for k in range(args.steps):
-            flush.zero_()
-            evs[k][0].record()
-            step.run()
-            evs[k][1].record()
-        torch.cuda.synchronize()
+        reb = _timed(step.rebuild, args.steps, flush)
     if world > 1:
         torch.distributed.barrier()
-    tess.tess_stage_timing(False)
-    stages = tess.tess_stage_times()
     launches = tess.tess_kernel_launch_count() - launches0
-    ms = sum(a.elapsed_time(b) for a, b in evs)
+    stage_ms = _stage_ms(tess.tess_stage_times())
+    ms = sum(reb)
     ms_max = max_over_ranks(ms, world, dev)
     n_total = sum_over_ranks(float(s.n * args.steps), world, dev)
     value = n_total / (ms_max / 1e3)
 
-    backward = None
+    # the same rebuilds with stage timing off (the events' cost is nil)
+    tess.tess_stage_timing(False)
+    plain_ms = sum(_timed(step.rebuild, args.steps, flush)) / args.steps
+
+    # the whole step (rebuild + skin check + aggregation), for context
+    tess.tess_stage_timing(True)
+    whole = _timed(step.run, args.steps, flush)
+    whole_stages = _stage_ms(tess.tess_stage_times())
+    tess.tess_stage_timing(False)
+    whole_ms = sum(whole) / args.steps
+
+    extras = _extras(args, step, flush, dev, world, ms_max)
+
+    # e2e: through the C ABI with host buffers (pinned); every rebuild's
+    # copies (positions in; perm, counts and the status words out -- the list
+    # itself stays on the device for the steps that use it) are inside the
+    # timed region, issued on a second stream with double buffers so that
+    # they overlap the neighboring rebuilds, as a stream-ordered caller would
+    e2e_val, e2e_steps = _e2e(step, s, args.steps, world, dev)
+
+    nbytes = _algorithmic_bytes(s.n, mean_count, s.F)
+    ps_ms = stage_ms.get("pair_search")
+    achieved = nbytes["pair_search"] / (ps_ms / 1e3) / 1e9 if ps_ms else None
+    rb = rebuild_bytes(s.n, mean_count)
+    reb_ms = ms_max / args.steps
+    traffic = _traffic_from_profile("pair_search", s.n, s.name)
+    clocks = clk.summary()
+
+    all_cfg = None
+    if args.all_configs:
+        all_cfg = []
+        for cfg in (1, 2, 3, 4, 5):
+            sc = s if cfg == args.config else synth.system(cfg)
+            stc = step if cfg == args.config else Step(sc, dev, pad_fill=not args.no_pad_fill,
+                                                       lane_search=args.lane_search, curve=args.curve)
+            all_cfg.append(_config_summary(stc, max(3, args.steps), flush, peak))
+            if stc is not step:
+                del stc
+                torch.cuda.empty_cache()
+
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": value,
+            "unit": "atoms/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": reb_ms,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic (seeded salt-solution generator; no dataset)",
+            "config": {
+                "workload": "%s: %d atoms, box %.3f x %.3f x %.3f A, rc %.2f, skin %.2f, cap %d; step = full "
+                            "neighbor rebuild: hilbert_sort + build_neighbors (pad-filled list)"
+                            % (s.name, s.n, s.box[0], s.box[1], s.box[2], s.rc, s.skin, s.cap),
+                "atoms": s.n,
+                "pad_fill": not args.no_pad_fill,
+                "pair_search": "per-lane" if args.lane_search else "tile",
+                "curve": args.curve,
+                "l2": "flushed before every timed rebuild (256 MB write, outside its events)",
+                "parallelism": "replicas (no collective in the data path)",
+                "mean_neighbors": mean_count,
+                "pairs_listed": pairs,
+                "overflow": ov,
+            },
+            "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+            "rebuild_ms_stage_timing_off": plain_ms,
+            "pairs_per_s": pairs / (reb_ms / 1e3),
+            "roofline": {
+                "bound": "hbm",
+                "kernel": "pair_search",
+                "achieved": achieved,
+                "peak": peak,
+                "peak_kind": peak_kind,
+                "unit": "GB/s",
+                "frac": achieved / peak if achieved else None,
+                "traffic": traffic,
+                "algorithmic_bytes": nbytes["pair_search"],
+                "ms": ps_ms,
+            },
+            "rebuild_roofline": {
+                "bound": "hbm", "ms": reb_ms, "algorithmic_bytes": rb,
+                "achieved": rb / (reb_ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                "frac": rb / (reb_ms / 1e3) / 1e9 / peak,
+            },
+            "step": {"what": "rebuild + skin check + edge aggregate (F %d)" % s.F, "ms": whole_ms,
+                     "atoms_per_s": s.n / (whole_ms / 1e3),
+                     "stages_ms": {k: round(v, 4) for k, v in whole_stages.items()}},
+            "e2e": {"value": e2e_val, "unit": "atoms/s", "steps": e2e_steps, "pipelined": True,
+                    "h2d_bytes_per_step": s.n * 12, "d2h_bytes_per_step": s.n * 8 + 8,
+                    "note": "positions in; perm, counts and status words out; the list stays on the device"},
+            "gpu_launches": launches,
+            "clocks": clocks,
+        }
+        line.update(extras)
+        if all_cfg is not None:
+            line["all_configs"] = all_cfg
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(args)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def _e2e(step, s, steps, world, dev):
+    import torch
+    host_pos = torch.from_numpy(s.pos).pin_memory()
+    host_perm = [torch.empty(s.n, dtype=torch.int32).pin_memory() for _ in range(2)]
+    host_counts = [torch.empty(s.n, dtype=torch.int32).pin_memory() for _ in range(2)]
+    host_flags = [torch.empty(2, dtype=torch.int32).pin_memory() for _ in range(2)]
+    pos_in = [torch.empty_like(step.pos3) for _ in range(2)]
+    st_perm = [torch.empty_like(step.perm) for _ in range(2)]
+    st_counts = [torch.empty_like(step.counts) for _ in range(2)]
+    st_flags = [torch.empty(2, dtype=torch.int32, device=dev) for _ in range(2)]
+    cs = torch.cuda.current_stream()
+    xs = torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    ev_read = [torch.cuda.Event() for _ in range(2)]
+    e2e_steps = max(1, steps)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(cs)
+    xs.wait_stream(cs)
+    with torch.cuda.stream(xs):
+        for b in range(min(2, e2e_steps)):
+            pos_in[b].copy_(host_pos, non_blocking=True)
+            ev_in[b].record(xs)
+    for t in range(e2e_steps):
+        b = t % 2
+        cs.wait_event(ev_in[b])
+        step.rebuild(pos3=pos_in[b])
+        if t >= 2:
+            cs.wait_event(ev_read[b])            # rebuild t-2's results have left the staging buffers
+        st_perm[b].copy_(step.perm)
+        st_counts[b].copy_(step.counts)
+        st_flags[b][0:1].copy_(step.overflow)
+        st_flags[b][1:2].copy_(step.status)
+        ev_out[b].record(cs)
+        with torch.cuda.stream(xs):
+            xs.wait_event(ev_out[b])
+            host_perm[b].copy_(st_perm[b], non_blocking=True)
+            host_counts[b].copy_(st_counts[b], non_blocking=True)
+            host_flags[b].copy_(st_flags[b], non_blocking=True)
+            ev_read[b].record(xs)
+            if t + 2 < e2e_steps:                  # rebuild t has read pos_in[b]: load t+2's positions
+                pos_in[b].copy_(host_pos, non_blocking=True)
+                ev_in[b].record(xs)
+    cs.wait_stream(xs)
+    e1.record(cs)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    return sum_over_ranks(float(s.n * e2e_steps), world, dev) / (e2e_ms / 1e3), e2e_steps
+
+
+def _extras(args, step, flush, dev, world, rebuild_ms_total):
+    """The optional measurements (--backward, --resort, --monitor,
+    --step-graph, --graph); each returns a dict under its own key."""
+    import ctypes
+    import torch
+    tess, s = step.tess, step.s
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+    stc = lambda: ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    out = {}
+
+    def mean_ms(call):
+        for _ in range(args.warmup):
+            assert call() == 0
+        return sum(_timed(call, args.steps, flush)) / args.steps
+
     if args.backward:
         # the aggregation's backward (force path) on the same list, timed alone
         gout = torch.randn((s.n, s.F), generator=torch.Generator(device=dev).manual_seed(2), device=dev)
         gfeat = torch.empty_like(gout)
         gpos = torch.empty((s.n, 3), dtype=torch.float32, device=dev)
-        import ctypes
-        P = lambda t: ctypes.c_void_p(t.data_ptr())
-        stc = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-        call = lambda: tess.tess_edge_aggregate_backward(P(step.pos_sorted), s.n, s.box, s.rc, P(step.nbr),
-                                                         P(step.counts), s.cap, P(step.feat), P(gout), s.F,
-                                                         P(gfeat), P(gpos), stc)
-        for _ in range(args.warmup):
-            assert call() == 0
-        bev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-        for k in range(args.steps):
-            flush.zero_()
-            bev[k][0].record()
-            call()
-            bev[k][1].record()
-        torch.cuda.synchronize()
-        bms = sum(a.elapsed_time(b) for a, b in bev) / args.steps
+        mean_count = float(step.counts.double().mean().item())
+        bms = mean_ms(lambda: tess.tess_edge_aggregate_backward(P(step.pos_sorted), s.n, s.box, s.rc, P(step.nbr),
+                                                                P(step.counts), s.cap, P(step.feat), P(gout), s.F,
+                                                                P(gfeat), P(gpos), stc()))
         bbytes = s.n * (3 * 4 * s.F + 16 + 4 * mean_count + 4 + 12)
-        backward = {"ms": bms, "algorithmic_bytes": bbytes, "achieved_gbs": bbytes / (bms / 1e3) / 1e9}
+        out["backward"] = {"ms": bms, "algorithmic_bytes": bbytes, "achieved_gbs": bbytes / (bms / 1e3) / 1e9}
 
-    resort = None
     if args.resort:
         # the re-sort at the next rebuild: every atom moved by a rebuild
         # interval of the trajectory's random walk (20 steps of sigma per axis)
@@ -286,131 +523,32 @@ def run_cuda(args, world, rank, local):
         keys1 = torch.empty_like(keys0)
         ps1 = torch.empty((s.n, 4), dtype=torch.float32, device=dev)
         st1 = torch.empty(1, dtype=torch.int32, device=dev)
-        import ctypes
-        P = lambda t: ctypes.c_void_p(t.data_ptr())
-        stc = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-        calls = {
-            "full_sort": lambda: tess.tess_hilbert_sort(P(pos1), s.n, s.box, 10, P(step.ws_sort), step.ws_sort.numel(),
-                                                        P(perm1), P(keys1), P(ps1), P(st1), stc),
-            "resort": lambda: tess.tess_hilbert_resort(P(pos1), s.n, s.box, 10, P(perm0), P(keys0), P(ws_rs),
-                                                       ws_rs.numel(), P(perm1), P(keys1), P(ps1), P(st1), stc),
-        }
-        resort = {"sigma_total": s.sigma * 20 ** 0.5}
-        for name, call in calls.items():
-            for _ in range(args.warmup):
-                assert call() == 0
-            rev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                   for _ in range(args.steps)]
-            for k in range(args.steps):
-                flush.zero_()
-                rev[k][0].record()
-                call()
-                rev[k][1].record()
-            torch.cuda.synchronize()
-            resort[name + "_ms"] = sum(a.elapsed_time(b) for a, b in rev) / args.steps
-            if name == "resort":
-                resort["incremental_path"] = not (int(st1.item()) & tess.TESS_DEV_FULL_SORT)
+        res = {"sigma_total": s.sigma * 20 ** 0.5}
+        res["full_sort_ms"] = mean_ms(lambda: tess.tess_hilbert_sort(P(pos1), s.n, s.box, 10, P(step.ws_sort),
+                                                                     step.ws_sort.numel(), P(perm1), P(keys1),
+                                                                     P(ps1), P(st1), stc()))
+        res["resort_ms"] = mean_ms(lambda: tess.tess_hilbert_resort(P(pos1), s.n, s.box, 10, P(perm0), P(keys0),
+                                                                    P(ws_rs), ws_rs.numel(), P(perm1), P(keys1),
+                                                                    P(ps1), P(st1), stc()))
+        res["incremental_path"] = not (int(st1.item()) & tess.TESS_DEV_FULL_SORT)
+        out["resort"] = res
 
-    monitor = None
     if args.monitor:
         # the closest listed pair on the step's list
         mws = torch.empty(tess.tess_min_pair_distance_workspace(), dtype=torch.uint8, device=dev)
         r2m = torch.empty(1, dtype=torch.float64, device=dev)
         pairm = torch.empty(2, dtype=torch.int32, device=dev)
-        import ctypes
-        P = lambda t: ctypes.c_void_p(t.data_ptr())
-        stc = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
-        call = lambda: tess.tess_min_pair_distance(P(step.pos_sorted), s.n, s.box, P(step.nbr), P(step.counts), s.cap,
-                                                   P(mws), mws.numel(), P(r2m), P(pairm), stc)
-        for _ in range(args.warmup):
-            assert call() == 0
-        mev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-        for k in range(args.steps):
-            flush.zero_()
-            mev[k][0].record()
-            call()
-            mev[k][1].record()
-        torch.cuda.synchronize()
-        mms = sum(a.elapsed_time(b) for a, b in mev) / args.steps
-        monitor = {"ms": mms, "min_distance": float(r2m.item()) ** 0.5, "pair": [int(v) for v in pairm.cpu()],
-                   "list_bytes_read_gbs": pairs * 4 / (mms / 1e3) / 1e9}
+        pairs = float(step.counts.double().sum().item())
+        mms = mean_ms(lambda: tess.tess_min_pair_distance(P(step.pos_sorted), s.n, s.box, P(step.nbr), P(step.counts),
+                                                          s.cap, P(mws), mws.numel(), P(r2m), P(pairm), stc()))
+        out["min_pair"] = {"ms": mms, "min_distance": float(r2m.item()) ** 0.5, "pair": [int(v) for v in pairm.cpu()],
+                           "list_bytes_read_gbs": pairs * 4 / (mms / 1e3) / 1e9}
 
-    step_graph = None
     if args.step_graph:
-        # a time-step loop over a random walk (sigma per axis per step): the
-        # step graph decides rebuilds on the device; the eager loop reads the
-        # skin check's flag back every step and calls the rebuild itself
-        nsteps = 30
-        gen = torch.Generator(device=dev).manual_seed(5)
-        L = torch.tensor(s.box, dtype=torch.float32, device=dev)
-        walk = [step.pos3.clone()]
-        for _ in range(nsteps):
-            x = walk[-1] + torch.randn(walk[-1].shape, generator=gen, device=dev) * s.sigma
-            walk.append(torch.remainder(x, L).contiguous())
-        sg = tess.StepGraph(walk[0], s.box, s.rc, s.skin, s.cap, step.feat)
-        try:
-            def run_graph():
-                for t in range(nsteps):
-                    sg.pos.copy_(walk[t])
-                    sg.launch()
-            with torch.cuda.stream(sg.stream):
-                run_graph()                                    # warm-up (and first rebuild)
-                sg.request_rebuild()
-            before = sg.rebuilds
-            with torch.cuda.stream(sg.stream):
-                a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a_ev.record()
-                run_graph()
-                b_ev.record()
-            sg.stream.synchronize()
-            g_ms = a_ev.elapsed_time(b_ev) / nsteps
-            g_rebuilds = sg.rebuilds - before
-        finally:
-            sg.close()
-        # the same loop driven from the host
-        ref4 = torch.empty((s.n, 4), dtype=torch.float32, device=dev)
-        cur4 = torch.zeros((s.n, 4), dtype=torch.float32, device=dev)
-        flag = torch.empty(1, dtype=torch.int32, device=dev)
-        md2 = torch.empty(1, dtype=torch.float64, device=dev)
-        import ctypes
-        P = lambda t_: ctypes.c_void_p(t_.data_ptr())
-        stc = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        out["step_graph"] = _step_graph_loop(step, dev)
 
-        def run_eager():
-            rebuilds = 0
-            for t in range(nsteps):
-                pos = walk[t]
-                if t == 0:
-                    r = 1
-                else:
-                    cur4[:, :3] = pos[step.perm.long()]
-                    assert tess.tess_skin_check(P(cur4), P(ref4), s.n, s.box, s.skin, P(flag), P(md2), stc) == 0
-                    r = int(flag.item())                     # the host round trip of a host-driven loop
-                if r:
-                    rebuilds += 1
-                    assert step.sort_fn(P(pos), s.n, s.box, 10, P(step.ws_sort), step.ws_sort.numel(), P(step.perm),
-                                        P(step.keys), P(ref4), P(step.status), stc) == 0
-                    assert tess.tess_build_neighbors(P(ref4), s.n, s.box, s.rc, s.skin, s.cap, 0, P(step.ws_nbr),
-                                                     step.ws_nbr.numel(), P(step.nbr), P(step.counts),
-                                                     P(step.overflow), stc) == 0
-                    cur4.copy_(ref4)
-                assert tess.tess_edge_aggregate(P(cur4), s.n, s.box, s.rc, P(step.nbr), P(step.counts), s.cap,
-                                                P(step.feat), s.F, P(step.out), None, None, None, stc) == 0
-            return rebuilds
-        run_eager()
-        torch.cuda.synchronize()
-        a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a_ev.record()
-        e_rebuilds = run_eager()
-        b_ev.record()
-        torch.cuda.synchronize()
-        e_ms = a_ev.elapsed_time(b_ev) / nsteps
-        step_graph = {"steps": nsteps, "sigma": s.sigma, "graph_ms_per_step": g_ms, "eager_ms_per_step": e_ms,
-                      "speedup": e_ms / g_ms, "graph_rebuilds": g_rebuilds, "eager_rebuilds": e_rebuilds}
-
-    graph = None
     if args.graph:
-        # the same step captured once as a CUDA graph and replayed
+        # the whole step captured once as a CUDA graph and replayed
         g = torch.cuda.CUDAGraph()
         side = torch.cuda.Stream()
         side.wait_stream(torch.cuda.current_stream())
@@ -423,145 +561,87 @@ def run_cuda(args, world, rank, local):
         for _ in range(args.warmup):
             flush.zero_()
             g.replay()
-        gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
         torch.cuda.synchronize()
-        for k in range(args.steps):
-            flush.zero_()
-            gev[k][0].record()
-            g.replay()
-            gev[k][1].record()
-        torch.cuda.synchronize()
-        gms = max_over_ranks(sum(a.elapsed_time(b) for a, b in gev), world, dev)
-        graph = {"ms_per_step": gms / args.steps, "eager_ms_per_step": ms_max / args.steps,
-                 "speedup": ms_max / gms}
+        gms = max_over_ranks(sum(_timed(g.replay, args.steps, flush)), world, dev)
+        eager = max_over_ranks(sum(_timed(step.run, args.steps, flush)), world, dev)
+        out["graph"] = {"ms_per_step": gms / args.steps, "eager_ms_per_step": eager / args.steps,
+                        "speedup": eager / gms}
         del g
+    return out
 
-    # e2e: through the C ABI with host buffers (pinned); every step's copies
-    # (positions in, perm / counts / flags out) are inside the timed region,
-    # issued on a second stream with double buffers so that they overlap the
-    # neighboring steps' kernels, as a stream-ordered caller would
-    host_pos = torch.from_numpy(s.pos).pin_memory()
-    host_perm = [torch.empty(s.n, dtype=torch.int32).pin_memory() for _ in range(2)]
-    host_counts = [torch.empty(s.n, dtype=torch.int32).pin_memory() for _ in range(2)]
-    host_flags = [torch.empty(2, dtype=torch.int32).pin_memory() for _ in range(2)]
-    pos_in = [torch.empty_like(step.pos3) for _ in range(2)]
-    st_perm = [torch.empty_like(step.perm) for _ in range(2)]
-    st_counts = [torch.empty_like(step.counts) for _ in range(2)]
-    st_flags = [torch.empty(2, dtype=torch.int32, device=dev) for _ in range(2)]
-    cs = torch.cuda.current_stream()
-    xs = torch.cuda.Stream(device=dev)
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_out = [torch.cuda.Event() for _ in range(2)]
-    ev_read = [torch.cuda.Event() for _ in range(2)]
-    e2e_steps = max(1, args.steps)
+
+def _step_graph_loop(step, dev):
+    """A time-step loop over a random walk (sigma per axis per step): the step
+    graph decides rebuilds on the device; the eager loop reads the skin
+    check's flag back every step and calls the rebuild itself."""
+    import ctypes
+    import torch
+    tess, s = step.tess, step.s
+    nsteps = 30
+    gen = torch.Generator(device=dev).manual_seed(5)
+    L = torch.tensor(s.box, dtype=torch.float32, device=dev)
+    walk = [step.pos3.clone()]
+    for _ in range(nsteps):
+        x = walk[-1] + torch.randn(walk[-1].shape, generator=gen, device=dev) * s.sigma
+        walk.append(torch.remainder(x, L).contiguous())
+    sg = tess.StepGraph(walk[0], s.box, s.rc, s.skin, s.cap, step.feat)
+    try:
+        def run_graph():
+            for t in range(nsteps):
+                sg.pos.copy_(walk[t])
+                sg.launch()
+        with torch.cuda.stream(sg.stream):
+            run_graph()                                    # warm-up (and first rebuild)
+            sg.request_rebuild()
+        before = sg.rebuilds
+        with torch.cuda.stream(sg.stream):
+            a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_ev.record()
+            run_graph()
+            b_ev.record()
+        sg.stream.synchronize()
+        g_ms = a_ev.elapsed_time(b_ev) / nsteps
+        g_rebuilds = sg.rebuilds - before
+    finally:
+        sg.close()
+    ref4 = torch.empty((s.n, 4), dtype=torch.float32, device=dev)
+    cur4 = torch.zeros((s.n, 4), dtype=torch.float32, device=dev)
+    flag = torch.empty(1, dtype=torch.int32, device=dev)
+    md2 = torch.empty(1, dtype=torch.float64, device=dev)
+    P = lambda t_: ctypes.c_void_p(t_.data_ptr())
+    stc = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+    def run_eager():
+        rebuilds = 0
+        for t in range(nsteps):
+            pos = walk[t]
+            if t == 0:
+                r = 1
+            else:
+                cur4[:, :3] = pos[step.perm.long()]
+                assert tess.tess_skin_check(P(cur4), P(ref4), s.n, s.box, s.skin, P(flag), P(md2), stc) == 0
+                r = int(flag.item())                     # the host round trip of a host-driven loop
+            if r:
+                rebuilds += 1
+                assert step.sort_fn(P(pos), s.n, s.box, 10, P(step.ws_sort), step.ws_sort.numel(), P(step.perm),
+                                    P(step.keys), P(ref4), P(step.status), stc) == 0
+                assert tess.tess_build_neighbors(P(ref4), s.n, s.box, s.rc, s.skin, s.cap, 0, P(step.ws_nbr),
+                                                 step.ws_nbr.numel(), P(step.nbr), P(step.counts),
+                                                 P(step.overflow), stc) == 0
+                cur4.copy_(ref4)
+            assert tess.tess_edge_aggregate(P(cur4), s.n, s.box, s.rc, P(step.nbr), P(step.counts), s.cap,
+                                            P(step.feat), s.F, P(step.out), None, None, None, stc) == 0
+        return rebuilds
+    run_eager()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(cs)
-    xs.wait_stream(cs)
-    with torch.cuda.stream(xs):
-        for b in range(min(2, e2e_steps)):
-            pos_in[b].copy_(host_pos, non_blocking=True)
-            ev_in[b].record(xs)
-    for t in range(e2e_steps):
-        b = t % 2
-        cs.wait_event(ev_in[b])
-        step.run(pos3=pos_in[b])
-        if t >= 2:
-            cs.wait_event(ev_read[b])            # step t-2's results have left the staging buffers
-        st_perm[b].copy_(step.perm)
-        st_counts[b].copy_(step.counts)
-        st_flags[b][0:1].copy_(step.overflow)
-        st_flags[b][1:2].copy_(step.rebuild)
-        ev_out[b].record(cs)
-        with torch.cuda.stream(xs):
-            xs.wait_event(ev_out[b])
-            host_perm[b].copy_(st_perm[b], non_blocking=True)
-            host_counts[b].copy_(st_counts[b], non_blocking=True)
-            host_flags[b].copy_(st_flags[b], non_blocking=True)
-            ev_read[b].record(xs)
-            if t + 2 < e2e_steps:                  # step t has read pos_in[b]: load step t+2's positions
-                pos_in[b].copy_(host_pos, non_blocking=True)
-                ev_in[b].record(xs)
-    cs.wait_stream(xs)
-    e1.record(cs)
+    a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a_ev.record()
+    e_rebuilds = run_eager()
+    b_ev.record()
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    e2e_val = sum_over_ranks(float(s.n * e2e_steps), world, dev) / (e2e_ms / 1e3)
-
-    peak, peak_kind = _peaks()
-    nbytes = _algorithmic_bytes(s.n, mean_count, s.F)
-    stage_ms = {k: (v[0] / max(v[1], 1)) for k, v in stages.items() if v[1] > 0}
-    dom = max(stage_ms, key=stage_ms.get)
-    achieved = nbytes[dom] / (stage_ms[dom] / 1e3) / 1e9
-    traffic = _traffic_from_profile(dom, s.n, s.name)
-    clocks = clk.summary()
-
-    if rank == 0:
-        line = {
-            "metric": METRIC,
-            "value": value,
-            "unit": "atoms/s",
-            "n_gpus": world,
-            "steps": args.steps,
-            "warmup": args.warmup,
-            "ms_per_step": ms_max / args.steps,
-            "higher_is_better": True,
-            "scaling": "weak",
-            "vs_baseline": None,
-            "dtype": "f32",
-            "data": "synthetic (seeded salt-solution generator; no dataset)",
-            "config": {
-                "workload": "%s: %d atoms, box %.3f x %.3f x %.3f A, rc %.2f, skin %.2f, cap %d, F %d; step = "
-                            "hilbert_sort + build_neighbors (pad-filled) + skin_check + edge_aggregate"
-                            % (s.name, s.n, s.box[0], s.box[1], s.box[2], s.rc, s.skin, s.cap, s.F),
-                "atoms": s.n,
-                "pad_fill": not args.no_pad_fill,
-                "pair_search": "tile" if args.tile_search else "per-lane",
-                "curve": args.curve,
-                "l2": "flushed between timed steps (256 MB write); each step also moves ~9 GB",
-                "parallelism": "replicas (no collective in the data path)",
-                "mean_neighbors": mean_count,
-                "pairs_listed": pairs,
-                "overflow": ov,
-            },
-            "stages_ms": {k: round(v, 4) for k, v in stage_ms.items()},
-            "rebuild_atoms_per_s": s.n / ((stage_ms.get("hilbert_keys", 0) + stage_ms.get("key_sort", 0)
-                                           + stage_ms.get("cell_binning", 0) + stage_ms.get("pair_search", 0)) / 1e3),
-            "pairs_per_s": pairs / (stage_ms.get("pair_search", float("nan")) / 1e3),
-            "roofline": {
-                "bound": "hbm",
-                "kernel": dom,
-                "achieved": achieved,
-                "peak": peak,
-                "peak_kind": peak_kind,
-                "unit": "GB/s",
-                "frac": achieved / peak,
-                "traffic": traffic,
-                "algorithmic_bytes": nbytes[dom],
-            },
-            "rebuild_roofline": _rebuild_roofline(s.n, mean_count, stage_ms, peak),
-            "e2e": {"value": e2e_val, "unit": "atoms/s", "steps": e2e_steps, "pipelined": True, "h2d_bytes_per_step": s.n * 12,
-                    "d2h_bytes_per_step": s.n * 8 + 8},
-            "gpu_launches": launches,
-            "graph": graph,
-            "backward": backward,
-            "resort": resort,
-            "min_pair": monitor,
-            "step_graph": step_graph,
-            "clocks": clocks,
-        }
-        if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(args)
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        torch.distributed.destroy_process_group()
-
-
-def _rebuild_roofline(n, mean_count, stage_ms, peak):
-    t = sum(stage_ms.get(k, 0.0) for k in ("hilbert_keys", "key_sort", "cell_binning", "pair_search"))
-    b = n * (24 + 12 + 36 + 28 + 16 + 4 * mean_count + 4)
-    return {"ms": t, "algorithmic_bytes": b, "achieved_gbs": b / (t / 1e3) / 1e9 if t else None,
-            "frac": (b / (t / 1e3) / 1e9) / peak if t else None}
+    e_ms = a_ev.elapsed_time(b_ev) / nsteps
+    return {"steps": nsteps, "sigma": s.sigma, "graph_ms_per_step": g_ms, "eager_ms_per_step": e_ms,
+            "speedup": e_ms / g_ms, "graph_rebuilds": g_rebuilds, "eager_rebuilds": e_rebuilds}
 
 
 def _traffic_from_profile(kernel_stage, n, workload=""):
@@ -588,12 +668,11 @@ def _traffic_from_profile(kernel_stage, n, workload=""):
 # ---------------------------------------------------------------- oracle arm
 
 
-def _oracle_step(s, feat):
-    """One step of the path on the CPU oracle (sort, list, skin, aggregate)."""
+def _oracle_step(s):
+    """One full rebuild on the CPU oracle: Hilbert sort, then the cell-list
+    Verlet list."""
     import oracle
     perm, keys, ps, nbr, cnt, ov = oracle.rebuild(s.pos, s.box, s.rc, s.skin, s.cap)
-    oracle.skin_check(ps, ps, s.box, s.skin)
-    oracle.edge_aggregate(ps, s.box, s.rc, nbr, cnt, feat)
     return int(cnt.sum())
 
 
@@ -608,12 +687,11 @@ def _sample_system(budget_steps: int):
 def cpu_baseline(args):
     import oracle
     s = _sample_system(1)
-    feat = s.features()
     t = time.perf_counter()
-    _oracle_step(s, feat)
+    _oracle_step(s)
     dt = time.perf_counter() - t
     return {"value": s.n / dt, "unit": "atoms/s", "cores": oracle.get_threads(), "kind": "oracle",
-            "sample": "one full step (sort, cell-list Verlet list, skin check, aggregation) of %s "
+            "sample": "one full rebuild (Hilbert sort, cell-list Verlet list) of %s "
                       "(%d atoms, same generator and rc/skin/cap/F family as the 10.24M workload), %.1f s"
                       % (s.name, s.n, dt)}
 
@@ -623,15 +701,14 @@ def run_reference(args, world, rank):
         return
     import oracle
     s = _sample_system(args.steps + args.warmup)
-    feat = s.features()
     for _ in range(args.warmup):
-        _oracle_step(s, feat)
+        _oracle_step(s)
     t = time.perf_counter()
     for _ in range(args.steps):
-        _oracle_step(s, feat)
+        _oracle_step(s)
     dt = time.perf_counter() - t
     value = s.n * args.steps / dt
-    sample = "%s (%d atoms) per step, the plain CPU oracle on %d host threads" % (s.name, s.n, oracle.get_threads())
+    sample = "%s (%d atoms) per rebuild, the plain CPU oracle on %d host threads" % (s.name, s.n, oracle.get_threads())
     line = {
         "impl": "reference",
         "metric": METRIC,
@@ -662,7 +739,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["tess", "reference"], default="tess")
     ap.add_argument("--config", type=int, default=WORKLOAD_CFG)
     ap.add_argument("--no-pad-fill", action="store_true")
-    ap.add_argument("--tile-search", action="store_true", help="use the warp-shared tile pair search")
+    ap.add_argument("--lane-search", action="store_true", help="use the per-lane stencil pair search")
     ap.add_argument("--curve", choices=["hilbert", "morton"], default="hilbert",
                     help="space-filling curve of the sort (morton: the comparison curve)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -673,6 +750,8 @@ def main(argv=None):
     ap.add_argument("--monitor", action="store_true", help="also time the closest-listed-pair check on the step's list")
     ap.add_argument("--resort", action="store_true",
                     help="also time the incremental re-sort against the full sort a rebuild interval later")
+    ap.add_argument("--all-configs", action="store_true",
+                    help="also report rebuild, skin check and aggregation on all five workloads")
     args = ap.parse_args(argv)
     world, rank, local = _dist_setup(args)
     if args.impl == "reference":

@@ -61,10 +61,12 @@ typedef struct {
 #define TESS_DEV_BAD_INPUT  2   /* some position outside [0, L) or not finite (clamped into the grid) */
 #define TESS_DEV_TIMEOUT    4   /* an inter-block wait gave up; outputs of that call are invalid */
 #define TESS_DEV_FULL_SORT  8   /* tess_hilbert_resort ran the full sort (its fast path did not apply) */
+#define TESS_DEV_CHECK     16   /* checked builds (-DTESS_CHECK) only: a kernel met an index out of range
+                                   and skipped that access */
 
 /* tess_build_neighbors flags */
 #define TESS_NO_PAD_FILL    1   /* leave slots >= min(count, max_neighbors) unwritten */
-#define TESS_TILE_SEARCH    2   /* use the warp-shared tile search instead of the per-lane search */
+#define TESS_LANE_SEARCH    2   /* use the per-lane stencil search instead of the warp tile search */
 
 /* Human-readable name of a status code (static string). */
 const char* tess_status_string(tess_status s);
@@ -172,8 +174,10 @@ tess_status tess_morton_sort(const float* pos, int n, tess_box box, int bits,
  *   n  1 .. TESS_HILBERT_SORT_STATIC_MAX_N; larger n returns
  *      TESS_ERR_TOO_LARGE (use tess_hilbert_sort with a workspace instead)
  *
- * The first call on a device looks up the array's device address (with that
- * device current); make that first call before any stream capture.  All calls
+ * Each call looks up the array's device address in the current context (a
+ * host-side query, so a context destroyed and created again never receives
+ * a stale address); the first call in a context may load the library's
+ * device code, so make it before any stream capture.  All calls
  * on a device share the array: calls that overlap on the GPU (different
  * streams, or unordered host threads) race on it and corrupt each other's
  * results, so order them on one stream.  Each call clears what must start at
@@ -200,8 +204,9 @@ tess_status tess_hilbert_sort_static(const float* pos, int n, tess_box box, int 
  *   pos            [n,4] float (x, y, z, ignored), 16-byte aligned
  *   rc, skin       cutoff and skin (rc > 0, skin >= 0); rs = rc + skin in fp32
  *   max_neighbors  row capacity cap >= 1
- *   flags          0, or'ed TESS_NO_PAD_FILL, TESS_TILE_SEARCH (same lists, other
- *                  search order; boxes shorter than 2 rs + 2e-3 always use it)
+ *   flags          0, or'ed TESS_NO_PAD_FILL, TESS_LANE_SEARCH (same lists, other
+ *                  order within rows; boxes shorter than 2 rs + 2e-3 always use
+ *                  the default tile search)
  *   ws, ws_bytes   scratch of at least tess_build_neighbors_workspace(...)
  *   nbr            [n, cap] int32 out: row i in nbr[i*cap .. i*cap+cap);
  *                  the first min(counts[i], cap) slots hold neighbors, the
@@ -403,7 +408,11 @@ tess_status tess_debug_lookback_timeout(void* ws, size_t ws_bytes, int32_t* dev_
  * 7 incremental re-sort (its fallback full sort records under 0 and 1),
  * 8 closest listed pair.  Returns the number of
  * stages written (<= max_stages).  ms_out[k] = total milliseconds,
- * calls_out[k] (nullable) = number of timed calls.
+ * calls_out[k] (nullable) = number of timed calls.  The events are kept in a
+ * process-wide pool and reused: after one timed round has been read back, a
+ * second round records without creating events.  The pool, the records and
+ * the on/off switch are the library's only process state (a mutex guards
+ * them); stage timing is off unless enabled.
  * ------------------------------------------------------------------------- */
 void tess_stage_timing(int enable);
 int tess_stage_times(double* ms_out, long long* calls_out, int max_stages);

@@ -4,6 +4,10 @@
 
 #include "common.cuh"
 
+#ifdef TESS_NVTX
+#include <nvtx3/nvToolsExt.h>
+#endif
+
 namespace tess {
 
 std::atomic<long long> g_launches{0};
@@ -40,6 +44,9 @@ tess_status edge_backward(const float* pos, int n, tess_box box, float rc, const
 // ---------------------------------------------------------------- stage timing
 
 namespace {
+// Stage timing state.  Events are recycled through a pool: a scope takes two
+// from the pool (creating them only when it is empty) and tess_stage_times
+// gives them back, so a warmed-up timing loop creates no events.
 struct Timing {
     std::mutex mu;
     bool enabled = false;
@@ -48,6 +55,20 @@ struct Timing {
         cudaEvent_t a, b;
     };
     std::vector<Rec> recs;
+    std::vector<cudaEvent_t> pool;
+    cudaEvent_t take() {
+        if (!pool.empty()) {
+            cudaEvent_t e = pool.back();
+            pool.pop_back();
+            return e;
+        }
+        cudaEvent_t e = nullptr;
+        if (cudaEventCreate(&e) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        return e;
+    }
 };
 Timing& timing() {
     static Timing t;
@@ -56,6 +77,9 @@ Timing& timing() {
 }  // namespace
 
 StageScope::StageScope(int stage_, cudaStream_t s_) : stage(stage_), s(s_) {
+#ifdef TESS_NVTX
+    nvtxRangePushA(stage_name(stage));
+#endif
     Timing& t = timing();
     std::lock_guard<std::mutex> g(t.mu);
     if (!t.enabled) return;
@@ -63,12 +87,21 @@ StageScope::StageScope(int stage_, cudaStream_t s_) : stage(stage_), s(s_) {
     // graph (conditional bodies), and a captured stage runs at replay time
     cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
     if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return;
-    cudaEventCreate(&a);
-    cudaEventCreate(&b);
+    a = t.take();
+    b = t.take();
+    if (!a || !b) {
+        if (a) t.pool.push_back(a);
+        if (b) t.pool.push_back(b);
+        a = b = nullptr;
+        return;
+    }
     cudaEventRecord(a, s);
 }
 
 StageScope::~StageScope() {
+#ifdef TESS_NVTX
+    nvtxRangePop();
+#endif
     if (!a) return;
     cudaEventRecord(b, s);
     Timing& t = timing();
@@ -195,8 +228,14 @@ int tess_stage_times(double* ms_out, long long* calls_out, int max_stages) {
             ms_out[r.stage] += ms;
             if (calls_out) calls_out[r.stage] += 1;
         }
-        cudaEventDestroy(r.a);
-        cudaEventDestroy(r.b);
+    }
+    cudaGetLastError();
+    {
+        std::lock_guard<std::mutex> g(t.mu);
+        for (auto& r : recs) {
+            t.pool.push_back(r.a);
+            t.pool.push_back(r.b);
+        }
     }
     return ns;
 }

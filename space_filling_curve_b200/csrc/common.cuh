@@ -20,7 +20,9 @@ inline void count_launch(long long k = 1) { g_launches.fetch_add(k, std::memory_
 // Stage ids for the optional event timing.
 enum Stage { ST_KEYS = 0, ST_SORT = 1, ST_CELLS = 2, ST_PAIRS = 3, ST_SKIN = 4, ST_EDGE = 5, ST_BACKWARD = 6, ST_RESORT = 7, ST_MONITOR = 8, ST_COUNT = 9 };
 
-// Records an event pair around a stage when stage timing is enabled.
+// Records an event pair around a stage when stage timing is enabled; in a
+// build with -DTESS_NVTX it also opens an NVTX range named after the stage
+// (host-side, around the launches), for timeline profilers.
 struct StageScope {
     int stage;
     cudaStream_t s;
@@ -28,6 +30,14 @@ struct StageScope {
     StageScope(int stage_, cudaStream_t s_);
     ~StageScope();
 };
+
+// Stage names, as the Python binding reports them.
+inline const char* stage_name(int stage) {
+    static const char* const names[ST_COUNT] = {"hilbert_keys", "key_sort", "cell_binning", "pair_search",
+                                                "skin_check", "edge_aggregate", "edge_backward", "resort",
+                                                "min_pair"};
+    return stage >= 0 && stage < ST_COUNT ? names[stage] : "tess";
+}
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -59,6 +69,20 @@ __device__ __forceinline__ unsigned lanemask_lt() {
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
     return m;
 }
+
+// Checked builds (-DTESS_CHECK): an index that a kernel scatters to or
+// gathers from is tested against its bound; a bad one sets TESS_DEV_CHECK in
+// the status word given and the access is skipped.  In the product build the
+// test compiles away.
+#ifdef TESS_CHECK
+__device__ __forceinline__ bool check_index(long long idx, long long bound, int32_t* status) {
+    if (idx >= 0 && idx < bound) return true;
+    if (status) atomicOr(status, TESS_DEV_CHECK);
+    return false;
+}
+#else
+__device__ __forceinline__ bool check_index(long long, long long, int32_t*) { return true; }
+#endif
 
 __device__ __forceinline__ int floor_div(int a, int b) {
     int q = a / b;

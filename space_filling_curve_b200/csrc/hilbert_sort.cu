@@ -12,7 +12,10 @@
 //                    pass writes perm / keys / float4 positions directly.
 // Elements carry the input index in the low word, so equal keys keep input
 // order (stable passes) and the permutation is unique.
+#include <algorithm>
+
 #include "common.cuh"
+#include "scan.cuh"
 
 namespace tess {
 
@@ -185,12 +188,16 @@ __global__ __launch_bounds__(SORT_THREADS, TESS_SORT_MINB) void onesweep_pass(co
     if (gate && *gate != want) return;
     if (n_dev) n = *n_dev;
 
+    // persistent: each block takes tiles in order from the counter until none
+    // is left (a block only takes a tile while it runs, so the look-back
+    // never waits on a tile that has not started)
+    for (;;) {
     if (tid == 0) S.tile = (int)atomicAdd(tile_counter, 1u);
     for (int k = tid; k < SORT_WARPS * RADIX; k += SORT_THREADS) (&S.wcnt[0][0])[k] = 0u;
     __syncthreads();
     const int tile = S.tile;
     const long long base = (long long)tile * TILE;
-    if (base >= n) return;     // a spare tile of a device-sized launch
+    if (base >= n) return;     // every tile is taken
     const long long wbase = base + (long long)warp * ITEMS * 32;
 
     unsigned long long e[ITEMS];
@@ -277,6 +284,7 @@ __global__ __launch_bounds__(SORT_THREADS, TESS_SORT_MINB) void onesweep_pass(co
         const unsigned long long v = S.elems[s];
         const unsigned d = (unsigned)(v >> shift) & 0xffu;
         const unsigned long long g = S.gbase[d] + (unsigned long long)(s - (int)S.lbase[d]);
+        if (!check_index((long long)g, n, status)) continue;
         if (FINAL) {
             const unsigned idx = (unsigned)v;
             perm[g] = (int32_t)idx;
@@ -289,6 +297,164 @@ __global__ __launch_bounds__(SORT_THREADS, TESS_SORT_MINB) void onesweep_pass(co
             out[g] = v;
         }
     }
+    __syncthreads();           // the next tile reuses the shared memory
+    }
+}
+
+// ---------------------------------------------------------------- bucket sort (default)
+//
+// The default path sorts in one bucketing pass plus local sorts:
+//   bucket_keys_kernel    key per atom, element (key << 32 | index), and the
+//                         count of its bucket (the top bits of the key)
+//   exclusive_scan        bucket offsets
+//   bucket_scatter_kernel every element into its bucket (any order inside)
+//   bucket_local_sort     one warp per bucket ranks its elements by the full
+//                         64-bit element (rank = number of smaller elements)
+//                         and writes perm / keys / float4 positions at
+//                         offset + rank
+// Elements are unique, so the order inside a bucket is fixed by the local
+// ranks whatever order the scatter left them in.  Buckets hold about 40
+// atoms; a bucket larger than BK_LOCAL_MAX (clustered input, a coarse grid)
+// sets a device flag, and the LSD onesweep sort above -- launched gated on
+// that flag -- then writes every output instead (no host synchronisation).
+
+constexpr int BK_THREADS = 256;
+constexpr int BK_LOCAL_MAX = 256;    // largest bucket a warp sorts (8 elements per lane)
+constexpr int BK_WARPS = 8;          // warps per block of the local sort
+constexpr int BK_TARGET = 40;        // mean bucket size the bucket bits aim for
+
+// Bits of the key that name the bucket: about n / BK_TARGET buckets, at most
+// the key's 3 * bits bits and 2^20 buckets.
+static int bucket_bits(int n, int bits) {
+    int db = 0;
+    while (db < 20 && ((long long)BK_TARGET << db) < (long long)n) ++db;
+    return std::min(db, 3 * bits);
+}
+
+template <int CURVE>
+__global__ __launch_bounds__(BK_THREADS) void bucket_keys_kernel(const float* __restrict__ pos, int n, float3 scale,
+                                                                 float3 L, int bits, int bshift,
+                                                                 unsigned long long* __restrict__ elems,
+                                                                 int* __restrict__ bcount, int32_t* status) {
+    const uint32_t top = (1u << bits) - 1u;
+    bool bad = false;
+    const int stride = gridDim.x * blockDim.x;
+    for (int base = blockIdx.x * blockDim.x; base < n; base += stride) {
+        const int i = base + (int)threadIdx.x;
+        const bool valid = i < n;
+        uint32_t b = 0;
+        if (valid) {
+            const float x = pos[3 * (size_t)i], y = pos[3 * (size_t)i + 1], z = pos[3 * (size_t)i + 2];
+            bad |= !(x >= 0.0f && x < L.x && y >= 0.0f && y < L.y && z >= 0.0f && z < L.z);
+            const uint32_t qx = quantize(x, scale.x, top), qy = quantize(y, scale.y, top),
+                           qz = quantize(z, scale.z, top);
+            const uint32_t key = CURVE == 0 ? hilbert_key(qx, qy, qz, bits) : morton_key(qx, qy, qz);
+            elems[i] = ((unsigned long long)key << 32) | (unsigned)i;
+            b = key >> bshift;
+        }
+        const unsigned act = __ballot_sync(FULL, valid);
+        if (valid) {
+            // one atomic per group of lanes in the same bucket
+            const unsigned peers = __match_any_sync(act, b);
+            if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&bcount[b], __popc(peers));
+        }
+    }
+    if (__any_sync(FULL, bad) && (threadIdx.x & 31) == 0 && status) atomicOr(status, TESS_DEV_BAD_INPUT);
+}
+
+__global__ __launch_bounds__(BK_THREADS) void bucket_scatter_kernel(const unsigned long long* __restrict__ in, int n,
+                                                                    int bshift, const int* __restrict__ bstart,
+                                                                    int* __restrict__ cursor,
+                                                                    unsigned long long* __restrict__ out,
+                                                                    int32_t* status) {
+    const int stride = gridDim.x * blockDim.x;
+    const int lane = threadIdx.x & 31;
+    for (int base = blockIdx.x * blockDim.x; base < n; base += stride) {
+        const int i = base + (int)threadIdx.x;
+        const bool valid = i < n;
+        const unsigned long long e = valid ? in[i] : 0ull;
+        const uint32_t b = (uint32_t)(e >> 32) >> bshift;
+        const unsigned act = __ballot_sync(FULL, valid);
+        if (valid) {
+            const unsigned peers = __match_any_sync(act, b);
+            const int leader = __ffs(peers) - 1;
+            int off = 0;
+            if (lane == leader) off = atomicAdd(&cursor[b], __popc(peers));
+            off = __shfl_sync(peers, off, leader) + __popc(peers & lanemask_lt());
+            const long long slot = (long long)bstart[b] + off;
+            if (check_index(slot, n, status)) out[slot] = e;
+        }
+    }
+}
+
+// Ranks of the lane's K elements among the bucket's m (shared memory s).
+template <int K>
+__device__ __forceinline__ void bucket_ranks(const unsigned long long* s, int m, const unsigned long long (&e)[8],
+                                             int (&r)[8]) {
+#pragma unroll 4
+    for (int t = 0; t < m; ++t) {
+        const unsigned long long v = s[t];
+#pragma unroll
+        for (int k = 0; k < K; ++k) r[k] += v < e[k] ? 1 : 0;
+    }
+}
+
+__global__ __launch_bounds__(BK_WARPS * 32) void bucket_local_sort(const unsigned long long* __restrict__ elems,
+                                                                   const int* __restrict__ bstart, int nb,
+                                                                   const float* __restrict__ pos3,
+                                                                   int32_t* __restrict__ perm,
+                                                                   uint32_t* __restrict__ keys_out,
+                                                                   float4* __restrict__ pos_sorted,
+                                                                   int32_t* fallback, int n, int32_t* status) {
+    __shared__ unsigned long long s_el[BK_WARPS][BK_LOCAL_MAX];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned long long* s = s_el[warp];
+    for (int b = blockIdx.x * BK_WARPS + warp; b < nb; b += gridDim.x * BK_WARPS) {
+        const int beg = bstart[b], m = bstart[b + 1] - beg;
+        if (m == 0) continue;
+        if (m > BK_LOCAL_MAX) {
+            if (lane == 0) atomicOr(fallback, 1);
+            continue;
+        }
+        for (int t = lane; t < m; t += 32) s[t] = elems[beg + t];
+        __syncwarp();
+        const int K = (m + 31) >> 5;
+        unsigned long long e[8];
+        int r[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int t = lane + 32 * k;
+            e[k] = (k < K && t < m) ? s[t] : ~0ull;
+            r[k] = 0;
+        }
+        if (K == 1) bucket_ranks<1>(s, m, e, r);
+        else if (K == 2) bucket_ranks<2>(s, m, e, r);
+        else if (K <= 4) bucket_ranks<4>(s, m, e, r);
+        else bucket_ranks<8>(s, m, e, r);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int t = lane + 32 * k;
+            if (k < K && t < m && check_index((long long)beg + r[k], n, status) &&
+                check_index((long long)(unsigned)e[k], n, status)) {
+                const int g = beg + r[k];
+                const unsigned idx = (unsigned)e[k];
+                perm[g] = (int32_t)idx;
+                if (keys_out) keys_out[g] = (uint32_t)(e[k] >> 32);
+                if (pos_sorted) {
+                    const float* p = pos3 + 3 * (size_t)idx;
+                    pos_sorted[g] = make_float4(p[0], p[1], p[2], 0.0f);
+                }
+            }
+        }
+        __syncwarp();
+    }
+}
+
+// Zeroes `words` 64-bit words when *gate == want (the fallback's state).
+__global__ void zero_if_kernel(unsigned long long* p, size_t words, const int32_t* gate, int want) {
+    if (*gate != want) return;
+    for (size_t k = blockIdx.x * (size_t)blockDim.x + threadIdx.x; k < words; k += (size_t)gridDim.x * blockDim.x)
+        p[k] = 0ull;
 }
 
 // ---------------------------------------------------------------- host
@@ -321,11 +487,6 @@ static SortLayout sort_layout(void* ws, int n) {
     L.zero_bytes = c.off - L.zero_begin;
     L.total = align_up(c.off, 256);
     return L;
-}
-
-size_t hilbert_sort_workspace(int n) {
-    if (n <= 0) return 0;
-    return sort_layout(nullptr, n).total;
 }
 
 static float3 grid_scale(tess_box box, int bits) {
@@ -362,6 +523,8 @@ static void sfc_sort_launch(const float* pos, int n, tess_box box, int bits, int
     {
         StageScope sc(ST_SORT, s);
         const long long tiles = tiles_for(n);
+        // persistent passes: at most the resident blocks, each looping over tiles
+        const unsigned grid = (unsigned)std::min<long long>(tiles, (long long)sms * TESS_SORT_MINB);
         const size_t smem = sizeof(SortShared);
         static_assert(sizeof(SortShared) <= 48 * 1024, "sort tile must fit the default shared-memory limit");
         unsigned long long* src = L.a;
@@ -369,11 +532,11 @@ static void sfc_sort_launch(const float* pos, int n, tess_box box, int bits, int
         for (int p = 0; p < npass; ++p) {
             unsigned long long* states = L.states + (size_t)p * tiles * RADIX;
             if (p == npass - 1) {
-                onesweep_pass<true><<<(unsigned)tiles, SORT_THREADS, smem, s>>>(
+                onesweep_pass<true><<<grid, SORT_THREADS, smem, s>>>(
                     src, nullptr, n, 32 + 8 * p, L.hist + p * RADIX, states, L.counters + p, status, perm,
                     keys_sorted, reinterpret_cast<float4*>(pos_sorted), pos, nullptr, gate, want);
             } else {
-                onesweep_pass<false><<<(unsigned)tiles, SORT_THREADS, smem, s>>>(
+                onesweep_pass<false><<<grid, SORT_THREADS, smem, s>>>(
                     src, dst, n, 32 + 8 * p, L.hist + p * RADIX, states, L.counters + p, status, nullptr, nullptr,
                     nullptr, nullptr, nullptr, gate, want);
             }
@@ -383,19 +546,85 @@ static void sfc_sort_launch(const float* pos, int n, tess_box box, int bits, int
     }
 }
 
+// Workspace of the default sort: the LSD sort's layout (its two element
+// buffers also carry the bucket pass), then the bucket counts / offsets.
+struct BucketLayout {
+    SortLayout lsd;
+    int* bcount;             // [nb] counts, then scatter cursors
+    int32_t* flag;           // 1: some bucket too large for the local sort
+    int* bstart;             // [nb + 1]
+    int* sums;               // scan scratch
+    size_t zero_begin, zero_bytes, total;
+};
+
+static BucketLayout bucket_layout(void* ws, int n) {
+    BucketLayout B{};
+    B.lsd = sort_layout(ws, n);
+    Carve c(ws);
+    c.off = B.lsd.total;
+    const long long nb = 1LL << bucket_bits(n, 10);
+    c.off = align_up(c.off, 256);
+    B.zero_begin = c.off;
+    B.bcount = c.take<int>((size_t)nb);
+    B.flag = c.take<int32_t>(1);
+    B.zero_bytes = c.off - B.zero_begin;
+    B.bstart = c.take<int>((size_t)nb + 1);
+    B.sums = c.take<int>((size_t)scan_sums_len(nb));
+    B.total = align_up(c.off, 256);
+    return B;
+}
+
+size_t hilbert_sort_workspace(int n) {
+    if (n <= 0) return 0;
+    return bucket_layout(nullptr, n).total;
+}
+
 tess_status sfc_sort(const float* pos, int n, tess_box box, int bits, int curve, void* ws, size_t ws_bytes,
                      int32_t* perm, uint32_t* keys_sorted, float* pos_sorted, int32_t* dev_status, cudaStream_t s) {
     if (n <= 0 || !pos || !perm || !ws || bits < 1 || bits > 10) return TESS_ERR_INVALID_ARG;
     if (!finite_pos(box.lx) || !finite_pos(box.ly) || !finite_pos(box.lz)) return TESS_ERR_INVALID_ARG;
     if (pos_sorted && !aligned(pos_sorted, 16)) return TESS_ERR_INVALID_ARG;
     if (!aligned(ws, 256)) return TESS_ERR_INVALID_ARG;
-    SortLayout L = sort_layout(ws, n);
-    if (ws_bytes < L.total) return TESS_ERR_WORKSPACE_TOO_SMALL;
+    BucketLayout B = bucket_layout(ws, n);
+    if (ws_bytes < B.total) return TESS_ERR_WORKSPACE_TOO_SMALL;
+    const SortLayout& L = B.lsd;
     int32_t* status = dev_status ? dev_status : L.status;
 
-    cudaMemsetAsync(static_cast<char*>(ws) + L.zero_begin, 0, L.zero_bytes, s);
+    const int db = bucket_bits(n, bits);
+    const long long nb = 1LL << db;
+    const int bshift = 3 * bits - db;
+    const float3 scale = grid_scale(box, bits);
+    const float3 Lb = make_float3(box.lx, box.ly, box.lz);
+    const int sms = sm_count();
+    const int blocks = (int)std::min<long long>(((long long)n + BK_THREADS - 1) / BK_THREADS, (long long)sms * 8);
+
+    cudaMemsetAsync(static_cast<char*>(ws) + B.zero_begin, 0, B.zero_bytes, s);
     if (dev_status) cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s);
-    sfc_sort_launch(pos, n, box, bits, curve, L, perm, keys_sorted, pos_sorted, status, nullptr, 0, s);
+    {
+        StageScope sc(ST_KEYS, s);
+        if (curve == 0)
+            bucket_keys_kernel<0><<<blocks, BK_THREADS, 0, s>>>(pos, n, scale, Lb, bits, bshift, L.a, B.bcount,
+                                                                 status);
+        else
+            bucket_keys_kernel<1><<<blocks, BK_THREADS, 0, s>>>(pos, n, scale, Lb, bits, bshift, L.a, B.bcount,
+                                                                 status);
+        count_launch();
+    }
+    {
+        StageScope sc(ST_SORT, s);
+        exclusive_scan(B.bcount, nb, B.sums, B.bstart, s);
+        bucket_scatter_kernel<<<blocks, BK_THREADS, 0, s>>>(L.a, n, bshift, B.bstart, B.bcount, L.b, status);
+        const int lblocks = (int)std::min<long long>((nb + BK_WARPS - 1) / BK_WARPS, (long long)sms * 16);
+        bucket_local_sort<<<lblocks, BK_WARPS * 32, 0, s>>>(L.b, B.bstart, (int)nb, pos, perm, keys_sorted,
+                                                           reinterpret_cast<float4*>(pos_sorted), B.flag, n, status);
+        count_launch(2);
+        // a bucket too large for the local sort: the LSD sort, gated on the flag
+        zero_if_kernel<<<sms * 2, 256, 0, s>>>(reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) +
+                                                                                     L.zero_begin),
+                                               L.zero_bytes / 8, B.flag, 1);
+        count_launch();
+    }
+    sfc_sort_launch(pos, n, box, bits, curve, L, perm, keys_sorted, pos_sorted, status, B.flag, 1, s);
     return launch_status();
 }
 
@@ -759,7 +988,8 @@ __global__ __launch_bounds__(RS_THREADS) void resort_merge_out(const unsigned lo
         const long long c = count_below(S, ms, v);
         bad |= (c < ms && S[c] == v) || (r + 1 < mo && !(v < Os[r + 1]));
         c_out[r] = (int)c;
-        write_sorted(r + c, v, pos3, perm, keys_out, pos_sorted);
+        if (check_index(r + c, ms + mo, nullptr)) write_sorted(r + c, v, pos3, perm, keys_out, pos_sorted);
+        else bad = true;          // checked builds: the full sort rewrites every slot
     }
     if (__any_sync(FULL, bad) && (threadIdx.x & 31) == 0) atomicExch(&ctl_w->fallback, 1);
 }
@@ -816,6 +1046,7 @@ __global__ __launch_bounds__(RS_THREADS) void resort_merge_local(const unsigned 
                 if (t >= t1) break;
                 const int below = staged ? lo + count_le(s_c, cnt, t) : count_le(c_out, mo, t);
                 const long long g = t + below;
+                if (!check_index(g, ctl->m_local + ctl->m_out, status)) continue;
                 perm[g] = (int32_t)(unsigned)v[u];
                 if (keys_out) keys_out[g] = (uint32_t)(v[u] >> 32);
                 if (pos_sorted) pos_sorted[g] = make_float4(q[u].x, q[u].y, q[u].z, 0.0f);

@@ -8,17 +8,22 @@
 //   cell_scatter   atom indices into their cells (any order within a cell)
 //   cell_order     within each cell, order by atom index and write the
 //                  positions in cell order as float4 (x, y, z, index bits)
-// Levels 1-3 (pair_search, one warp per tile of 32 consecutive atoms, lane =
-// atom i):
+// Levels 1-3 (pair_tile_kernel, the default; one warp per tile of 32
+// consecutive atoms, lane = atom i):
 //   1. tile: bounding box of the 32 atoms (Hilbert-consecutive, so compact)
-//   2. cells: every cell row overlapping box +- rs; each cell row is one
-//      contiguous range of the cell-ordered positions, shifted by its
-//      periodic image; candidates are culled against box +- rs and compacted
-//      (ballot + popc) into a shared-memory chunk
-//   3. pairs: every lane tests its atom against the chunk (broadcast reads)
-//      and appends accepted indices to its row in shared memory; the 32 rows
-//      are one contiguous block of the output and leave with 16-byte stores.
+//      and a frame centred on it
+//   2. cells: the cell rows within reach of the box, each clipped to the
+//      box's chord at its distance; each piece of a row is one contiguous
+//      range of the cell-ordered positions, shifted by its periodic image;
+//      candidates are culled against the rounded box and compacted (ballot
+//      + popc) into a shared-memory chunk
+//   3. pairs: every lane tests its atom against the chunk (broadcast reads,
+//      packed f32x2), 32 candidates per accept mask, and turns the set bits
+//      into indices that leave for its row in aligned 32-byte groups.
+// pair_search_lane_kernel (TESS_LANE_SEARCH) walks a stencil of cell rows
+// per lane instead; it gives the same lists in another order.
 #include "common.cuh"
+#include "scan.cuh"
 
 namespace tess {
 
@@ -98,95 +103,14 @@ __global__ void cell_count_kernel(const float4* __restrict__ pos, int n, int3 nc
     if (__any_sync(FULL, bad) && (threadIdx.x & 31) == 0 && status) atomicOr(status, TESS_DEV_BAD_INPUT);
 }
 
-constexpr int SCAN_THREADS = 1024;
-constexpr int SCAN_ITEMS = 4;
-constexpr int SCAN_TILE = SCAN_THREADS * SCAN_ITEMS;
-
-__device__ __forceinline__ int block_scan_incl(int v, int* s_warp) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        int y = __shfl_up_sync(FULL, v, o);
-        if (lane >= o) v += y;
-    }
-    if (lane == 31) s_warp[warp] = v;
-    __syncthreads();
-    if (warp == 0) {
-        int w = (lane < (int)(blockDim.x >> 5)) ? s_warp[lane] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            int y = __shfl_up_sync(FULL, w, o);
-            if (lane >= o) w += y;
-        }
-        s_warp[lane] = w;
-    }
-    __syncthreads();
-    const int add = warp > 0 ? s_warp[warp - 1] : 0;
-    __syncthreads();
-    return v + add;
-}
-
-// per-tile sums of the counts
-__global__ __launch_bounds__(SCAN_THREADS) void scan_reduce_kernel(const int* __restrict__ cnt, long long m,
-                                                                   int* __restrict__ sums) {
-    __shared__ int s_warp[32];
-    const long long b = (long long)blockIdx.x * SCAN_TILE + (long long)threadIdx.x * SCAN_ITEMS;
-    int v = 0;
-#pragma unroll
-    for (int k = 0; k < SCAN_ITEMS; ++k) v += (b + k < m) ? cnt[b + k] : 0;
-    const int tot = block_scan_incl(v, s_warp);
-    if (threadIdx.x == blockDim.x - 1) sums[blockIdx.x] = tot;
-}
-
-// exclusive scan of the per-tile sums, one block, any length
-__global__ __launch_bounds__(SCAN_THREADS) void scan_sums_kernel(int* sums, long long nt) {
-    __shared__ int s_warp[32];
-    __shared__ int s_carry;
-    if (threadIdx.x == 0) s_carry = 0;
-    __syncthreads();
-    for (long long b = 0; b < nt; b += SCAN_THREADS) {
-        const long long k = b + threadIdx.x;
-        const int v = k < nt ? sums[k] : 0;
-        const int inc = block_scan_incl(v, s_warp);
-        const int carry = s_carry;
-        if (k < nt) sums[k] = carry + inc - v;
-        __syncthreads();
-        if (threadIdx.x == blockDim.x - 1) s_carry = carry + inc;
-        __syncthreads();
-    }
-}
-
-// cell_start[c] = exclusive prefix; cnt[c] reset to 0 for the scatter cursor
-__global__ __launch_bounds__(SCAN_THREADS) void scan_apply_kernel(int* __restrict__ cnt, long long m,
-                                                                  const int* __restrict__ sums,
-                                                                  int* __restrict__ cell_start) {
-    __shared__ int s_warp[32];
-    const long long b = (long long)blockIdx.x * SCAN_TILE + (long long)threadIdx.x * SCAN_ITEMS;
-    int v[SCAN_ITEMS];
-    int tot = 0;
-#pragma unroll
-    for (int k = 0; k < SCAN_ITEMS; ++k) {
-        v[k] = (b + k < m) ? cnt[b + k] : 0;
-        tot += v[k];
-    }
-    const int inc = block_scan_incl(tot, s_warp);
-    int run = sums[blockIdx.x] + inc - tot;
-#pragma unroll
-    for (int k = 0; k < SCAN_ITEMS; ++k) {
-        if (b + k < m) {
-            cell_start[b + k] = run;
-            cnt[b + k] = 0;
-        }
-        run += v[k];
-    }
-    if (b < m && b + SCAN_ITEMS >= m) cell_start[m] = run;   // the thread holding the last cell
-}
-
 __global__ void cell_scatter_kernel(const int* __restrict__ cell_id, const int* __restrict__ cell_rank, int n,
-                                    const int* __restrict__ cell_start, int* __restrict__ slot_atom) {
+                                    const int* __restrict__ cell_start, int* __restrict__ slot_atom,
+                                    int32_t* status) {
     const int stride = gridDim.x * blockDim.x;
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
-        slot_atom[cell_start[cell_id[i]] + cell_rank[i]] = i;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+        const long long slot = (long long)cell_start[cell_id[i]] + cell_rank[i];
+        if (check_index(slot, n, status)) slot_atom[slot] = i;
+    }
 }
 
 // Deterministic order inside each cell: the slot of atom i is the cell start
@@ -208,13 +132,8 @@ __global__ void cell_order_kernel(const int* __restrict__ slot_atom, int n, cons
 
 // ---------------------------------------------------------------- pair search
 
-constexpr int PS_WARPS = 4;          // warps per block (each warp owns its tiles)
-constexpr int PS_CHUNK = 256;        // culled candidates staged per warp before testing
-constexpr int PS_MAXSEG = 64;        // cell-row segments per table batch
-constexpr int PS_UNROLL = 4;         // candidate loads in flight per lane
-constexpr int PS_BUF = 32;           // per-lane staging of accepted indices (linear)
+constexpr int PS_BUF = 32;           // per-lane staging of accepted indices, per-lane search
 constexpr int PS_GROUP = 8;          // accepted indices leave in aligned groups of 8 (32 bytes)
-constexpr int PS_TEST_UNROLL = 4;    // candidate pairs tested between fullness votes (the loop is written for 4)
 
 struct PairArgs {
     const float4* pos;
@@ -240,44 +159,6 @@ struct SegEntry {
     float sx, sy, sz, pad0, pad1, pad2;
 };
 
-// Per-warp shared memory: candidates as pairs in structure-of-arrays form so
-// that one 16-byte read gives (x0, x1, y0, y1) and another (z0, z1, j0, j1),
-// ready for packed f32x2 arithmetic; the segment table; the index rings.
-struct PairWarpSmem {
-    float4 ca[PS_CHUNK / 2];
-    float4 cb[PS_CHUNK / 2];
-    SegEntry seg[PS_MAXSEG + 1];
-    int buf[32 * PS_BUF];
-};
-
-__device__ __forceinline__ unsigned long long pk(float lo, float hi) {
-    return (unsigned long long)__float_as_uint(lo) | ((unsigned long long)__float_as_uint(hi) << 32);
-}
-__device__ __forceinline__ float pk_lo(unsigned long long v) { return __uint_as_float((unsigned)v); }
-__device__ __forceinline__ float pk_hi(unsigned long long v) { return __uint_as_float((unsigned)(v >> 32)); }
-__device__ __forceinline__ unsigned long long f2_sub(unsigned long long a, unsigned long long b) {
-    unsigned long long d;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
-    unsigned long long d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
-                                                     unsigned long long c) {
-    unsigned long long d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-
-// Two 8-byte words from shared memory at base + OFF (OFF an immediate).
-template <int OFF>
-__device__ __forceinline__ void ld_pair(unsigned base, unsigned long long& a, unsigned long long& b) {
-    asm volatile("ld.shared.v2.u64 {%0, %1}, [%2+%3];" : "=l"(a), "=l"(b) : "r"(base), "n"(OFF));
-}
-
 // Append candidate j at the buffer slot *wsa and advance the slot by one
 // lane-interleaved step (128 bytes) if r2 < rs2 and j is not the atom itself.
 // The store happens either way; a rejected index is overwritten by the next.
@@ -293,67 +174,120 @@ __device__ __forceinline__ void append_if(unsigned& wsa, float r2, float rs2, in
         : "memory");
 }
 
-// Test one candidate pair (x0,x1), (y0,y1), (z0,z1), (j0,j1) against the atom
-// at (px, py, pz) (each duplicated into both halves) with packed f32x2
-// arithmetic, and append the accepted indices at *wsa (see append_if).  One
-// PTX block, so the halves are never moved out of their register pairs.
-__device__ __forceinline__ void test_pair(unsigned& wsa, unsigned long long xx, unsigned long long yy,
-                                          unsigned long long zz, unsigned long long jj, unsigned long long px2,
-                                          unsigned long long py2, unsigned long long pz2, float rs2, int self) {
-    asm volatile(
-        "{\n\t.reg .b64 dx, dy, dz, r2;\n\t.reg .f32 r0, r1;\n\t.reg .b32 j0, j1;\n\t.reg .pred p, q;\n\t"
-        "sub.rn.f32x2 dx, %1, %5;\n\t"
-        "sub.rn.f32x2 dy, %2, %6;\n\t"
-        "sub.rn.f32x2 dz, %3, %7;\n\t"
-        "mul.rn.f32x2 r2, dx, dx;\n\t"
-        "fma.rn.f32x2 r2, dy, dy, r2;\n\t"
-        "fma.rn.f32x2 r2, dz, dz, r2;\n\t"
-        "mov.b64 {r0, r1}, r2;\n\t"
-        "mov.b64 {j0, j1}, %4;\n\t"
-        "setp.lt.f32 p, r0, %8;\n\t"
-        "setp.ne.and.s32 p, j0, %9, p;\n\t"
-        "st.shared.b32 [%0], j0;\n\t"
-        "@p add.u32 %0, %0, 128;\n\t"
-        "setp.lt.f32 q, r1, %8;\n\t"
-        "setp.ne.and.s32 q, j1, %9, q;\n\t"
-        "st.shared.b32 [%0], j1;\n\t"
-        "@q add.u32 %0, %0, 128;\n\t}"
-        : "+r"(wsa)
-        : "l"(xx), "l"(yy), "l"(zz), "l"(jj), "l"(px2), "l"(py2), "l"(pz2), "f"(rs2), "r"(self)
-        : "memory");
+// ------------------------------------------------ tile search with accept masks
+//
+// One warp per tile of 32 consecutive atoms (Hilbert-consecutive when the
+// input is sorted, so the tile is compact), lane = atom i.
+//   1. tile frame: bounding box of the 32 atoms (shuffles) and its centre o;
+//      every coordinate below is taken relative to o, so the pair test works
+//      on numbers of a few Angstrom.
+//   2. candidates: the cell rows within reach of the box, each row clipped to
+//      the chord of the rounded box at that row's y/z distance; every atom
+//      read is culled against the rounded box (distance to the box < reach)
+//      and the survivors are compacted (ballot + popc) into a shared-memory
+//      chunk in groups of four: x0 x1 y0 y1 | z0 z1 x2 x3 | y2 y3 z2 z3, so
+//      that three broadcast 16-byte reads feed packed f32x2 arithmetic for
+//      four candidates.
+//   3. pairs: per block of 32 staged candidates every lane builds a 32-bit
+//      accept mask (r^2 < rs^2), then walks its set bits, skipping itself,
+//      into a lane-interleaved buffer that drains to the row in aligned
+//      32-byte groups.  Pads follow as coalesced stores, row by row.
+
+constexpr int TM_WARPS = 4;          // warps per block, each on its own tiles
+constexpr int TM_CH = 256;           // staged candidates per chunk (a multiple of 32)
+constexpr int TM_MAXSEG = 64;        // cell-row segments per table batch
+constexpr int TM_UNROLL = 4;         // candidate loads in flight per lane while culling
+constexpr int TM_BUF = 48;           // per-lane buffer of accepted indices (>= 32 + TM_GROUP)
+constexpr int TM_GROUP = 8;          // indices leave in aligned groups of 8 (32 bytes)
+
+struct TileWarpSmem {
+    float cq[TM_CH * 3];             // staged candidates, 48 bytes per group of four (tile frame)
+    int cj[TM_CH];                   // their atom indices
+    SegEntry seg[TM_MAXSEG + 1];
+    int buf[32 * TM_BUF];            // entry e of lane l at buf[e * 32 + l]
+};
+constexpr size_t TM_SMEM = sizeof(TileWarpSmem) * TM_WARPS;
+
+// Candidate s of the chunk: group s / 4, slot s % 4 of the 12-float layout.
+__device__ __forceinline__ void stage_cand(TileWarpSmem& W, int s, float x, float y, float z, int j) {
+    const int k = s & 3;
+    const int off = 12 * (s >> 2) + (k & 1) + (k >> 1) * 6;
+    W.cq[off] = x;
+    W.cq[off + 2] = y;
+    W.cq[off + 4] = z;
+    W.cj[s] = j;
 }
 
-// Store one accepted index into slot `slot` of a candidate pair array.
-__device__ __forceinline__ void put_cand(PairWarpSmem& W, int slot, float4 q) {
-    float* a = reinterpret_cast<float*>(&W.ca[slot >> 1]) + (slot & 1);
-    float* b = reinterpret_cast<float*>(&W.cb[slot >> 1]) + (slot & 1);
-    a[0] = q.x;
-    a[2] = q.y;
-    b[0] = q.z;
-    b[2] = q.w;
+// Tests the four candidates of group G of a 32-candidate block against the
+// lane's atom (px2, py2, pz2: its tile-frame coordinates in both halves) and
+// sets bits 4G .. 4G+3 of m for those with r^2 < rs^2.
+template <int G>
+__device__ __forceinline__ void test4(unsigned& m, const ulonglong2* q, unsigned long long px2,
+                                      unsigned long long py2, unsigned long long pz2, float rs2) {
+    const ulonglong2 a = q[3 * G], b = q[3 * G + 1], c = q[3 * G + 2];
+    asm("{\n\t.reg .b64 dx, dy, dz, r;\n\t.reg .f32 r0, r1;\n\t.reg .pred p;\n\t"
+        "sub.rn.f32x2 dx, %1, %7;\n\t"
+        "sub.rn.f32x2 dy, %2, %8;\n\t"
+        "sub.rn.f32x2 dz, %3, %9;\n\t"
+        "mul.rn.f32x2 r, dx, dx;\n\t"
+        "fma.rn.f32x2 r, dy, dy, r;\n\t"
+        "fma.rn.f32x2 r, dz, dz, r;\n\t"
+        "mov.b64 {r0, r1}, r;\n\t"
+        "setp.lt.f32 p, r0, %10;\n\t"
+        "@p or.b32 %0, %0, %11;\n\t"
+        "setp.lt.f32 p, r1, %10;\n\t"
+        "@p or.b32 %0, %0, %12;\n\t"
+        "sub.rn.f32x2 dx, %4, %7;\n\t"
+        "sub.rn.f32x2 dy, %5, %8;\n\t"
+        "sub.rn.f32x2 dz, %6, %9;\n\t"
+        "mul.rn.f32x2 r, dx, dx;\n\t"
+        "fma.rn.f32x2 r, dy, dy, r;\n\t"
+        "fma.rn.f32x2 r, dz, dz, r;\n\t"
+        "mov.b64 {r0, r1}, r;\n\t"
+        "setp.lt.f32 p, r0, %10;\n\t"
+        "@p or.b32 %0, %0, %13;\n\t"
+        "setp.lt.f32 p, r1, %10;\n\t"
+        "@p or.b32 %0, %0, %14;\n\t}"
+        : "+r"(m)
+        : "l"(a.x), "l"(a.y), "l"(b.x), "l"(b.y), "l"(c.x), "l"(c.y), "l"(px2), "l"(py2), "l"(pz2), "f"(rs2),
+          "n"(1u << (4 * G)), "n"(1u << (4 * G + 1)), "n"(1u << (4 * G + 2)), "n"(1u << (4 * G + 3)));
 }
 
-__global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs A) {
-    __shared__ PairWarpSmem smem_w[PS_WARPS];
+__device__ __forceinline__ unsigned long long pk2(float v) {
+    return (unsigned long long)__float_as_uint(v) | ((unsigned long long)__float_as_uint(v) << 32);
+}
+
+// Eight consecutive ints to a 32-byte aligned global address.
+__device__ __forceinline__ void st_global_v8(int* p, int a0, int a1, int a2, int a3, int a4, int a5, int a6, int a7) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a0), "r"(a1), "r"(a2),
+                 "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7)
+                 : "memory");
+}
+
+// VW: row store width in ints (8: rows 32-byte aligned, cap % 8 == 0;
+// 4: 16-byte aligned, cap % 4 == 0; 1: anything).
+template <int VW>
+__global__ __launch_bounds__(TM_WARPS * 32, 4) void pair_tile_kernel(PairArgs A) {
+    extern __shared__ __align__(16) unsigned char tm_smem_raw[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const unsigned lt_mask = lanemask_lt();
-    PairWarpSmem& W = smem_w[warp];
-    // slot s of this lane's buffer is W.buf[s * 32 + lane]: lanes interleaved
-    // across the 32 banks, so the appends of a warp never conflict
+    TileWarpSmem& W = reinterpret_cast<TileWarpSmem*>(tm_smem_raw)[warp];
     int* const buf = W.buf + lane;
     const int cap = A.cap;
     const long long ntiles = ((long long)A.n + 31) / 32;
     const float nanf_ = __int_as_float(0x7fc00000);
+    const float wy = A.L.y / (float)A.nc.y, wz = A.L.z / (float)A.nc.z;
+    const float reach2 = A.reach * A.reach;
 
-    for (long long tile = (long long)blockIdx.x * PS_WARPS + warp; tile < ntiles;
-         tile += (long long)gridDim.x * PS_WARPS) {
+    for (long long tile = (long long)blockIdx.x * TM_WARPS + warp; tile < ntiles;
+         tile += (long long)gridDim.x * TM_WARPS) {
         const int base = (int)(tile * 32);
         const int i = base + lane;
         const bool valid = i < A.n;
         const float4 p = valid ? A.pos[i] : make_float4(nanf_, nanf_, nanf_, 0.f);
-        int* row = A.nbr + (size_t)(valid ? i : 0) * cap;
+        int* const row = A.nbr + (size_t)(valid ? i : 0) * cap;
 
-        // level 1: tile bounding box
+        // level 1: tile bounding box and frame
         float lox = valid ? p.x : INFINITY, loy = valid ? p.y : INFINITY, loz = valid ? p.z : INFINITY;
         float hix = valid ? p.x : -INFINITY, hiy = valid ? p.y : -INFINITY, hiz = valid ? p.z : -INFINITY;
 #pragma unroll
@@ -373,90 +307,107 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
         }
         lox = fmaxf(lox, -A.L.x); loy = fmaxf(loy, -A.L.y); loz = fmaxf(loz, -A.L.z);
         hix = fminf(hix, 2.f * A.L.x); hiy = fminf(hiy, 2.f * A.L.y); hiz = fminf(hiz, 2.f * A.L.z);
-
-        int done = 0;      // accepted indices already written to the row (a multiple of 8 until the end)
-        // next free slot of this lane's buffer, as a 32-bit shared-memory address
-        const unsigned buf_sa = (unsigned)__cvta_generic_to_shared(buf);
-        unsigned wsa = buf_sa;
-        int ncand = 0;     // staged candidates (warp-uniform)
-        const unsigned long long px2 = pk(p.x, p.x), py2 = pk(p.y, p.y), pz2 = pk(p.z, p.z);
+        const float ox = 0.5f * (lox + hix), oy = 0.5f * (loy + hiy), oz = 0.5f * (loz + hiz);
+        const unsigned long long px2 = pk2(p.x - ox), py2 = pk2(p.y - oy), pz2 = pk2(p.z - oz);
         const float rs2 = A.rs2;
 
-        // write the complete groups of 8 buffered indices to the row; with
-        // `all`, the remainder too.  The remainder of a partial drain moves
-        // to the front of the buffer.
-        auto drain = [&](bool all) {
-            const int pend = (int)((wsa - buf_sa) >> 7);
-            const int groups = pend / PS_GROUP;
+        int done = 0;      // accepted indices handed to the row (a multiple of TM_GROUP until the end)
+        int pend = 0;      // indices waiting in this lane's buffer
+        int ncand = 0;     // staged candidates (warp-uniform)
+
+        // write the complete groups of TM_GROUP buffered indices to the row;
+        // the rest moves to the front of the buffer
+        auto drain = [&]() {
+            const int groups = pend / TM_GROUP;
             for (int gi = 0; gi < groups; ++gi) {
-                const int* src = buf + gi * PS_GROUP * 32;
-                if (done + PS_GROUP <= cap && A.vec_rows) {
-                    const int4 a = make_int4(src[0], src[32], src[64], src[96]);
-                    const int4 b = make_int4(src[128], src[160], src[192], src[224]);
-                    *reinterpret_cast<int4*>(row + done) = a;
-                    *reinterpret_cast<int4*>(row + done + 4) = b;
+                const int* src = buf + gi * TM_GROUP * 32;
+                if (VW == 8 && done + TM_GROUP <= cap) {
+                    st_global_v8(row + done, src[0], src[32], src[64], src[96], src[128], src[160], src[192],
+                                 src[224]);
+                } else if (VW == 4 && done + TM_GROUP <= cap) {
+                    *reinterpret_cast<int4*>(row + done) = make_int4(src[0], src[32], src[64], src[96]);
+                    *reinterpret_cast<int4*>(row + done + 4) = make_int4(src[128], src[160], src[192], src[224]);
                 } else {
-                    for (int e = 0; e < PS_GROUP; ++e)
+#pragma unroll
+                    for (int e = 0; e < TM_GROUP; ++e)
                         if (done + e < cap) row[done + e] = src[e * 32];
                 }
-                done += PS_GROUP;
+                done += TM_GROUP;
             }
-            const int rest = pend - groups * PS_GROUP;
-            if (all) {
-                for (int e = 0; e < rest; ++e)
-                    if (done + e < cap) row[done + e] = buf[(groups * PS_GROUP + e) * 32];
-                done += rest;
-                wsa = buf_sa;
+            const int rest = pend - groups * TM_GROUP;
+            for (int e = 0; e < rest; ++e) buf[e * 32] = buf[(groups * TM_GROUP + e) * 32];
+            pend = rest;
+        };
+
+        // level 3: test the staged candidates in blocks of 32.  With `last`
+        // the final partial block is padded with candidates that are never
+        // accepted (NaN); otherwise it moves to the front of the chunk.
+        auto test_chunk = [&](bool last) {
+            __syncwarp();
+            int nblk = ncand >> 5;
+            if (last && (ncand & 31)) {
+                const int pad_to = (ncand + 31) & ~31;
+                if (lane < pad_to - ncand) stage_cand(W, ncand + lane, nanf_, nanf_, nanf_, -1);
+                nblk = pad_to >> 5;
+                __syncwarp();
+            }
+            for (int blk = 0; blk < nblk; ++blk) {
+                if (__any_sync(FULL, pend > TM_BUF - 32)) drain();
+                const ulonglong2* q = reinterpret_cast<const ulonglong2*>(W.cq + blk * 96);
+                // eight independent nibbles, joined by a tree of ORs
+                unsigned m0 = 0u, m1 = 0u, m2 = 0u, m3 = 0u, m4 = 0u, m5 = 0u, m6 = 0u, m7 = 0u;
+                test4<0>(m0, q, px2, py2, pz2, rs2);
+                test4<1>(m1, q, px2, py2, pz2, rs2);
+                test4<2>(m2, q, px2, py2, pz2, rs2);
+                test4<3>(m3, q, px2, py2, pz2, rs2);
+                test4<4>(m4, q, px2, py2, pz2, rs2);
+                test4<5>(m5, q, px2, py2, pz2, rs2);
+                test4<6>(m6, q, px2, py2, pz2, rs2);
+                test4<7>(m7, q, px2, py2, pz2, rs2);
+                unsigned m = ((m0 | m1) | (m2 | m3)) | ((m4 | m5) | (m6 | m7));
+                const int* cjb = W.cj + blk * 32;
+                while (m) {
+                    const int b = __ffs(m) - 1;
+                    m &= m - 1u;
+                    const int j = cjb[b];
+                    if (j != i && check_index(j, A.n, A.status)) {
+                        buf[pend * 32] = j;
+                        ++pend;
+                    }
+                }
+            }
+            if (last) {
+                ncand = 0;
             } else {
-                for (int e = 0; e < rest; ++e) buf[e * 32] = buf[(groups * PS_GROUP + e) * 32];
-                wsa = buf_sa + 128u * (unsigned)rest;
+                // the partial block (fewer than 32) moves to the front: whole
+                // 48-byte groups and their indices
+                const int rem = ncand - (nblk << 5);
+                __syncwarp();
+                float4* cq4 = reinterpret_cast<float4*>(W.cq);
+                const int nq = ((rem + 3) >> 2) * 3;
+                float4 t4 = make_float4(0.f, 0.f, 0.f, 0.f);
+                int tj = 0;
+                if (lane < nq) t4 = cq4[nblk * 24 + lane];
+                if (lane < rem) tj = W.cj[(nblk << 5) + lane];
+                __syncwarp();
+                if (lane < nq) cq4[lane] = t4;
+                if (lane < rem) W.cj[lane] = tj;
+                ncand = rem;
             }
-        };
-
-        // level 3: test the staged candidates, two at a time in f32x2.  An
-        // accepted index is stored at the buffer pointer, which then advances
-        // (stores for rejected candidates are overwritten by the next one).
-        auto test_chunk = [&]() {
-            __syncwarp();
-            // pad to a whole number of unrolled steps with candidates that are
-            // never accepted (NaN position), so the loop needs no bounds tests
-            const int padded = (ncand + 2 * PS_TEST_UNROLL - 1) & ~(2 * PS_TEST_UNROLL - 1);
-            if (lane < padded - ncand)
-                put_cand(W, ncand + lane, make_float4(nanf_, nanf_, nanf_, __int_as_float(-1)));
-            __syncwarp();
-            const unsigned ca_sa = (unsigned)__cvta_generic_to_shared(&W.ca[0]);
-            const unsigned cb_sa = (unsigned)__cvta_generic_to_shared(&W.cb[0]);
-            for (int c = 0; c < (padded >> 1); c += PS_TEST_UNROLL) {
-                // room for 2 * PS_TEST_UNROLL more in every lane's buffer?
-                if (__any_sync(FULL, (int)((wsa - buf_sa) >> 7) > PS_BUF - 2 * PS_TEST_UNROLL)) drain(false);
-                unsigned long long xx[4], yy[4], zz[4], jj[4];
-                const unsigned ab = ca_sa + 16u * (unsigned)c, bb = cb_sa + 16u * (unsigned)c;
-                ld_pair<0>(ab, xx[0], yy[0]);
-                ld_pair<0>(bb, zz[0], jj[0]);
-                ld_pair<16>(ab, xx[1], yy[1]);
-                ld_pair<16>(bb, zz[1], jj[1]);
-                ld_pair<32>(ab, xx[2], yy[2]);
-                ld_pair<32>(bb, zz[2], jj[2]);
-                ld_pair<48>(ab, xx[3], yy[3]);
-                ld_pair<48>(bb, zz[3], jj[3]);
-#pragma unroll
-                for (int u = 0; u < 4; ++u) test_pair(wsa, xx[u], yy[u], zz[u], jj[u], px2, py2, pz2, rs2, i);
-            }
-            ncand = 0;
             __syncwarp();
         };
 
-        // level 2: cell rows overlapping the box +- reach
+        // level 2: cell rows within reach of the box, each clipped to its chord
         const int ux0 = (int)floorf((lox - A.reach) * A.inv_w.x), ux1 = (int)floorf((hix + A.reach) * A.inv_w.x);
         const int uy0 = (int)floorf((loy - A.reach) * A.inv_w.y), uy1 = (int)floorf((hiy + A.reach) * A.inv_w.y);
         const int uz0 = (int)floorf((loz - A.reach) * A.inv_w.z), uz1 = (int)floorf((hiz + A.reach) * A.inv_w.z);
         const int ny = uy1 - uy0 + 1, nz = uz1 - uz0 + 1;
-        const int npieces = floor_div(ux1, A.nc.x) - floor_div(ux0, A.nc.x) + 1;
+        const int kx0 = floor_div(ux0, A.nc.x);
+        const int npieces = floor_div(ux1, A.nc.x) - kx0 + 1;
         const int nseg = ny * nz * npieces;
-        const float reach2 = A.reach * A.reach;
 
-        for (int sb = 0; sb < nseg; sb += PS_MAXSEG) {
-            const int nb = min(PS_MAXSEG, nseg - sb);
+        for (int sb = 0; sb < nseg; sb += TM_MAXSEG) {
+            const int nb = min(TM_MAXSEG, nseg - sb);
             int run = 0;
             for (int s0 = 0; s0 < nb; s0 += 32) {
                 const int sl = s0 + lane;
@@ -467,17 +418,29 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
                     const int piece = s % npieces;
                     const int rw = s / npieces;
                     const int uy = uy0 + rw % ny, uz = uz0 + rw / ny;
-                    const int ky = floor_div(uy, A.nc.y), kz = floor_div(uz, A.nc.z);
-                    const int cy = uy - ky * A.nc.y, cz = uz - kz * A.nc.z;
-                    const int kx = floor_div(ux0, A.nc.x) + piece;
-                    const int xa = max(ux0, kx * A.nc.x) - kx * A.nc.x;
-                    const int xb = min(ux1, (kx + 1) * A.nc.x - 1) - kx * A.nc.x;
-                    const int rowbase = (cz * A.nc.y + cy) * A.nc.x;
-                    beg = A.cell_start[rowbase + xa];
-                    len = A.cell_start[rowbase + xb + 1] - beg;
-                    sx = (float)kx * A.L.x;
-                    sy = (float)ky * A.L.y;
-                    sz = (float)kz * A.L.z;
+                    // the row's distance to the box in y and z (unwrapped cell geometry)
+                    const float ylo = (float)uy * wy, zlo = (float)uz * wz;
+                    const float ddy = fmaxf(fmaxf(ylo - hiy, loy - (ylo + wy)), 0.f);
+                    const float ddz = fmaxf(fmaxf(zlo - hiz, loz - (zlo + wz)), 0.f);
+                    const float ch2 = reach2 - ddy * ddy - ddz * ddz;
+                    if (ch2 > 0.f) {
+                        const float ch = fmaf(ch2 * rsqrtf(ch2), 1.0001f, 1e-4f);
+                        const int ca = max(ux0, (int)floorf((lox - ch) * A.inv_w.x));
+                        const int cb = min(ux1, (int)floorf((hix + ch) * A.inv_w.x));
+                        const int ky = floor_div(uy, A.nc.y), kz = floor_div(uz, A.nc.z);
+                        const int cy = uy - ky * A.nc.y, cz = uz - kz * A.nc.z;
+                        const int kx = kx0 + piece;
+                        const int xa = max(ca, kx * A.nc.x) - kx * A.nc.x;
+                        const int xb = min(cb, (kx + 1) * A.nc.x - 1) - kx * A.nc.x;
+                        if (xa <= xb) {
+                            const int rowbase = (cz * A.nc.y + cy) * A.nc.x;
+                            beg = A.cell_start[rowbase + xa];
+                            len = A.cell_start[rowbase + xb + 1] - beg;
+                            sx = (float)kx * A.L.x;
+                            sy = (float)ky * A.L.y;
+                            sz = (float)kz * A.L.z;
+                        }
+                    }
                 }
                 int inc = len;
 #pragma unroll
@@ -498,12 +461,12 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
             const int total = run;
 
             int sc = 0;   // this lane's segment cursor
-            for (int t0 = 0; t0 < total; t0 += 32 * PS_UNROLL) {
-                if (ncand > PS_CHUNK - 2 * PS_TEST_UNROLL - 32 * PS_UNROLL) test_chunk();
-                float4 q[PS_UNROLL];
-                bool ok[PS_UNROLL];
+            for (int t0 = 0; t0 < total; t0 += 32 * TM_UNROLL) {
+                if (ncand > TM_CH - 32 * TM_UNROLL) test_chunk(false);
+                float4 q[TM_UNROLL];
+                bool ok[TM_UNROLL];
 #pragma unroll
-                for (int u = 0; u < PS_UNROLL; ++u) {
+                for (int u = 0; u < TM_UNROLL; ++u) {
                     const int t = t0 + u * 32 + lane;
                     ok[u] = t < total;
                     if (ok[u]) {
@@ -514,7 +477,7 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
                     }
                 }
 #pragma unroll
-                for (int u = 0; u < PS_UNROLL; ++u) {
+                for (int u = 0; u < TM_UNROLL; ++u) {
                     bool keep = false;
                     if (ok[u]) {
                         const float ex = fmaxf(fmaxf(lox - q[u].x, q[u].x - hix), 0.f);
@@ -523,29 +486,59 @@ __global__ __launch_bounds__(PS_WARPS * 32, 6) void pair_search_kernel(PairArgs 
                         keep = fmaf(ez, ez, fmaf(ey, ey, ex * ex)) < reach2;
                     }
                     const unsigned bm = __ballot_sync(FULL, keep);
-                    if (keep) put_cand(W, ncand + __popc(bm & lt_mask), q[u]);
+                    if (keep)
+                        stage_cand(W, ncand + __popc(bm & lt_mask), q[u].x - ox, q[u].y - oy, q[u].z - oz,
+                                   __float_as_int(q[u].w));
                     ncand += __popc(bm);
                 }
             }
             __syncwarp();
         }
-        test_chunk();
-        drain(true);
-        const int cnt = done;
+        test_chunk(true);
 
-        if (valid) {
-            A.counts[i] = cnt;
-            if (A.pad_fill) {
-                int e = min(cnt, cap);
-                if (A.vec_rows) {
-                    for (; e < cap && (e & 3); ++e) row[e] = -1;
-                    for (; e + 4 <= cap; e += 4) *reinterpret_cast<int4*>(row + e) = make_int4(-1, -1, -1, -1);
+        // the rest of the buffer: a last group of TM_GROUP completed with pads
+        // where the row has room for it (pad-filled rows), else one by one
+        drain();
+        int filled = done;                 // slots of the row written so far (from 0)
+        if (VW >= 4 && A.pad_fill && pend > 0 && done + TM_GROUP <= cap) {
+            int v[TM_GROUP];
+#pragma unroll
+            for (int e = 0; e < TM_GROUP; ++e) v[e] = e < pend ? buf[e * 32] : -1;
+            if (VW == 8) {
+                st_global_v8(row + done, v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+            } else {
+                *reinterpret_cast<int4*>(row + done) = make_int4(v[0], v[1], v[2], v[3]);
+                *reinterpret_cast<int4*>(row + done + 4) = make_int4(v[4], v[5], v[6], v[7]);
+            }
+            filled = done + TM_GROUP;
+        } else {
+            for (int e = 0; e < pend; ++e)
+                if (done + e < cap) row[done + e] = buf[e * 32];
+            filled = min(done + pend, cap);
+        }
+        const int cnt = done + pend;
+        if (!valid) filled = cap;
+
+        if (valid) A.counts[i] = cnt;
+        if (A.pad_fill) {
+            // pads row by row, the whole warp on one row at a time (coalesced)
+            for (int r = 0; r < 32; ++r) {
+                const int fr = __shfl_sync(FULL, filled, r);
+                if (fr >= cap) continue;
+                int* rowr = A.nbr + (size_t)(base + r) * cap;
+                if (VW >= 4) {
+                    const int f4 = min((fr + 3) & ~3, cap);
+                    if (lane < f4 - fr) rowr[fr + lane] = -1;
+                    for (int e = f4 + 4 * lane; e < cap; e += 128)
+                        *reinterpret_cast<int4*>(rowr + e) = make_int4(-1, -1, -1, -1);
+                } else {
+                    for (int e = fr + lane; e < cap; e += 32) rowr[e] = -1;
                 }
-                for (; e < cap; ++e) row[e] = -1;
             }
         }
         const unsigned ov = __ballot_sync(FULL, valid && cnt > cap);
         if (ov && lane == 0) atomicOr(A.status, TESS_DEV_OVERFLOW);
+        __syncwarp();
     }
 }
 
@@ -756,7 +749,7 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
     if (n <= 0 || !pos || !ws || !nbr || !counts || !overflow || cap < 1) return TESS_ERR_INVALID_ARG;
     if (!box_ok(box) || !(rc > 0.f) || !(skin >= 0.f) || !std::isfinite(rc) || !std::isfinite(skin))
         return TESS_ERR_INVALID_ARG;
-    if ((flags & ~(TESS_NO_PAD_FILL | TESS_TILE_SEARCH)) != 0) return TESS_ERR_INVALID_ARG;
+    if ((flags & ~(TESS_NO_PAD_FILL | TESS_LANE_SEARCH)) != 0) return TESS_ERR_INVALID_ARG;
     if (!aligned(pos, 16) || !aligned(ws, 256) || !aligned(nbr, 4) || !aligned(counts, 4)) return TESS_ERR_INVALID_ARG;
     const float rs = rc + skin;
     if (box.lx < 2.f * rs || box.ly < 2.f * rs || box.lz < 2.f * rs) return TESS_ERR_BOX_TOO_SMALL;
@@ -783,7 +776,7 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
         scan_reduce_kernel<<<(unsigned)scan_tiles, SCAN_THREADS, 0, s>>>(L.cnt, m, L.sums);
         scan_sums_kernel<<<1, SCAN_THREADS, 0, s>>>(L.sums, scan_tiles);
         scan_apply_kernel<<<(unsigned)scan_tiles, SCAN_THREADS, 0, s>>>(L.cnt, m, L.sums, L.cell_start);
-        cell_scatter_kernel<<<blocks, 256, 0, s>>>(L.cell_id, L.cell_rank, n, L.cell_start, L.slot_atom);
+        cell_scatter_kernel<<<blocks, 256, 0, s>>>(L.cell_id, L.cell_rank, n, L.cell_start, L.slot_atom, overflow);
         cell_order_kernel<<<blocks, 256, 0, s>>>(L.slot_atom, n, L.cell_id, L.cell_start, pos4, L.pos_cell);
         count_launch(6);
     }
@@ -810,12 +803,19 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
         // the per-lane search needs every box length >= 2 reach (a window
         // then wraps at most once); otherwise the tile search handles it
         const bool lane_ok = box.lx >= 2.f * A.reach && box.ly >= 2.f * A.reach && box.lz >= 2.f * A.reach;
-        if ((flags & TESS_TILE_SEARCH) || !lane_ok) {
-            const long long blocks = (ntiles + PS_WARPS - 1) / PS_WARPS;
-            pair_search_kernel<<<(unsigned)std::min<long long>(blocks, 1LL << 30), PS_WARPS * 32, 0, s>>>(A);
-        } else {
+        if ((flags & TESS_LANE_SEARCH) && lane_ok) {
             const long long blocks = (ntiles + PL_WARPS - 1) / PL_WARPS;
             pair_search_lane_kernel<<<(unsigned)std::min<long long>(blocks, 1LL << 30), PL_WARPS * 32, 0, s>>>(A);
+        } else {
+            const long long blocks = std::min<long long>((ntiles + TM_WARPS - 1) / TM_WARPS, 1LL << 30);
+            const bool v8 = cap % 8 == 0 && aligned(nbr, 32), v4 = cap % 4 == 0 && aligned(nbr, 16);
+            auto launch = [&](auto kern) {
+                cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TM_SMEM);
+                kern<<<(unsigned)blocks, TM_WARPS * 32, TM_SMEM, s>>>(A);
+            };
+            if (v8) launch(pair_tile_kernel<8>);
+            else if (v4) launch(pair_tile_kernel<4>);
+            else launch(pair_tile_kernel<1>);
         }
         count_launch();
     }

@@ -17,8 +17,6 @@
 // Two calls whose kernels overlap on the GPU -- on different streams, or from
 // different host threads without ordering -- race on the array and corrupt
 // each other's results: order them on one stream.
-#include <mutex>
-
 #include "common.cuh"
 
 namespace tess {
@@ -35,29 +33,20 @@ constexpr size_t STATIC_SORT_SCRATCH_BYTES = TESS_HILBERT_SORT_STATIC_BYTES;
 static __device__ __align__(256) unsigned char g_sort_scratch[STATIC_SORT_SCRATCH_BYTES];
 
 namespace {
-constexpr int MAX_DEVICES = 64;
-std::mutex g_scratch_mu;
-void* g_scratch_addr[MAX_DEVICES] = {};
-
-// Device address of the scratch array on the current device, looked up once
-// per device (the first call on a device does this set-up).
+// Device address of the scratch array in the current context.  It is looked
+// up on every call (a host-side query that enqueues no work) rather than
+// cached: a cached address would go stale once the context that holds the
+// module is destroyed and created again (cudaDeviceReset, or the primary
+// context released and retained), and the next call would then write
+// through it.
 tess_status scratch_address(void** out) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_sort_scratch);
+    if (e != cudaSuccess || p == nullptr) {
         cudaGetLastError();
         return TESS_ERR_CUDA;
     }
-    std::lock_guard<std::mutex> guard(g_scratch_mu);
-    if (!g_scratch_addr[dev]) {
-        void* p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_sort_scratch);
-        if (e != cudaSuccess || p == nullptr) {
-            cudaGetLastError();
-            return TESS_ERR_CUDA;
-        }
-        g_scratch_addr[dev] = p;
-    }
-    *out = g_scratch_addr[dev];
+    *out = p;
     return TESS_OK;
 }
 }  // namespace

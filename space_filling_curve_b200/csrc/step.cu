@@ -89,31 +89,55 @@ __device__ __forceinline__ float min_image_f(float d, float L) {
     return d;
 }
 
-// Smooth cosine cutoff f_c = (cos(pi r / rc) + 1) / 2 for r < rc, as a
-// function of u = (r / rc)^2 in [0, 1): cos(pi sqrt(u)) is the Taylor series
-// sum_k (-pi^2 u)^k / (2k)!, which converges on the whole interval; eleven
-// terms leave a truncation error below 4e-9 at u = 1 and the fp32 Horner
-// evaluation adds a few 1e-7 at most (the largest partial terms are ~4).
-// No square root or trigonometric call is needed on the aggregation path.
-__host__ __device__ constexpr double cos_pi_sqrt_coef(int k) {
-    double c = 1.0;
-    for (int m = 1; m <= k; ++m) c *= -9.8696044010893586188 / ((2.0 * m - 1.0) * (2.0 * m));
-    return c;
+// Smooth cosine cutoff f_c = (cos(pi r / rc) + 1) / 2 for r < rc, written
+// in w = 1 - (r / rc)^2 in (0, 1]: f_c = cos^2(pi sqrt(1 - w) / 2) is an
+// entire function of w whose Taylor series at w = 0 is w^2 (b_2 + b_3 w +
+// ...).  Its coefficients follow from cos(pi sqrt(u)) = sum_k c_k u^k, c_k =
+// (-pi^2)^k / (2k)!, by putting u = 1 - w: b_j = (-1)^j / 2 sum_{k >= j} c_k
+// C(k, j) (b_0 = b_1 = 0, b_2 = pi^2 / 16).  Every b_j is positive, so the
+// fp32 Horner sum has no cancellation and stays within ~2e-7 relative error
+// on the whole range -- also next to the cutoff, where f_c ~ (pi^2/16) w^2
+// vanishes.  Eight terms (b_2 .. b_9): truncation below 2e-9.  w itself is
+// one fused multiply-add, 1 - r^2 / rc^2; no square root or trigonometric
+// call is needed on the aggregation path.
+__host__ __device__ constexpr double fc_w_coef(int j) {
+    double s = 0.0;
+    double c = 1.0;                  // c_k
+    for (int k = 0; k <= 40; ++k) {
+        if (k > 0) c *= -9.8696044010893586188 / ((2.0 * k - 1.0) * (2.0 * k));
+        if (k >= j) {
+            double bn = 1.0;         // C(k, j)
+            for (int t = 1; t <= j; ++t) bn = bn * (double)(k - j + t) / (double)t;
+            s += c * bn;
+        }
+    }
+    return ((j & 1) ? -s : s) * 0.5;
 }
 
-__device__ __forceinline__ float cutoff_u(float u) {
-    float p = (float)cos_pi_sqrt_coef(10);
-    p = fmaf(p, u, (float)cos_pi_sqrt_coef(9));
-    p = fmaf(p, u, (float)cos_pi_sqrt_coef(8));
-    p = fmaf(p, u, (float)cos_pi_sqrt_coef(7));
-    p = fmaf(p, u, (float)cos_pi_sqrt_coef(6));
-    p = fmaf(p, u, (float)cos_pi_sqrt_coef(5));
-    p = fmaf(p, u, (float)cos_pi_sqrt_coef(4));
-    p = fmaf(p, u, (float)cos_pi_sqrt_coef(3));
-    p = fmaf(p, u, (float)cos_pi_sqrt_coef(2));
-    p = fmaf(p, u, (float)cos_pi_sqrt_coef(1));
-    p = fmaf(p, u, 1.0f);
-    return 0.5f * (p + 1.0f);
+__device__ __forceinline__ float cutoff_w(float w) {
+    float q = (float)fc_w_coef(9);
+    q = fmaf(q, w, (float)fc_w_coef(8));
+    q = fmaf(q, w, (float)fc_w_coef(7));
+    q = fmaf(q, w, (float)fc_w_coef(6));
+    q = fmaf(q, w, (float)fc_w_coef(5));
+    q = fmaf(q, w, (float)fc_w_coef(4));
+    q = fmaf(q, w, (float)fc_w_coef(3));
+    q = fmaf(q, w, (float)fc_w_coef(2));
+    return (w * w) * q;
+}
+
+// d f_c / d w = w (2 b_2 + 3 b_3 w + ...), also all positive terms; then
+// (d f_c / d r) / r = -(2 / rc^2) d f_c / d w.
+__device__ __forceinline__ float cutoff_dw(float w) {
+    float q = (float)(9.0 * fc_w_coef(9));
+    q = fmaf(q, w, (float)(8.0 * fc_w_coef(8)));
+    q = fmaf(q, w, (float)(7.0 * fc_w_coef(7)));
+    q = fmaf(q, w, (float)(6.0 * fc_w_coef(6)));
+    q = fmaf(q, w, (float)(5.0 * fc_w_coef(5)));
+    q = fmaf(q, w, (float)(4.0 * fc_w_coef(4)));
+    q = fmaf(q, w, (float)(3.0 * fc_w_coef(3)));
+    q = fmaf(q, w, (float)(2.0 * fc_w_coef(2)));
+    return w * q;
 }
 
 constexpr int EDGE_WARPS = 8;
@@ -150,8 +174,8 @@ __global__ __launch_bounds__(EDGE_WARPS * 32) void edge_kernel(EdgeArgs A) {
                     const float dy = min_image_f(pj.y - pi.y, A.L.y);
                     const float dz = min_image_f(pj.z - pi.z, A.L.z);
                     const float r2 = fmaf(dz, dz, fmaf(dy, dy, dx * dx));
-                    const float u = r2 * A.inv_rc2;
-                    fc = u < 1.0f ? cutoff_u(u) : 0.0f;
+                    const float w = fmaf(-r2, A.inv_rc2, 1.0f);
+                    fc = w > 0.0f ? cutoff_w(w) : 0.0f;
                     if (fc0 == 0 && edges) {
                         const float r = sqrtf(r2);
                         const float inv_r = r > 0.f ? 1.0f / r : 0.f;
@@ -221,47 +245,72 @@ constexpr int EV_CHUNK = TESS_EV_CHUNK;
 constexpr int EV_GEO_UNROLL = TESS_EV_GEO_UNROLL;     // neighbor/position loads in flight per lane
 constexpr int EV_ACC_UNROLL = TESS_EV_ACC_UNROLL;     // feature rows in flight per lane group
 
-// W consecutive floats of a feature row (W = 4: one 16-byte load; W = 8: one
-// 32-byte load, which sm_100 issues as a single instruction).
+// W consecutive floats of a feature row, held as W/2 packed pairs so that
+// sm_100's paired fp32 instructions (fma.rn.f32x2, add.rn.f32x2) work on two
+// features at once.  W = 4: one 16-byte load; W = 8: one 32-byte load, which
+// sm_100 issues as a single instruction.
+__device__ __forceinline__ unsigned long long f2_dup(float v) {
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(v));
+    return r;
+}
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
+                                                     unsigned long long c) {
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
+    unsigned long long d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float f2_sum(unsigned long long a) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(a));
+    return lo + hi;
+}
+__device__ __forceinline__ unsigned long long f2_shfl_xor(unsigned long long a, int o) {
+    unsigned lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(a));
+    lo = __shfl_xor_sync(FULL, lo, o);
+    hi = __shfl_xor_sync(FULL, hi, o);
+    unsigned long long r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+
 template <int W>
 struct FVec {
-    float4 q[W / 4];
+    unsigned long long p[W / 2];
     __device__ __forceinline__ void zero() {
 #pragma unroll
-        for (int k = 0; k < W / 4; ++k) q[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int k = 0; k < W / 2; ++k) p[k] = 0ull;
     }
+    // this += w * h, two features per instruction
     __device__ __forceinline__ void fma(float w, const FVec& h) {
+        const unsigned long long w2 = f2_dup(w);
 #pragma unroll
-        for (int k = 0; k < W / 4; ++k) {
-            q[k].x = fmaf(w, h.q[k].x, q[k].x);
-            q[k].y = fmaf(w, h.q[k].y, q[k].y);
-            q[k].z = fmaf(w, h.q[k].z, q[k].z);
-            q[k].w = fmaf(w, h.q[k].w, q[k].w);
-        }
+        for (int k = 0; k < W / 2; ++k) p[k] = f2_fma(w2, h.p[k], p[k]);
     }
-    // acc + sum_k a_k b_k
-    __device__ __forceinline__ static float dot(const FVec& a, const FVec& b, float acc) {
+    // acc2 + the products a_k b_k, summed pairwise into a packed pair
+    __device__ __forceinline__ static unsigned long long dot2(const FVec& a, const FVec& b, unsigned long long acc2) {
 #pragma unroll
-        for (int k = 0; k < W / 4; ++k) {
-            acc = fmaf(a.q[k].x, b.q[k].x, acc);
-            acc = fmaf(a.q[k].y, b.q[k].y, acc);
-            acc = fmaf(a.q[k].z, b.q[k].z, acc);
-            acc = fmaf(a.q[k].w, b.q[k].w, acc);
-        }
-        return acc;
+        for (int k = 0; k < W / 2; ++k) acc2 = f2_fma(a.p[k], b.p[k], acc2);
+        return acc2;
     }
     __device__ __forceinline__ void shfl_add(int o) {
 #pragma unroll
-        for (int k = 0; k < W / 4; ++k) {
-            q[k].x += __shfl_xor_sync(FULL, q[k].x, o);
-            q[k].y += __shfl_xor_sync(FULL, q[k].y, o);
-            q[k].z += __shfl_xor_sync(FULL, q[k].z, o);
-            q[k].w += __shfl_xor_sync(FULL, q[k].w, o);
-        }
+        for (int k = 0; k < W / 2; ++k) p[k] = f2_add(p[k], f2_shfl_xor(p[k], o));
     }
-    __device__ __forceinline__ void store(float* p) const {
-#pragma unroll
-        for (int k = 0; k < W / 4; ++k) reinterpret_cast<float4*>(p)[k] = q[k];
+    __device__ __forceinline__ void store(float* ptr) const {
+        if (W == 4) {
+            asm volatile("st.global.v2.b64 [%0], {%1, %2};" ::"l"(ptr), "l"(p[0]), "l"(p[1]) : "memory");
+        } else {
+            asm volatile("st.global.v2.b64 [%0], {%1, %2};" ::"l"(ptr), "l"(p[0]), "l"(p[1]) : "memory");
+            asm volatile("st.global.v2.b64 [%0], {%1, %2};" ::"l"(ptr + 4), "l"(p[W / 2 - 2]), "l"(p[W / 2 - 1])
+                         : "memory");
+        }
     }
 };
 
@@ -271,7 +320,7 @@ __device__ __forceinline__ FVec<W> ld_vec(const float* p);
 template <>
 __device__ __forceinline__ FVec<4> ld_vec<4>(const float* p) {
     FVec<4> r;
-    r.q[0] = *reinterpret_cast<const float4*>(p);
+    asm("ld.global.v2.b64 {%0, %1}, [%2];" : "=l"(r.p[0]), "=l"(r.p[1]) : "l"(p));
     return r;
 }
 
@@ -280,10 +329,7 @@ __device__ __forceinline__ FVec<4> ld_vec<4>(const float* p) {
 template <>
 __device__ __forceinline__ FVec<8> ld_vec<8>(const float* p) {
     FVec<8> r;
-    asm("ld.global.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-        : "=f"(r.q[0].x), "=f"(r.q[0].y), "=f"(r.q[0].z), "=f"(r.q[0].w), "=f"(r.q[1].x), "=f"(r.q[1].y),
-          "=f"(r.q[1].z), "=f"(r.q[1].w)
-        : "l"(p));
+    asm("ld.global.v4.b64 {%0, %1, %2, %3}, [%4];" : "=l"(r.p[0]), "=l"(r.p[1]), "=l"(r.p[2]), "=l"(r.p[3]) : "l"(p));
     return r;
 }
 
@@ -331,8 +377,8 @@ __global__ __launch_bounds__(EV_WARPS * 32, TESS_EV_MINB) void edge_vec_kernel(E
                     const float dy = min_image_f(pj[u].y - pi.y, A.L.y);
                     const float dz = min_image_f(pj[u].z - pi.z, A.L.z);
                     const float r2 = fmaf(dz, dz, fmaf(dy, dy, dx * dx));
-                    const float u2 = r2 * A.inv_rc2;
-                    fc = u2 < 1.0f ? cutoff_u(u2) : 0.0f;
+                    const float w = fmaf(-r2, A.inv_rc2, 1.0f);
+                    fc = w > 0.0f ? cutoff_w(w) : 0.0f;
                     if (edges) {
                         const size_t e = (size_t)i * A.cap + s;
                         const float r = sqrtf(r2);
@@ -394,29 +440,6 @@ __global__ __launch_bounds__(EV_WARPS * 32, TESS_EV_MINB) void edge_vec_kernel(E
 
 // ---------------------------------------------------------------- backward (force path)
 
-// sin(pi sqrt(u)) / (pi sqrt(u)) as the Taylor series sum_k (-pi^2 u)^k /
-// (2k+1)!, eleven terms (truncation below 2e-10 at u = 1), so that
-// d f_c / d r divided by r is -(pi^2 / (2 rc^2)) times this, with no root.
-__host__ __device__ constexpr double sinc_pi_sqrt_coef(int k) {
-    double c = 1.0;
-    for (int m = 1; m <= k; ++m) c *= -9.8696044010893586188 / ((2.0 * m) * (2.0 * m + 1.0));
-    return c;
-}
-
-__device__ __forceinline__ float sinc_u(float u) {
-    float p = (float)sinc_pi_sqrt_coef(10);
-    p = fmaf(p, u, (float)sinc_pi_sqrt_coef(9));
-    p = fmaf(p, u, (float)sinc_pi_sqrt_coef(8));
-    p = fmaf(p, u, (float)sinc_pi_sqrt_coef(7));
-    p = fmaf(p, u, (float)sinc_pi_sqrt_coef(6));
-    p = fmaf(p, u, (float)sinc_pi_sqrt_coef(5));
-    p = fmaf(p, u, (float)sinc_pi_sqrt_coef(4));
-    p = fmaf(p, u, (float)sinc_pi_sqrt_coef(3));
-    p = fmaf(p, u, (float)sinc_pi_sqrt_coef(2));
-    p = fmaf(p, u, (float)sinc_pi_sqrt_coef(1));
-    return fmaf(p, u, 1.0f);
-}
-
 struct BackArgs {
     const float4* pos;
     const int* nbr;
@@ -428,7 +451,7 @@ struct BackArgs {
     int n, cap, F;
     float3 L;
     float inv_rc2;
-    float dfc_scale;     // -(pi^2 / (2 rc^2)): (d f_c / d r) / r = dfc_scale * sinc_u(u)
+    float dfc_scale;     // -2 / rc^2: (d f_c / d r) / r = dfc_scale * cutoff_dw(w)
 };
 
 // Vector-Jacobian product of the aggregation over a full symmetric list
@@ -480,10 +503,10 @@ __global__ __launch_bounds__(BK_WARPS * 32, TESS_BK_MINB) void edge_backward_ker
                 const float dx = min_image_f(pj.x - pi.x, A.L.x);
                 const float dy = min_image_f(pj.y - pi.y, A.L.y);
                 const float dz = min_image_f(pj.z - pi.z, A.L.z);
-                const float u2 = fmaf(dz, dz, fmaf(dy, dy, dx * dx)) * A.inv_rc2;
-                if (u2 < 1.0f) {
-                    const float dr = A.dfc_scale * sinc_u(u2);
-                    w = make_float4(cutoff_u(u2), dr * dx, dr * dy, dr * dz);
+                const float ww = fmaf(-fmaf(dz, dz, fmaf(dy, dy, dx * dx)), A.inv_rc2, 1.0f);
+                if (ww > 0.0f) {
+                    const float dr = A.dfc_scale * cutoff_dw(ww);
+                    w = make_float4(cutoff_w(ww), dr * dx, dr * dy, dr * dz);
                     live = true;
                 }
             }
@@ -518,13 +541,14 @@ __global__ __launch_bounds__(BK_WARPS * 32, TESS_BK_MINB) void edge_backward_ker
                 gj[v] = ld_vec<W>(A.grad_out + base + v * LPE * W);
             }
             if (ok) {
-                float dot = 0.f;
+                unsigned long long d2 = 0ull;
 #pragma unroll
                 for (int v = 0; v < VPL; ++v) {
                     acc[v].fma(w.x, gj[v]);
-                    dot = FVec<W>::dot(gi[v], hj[v], dot);
-                    dot = FVec<W>::dot(gj[v], hi[v], dot);
+                    d2 = FVec<W>::dot2(gi[v], hj[v], d2);
+                    d2 = FVec<W>::dot2(gj[v], hi[v], d2);
                 }
+                const float dot = f2_sum(d2);
                 fx = fmaf(dot, w.y, fx);
                 fy = fmaf(dot, w.z, fy);
                 fz = fmaf(dot, w.w, fz);
@@ -670,7 +694,7 @@ tess_status edge_backward(const float* pos, int n, tess_box box, float rc, const
     A.F = F;
     A.L = make_float3(box.lx, box.ly, box.lz);
     A.inv_rc2 = 1.0f / (rc * rc);
-    A.dfc_scale = (float)(-9.8696044010893586188 / (2.0 * (double)rc * (double)rc));
+    A.dfc_scale = (float)(-2.0 / ((double)rc * (double)rc));
     StageScope sc(ST_BACKWARD, s);
     const size_t smem = (size_t)BK_WARPS * cap * (sizeof(float4) + sizeof(int));
     auto launch = [&](auto w, auto lpe, auto vpl) {

@@ -5,8 +5,9 @@ configuration as bench.py.
 Outputs the oracle can compute one by one are compared on samples: the whole
 permutation and key array (the oracle sorts 10M keys in seconds), neighbor rows
 of 3,000 sampled atoms plus the first and last tiles (brute force over all
-atoms), the skin flags and maximum displacements of a 6-step trajectory with
-rebuilds (exact, fp64), and aggregated features of sampled rows.  Properties
+atoms), the skin flags and maximum displacements of the workload's whole
+50-step trajectory with its rebuilds (exact, fp64), and aggregated features
+of sampled rows.  Properties
 that hold at any size are checked on the whole list: pads, counts >= 0, total
 pair count even, symmetry of sampled rows.
 """
@@ -91,7 +92,9 @@ def test_fullsize_pipeline_against_oracle(system):
     o_ref = p4
     o_perm = operm
     flags = []
-    for t, frame in s.trajectory(6, condition=False):
+    # the skin check compares exact fp64 values on both sides, so the frames
+    # need no band conditioning (that is for the lists)
+    for t, frame in s.trajectory(s.steps, condition=False):
         cur = torch.zeros_like(ref4)
         cur[:, :3] = torch.from_numpy(frame).to(dev)[cur_perm.long()]
         rb, md = tess.skin_check(cur, ref4, s.box, s.skin)
@@ -106,3 +109,5 @@ def test_fullsize_pipeline_against_oracle(system):
             assert np.array_equal(cur_perm.cpu().numpy(), o_perm)
             o_ref = np.zeros_like(o_ref)
             o_ref[:, :3] = frame[o_perm]
+    assert len(flags) == s.steps == 50
+    assert any(flags), "50 steps at sigma 0.01 A should trigger a rebuild"
