@@ -125,7 +125,7 @@ def sum_over_ranks(value: float, world: int, device=None) -> float:
 class Step:
     """All device buffers of one replica, and the path through the C ABI."""
 
-    def __init__(self, s, device, pad_fill=True, lane_search=False, curve="hilbert"):
+    def __init__(self, s, device, pad_fill=True, search="default", curve="hilbert"):
         import torch
         import space_filling_curve_b200 as tess
         self.tess = tess
@@ -152,7 +152,8 @@ class Step:
         # features live in the sorted index space (produced there by the model)
         self.feat = torch.randn((n, F), generator=g, device=device, dtype=torch.float32)
         self.out = torch.empty((n, F), dtype=torch.float32, device=device)
-        self.flags = (0 if pad_fill else tess.TESS_NO_PAD_FILL) | (tess.TESS_LANE_SEARCH if lane_search else 0)
+        self.flags = (0 if pad_fill else tess.TESS_NO_PAD_FILL) | {"default": 0, "lane": tess.TESS_LANE_SEARCH,
+                                                                    "tile": tess.TESS_TILE_SEARCH}[search]
         self.sort_fn = tess.tess_hilbert_sort if curve == "hilbert" else tess.tess_morton_sort
         # the next frame of the trajectory, in the sorted order of frame 0
         t1 = next(iter(s.trajectory(1, condition=False)))[1]
@@ -289,7 +290,7 @@ def run_cuda(args, world, rank, local):
     import synth
     import space_filling_curve_b200 as tess
     s = synth.system(args.config)
-    step = Step(s, dev, pad_fill=not args.no_pad_fill, lane_search=args.lane_search, curve=args.curve)
+    step = Step(s, dev, pad_fill=not args.no_pad_fill, search=args.search, curve=args.curve)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     peak, peak_kind = _peaks()
 
@@ -358,7 +359,7 @@ def run_cuda(args, world, rank, local):
         for cfg in (1, 2, 3, 4, 5):
             sc = s if cfg == args.config else synth.system(cfg)
             stc = step if cfg == args.config else Step(sc, dev, pad_fill=not args.no_pad_fill,
-                                                       lane_search=args.lane_search, curve=args.curve)
+                                                       search=args.search, curve=args.curve)
             all_cfg.append(_config_summary(stc, max(3, args.steps), flush, peak))
             if stc is not step:
                 del stc
@@ -384,7 +385,7 @@ def run_cuda(args, world, rank, local):
                             % (s.name, s.n, s.box[0], s.box[1], s.box[2], s.rc, s.skin, s.cap),
                 "atoms": s.n,
                 "pad_fill": not args.no_pad_fill,
-                "pair_search": "per-lane" if args.lane_search else "tile",
+                "pair_search": args.search, "library": tess.tess_version(),
                 "curve": args.curve,
                 "l2": "flushed before every timed rebuild (256 MB write, outside its events)",
                 "parallelism": "replicas (no collective in the data path)",
@@ -739,7 +740,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["tess", "reference"], default="tess")
     ap.add_argument("--config", type=int, default=WORKLOAD_CFG)
     ap.add_argument("--no-pad-fill", action="store_true")
-    ap.add_argument("--lane-search", action="store_true", help="use the per-lane stencil pair search")
+    ap.add_argument("--search", choices=["default", "tile", "lane"], default="default",
+                    help="pair search kernel (default: the library's choice)")
     ap.add_argument("--curve", choices=["hilbert", "morton"], default="hilbert",
                     help="space-filling curve of the sort (morton: the comparison curve)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

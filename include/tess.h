@@ -66,7 +66,8 @@ typedef struct {
 
 /* tess_build_neighbors flags */
 #define TESS_NO_PAD_FILL    1   /* leave slots >= min(count, max_neighbors) unwritten */
-#define TESS_LANE_SEARCH    2   /* use the per-lane stencil search instead of the warp tile search */
+#define TESS_LANE_SEARCH    2   /* use the per-lane stencil search */
+#define TESS_TILE_SEARCH    4   /* use the warp tile search (accept per 32-candidate block) */
 
 /* Human-readable name of a status code (static string). */
 const char* tess_status_string(tess_status s);
@@ -204,9 +205,11 @@ tess_status tess_hilbert_sort_static(const float* pos, int n, tess_box box, int 
  *   pos            [n,4] float (x, y, z, ignored), 16-byte aligned
  *   rc, skin       cutoff and skin (rc > 0, skin >= 0); rs = rc + skin in fp32
  *   max_neighbors  row capacity cap >= 1
- *   flags          0, or'ed TESS_NO_PAD_FILL, TESS_LANE_SEARCH (same lists, other
- *                  order within rows; boxes shorter than 2 rs + 2e-3 always use
- *                  the default tile search)
+ *   flags          0, or'ed TESS_NO_PAD_FILL and one of TESS_LANE_SEARCH,
+ *                  TESS_TILE_SEARCH (two search kernels: the same lists in
+ *                  another order within rows; 0 picks the library's default,
+ *                  and boxes shorter than 2 rs + 2e-3 always take the tile
+ *                  search)
  *   ws, ws_bytes   scratch of at least tess_build_neighbors_workspace(...)
  *   nbr            [n, cap] int32 out: row i in nbr[i*cap .. i*cap+cap);
  *                  the first min(counts[i], cap) slots hold neighbors, the

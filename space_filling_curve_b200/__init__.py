@@ -34,7 +34,7 @@ __all__ = [
     "tess_skin_check", "tess_edge_aggregate", "tess_stage_timing", "tess_stage_times",
     "hilbert_sort", "build_neighbors", "skin_check", "edge_aggregate",
     "tess_edge_aggregate_backward", "edge_aggregate_backward",
-    "TESS_DEV_OVERFLOW", "TESS_DEV_BAD_INPUT", "TESS_DEV_TIMEOUT", "TESS_NO_PAD_FILL", "TESS_LANE_SEARCH", "STAGES",
+    "TESS_DEV_OVERFLOW", "TESS_DEV_BAD_INPUT", "TESS_DEV_TIMEOUT", "TESS_NO_PAD_FILL", "TESS_LANE_SEARCH", "TESS_TILE_SEARCH", "STAGES",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -47,6 +47,7 @@ TESS_DEV_BAD_INPUT = 2
 TESS_DEV_TIMEOUT = 4
 TESS_NO_PAD_FILL = 1
 TESS_LANE_SEARCH = 2
+TESS_TILE_SEARCH = 4
 STAGES = ("hilbert_keys", "key_sort", "cell_binning", "pair_search", "skin_check", "edge_aggregate", "edge_backward",
           "resort", "min_pair")
 _STATUS = {0: "ok", 1: "invalid argument", 2: "box too small", 3: "workspace too small", 4: "CUDA launch error",
@@ -362,7 +363,7 @@ def morton_sort(pos, box, bits: int = 10, **kw):
 
 
 def build_neighbors(pos4, box, rc: float, skin: float, max_neighbors: int, *, pad_fill: bool = True,
-                    lane_search: bool = False, ws=None, nbr=None, counts=None, overflow=None, stream=None):
+                    search: str = "default", ws=None, nbr=None, counts=None, overflow=None, stream=None):
     """Padded Verlet list at rc + skin.  ``pos4``: float32 [n, 4] CUDA
     tensor.  Returns (nbr int32 [n, cap], counts int32 [n], overflow int32 [1])."""
     torch = _torch()
@@ -373,7 +374,7 @@ def build_neighbors(pos4, box, rc: float, skin: float, max_neighbors: int, *, pa
     nbr = torch.empty((n, max_neighbors), dtype=torch.int32, device=dev) if nbr is None else nbr
     counts = torch.empty(n, dtype=torch.int32, device=dev) if counts is None else counts
     overflow = torch.empty(1, dtype=torch.int32, device=dev) if overflow is None else overflow
-    flags = (0 if pad_fill else TESS_NO_PAD_FILL) | (TESS_LANE_SEARCH if lane_search else 0)
+    flags = (0 if pad_fill else TESS_NO_PAD_FILL) | {"default": 0, "lane": TESS_LANE_SEARCH, "tile": TESS_TILE_SEARCH}[search]
     code = tess_build_neighbors(_ptr(pos4), n, box, float(rc), float(skin), int(max_neighbors), flags, _ptr(ws),
                                 ws.numel() * ws.element_size(), _ptr(nbr), _ptr(counts), _ptr(overflow),
                                 _stream(stream))

@@ -127,7 +127,10 @@ const char* tess_status_string(tess_status s) {
     return "unknown status";
 }
 
-const char* tess_version(void) { return "tess-b200 0.1 (sm_100a)"; }
+const char* tess_version(void) {
+    return TESS_DEFAULT_LANE ? "tess-b200 0.2 (sm_100a; default pair search: per-lane)"
+                             : "tess-b200 0.2 (sm_100a; default pair search: tile)";
+}
 
 long long tess_kernel_launch_count(void) { return g_launches.load(); }
 

@@ -387,19 +387,61 @@ __global__ __launch_bounds__(BK_THREADS) void bucket_scatter_kernel(const unsign
     }
 }
 
-// Ranks of the lane's K elements among the bucket's m (shared memory s).
-template <int K>
-__device__ __forceinline__ void bucket_ranks(const unsigned long long* s, int m, const unsigned long long (&e)[8],
-                                             int (&r)[8]) {
+// One bucket of m elements (in shared memory s) with K elements per lane:
+// each element's rank is the number of smaller elements, and it lands in
+// slot beg + rank.  With EARLY the positions of the lane's atoms are fetched
+// before the ranking, so that their (random) loads overlap it; the rare
+// large buckets fetch them at the end and keep fewer registers.
+template <int K, bool EARLY>
+__device__ __forceinline__ void bucket_rank_write(const unsigned long long* s, int m, int beg, int lane,
+                                                  const float* __restrict__ pos3, int32_t* __restrict__ perm,
+                                                  uint32_t* __restrict__ keys_out, float4* __restrict__ pos_sorted,
+                                                  int n, int32_t* status) {
+    unsigned long long e[K];
+    int r[K];
+    float px[K], py[K], pz[K];
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+        const int t = lane + 32 * k;
+        e[k] = t < m ? s[t] : ~0ull;
+        r[k] = 0;
+        if (EARLY && pos_sorted && t < m) {
+            const unsigned idx = (unsigned)e[k];
+            if (check_index(idx, n, status)) {
+                const float* p = pos3 + 3 * (size_t)idx;
+                px[k] = p[0];
+                py[k] = p[1];
+                pz[k] = p[2];
+            }
+        }
+    }
 #pragma unroll 4
     for (int t = 0; t < m; ++t) {
         const unsigned long long v = s[t];
 #pragma unroll
         for (int k = 0; k < K; ++k) r[k] += v < e[k] ? 1 : 0;
     }
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+        const int t = lane + 32 * k;
+        if (t < m && check_index((long long)beg + r[k], n, status) && check_index((unsigned)e[k], n, status)) {
+            const int g = beg + r[k];
+            perm[g] = (int32_t)(unsigned)e[k];
+            if (keys_out) keys_out[g] = (uint32_t)(e[k] >> 32);
+            if (pos_sorted) {
+                if (!EARLY) {
+                    const float* p = pos3 + 3 * (size_t)(unsigned)e[k];
+                    px[k] = p[0];
+                    py[k] = p[1];
+                    pz[k] = p[2];
+                }
+                pos_sorted[g] = make_float4(px[k], py[k], pz[k], 0.0f);
+            }
+        }
+    }
 }
 
-__global__ __launch_bounds__(BK_WARPS * 32) void bucket_local_sort(const unsigned long long* __restrict__ elems,
+__global__ __launch_bounds__(BK_WARPS * 32, 4) void bucket_local_sort(const unsigned long long* __restrict__ elems,
                                                                    const int* __restrict__ bstart, int nb,
                                                                    const float* __restrict__ pos3,
                                                                    int32_t* __restrict__ perm,
@@ -418,34 +460,10 @@ __global__ __launch_bounds__(BK_WARPS * 32) void bucket_local_sort(const unsigne
         }
         for (int t = lane; t < m; t += 32) s[t] = elems[beg + t];
         __syncwarp();
-        const int K = (m + 31) >> 5;
-        unsigned long long e[8];
-        int r[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int t = lane + 32 * k;
-            e[k] = (k < K && t < m) ? s[t] : ~0ull;
-            r[k] = 0;
-        }
-        if (K == 1) bucket_ranks<1>(s, m, e, r);
-        else if (K == 2) bucket_ranks<2>(s, m, e, r);
-        else if (K <= 4) bucket_ranks<4>(s, m, e, r);
-        else bucket_ranks<8>(s, m, e, r);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int t = lane + 32 * k;
-            if (k < K && t < m && check_index((long long)beg + r[k], n, status) &&
-                check_index((long long)(unsigned)e[k], n, status)) {
-                const int g = beg + r[k];
-                const unsigned idx = (unsigned)e[k];
-                perm[g] = (int32_t)idx;
-                if (keys_out) keys_out[g] = (uint32_t)(e[k] >> 32);
-                if (pos_sorted) {
-                    const float* p = pos3 + 3 * (size_t)idx;
-                    pos_sorted[g] = make_float4(p[0], p[1], p[2], 0.0f);
-                }
-            }
-        }
+        if (m <= 32) bucket_rank_write<1, true>(s, m, beg, lane, pos3, perm, keys_out, pos_sorted, n, status);
+        else if (m <= 64) bucket_rank_write<2, true>(s, m, beg, lane, pos3, perm, keys_out, pos_sorted, n, status);
+        else if (m <= 128) bucket_rank_write<4, false>(s, m, beg, lane, pos3, perm, keys_out, pos_sorted, n, status);
+        else bucket_rank_write<8, false>(s, m, beg, lane, pos3, perm, keys_out, pos_sorted, n, status);
         __syncwarp();
     }
 }

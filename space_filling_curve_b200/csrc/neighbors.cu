@@ -21,7 +21,10 @@
 //      packed f32x2), 32 candidates per accept mask, and turns the set bits
 //      into indices that leave for its row in aligned 32-byte groups.
 // pair_search_lane_kernel (TESS_LANE_SEARCH) walks a stencil of cell rows
-// per lane instead; it gives the same lists in another order.
+// per lane instead; it gives the same lists in another order.  Which of the
+// two runs when the caller asks for neither is TESS_DEFAULT_LANE.
+#include <climits>
+
 #include "common.cuh"
 #include "scan.cuh"
 
@@ -113,20 +116,50 @@ __global__ void cell_scatter_kernel(const int* __restrict__ cell_id, const int* 
     }
 }
 
-// Deterministic order inside each cell: the slot of atom i is the cell start
-// plus the number of atoms of the same cell with a smaller index.
-__global__ void cell_order_kernel(const int* __restrict__ slot_atom, int n, const int* __restrict__ cell_id,
+// Deterministic order inside each cell: the atoms of a cell in ascending
+// index order, positions written in that order as float4 (x, y, z, index
+// bits).  One thread per cell; cells of up to 8 atoms (nearly all) are sorted
+// in registers by a fixed network, larger ones rank each atom by counting.
+__device__ __forceinline__ void cswap(int& a, int& b) {
+    const int lo = min(a, b), hi = max(a, b);
+    a = lo;
+    b = hi;
+}
+
+__global__ void cell_order_kernel(const int* __restrict__ slot_atom, long long ncell,
                                   const int* __restrict__ cell_start, const float4* __restrict__ pos,
                                   float4* __restrict__ pos_cell) {
-    const int stride = gridDim.x * blockDim.x;
-    for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < n; k += stride) {
-        const int i = slot_atom[k];
-        const int c = cell_id[i];
-        const int b = cell_start[c], e = cell_start[c + 1];
-        int r = 0;
-        for (int s = b; s < e; ++s) r += slot_atom[s] < i;
-        const float4 p = pos[i];
-        pos_cell[b + r] = make_float4(p.x, p.y, p.z, __int_as_float(i));
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long c = (long long)blockIdx.x * blockDim.x + threadIdx.x; c < ncell; c += stride) {
+        const int b = cell_start[c], e = cell_start[c + 1], m = e - b;
+        if (m <= 0) continue;
+        if (m <= 8) {
+            int v[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[k] = k < m ? slot_atom[b + k] : INT_MAX;
+            // Batcher's odd-even merge network for 8 (19 comparators)
+            cswap(v[0], v[1]); cswap(v[2], v[3]); cswap(v[4], v[5]); cswap(v[6], v[7]);
+            cswap(v[0], v[2]); cswap(v[1], v[3]); cswap(v[4], v[6]); cswap(v[5], v[7]);
+            cswap(v[1], v[2]); cswap(v[5], v[6]);
+            cswap(v[0], v[4]); cswap(v[1], v[5]); cswap(v[2], v[6]); cswap(v[3], v[7]);
+            cswap(v[2], v[4]); cswap(v[3], v[5]);
+            cswap(v[1], v[2]); cswap(v[3], v[4]); cswap(v[5], v[6]);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                if (k < m) {
+                    const float4 p = pos[v[k]];
+                    pos_cell[b + k] = make_float4(p.x, p.y, p.z, __int_as_float(v[k]));
+                }
+            }
+        } else {
+            for (int s = b; s < e; ++s) {
+                const int i = slot_atom[s];
+                int r = 0;
+                for (int t = b; t < e; ++t) r += slot_atom[t] < i;
+                const float4 p = pos[i];
+                pos_cell[b + r] = make_float4(p.x, p.y, p.z, __int_as_float(i));
+            }
+        }
     }
 }
 
@@ -196,36 +229,93 @@ __device__ __forceinline__ void append_if(unsigned& wsa, float r2, float rs2, in
 constexpr int TM_WARPS = 4;          // warps per block, each on its own tiles
 constexpr int TM_CH = 256;           // staged candidates per chunk (a multiple of 32)
 constexpr int TM_MAXSEG = 64;        // cell-row segments per table batch
-constexpr int TM_UNROLL = 4;         // candidate loads in flight per lane while culling
+#ifndef TESS_TM_RANGES
+#define TESS_TM_RANGES 0
+#endif
+#ifndef TESS_TM_UNROLL
+#define TESS_TM_UNROLL 4
+#endif
+constexpr int TM_UNROLL = TESS_TM_UNROLL;  // candidate loads in flight per lane while culling
 constexpr int TM_BUF = 48;           // per-lane buffer of accepted indices (>= 32 + TM_GROUP)
 constexpr int TM_GROUP = 8;          // indices leave in aligned groups of 8 (32 bytes)
+constexpr float TM_FFMA_H = 12.f;    // largest tile half-diagonal (A) for the fused pair test
 
 struct TileWarpSmem {
-    float cq[TM_CH * 3];             // staged candidates, 48 bytes per group of four (tile frame)
+    float cq[TM_CH * 4];             // staged candidates, 64 bytes per group of four (tile frame)
     int cj[TM_CH];                   // their atom indices
     SegEntry seg[TM_MAXSEG + 1];
     int buf[32 * TM_BUF];            // entry e of lane l at buf[e * 32 + l]
 };
 constexpr size_t TM_SMEM = sizeof(TileWarpSmem) * TM_WARPS;
 
-// Candidate s of the chunk: group s / 4, slot s % 4 of the 12-float layout.
+// Candidate s of the chunk: group s / 4 holds x0 x1 y0 y1 | z0 z1 n0 n1 |
+// x2 x3 y2 y3 | z2 z3 n2 n3 (tile frame, n = x^2 + y^2 + z^2), so that each
+// 16-byte read gives two candidates' values of one kind, ready for packed
+// f32x2 arithmetic.
 __device__ __forceinline__ void stage_cand(TileWarpSmem& W, int s, float x, float y, float z, int j) {
     const int k = s & 3;
-    const int off = 12 * (s >> 2) + (k & 1) + (k >> 1) * 6;
+    const int off = 16 * (s >> 2) + (k & 1) + (k >> 1) * 8;
     W.cq[off] = x;
     W.cq[off + 2] = y;
     W.cq[off + 4] = z;
+    W.cq[off + 6] = fmaf(z, z, fmaf(y, y, x * x));
     W.cj[s] = j;
 }
 
-// Tests the four candidates of group G of a 32-candidate block against the
-// lane's atom (px2, py2, pz2: its tile-frame coordinates in both halves) and
-// sets bits 4G .. 4G+3 of m for those with r^2 < rs^2.
+// Both pair tests below append each accepted index to the lane's buffer: it
+// is stored at the lane's next slot (*wsa) and the slot advances by one
+// lane-interleaved step (128 bytes).
+
+// Compact tiles: r^2 < rs^2  <=>  |c|^2 - 2 c.p < rs^2 - |p|^2 = T in the tile
+// frame (|c|, |p| of a few Angstrom), three packed fused multiply-adds per
+// two candidates: v = n + c.m with m = -2 p (m2x, m2y, m2z in both halves).
+// The tile's own atoms are not among the candidates (they are tested by
+// intra_tile), so no index comparison is needed.
 template <int G>
-__device__ __forceinline__ void test4(unsigned& m, const ulonglong2* q, unsigned long long px2,
-                                      unsigned long long py2, unsigned long long pz2, float rs2) {
-    const ulonglong2 a = q[3 * G], b = q[3 * G + 1], c = q[3 * G + 2];
-    asm("{\n\t.reg .b64 dx, dy, dz, r;\n\t.reg .f32 r0, r1;\n\t.reg .pred p;\n\t"
+__device__ __forceinline__ void test4_ffma(unsigned& wsa, const ulonglong2* q, const int4* qj,
+                                           unsigned long long m2x, unsigned long long m2y,
+                                           unsigned long long m2z, float T) {
+    const ulonglong2 a = q[4 * G], b = q[4 * G + 1], c = q[4 * G + 2], d = q[4 * G + 3];
+    const int4 j = qj[G];
+    asm volatile(
+        "{\n\t.reg .b64 v;\n\t.reg .f32 v0, v1;\n\t.reg .pred p;\n\t"
+        "fma.rn.f32x2 v, %1, %9, %4;\n\t"
+        "fma.rn.f32x2 v, %2, %10, v;\n\t"
+        "fma.rn.f32x2 v, %3, %11, v;\n\t"
+        "mov.b64 {v0, v1}, v;\n\t"
+        "setp.lt.f32 p, v0, %12;\n\t"
+        "@p st.shared.b32 [%0], %13;\n\t"
+        "@p add.u32 %0, %0, 128;\n\t"
+        "setp.lt.f32 p, v1, %12;\n\t"
+        "@p st.shared.b32 [%0], %14;\n\t"
+        "@p add.u32 %0, %0, 128;\n\t"
+        "fma.rn.f32x2 v, %5, %9, %8;\n\t"
+        "fma.rn.f32x2 v, %6, %10, v;\n\t"
+        "fma.rn.f32x2 v, %7, %11, v;\n\t"
+        "mov.b64 {v0, v1}, v;\n\t"
+        "setp.lt.f32 p, v0, %12;\n\t"
+        "@p st.shared.b32 [%0], %15;\n\t"
+        "@p add.u32 %0, %0, 128;\n\t"
+        "setp.lt.f32 p, v1, %12;\n\t"
+        "@p st.shared.b32 [%0], %16;\n\t"
+        "@p add.u32 %0, %0, 128;\n\t}"
+        : "+r"(wsa)
+        : "l"(a.x), "l"(a.y), "l"(b.x), "l"(b.y), "l"(c.x), "l"(c.y), "l"(d.x), "l"(d.y), "l"(m2x), "l"(m2y),
+          "l"(m2z), "f"(T), "r"(j.x), "r"(j.y), "r"(j.z), "r"(j.w)
+        : "memory");
+}
+
+// Any tile: differences (x, y, z of candidate minus atom, both in the tile
+// frame), r^2 = (dx^2 + dy^2) + dz^2 with packed arithmetic, r^2 < rs^2, and
+// the atom itself (index `self`) skipped.
+template <int G>
+__device__ __forceinline__ void test4_sub(unsigned& wsa, const ulonglong2* q, const int4* qj,
+                                          unsigned long long px2, unsigned long long py2,
+                                          unsigned long long pz2, float rs2, int self) {
+    const ulonglong2 a = q[4 * G], b = q[4 * G + 1], c = q[4 * G + 2], d = q[4 * G + 3];
+    const int4 j = qj[G];
+    asm volatile(
+        "{\n\t.reg .b64 dx, dy, dz, r;\n\t.reg .f32 r0, r1;\n\t.reg .pred p;\n\t"
         "sub.rn.f32x2 dx, %1, %7;\n\t"
         "sub.rn.f32x2 dy, %2, %8;\n\t"
         "sub.rn.f32x2 dz, %3, %9;\n\t"
@@ -234,9 +324,13 @@ __device__ __forceinline__ void test4(unsigned& m, const ulonglong2* q, unsigned
         "fma.rn.f32x2 r, dz, dz, r;\n\t"
         "mov.b64 {r0, r1}, r;\n\t"
         "setp.lt.f32 p, r0, %10;\n\t"
-        "@p or.b32 %0, %0, %11;\n\t"
+        "setp.ne.and.s32 p, %11, %15, p;\n\t"
+        "@p st.shared.b32 [%0], %11;\n\t"
+        "@p add.u32 %0, %0, 128;\n\t"
         "setp.lt.f32 p, r1, %10;\n\t"
-        "@p or.b32 %0, %0, %12;\n\t"
+        "setp.ne.and.s32 p, %12, %15, p;\n\t"
+        "@p st.shared.b32 [%0], %12;\n\t"
+        "@p add.u32 %0, %0, 128;\n\t"
         "sub.rn.f32x2 dx, %4, %7;\n\t"
         "sub.rn.f32x2 dy, %5, %8;\n\t"
         "sub.rn.f32x2 dz, %6, %9;\n\t"
@@ -245,22 +339,54 @@ __device__ __forceinline__ void test4(unsigned& m, const ulonglong2* q, unsigned
         "fma.rn.f32x2 r, dz, dz, r;\n\t"
         "mov.b64 {r0, r1}, r;\n\t"
         "setp.lt.f32 p, r0, %10;\n\t"
-        "@p or.b32 %0, %0, %13;\n\t"
+        "setp.ne.and.s32 p, %13, %15, p;\n\t"
+        "@p st.shared.b32 [%0], %13;\n\t"
+        "@p add.u32 %0, %0, 128;\n\t"
         "setp.lt.f32 p, r1, %10;\n\t"
-        "@p or.b32 %0, %0, %14;\n\t}"
-        : "+r"(m)
-        : "l"(a.x), "l"(a.y), "l"(b.x), "l"(b.y), "l"(c.x), "l"(c.y), "l"(px2), "l"(py2), "l"(pz2), "f"(rs2),
-          "n"(1u << (4 * G)), "n"(1u << (4 * G + 1)), "n"(1u << (4 * G + 2)), "n"(1u << (4 * G + 3)));
+        "setp.ne.and.s32 p, %14, %15, p;\n\t"
+        "@p st.shared.b32 [%0], %14;\n\t"
+        "@p add.u32 %0, %0, 128;\n\t}"
+        : "+r"(wsa)
+        : "l"(a.x), "l"(a.y), "l"(b.x), "l"(c.x), "l"(c.y), "l"(d.x), "l"(px2), "l"(py2), "l"(pz2), "f"(rs2),
+          "r"(j.x), "r"(j.y), "r"(j.z), "r"(j.w), "r"(self)
+        : "memory");
+}
+
+// q = a / b, r = a % b for 0 <= a < 2^22 and a small divisor b > 0, through
+// the fp32 reciprocal and one correction step (cheaper than integer division).
+__device__ __forceinline__ void div_small(int a, int b, float inv_b, int& q, int& r) {
+    q = (int)((float)a * inv_b);
+    r = a - q * b;
+    if (r < 0) { --q; r += b; }
+    else if (r >= b) { ++q; r -= b; }
 }
 
 __device__ __forceinline__ unsigned long long pk2(float v) {
     return (unsigned long long)__float_as_uint(v) | ((unsigned long long)__float_as_uint(v) << 32);
 }
 
+// The list is written once and read by later kernels; its stores are marked
+// streaming (evict first) so that they do not push the candidate positions,
+// which every tile reads again, out of L2.
+#ifndef TESS_TM_CS
+#define TESS_TM_CS 1
+#endif
+#if TESS_TM_CS
+#define TESS_ST_COP ".cs"
+#else
+#define TESS_ST_COP ""
+#endif
+
 // Eight consecutive ints to a 32-byte aligned global address.
 __device__ __forceinline__ void st_global_v8(int* p, int a0, int a1, int a2, int a3, int a4, int a5, int a6, int a7) {
-    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a0), "r"(a1), "r"(a2),
-                 "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7)
+    asm volatile("st.global" TESS_ST_COP ".v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a0),
+                 "r"(a1), "r"(a2), "r"(a3), "r"(a4), "r"(a5), "r"(a6), "r"(a7)
+                 : "memory");
+}
+// Four consecutive ints to a 16-byte aligned global address.
+__device__ __forceinline__ void st_global_v4(int* p, int a0, int a1, int a2, int a3) {
+    asm volatile("st.global" TESS_ST_COP ".v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a0), "r"(a1), "r"(a2),
+                 "r"(a3)
                  : "memory");
 }
 
@@ -273,14 +399,24 @@ __global__ __launch_bounds__(TM_WARPS * 32, 4) void pair_tile_kernel(PairArgs A)
     const unsigned lt_mask = lanemask_lt();
     TileWarpSmem& W = reinterpret_cast<TileWarpSmem*>(tm_smem_raw)[warp];
     int* const buf = W.buf + lane;
+    const unsigned buf_sa = (unsigned)__cvta_generic_to_shared(buf);
     const int cap = A.cap;
     const long long ntiles = ((long long)A.n + 31) / 32;
     const float nanf_ = __int_as_float(0x7fc00000);
     const float wy = A.L.y / (float)A.nc.y, wz = A.L.z / (float)A.nc.z;
     const float reach2 = A.reach * A.reach;
 
+#if TESS_TM_RANGES
+    // each block walks its own contiguous range of tiles (its warps side by
+    // side), so that an SM works on neighboring tiles whose candidate cells
+    // overlap and stay in its L1
+    const long long per_block = (ntiles + gridDim.x - 1) / gridDim.x;
+    const long long t_end = min(ntiles, (long long)(blockIdx.x + 1) * per_block);
+    for (long long tile = (long long)blockIdx.x * per_block + warp; tile < t_end; tile += TM_WARPS) {
+#else
     for (long long tile = (long long)blockIdx.x * TM_WARPS + warp; tile < ntiles;
          tile += (long long)gridDim.x * TM_WARPS) {
+#endif
         const int base = (int)(tile * 32);
         const int i = base + lane;
         const bool valid = i < A.n;
@@ -308,8 +444,23 @@ __global__ __launch_bounds__(TM_WARPS * 32, 4) void pair_tile_kernel(PairArgs A)
         lox = fmaxf(lox, -A.L.x); loy = fmaxf(loy, -A.L.y); loz = fmaxf(loz, -A.L.z);
         hix = fminf(hix, 2.f * A.L.x); hiy = fminf(hiy, 2.f * A.L.y); hiz = fminf(hiz, 2.f * A.L.z);
         const float ox = 0.5f * (lox + hix), oy = 0.5f * (loy + hiy), oz = 0.5f * (loz + hiz);
-        const unsigned long long px2 = pk2(p.x - ox), py2 = pk2(p.y - oy), pz2 = pk2(p.z - oz);
+        const float qx = p.x - ox, qy = p.y - oy, qz = p.z - oz;     // the atom in the tile frame
+        const unsigned long long px2 = pk2(qx), py2 = pk2(qy), pz2 = pk2(qz);
         const float rs2 = A.rs2;
+        // A compact tile (the usual case) uses the fused form of the pair
+        // test, whose fp32 error grows with the frame's size: for a
+        // half-diagonal up to TM_FFMA_H the terms stay below ~800 A^2 and the
+        // rounding of n, T and the three products moves r^2 by at most
+        // ~1.6e-4 A^2, about 1.3e-5 A in r near rs -- well inside the 1e-4 A
+        // band that the inputs keep around rs.  It also leaves its own atoms
+        // out of the candidates: they are tested against each other directly,
+        // which needs every pair inside the tile to be its own minimum image.
+        const float hx = 0.5f * (hix - lox), hy = 0.5f * (hiy - loy), hz = 0.5f * (hiz - loz);
+        const bool compact = fmaf(hz, hz, fmaf(hy, hy, hx * hx)) <= TM_FFMA_H * TM_FFMA_H &&
+                             4.f * hx < A.L.x - 2.f * A.reach && 4.f * hy < A.L.y - 2.f * A.reach &&
+                             4.f * hz < A.L.z - 2.f * A.reach;
+        const unsigned long long m2x = pk2(-2.f * qx), m2y = pk2(-2.f * qy), m2z = pk2(-2.f * qz);
+        const float T = rs2 - fmaf(qz, qz, fmaf(qy, qy, qx * qx));
 
         int done = 0;      // accepted indices handed to the row (a multiple of TM_GROUP until the end)
         int pend = 0;      // indices waiting in this lane's buffer
@@ -325,8 +476,8 @@ __global__ __launch_bounds__(TM_WARPS * 32, 4) void pair_tile_kernel(PairArgs A)
                     st_global_v8(row + done, src[0], src[32], src[64], src[96], src[128], src[160], src[192],
                                  src[224]);
                 } else if (VW == 4 && done + TM_GROUP <= cap) {
-                    *reinterpret_cast<int4*>(row + done) = make_int4(src[0], src[32], src[64], src[96]);
-                    *reinterpret_cast<int4*>(row + done + 4) = make_int4(src[128], src[160], src[192], src[224]);
+                    st_global_v4(row + done, src[0], src[32], src[64], src[96]);
+                    st_global_v4(row + done + 4, src[128], src[160], src[192], src[224]);
                 } else {
 #pragma unroll
                     for (int e = 0; e < TM_GROUP; ++e)
@@ -353,41 +504,42 @@ __global__ __launch_bounds__(TM_WARPS * 32, 4) void pair_tile_kernel(PairArgs A)
             }
             for (int blk = 0; blk < nblk; ++blk) {
                 if (__any_sync(FULL, pend > TM_BUF - 32)) drain();
-                const ulonglong2* q = reinterpret_cast<const ulonglong2*>(W.cq + blk * 96);
-                // eight independent nibbles, joined by a tree of ORs
-                unsigned m0 = 0u, m1 = 0u, m2 = 0u, m3 = 0u, m4 = 0u, m5 = 0u, m6 = 0u, m7 = 0u;
-                test4<0>(m0, q, px2, py2, pz2, rs2);
-                test4<1>(m1, q, px2, py2, pz2, rs2);
-                test4<2>(m2, q, px2, py2, pz2, rs2);
-                test4<3>(m3, q, px2, py2, pz2, rs2);
-                test4<4>(m4, q, px2, py2, pz2, rs2);
-                test4<5>(m5, q, px2, py2, pz2, rs2);
-                test4<6>(m6, q, px2, py2, pz2, rs2);
-                test4<7>(m7, q, px2, py2, pz2, rs2);
-                unsigned m = ((m0 | m1) | (m2 | m3)) | ((m4 | m5) | (m6 | m7));
-                const int* cjb = W.cj + blk * 32;
-                while (m) {
-                    const int b = __ffs(m) - 1;
-                    m &= m - 1u;
-                    const int j = cjb[b];
-                    if (j != i && check_index(j, A.n, A.status)) {
-                        buf[pend * 32] = j;
-                        ++pend;
-                    }
+                const ulonglong2* q = reinterpret_cast<const ulonglong2*>(W.cq + blk * 128);
+                const int4* qj = reinterpret_cast<const int4*>(W.cj + blk * 32);
+                unsigned wsa = buf_sa + 128u * (unsigned)pend;
+                if (compact) {
+                    test4_ffma<0>(wsa, q, qj, m2x, m2y, m2z, T);
+                    test4_ffma<1>(wsa, q, qj, m2x, m2y, m2z, T);
+                    test4_ffma<2>(wsa, q, qj, m2x, m2y, m2z, T);
+                    test4_ffma<3>(wsa, q, qj, m2x, m2y, m2z, T);
+                    test4_ffma<4>(wsa, q, qj, m2x, m2y, m2z, T);
+                    test4_ffma<5>(wsa, q, qj, m2x, m2y, m2z, T);
+                    test4_ffma<6>(wsa, q, qj, m2x, m2y, m2z, T);
+                    test4_ffma<7>(wsa, q, qj, m2x, m2y, m2z, T);
+                } else {
+                    test4_sub<0>(wsa, q, qj, px2, py2, pz2, rs2, i);
+                    test4_sub<1>(wsa, q, qj, px2, py2, pz2, rs2, i);
+                    test4_sub<2>(wsa, q, qj, px2, py2, pz2, rs2, i);
+                    test4_sub<3>(wsa, q, qj, px2, py2, pz2, rs2, i);
+                    test4_sub<4>(wsa, q, qj, px2, py2, pz2, rs2, i);
+                    test4_sub<5>(wsa, q, qj, px2, py2, pz2, rs2, i);
+                    test4_sub<6>(wsa, q, qj, px2, py2, pz2, rs2, i);
+                    test4_sub<7>(wsa, q, qj, px2, py2, pz2, rs2, i);
                 }
+                pend = (int)((wsa - buf_sa) >> 7);
             }
             if (last) {
                 ncand = 0;
             } else {
                 // the partial block (fewer than 32) moves to the front: whole
-                // 48-byte groups and their indices
+                // 64-byte groups and their indices
                 const int rem = ncand - (nblk << 5);
                 __syncwarp();
                 float4* cq4 = reinterpret_cast<float4*>(W.cq);
-                const int nq = ((rem + 3) >> 2) * 3;
+                const int nq = ((rem + 3) >> 2) * 4;
                 float4 t4 = make_float4(0.f, 0.f, 0.f, 0.f);
                 int tj = 0;
-                if (lane < nq) t4 = cq4[nblk * 24 + lane];
+                if (lane < nq) t4 = cq4[nblk * 32 + lane];
                 if (lane < rem) tj = W.cj[(nblk << 5) + lane];
                 __syncwarp();
                 if (lane < nq) cq4[lane] = t4;
@@ -397,6 +549,22 @@ __global__ __launch_bounds__(TM_WARPS * 32, 4) void pair_tile_kernel(PairArgs A)
             __syncwarp();
         };
 
+        // the tile's own atoms against each other (compact tiles): the other
+        // 31 lanes' frame coordinates by shuffles, the same fp32 difference
+        // form as test4_sub; its indices enter the (empty) buffer first
+        if (compact) {
+            unsigned wsa = buf_sa;
+            for (int o = 1; o < 32; ++o) {
+                const int src = (lane + o) & 31;
+                const float dx = __shfl_sync(FULL, qx, src) - qx;
+                const float dy = __shfl_sync(FULL, qy, src) - qy;
+                const float dz = __shfl_sync(FULL, qz, src) - qz;
+                const float r2 = fmaf(dz, dz, fmaf(dy, dy, dx * dx));
+                append_if(wsa, r2, rs2, base + src, i);
+            }
+            pend = (int)((wsa - buf_sa) >> 7);
+        }
+
         // level 2: cell rows within reach of the box, each clipped to its chord
         const int ux0 = (int)floorf((lox - A.reach) * A.inv_w.x), ux1 = (int)floorf((hix + A.reach) * A.inv_w.x);
         const int uy0 = (int)floorf((loy - A.reach) * A.inv_w.y), uy1 = (int)floorf((hiy + A.reach) * A.inv_w.y);
@@ -405,6 +573,7 @@ __global__ __launch_bounds__(TM_WARPS * 32, 4) void pair_tile_kernel(PairArgs A)
         const int kx0 = floor_div(ux0, A.nc.x);
         const int npieces = floor_div(ux1, A.nc.x) - kx0 + 1;
         const int nseg = ny * nz * npieces;
+        const float inv_np = 1.0f / (float)npieces, inv_ny = 1.0f / (float)ny;
 
         for (int sb = 0; sb < nseg; sb += TM_MAXSEG) {
             const int nb = min(TM_MAXSEG, nseg - sb);
@@ -415,9 +584,11 @@ __global__ __launch_bounds__(TM_WARPS * 32, 4) void pair_tile_kernel(PairArgs A)
                 float sx = 0.f, sy = 0.f, sz = 0.f;
                 if (sl < nb) {
                     const int s = sb + sl;
-                    const int piece = s % npieces;
-                    const int rw = s / npieces;
-                    const int uy = uy0 + rw % ny, uz = uz0 + rw / ny;
+                    // s = rw * npieces + piece, rw = (uz - uz0) * ny + (uy - uy0)
+                    int rw, piece, rz, ry;
+                    div_small(s, npieces, inv_np, rw, piece);
+                    div_small(rw, ny, inv_ny, rz, ry);
+                    const int uy = uy0 + ry, uz = uz0 + rz;
                     // the row's distance to the box in y and z (unwrapped cell geometry)
                     const float ylo = (float)uy * wy, zlo = (float)uz * wz;
                     const float ddy = fmaxf(fmaxf(ylo - hiy, loy - (ylo + wy)), 0.f);
@@ -427,8 +598,11 @@ __global__ __launch_bounds__(TM_WARPS * 32, 4) void pair_tile_kernel(PairArgs A)
                         const float ch = fmaf(ch2 * rsqrtf(ch2), 1.0001f, 1e-4f);
                         const int ca = max(ux0, (int)floorf((lox - ch) * A.inv_w.x));
                         const int cb = min(ux1, (int)floorf((hix + ch) * A.inv_w.x));
-                        const int ky = floor_div(uy, A.nc.y), kz = floor_div(uz, A.nc.z);
-                        const int cy = uy - ky * A.nc.y, cz = uz - kz * A.nc.z;
+                        int ky = 0, kz = 0, cy = uy, cz = uz;
+                        while (cy < 0) { cy += A.nc.y; --ky; }
+                        while (cy >= A.nc.y) { cy -= A.nc.y; ++ky; }
+                        while (cz < 0) { cz += A.nc.z; --kz; }
+                        while (cz >= A.nc.z) { cz -= A.nc.z; ++kz; }
                         const int kx = kx0 + piece;
                         const int xa = max(ca, kx * A.nc.x) - kx * A.nc.x;
                         const int xb = min(cb, (kx + 1) * A.nc.x - 1) - kx * A.nc.x;
@@ -460,35 +634,54 @@ __global__ __launch_bounds__(TM_WARPS * 32, 4) void pair_tile_kernel(PairArgs A)
             __syncwarp();
             const int total = run;
 
+            // candidates are loaded one round ahead of their culling, so that
+            // the loads of round k+1 are in flight while round k is culled and
+            // the chunk is tested
             int sc = 0;   // this lane's segment cursor
-            for (int t0 = 0; t0 < total; t0 += 32 * TM_UNROLL) {
-                if (ncand > TM_CH - 32 * TM_UNROLL) test_chunk(false);
-                float4 q[TM_UNROLL];
-                bool ok[TM_UNROLL];
+            float4 nq[TM_UNROLL];
+            int ns[TM_UNROLL];
+            auto load_round = [&](int t0) {
 #pragma unroll
                 for (int u = 0; u < TM_UNROLL; ++u) {
                     const int t = t0 + u * 32 + lane;
-                    ok[u] = t < total;
-                    if (ok[u]) {
+                    ns[u] = -1;
+                    if (t < total) {
                         while (W.seg[sc + 1].pre <= t) ++sc;
-                        const SegEntry& e = W.seg[sc];
-                        const float4 c = A.pos_cell[e.beg + (t - e.pre)];
-                        q[u] = make_float4(c.x + e.sx, c.y + e.sy, c.z + e.sz, c.w);
+                        ns[u] = sc;
+                        nq[u] = A.pos_cell[W.seg[sc].beg + (t - W.seg[sc].pre)];
                     }
                 }
+            };
+            load_round(0);
+            for (int t0 = 0; t0 < total; t0 += 32 * TM_UNROLL) {
+                float4 q[TM_UNROLL];
+                int qs[TM_UNROLL];
+#pragma unroll
+                for (int u = 0; u < TM_UNROLL; ++u) {
+                    q[u] = nq[u];
+                    qs[u] = ns[u];
+                }
+                if (t0 + 32 * TM_UNROLL < total) load_round(t0 + 32 * TM_UNROLL);
+                if (ncand > TM_CH - 32 * TM_UNROLL) test_chunk(false);
 #pragma unroll
                 for (int u = 0; u < TM_UNROLL; ++u) {
                     bool keep = false;
-                    if (ok[u]) {
-                        const float ex = fmaxf(fmaxf(lox - q[u].x, q[u].x - hix), 0.f);
-                        const float ey = fmaxf(fmaxf(loy - q[u].y, q[u].y - hiy), 0.f);
-                        const float ez = fmaxf(fmaxf(loz - q[u].z, q[u].z - hiz), 0.f);
-                        keep = fmaf(ez, ez, fmaf(ey, ey, ex * ex)) < reach2;
+                    float4 c = q[u];
+                    if (qs[u] >= 0) {
+                        const SegEntry& e = W.seg[qs[u]];
+                        c.x += e.sx;
+                        c.y += e.sy;
+                        c.z += e.sz;
+                        const float ex = fmaxf(fmaxf(lox - c.x, c.x - hix), 0.f);
+                        const float ey = fmaxf(fmaxf(loy - c.y, c.y - hiy), 0.f);
+                        const float ez = fmaxf(fmaxf(loz - c.z, c.z - hiz), 0.f);
+                        keep = fmaf(ez, ez, fmaf(ey, ey, ex * ex)) < reach2 &&
+                               !(compact && (unsigned)(__float_as_int(c.w) - base) < 32u);
                     }
                     const unsigned bm = __ballot_sync(FULL, keep);
                     if (keep)
-                        stage_cand(W, ncand + __popc(bm & lt_mask), q[u].x - ox, q[u].y - oy, q[u].z - oz,
-                                   __float_as_int(q[u].w));
+                        stage_cand(W, ncand + __popc(bm & lt_mask), c.x - ox, c.y - oy, c.z - oz,
+                                   __float_as_int(c.w));
                     ncand += __popc(bm);
                 }
             }
@@ -507,8 +700,8 @@ __global__ __launch_bounds__(TM_WARPS * 32, 4) void pair_tile_kernel(PairArgs A)
             if (VW == 8) {
                 st_global_v8(row + done, v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
             } else {
-                *reinterpret_cast<int4*>(row + done) = make_int4(v[0], v[1], v[2], v[3]);
-                *reinterpret_cast<int4*>(row + done + 4) = make_int4(v[4], v[5], v[6], v[7]);
+                st_global_v4(row + done, v[0], v[1], v[2], v[3]);
+                st_global_v4(row + done + 4, v[4], v[5], v[6], v[7]);
             }
             filled = done + TM_GROUP;
         } else {
@@ -520,21 +713,19 @@ __global__ __launch_bounds__(TM_WARPS * 32, 4) void pair_tile_kernel(PairArgs A)
         if (!valid) filled = cap;
 
         if (valid) A.counts[i] = cnt;
-        if (A.pad_fill) {
-            // pads row by row, the whole warp on one row at a time (coalesced)
-            for (int r = 0; r < 32; ++r) {
-                const int fr = __shfl_sync(FULL, filled, r);
-                if (fr >= cap) continue;
-                int* rowr = A.nbr + (size_t)(base + r) * cap;
-                if (VW >= 4) {
-                    const int f4 = min((fr + 3) & ~3, cap);
-                    if (lane < f4 - fr) rowr[fr + lane] = -1;
-                    for (int e = f4 + 4 * lane; e < cap; e += 128)
-                        *reinterpret_cast<int4*>(rowr + e) = make_int4(-1, -1, -1, -1);
-                } else {
-                    for (int e = fr + lane; e < cap; e += 32) rowr[e] = -1;
-                }
+        if (A.pad_fill && valid) {
+            // each lane pads its own row (the kernel is bound by instruction
+            // issue, not by the L1 pipe, so few wide stores beat a coalesced
+            // pass over the 32 rows)
+            int e = filled;
+            if (VW == 8) {
+                for (; e < cap && (e & 7); ++e) row[e] = -1;
+                for (; e + 8 <= cap; e += 8) st_global_v8(row + e, -1, -1, -1, -1, -1, -1, -1, -1);
+            } else if (VW == 4) {
+                for (; e < cap && (e & 3); ++e) row[e] = -1;
+                for (; e + 4 <= cap; e += 4) st_global_v4(row + e, -1, -1, -1, -1);
             }
+            for (; e < cap; ++e) row[e] = -1;
         }
         const unsigned ov = __ballot_sync(FULL, valid && cnt > cap);
         if (ov && lane == 0) atomicOr(A.status, TESS_DEV_OVERFLOW);
@@ -749,7 +940,8 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
     if (n <= 0 || !pos || !ws || !nbr || !counts || !overflow || cap < 1) return TESS_ERR_INVALID_ARG;
     if (!box_ok(box) || !(rc > 0.f) || !(skin >= 0.f) || !std::isfinite(rc) || !std::isfinite(skin))
         return TESS_ERR_INVALID_ARG;
-    if ((flags & ~(TESS_NO_PAD_FILL | TESS_LANE_SEARCH)) != 0) return TESS_ERR_INVALID_ARG;
+    if ((flags & ~(TESS_NO_PAD_FILL | TESS_LANE_SEARCH | TESS_TILE_SEARCH)) != 0) return TESS_ERR_INVALID_ARG;
+    if ((flags & TESS_LANE_SEARCH) && (flags & TESS_TILE_SEARCH)) return TESS_ERR_INVALID_ARG;
     if (!aligned(pos, 16) || !aligned(ws, 256) || !aligned(nbr, 4) || !aligned(counts, 4)) return TESS_ERR_INVALID_ARG;
     const float rs = rc + skin;
     if (box.lx < 2.f * rs || box.ly < 2.f * rs || box.lz < 2.f * rs) return TESS_ERR_BOX_TOO_SMALL;
@@ -777,7 +969,8 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
         scan_sums_kernel<<<1, SCAN_THREADS, 0, s>>>(L.sums, scan_tiles);
         scan_apply_kernel<<<(unsigned)scan_tiles, SCAN_THREADS, 0, s>>>(L.cnt, m, L.sums, L.cell_start);
         cell_scatter_kernel<<<blocks, 256, 0, s>>>(L.cell_id, L.cell_rank, n, L.cell_start, L.slot_atom, overflow);
-        cell_order_kernel<<<blocks, 256, 0, s>>>(L.slot_atom, n, L.cell_id, L.cell_start, pos4, L.pos_cell);
+        cell_order_kernel<<<(int)std::min<long long>((m + 255) / 256, (long long)sms * 16), 256, 0, s>>>(
+            L.slot_atom, m, L.cell_start, pos4, L.pos_cell);
         count_launch(6);
     }
     {
@@ -803,11 +996,16 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
         // the per-lane search needs every box length >= 2 reach (a window
         // then wraps at most once); otherwise the tile search handles it
         const bool lane_ok = box.lx >= 2.f * A.reach && box.ly >= 2.f * A.reach && box.lz >= 2.f * A.reach;
-        if ((flags & TESS_LANE_SEARCH) && lane_ok) {
+        const bool want_lane = (flags & TESS_LANE_SEARCH) || (!(flags & TESS_TILE_SEARCH) && TESS_DEFAULT_LANE);
+        if (want_lane && lane_ok) {
             const long long blocks = (ntiles + PL_WARPS - 1) / PL_WARPS;
             pair_search_lane_kernel<<<(unsigned)std::min<long long>(blocks, 1LL << 30), PL_WARPS * 32, 0, s>>>(A);
         } else {
+#if TESS_TM_RANGES
+            const long long blocks = std::min<long long>((ntiles + TM_WARPS - 1) / TM_WARPS, (long long)sms * 4);
+#else
             const long long blocks = std::min<long long>((ntiles + TM_WARPS - 1) / TM_WARPS, 1LL << 30);
+#endif
             const bool v8 = cap % 8 == 0 && aligned(nbr, 32), v4 = cap % 4 == 0 && aligned(nbr, 16);
             auto launch = [&](auto kern) {
                 cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TM_SMEM);

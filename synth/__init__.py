@@ -105,6 +105,31 @@ def mark_forbidden(pos32: np.ndarray, box, r_band: float, dmin: float = DMIN, ba
     return close.astype(bool), bandm.astype(bool)
 
 
+def band_clean(pos, box, rs: float, seed: int = 0, max_iter: int = 200) -> np.ndarray:
+    """Nudge atoms of hand-made test inputs until no pair lies within BAND of
+    rs (the rule every generated input keeps, so that fp32 distances cannot
+    flip a list decision).  pos: float32 [n, 3] or [n, 4]; returns a float32
+    copy of the same shape.  Non-finite positions are left alone."""
+    p = np.array(pos, dtype=np.float32, copy=True)
+    rng = np.random.default_rng([seed, 77])
+    L32 = np.asarray(box, dtype=np.float32)
+    fin = np.isfinite(p[:, :3]).all(1)
+    inside = fin & ((p[:, :3] >= 0) & (p[:, :3] < L32)).all(1)
+    for _ in range(max_iter):
+        q = np.where(fin[:, None], p[:, :3], np.float32(0.0))
+        _, bandm = mark_forbidden(q, box, rs, dmin=0.0)
+        bandm &= fin
+        if not bandm.any():
+            return p
+        idx = np.nonzero(bandm)[0]
+        moved = p[idx, :3].astype(np.float64) + rng.uniform(-0.003, 0.003, size=(len(idx), 3))
+        # atoms that were in [0, L) stay there
+        ins = inside[idx]
+        moved[ins] = wrap_cast(moved[ins], box)
+        p[idx, :3] = moved.astype(np.float32)
+    raise RuntimeError("band conditioning did not converge")
+
+
 def wrap_cast(x64: np.ndarray, box) -> np.ndarray:
     """fp64 positions -> fp32 in [0, L): wrap in fp64, cast, fold L to 0."""
     L = np.asarray(box, dtype=np.float64)

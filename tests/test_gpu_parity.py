@@ -96,7 +96,7 @@ def test_sort_configs(cfg):
 
 def _gpu_list(pos4, box, rc, skin, cap, pad_fill=True, lane=False):
     tess = _tess()
-    nbr, cnt, ov = tess.build_neighbors(_dev(pos4), box, rc, skin, cap, pad_fill=pad_fill, lane_search=lane)
+    nbr, cnt, ov = tess.build_neighbors(_dev(pos4), box, rc, skin, cap, pad_fill=pad_fill, search="lane" if lane else "tile")
     torch_cuda().cuda.synchronize()
     return nbr, cnt, int(ov.item())
 
@@ -153,6 +153,7 @@ def test_neighbors_ragged(n, lane):
     L = 30.0
     p = np.zeros((n, 4), np.float32)
     p[:, :3] = rng.uniform(0, L, (n, 3))
+    p = synth.band_clean(p, (L, L, L), 4.5)       # no pair within 1e-4 A of rs, like every generated input
     _check_list(p, (L, L, L), 4.0, 0.5, 64, method="brute", lane=lane)
 
 
@@ -165,12 +166,13 @@ def test_neighbors_flag_invalid_positions(lane):
     n, L, rc, skin = 2000, 30.0, 4.0, 0.5
     p = np.zeros((n, 4), np.float32)
     p[:, :3] = rng.uniform(0, L, (n, 3))
+    p = synth.band_clean(p, (L, L, L), rc + skin)
     bad = [5, 9, 13]
     p[5, 0] = np.nan
     p[9, 0] = -0.5
     p[13, 1] = L + 1.0
     nbr_d, cnt_d, ov = tess.build_neighbors(_dev(p), (L, L, L), rc, skin, 128,
-                                            lane_search=lane)
+                                            search="lane" if lane else "tile")
     assert int(ov.item()) & 2
     onbr, ocnt, _ = oracle.neighbors_brute(p, (L, L, L), rc, skin, 128)
     good = np.ones(n, bool)
@@ -204,6 +206,7 @@ def test_neighbors_small_boxes(L, rc, lane):
     n = int(0.1 * L ** 3)
     p = np.zeros((n, 4), np.float32)
     p[:, :3] = rng.uniform(0, L, (n, 3))
+    p = synth.band_clean(p, (L, L, L), float(np.float32(rc) + np.float32(0.5)))
     p = p[oracle.hilbert_sort(p, (L, L, L), 10)[0]]
     _check_list(p, (L, L, L), rc, 0.5, 256, method="brute", lane=lane)
 
@@ -222,6 +225,7 @@ def test_neighbors_dense_rows_drain_the_buffer():
     n = 4000
     p = np.zeros((n, 4), np.float32)
     p[:, :3] = rng.uniform(0, 1, (n, 3)) * np.array([L, L, 6.0]) + np.array([0, 0, 10.0])
+    p = synth.band_clean(p, (L, L, L), 5.5)
     p = p[oracle.hilbert_sort(p, (L, L, L), 10)[0]]
     for lane in (False, True):
         _check_list(p, (L, L, L), 5.0, 0.5, 512, method="brute", lane=lane)
