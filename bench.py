@@ -152,8 +152,7 @@ class Step:
         # features live in the sorted index space (produced there by the model)
         self.feat = torch.randn((n, F), generator=g, device=device, dtype=torch.float32)
         self.out = torch.empty((n, F), dtype=torch.float32, device=device)
-        self.flags = (0 if pad_fill else tess.TESS_NO_PAD_FILL) | {"default": 0, "lane": tess.TESS_LANE_SEARCH,
-                                                                    "tile": tess.TESS_TILE_SEARCH}[search]
+        self.flags = (0 if pad_fill else tess.TESS_NO_PAD_FILL) | tess.SEARCH_FLAGS[search]
         self.sort_fn = tess.tess_hilbert_sort if curve == "hilbert" else tess.tess_morton_sort
         # the next frame of the trajectory, in the sorted order of frame 0
         t1 = next(iter(s.trajectory(1, condition=False)))[1]
@@ -740,7 +739,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["tess", "reference"], default="tess")
     ap.add_argument("--config", type=int, default=WORKLOAD_CFG)
     ap.add_argument("--no-pad-fill", action="store_true")
-    ap.add_argument("--search", choices=["default", "tile", "lane"], default="default",
+    ap.add_argument("--search", choices=["default", "tile", "lane", "lane2"], default="default",
                     help="pair search kernel (default: the library's choice)")
     ap.add_argument("--curve", choices=["hilbert", "morton"], default="hilbert",
                     help="space-filling curve of the sort (morton: the comparison curve)")

@@ -68,6 +68,7 @@ typedef struct {
 #define TESS_NO_PAD_FILL    1   /* leave slots >= min(count, max_neighbors) unwritten */
 #define TESS_LANE_SEARCH    2   /* use the per-lane stencil search */
 #define TESS_TILE_SEARCH    4   /* use the warp tile search (accept per 32-candidate block) */
+#define TESS_LANE2_SEARCH   8   /* use the per-lane stencil search with two atoms per lane */
 
 /* Human-readable name of a status code (static string). */
 const char* tess_status_string(tess_status s);
@@ -205,10 +206,11 @@ tess_status tess_hilbert_sort_static(const float* pos, int n, tess_box box, int 
  *   pos            [n,4] float (x, y, z, ignored), 16-byte aligned
  *   rc, skin       cutoff and skin (rc > 0, skin >= 0); rs = rc + skin in fp32
  *   max_neighbors  row capacity cap >= 1
- *   flags          0, or'ed TESS_NO_PAD_FILL and one of TESS_LANE_SEARCH,
- *                  TESS_TILE_SEARCH (two search kernels: the same lists in
- *                  another order within rows; 0 picks the library's default,
- *                  and boxes shorter than 2 rs + 2e-3 always take the tile
+ *   flags          0, or'ed TESS_NO_PAD_FILL and at most one of
+ *                  TESS_LANE2_SEARCH, TESS_LANE_SEARCH, TESS_TILE_SEARCH
+ *                  (three search kernels: the same lists in other orders
+ *                  within rows; none named picks the library's default, and
+ *                  boxes shorter than 2 rs + 2e-3 always take the tile
  *                  search)
  *   ws, ws_bytes   scratch of at least tess_build_neighbors_workspace(...)
  *   nbr            [n, cap] int32 out: row i in nbr[i*cap .. i*cap+cap);

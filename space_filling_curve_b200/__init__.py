@@ -34,7 +34,7 @@ __all__ = [
     "tess_skin_check", "tess_edge_aggregate", "tess_stage_timing", "tess_stage_times",
     "hilbert_sort", "build_neighbors", "skin_check", "edge_aggregate",
     "tess_edge_aggregate_backward", "edge_aggregate_backward",
-    "TESS_DEV_OVERFLOW", "TESS_DEV_BAD_INPUT", "TESS_DEV_TIMEOUT", "TESS_NO_PAD_FILL", "TESS_LANE_SEARCH", "TESS_TILE_SEARCH", "STAGES",
+    "TESS_DEV_OVERFLOW", "TESS_DEV_BAD_INPUT", "TESS_DEV_TIMEOUT", "TESS_NO_PAD_FILL", "TESS_LANE_SEARCH", "TESS_TILE_SEARCH", "TESS_LANE2_SEARCH", "STAGES",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -48,6 +48,8 @@ TESS_DEV_TIMEOUT = 4
 TESS_NO_PAD_FILL = 1
 TESS_LANE_SEARCH = 2
 TESS_TILE_SEARCH = 4
+TESS_LANE2_SEARCH = 8
+SEARCH_FLAGS = {"default": 0, "lane": TESS_LANE_SEARCH, "tile": TESS_TILE_SEARCH, "lane2": TESS_LANE2_SEARCH}
 STAGES = ("hilbert_keys", "key_sort", "cell_binning", "pair_search", "skin_check", "edge_aggregate", "edge_backward",
           "resort", "min_pair")
 _STATUS = {0: "ok", 1: "invalid argument", 2: "box too small", 3: "workspace too small", 4: "CUDA launch error",
@@ -374,7 +376,7 @@ def build_neighbors(pos4, box, rc: float, skin: float, max_neighbors: int, *, pa
     nbr = torch.empty((n, max_neighbors), dtype=torch.int32, device=dev) if nbr is None else nbr
     counts = torch.empty(n, dtype=torch.int32, device=dev) if counts is None else counts
     overflow = torch.empty(1, dtype=torch.int32, device=dev) if overflow is None else overflow
-    flags = (0 if pad_fill else TESS_NO_PAD_FILL) | {"default": 0, "lane": TESS_LANE_SEARCH, "tile": TESS_TILE_SEARCH}[search]
+    flags = (0 if pad_fill else TESS_NO_PAD_FILL) | SEARCH_FLAGS[search]
     code = tess_build_neighbors(_ptr(pos4), n, box, float(rc), float(skin), int(max_neighbors), flags, _ptr(ws),
                                 ws.numel() * ws.element_size(), _ptr(nbr), _ptr(counts), _ptr(overflow),
                                 _stream(stream))

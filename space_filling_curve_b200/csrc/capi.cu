@@ -128,8 +128,9 @@ const char* tess_status_string(tess_status s) {
 }
 
 const char* tess_version(void) {
-    return TESS_DEFAULT_LANE ? "tess-b200 0.2 (sm_100a; default pair search: per-lane)"
-                             : "tess-b200 0.2 (sm_100a; default pair search: tile)";
+    return TESS_DEFAULT_SEARCH == TESS_LANE2_SEARCH ? "tess-b200 0.3 (sm_100a; default pair search: two atoms per lane)"
+           : TESS_DEFAULT_SEARCH == TESS_LANE_SEARCH ? "tess-b200 0.3 (sm_100a; default pair search: per-lane)"
+                                                     : "tess-b200 0.3 (sm_100a; default pair search: tile)";
 }
 
 long long tess_kernel_launch_count(void) { return g_launches.load(); }

@@ -9,11 +9,11 @@
 
 #include "tess.h"
 
-// The pair search that tess_build_neighbors runs when its flags name neither
-// (1: per-lane stencil, 0: warp tile), the faster one on the 10.24M-atom salt
-// solution as last measured.
-#ifndef TESS_DEFAULT_LANE
-#define TESS_DEFAULT_LANE 1
+// The pair search that tess_build_neighbors runs when its flags name none
+// (TESS_LANE2_SEARCH, TESS_LANE_SEARCH or TESS_TILE_SEARCH): the fastest on
+// the 10.24M-atom salt solution as last measured.
+#ifndef TESS_DEFAULT_SEARCH
+#define TESS_DEFAULT_SEARCH TESS_LANE2_SEARCH
 #endif
 
 namespace tess {

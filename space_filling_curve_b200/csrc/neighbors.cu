@@ -21,9 +21,12 @@
 //      packed f32x2), 32 candidates per accept mask, and turns the set bits
 //      into indices that leave for its row in aligned 32-byte groups.
 // pair_search_lane_kernel (TESS_LANE_SEARCH) walks a stencil of cell rows
-// per lane instead; it gives the same lists in another order.  Which of the
-// two runs when the caller asks for neither is TESS_DEFAULT_LANE.
+// per lane instead, and pair_search_duo_kernel (TESS_LANE2_SEARCH) does so
+// with two atoms per lane over a record layout of the cell order; all three
+// give the same lists (in different orders).  Which one runs when the caller
+// names none is TESS_DEFAULT_SEARCH.
 #include <climits>
+#include <type_traits>
 
 #include "common.cuh"
 #include "scan.cuh"
@@ -107,12 +110,12 @@ __global__ void cell_count_kernel(const float4* __restrict__ pos, int n, int3 nc
 }
 
 __global__ void cell_scatter_kernel(const int* __restrict__ cell_id, const int* __restrict__ cell_rank, int n,
-                                    const int* __restrict__ cell_start, int* __restrict__ slot_atom,
-                                    int32_t* status) {
+                                    long long nslots, const int* __restrict__ cell_start,
+                                    int* __restrict__ slot_atom, int32_t* status) {
     const int stride = gridDim.x * blockDim.x;
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
         const long long slot = (long long)cell_start[cell_id[i]] + cell_rank[i];
-        if (check_index(slot, n, status)) slot_atom[slot] = i;
+        if (check_index(slot, nslots, status)) slot_atom[slot] = i;
     }
 }
 
@@ -126,6 +129,16 @@ __device__ __forceinline__ void cswap(int& a, int& b) {
     b = hi;
 }
 
+// Batcher's odd-even merge network for 8 keys (19 comparators).
+__device__ __forceinline__ void sort8(int (&v)[8]) {
+    cswap(v[0], v[1]); cswap(v[2], v[3]); cswap(v[4], v[5]); cswap(v[6], v[7]);
+    cswap(v[0], v[2]); cswap(v[1], v[3]); cswap(v[4], v[6]); cswap(v[5], v[7]);
+    cswap(v[1], v[2]); cswap(v[5], v[6]);
+    cswap(v[0], v[4]); cswap(v[1], v[5]); cswap(v[2], v[6]); cswap(v[3], v[7]);
+    cswap(v[2], v[4]); cswap(v[3], v[5]);
+    cswap(v[1], v[2]); cswap(v[3], v[4]); cswap(v[5], v[6]);
+}
+
 __global__ void cell_order_kernel(const int* __restrict__ slot_atom, long long ncell,
                                   const int* __restrict__ cell_start, const float4* __restrict__ pos,
                                   float4* __restrict__ pos_cell) {
@@ -137,13 +150,7 @@ __global__ void cell_order_kernel(const int* __restrict__ slot_atom, long long n
             int v[8];
 #pragma unroll
             for (int k = 0; k < 8; ++k) v[k] = k < m ? slot_atom[b + k] : INT_MAX;
-            // Batcher's odd-even merge network for 8 (19 comparators)
-            cswap(v[0], v[1]); cswap(v[2], v[3]); cswap(v[4], v[5]); cswap(v[6], v[7]);
-            cswap(v[0], v[2]); cswap(v[1], v[3]); cswap(v[4], v[6]); cswap(v[5], v[7]);
-            cswap(v[1], v[2]); cswap(v[5], v[6]);
-            cswap(v[0], v[4]); cswap(v[1], v[5]); cswap(v[2], v[6]); cswap(v[3], v[7]);
-            cswap(v[2], v[4]); cswap(v[3], v[5]);
-            cswap(v[1], v[2]); cswap(v[3], v[4]); cswap(v[5], v[6]);
+            sort8(v);
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 if (k < m) {
@@ -163,19 +170,132 @@ __global__ void cell_order_kernel(const int* __restrict__ slot_atom, long long n
     }
 }
 
+// Two-slot records for the two-atoms-per-lane search: slots 2m and 2m + 1
+// of the cell order in one 32-byte record, coordinates and indices paired so
+// that one 256-bit load yields (x0 x1), (y0 y1), (z0 z1) as packed f32x2
+// operands.  In this layout every cell row starts at an even slot: a row
+// holding an odd number of atoms ends with one pad slot (index -1, NaN
+// coordinates), which fails every distance test.
+struct alignas(32) SlotPair {
+    float x[2], y[2], z[2];
+    int i[2];
+};
+
+// One warp per cell row: the row's atom count; an odd count gets its pad
+// slot counted in the row's last cell, so the scan of the counts starts every
+// row at an even slot.  rowpad[r] = 1 marks such a row.
+__global__ void row_pad_kernel(int* __restrict__ cnt, int ncx, long long nrows, int* __restrict__ rowpad) {
+    const int lane = threadIdx.x & 31;
+    const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < nrows; r += warps) {
+        const int* row = cnt + r * ncx;
+        int sum = 0;
+        for (int x = lane; x < ncx; x += 32) sum += row[x];
+        sum = (int)__reduce_add_sync(FULL, (unsigned)sum);
+        if (lane == 0) {
+            rowpad[r] = sum & 1;
+            if (sum & 1) cnt[r * ncx + ncx - 1] += 1;
+        }
+    }
+}
+
+__device__ __forceinline__ void put_slot(SlotPair* pairs, int s, float x, float y, float z, int i) {
+    float* f = reinterpret_cast<float*>(pairs + (s >> 1)) + (s & 1);
+    f[0] = x;
+    f[2] = y;
+    f[4] = z;
+    reinterpret_cast<int*>(f)[6] = i;
+}
+
+// Both slots of record r in one 32-byte store (a plain store: the search
+// reads the records next).
+__device__ __forceinline__ void put_record(SlotPair* pairs, int r, float4 p0, int i0, float4 p1, int i1) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(pairs + r),
+                 "r"(__float_as_int(p0.x)), "r"(__float_as_int(p1.x)), "r"(__float_as_int(p0.y)),
+                 "r"(__float_as_int(p1.y)), "r"(__float_as_int(p0.z)), "r"(__float_as_int(p1.z)), "r"(i0), "r"(i1)
+                 : "memory");
+}
+
+// cell_order for the record layout: the same order inside each cell, the
+// positions written as two-slot records (a record whose two slots both
+// belong to the cell, its pad slot included, in one store; a record shared
+// with a neighboring cell half by half), and the pad slot of an odd row
+// (the last slot of the row's last cell) filled.
+__global__ void cell_order_pairs_kernel(const int* __restrict__ slot_atom, long long ncell, int ncx,
+                                        const int* __restrict__ cell_start, const int* __restrict__ rowpad,
+                                        const float4* __restrict__ pos, SlotPair* __restrict__ pairs) {
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    const float nan = __int_as_float(0x7fc00000);
+    const float4 pnan = make_float4(nan, nan, nan, nan);
+    for (long long c = (long long)blockIdx.x * blockDim.x + threadIdx.x; c < ncell; c += stride) {
+        const int b = cell_start[c];
+        int e = cell_start[c + 1];
+        const long long r = c / ncx;
+        const bool pad = c - r * ncx == ncx - 1 && rowpad[r];
+        if (pad) --e;                      // slot e is the row's pad
+        const int m = e - b;
+        if (m <= 0) {
+            if (pad) put_slot(pairs, e, nan, nan, nan, -1);
+            continue;
+        }
+        if (m <= 8) {
+            int v[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[k] = k < m ? slot_atom[b + k] : INT_MAX;
+            sort8(v);
+            // slots b .. e-1 hold v[0 .. m-1], slot e the pad when there is one
+            // (the pad is always the second half of its record)
+            auto emit = [&](auto first) {
+                constexpr int K0 = decltype(first)::value;
+                if (K0 == 1) {             // slot b: the second half of a record shared with the cell before
+                    const float4 p = pos[v[0]];
+                    put_slot(pairs, b, p.x, p.y, p.z, v[0]);
+                }
+#pragma unroll
+                for (int kk = K0; kk < 8; kk += 2) {
+                    if (kk + 1 < m) {
+                        put_record(pairs, (b + kk) >> 1, pos[v[kk]], v[kk], pos[v[kk + 1]], v[kk + 1]);
+                    } else if (kk + 1 == m) {
+                        const float4 p = pos[v[kk]];
+                        if (pad) put_record(pairs, (b + kk) >> 1, p, v[kk], pnan, -1);
+                        else put_slot(pairs, b + kk, p.x, p.y, p.z, v[kk]);   // shared with the cell after
+                    }
+                }
+            };
+            if (b & 1) emit(std::integral_constant<int, 1>{});
+            else emit(std::integral_constant<int, 0>{});
+        } else {
+            for (int s = b; s < e; ++s) {
+                const int i = slot_atom[s];
+                int rk = 0;
+                for (int t = b; t < e; ++t) rk += slot_atom[t] < i;
+                const float4 p = pos[i];
+                put_slot(pairs, b + rk, p.x, p.y, p.z, i);
+            }
+            if (pad) put_slot(pairs, e, nan, nan, nan, -1);
+        }
+    }
+}
+
 // ---------------------------------------------------------------- pair search
 
 constexpr int PS_BUF = 32;           // per-lane staging of accepted indices, per-lane search
 constexpr int PS_GROUP = 8;          // accepted indices leave in aligned groups of 8 (32 bytes)
 
+struct SlotPair;
+
 struct PairArgs {
     const float4* pos;
     const float4* pos_cell;
+    const SlotPair* pairs;   // two-slot records (the two-atoms-per-lane search)
+    const int* nslots;       // slots of the record layout, pads included (device)
     const int* cell_start;
     int n;
     int cap;
     int pad_fill;
     int vec_rows;      // rows can take 16-byte stores (cap % 4 == 0, 16-byte aligned nbr)
+    int vec8;          // rows can take 32-byte stores (cap % 8 == 0, 32-byte aligned nbr)
+    int row_tiles;     // tiles of 32 records per cell row, on average (at least 1)
     int3 nc;
     float3 inv_w;
     float3 L;
@@ -896,6 +1016,319 @@ __global__ __launch_bounds__(PL_WARPS * 32, 6) void pair_search_lane_kernel(Pair
     }
 }
 
+// ------------------------------------------------ two atoms per lane
+//
+// pair_search_duo_kernel (TESS_LANE2_SEARCH): the per-lane stencil walk with
+// two atoms per lane, over the two-slot records.  A warp takes 32
+// consecutive records (64 slots) of the cell order; lane l owns the atoms in
+// slots 2l and 2l + 1 of them, which lie in one cell row (every row starts at
+// an even slot).  For each of the 5 x 5 cell rows around that row the lane
+// walks the union of its two atoms' x windows (each clipped to that atom's
+// chord at the row's distance) record by record: one 32-byte load feeds four
+// distance tests -- two candidates against two atoms -- in packed f32x2
+// arithmetic.  Where the two windows together would span more than a row
+// (two atoms far apart in a sparse row) the lane walks them one after the
+// other instead.  Accepted indices are staged per atom in shared memory and
+// leave for the atom's row in aligned 32-byte groups.
+
+#ifndef TESS_PD_WARPS
+#define TESS_PD_WARPS 4
+#endif
+#ifndef TESS_PD_BUF
+#define TESS_PD_BUF 24
+#endif
+#ifndef TESS_PD_GROUP
+#define TESS_PD_GROUP 1
+#endif
+constexpr int PD_WARPS = TESS_PD_WARPS;
+constexpr int PD_BUF = TESS_PD_BUF;        // staged indices per atom (two buffers per lane)
+#ifndef TESS_PD_CHUNK
+#define TESS_PD_CHUNK 2
+#endif
+constexpr int PD_CHUNK = TESS_PD_CHUNK;    // records per lane between buffer votes
+
+typedef unsigned long long u64;
+
+// The record at a (32-byte aligned) into four packed pairs when p; the
+// registers keep their values otherwise.
+__device__ __forceinline__ void ld_pair_if(bool p, const SlotPair* a, u64& x, u64& y, u64& z, u64& j) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %5, 0;\n\t"
+        "@p ld.global.nc.v4.b64 {%0, %1, %2, %3}, [%4];\n\t}"
+        : "+l"(x), "+l"(y), "+l"(z), "+l"(j)
+        : "l"(a), "r"((int)p));
+}
+
+// Four tests of one record (slots k, k + 1) against atoms a and b: element 0
+// counts when beg <= k < end, element 1 when k + 1 < end; with SELF the
+// lane's own record (k == own) skips a against itself (element 0) and b
+// against itself (element 1).  Each accepted index is appended to its atom's
+// staging column (wa, wb: shared addresses, 128-byte steps).
+// Four tests of one record against atoms a and b (packed pairs qa*, qb*),
+// counted when `live`; with SELF the lane's own record (k == own) skips a
+// against itself (element 0) and b against itself (element 1).  Each accepted
+// index is appended to its atom's staging column (wa, wb: shared addresses,
+// 128-byte steps; the store happens either way and a rejected index is
+// overwritten by the next).
+#define TESS_DUO_BODY(SA, SB)                                \
+    "{\n\t.reg .b64 dx, dy, dz, r;\n\t.reg .f32 r0, r1;\n\t"  \
+    ".reg .b32 j0, j1;\n\t.reg .pred v, sa, sb, p;\n\t"      \
+    "setp.ne.b32 v, %13, 0;\n\t"                              \
+    SA SB                                                     \
+    "mov.b64 {j0, j1}, %5;\n\t"                               \
+    "sub.rn.f32x2 dx, %2, %6;\n\t"                            \
+    "sub.rn.f32x2 dy, %3, %7;\n\t"                            \
+    "sub.rn.f32x2 dz, %4, %8;\n\t"                            \
+    "mul.rn.f32x2 r, dx, dx;\n\t"                             \
+    "fma.rn.f32x2 r, dy, dy, r;\n\t"                          \
+    "fma.rn.f32x2 r, dz, dz, r;\n\t"                          \
+    "mov.b64 {r0, r1}, r;\n\t"                                \
+    "setp.lt.and.f32 p, r0, %12, sa;\n\t"                     \
+    "st.shared.b32 [%0], j0;\n\t"                             \
+    "@p add.u32 %0, %0, 128;\n\t"                             \
+    "setp.lt.and.f32 p, r1, %12, v;\n\t"                      \
+    "st.shared.b32 [%0], j1;\n\t"                             \
+    "@p add.u32 %0, %0, 128;\n\t"                             \
+    "sub.rn.f32x2 dx, %2, %9;\n\t"                            \
+    "sub.rn.f32x2 dy, %3, %10;\n\t"                           \
+    "sub.rn.f32x2 dz, %4, %11;\n\t"                           \
+    "mul.rn.f32x2 r, dx, dx;\n\t"                             \
+    "fma.rn.f32x2 r, dy, dy, r;\n\t"                          \
+    "fma.rn.f32x2 r, dz, dz, r;\n\t"                          \
+    "mov.b64 {r0, r1}, r;\n\t"                                \
+    "setp.lt.and.f32 p, r0, %12, v;\n\t"                      \
+    "st.shared.b32 [%1], j0;\n\t"                             \
+    "@p add.u32 %1, %1, 128;\n\t"                             \
+    "setp.lt.and.f32 p, r1, %12, sb;\n\t"                     \
+    "st.shared.b32 [%1], j1;\n\t"                             \
+    "@p add.u32 %1, %1, 128;\n\t}"
+
+template <bool SELF>
+__device__ __forceinline__ void duo_test(unsigned& wa, unsigned& wb, u64 x, u64 y, u64 z, u64 j, u64 qax,
+                                         u64 qay, u64 qaz, u64 qbx, u64 qby, u64 qbz, float rs2, bool live, int k,
+                                         int own) {
+    if (SELF) {
+        asm volatile(TESS_DUO_BODY("setp.ne.and.s32 sa, %14, %15, v;\n\t", "setp.ne.and.s32 sb, %14, %15, v;\n\t")
+                     : "+r"(wa), "+r"(wb)
+                     : "l"(x), "l"(y), "l"(z), "l"(j), "l"(qax), "l"(qay), "l"(qaz), "l"(qbx), "l"(qby), "l"(qbz),
+                       "f"(rs2), "r"((int)live), "r"(k), "r"(own)
+                     : "memory");
+    } else {
+        asm volatile(TESS_DUO_BODY("mov.pred sa, v;\n\t", "mov.pred sb, v;\n\t")
+                     : "+r"(wa), "+r"(wb)
+                     : "l"(x), "l"(y), "l"(z), "l"(j), "l"(qax), "l"(qay), "l"(qaz), "l"(qbx), "l"(qby), "l"(qbz),
+                       "f"(rs2), "r"((int)live), "r"(k), "r"(own)
+                     : "memory");
+    }
+}
+#undef TESS_DUO_BODY
+
+#ifndef TESS_PD_MINB
+#define TESS_PD_MINB 6
+#endif
+
+__global__ __launch_bounds__(PD_WARPS * 32, TESS_PD_MINB) void pair_search_duo_kernel(PairArgs A) {
+    __shared__ int s_buf[PD_WARPS][2][32 * PD_BUF];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int* const bufa = &s_buf[warp][0][lane];
+    int* const bufb = &s_buf[warp][1][lane];
+    const unsigned basea = (unsigned)__cvta_generic_to_shared(bufa);
+    const unsigned baseb = (unsigned)__cvta_generic_to_shared(bufb);
+    const int cap = A.cap, ncx = A.nc.x;
+    const int nrec = *A.nslots >> 1;
+    const long long ntiles = ((long long)nrec + 31) / 32;
+    const float wy = (float)A.L.y / (float)A.nc.y, wz = (float)A.L.z / (float)A.nc.z;
+    const float reach2 = A.reach * A.reach;
+    const float nan = __int_as_float(0x7fc00000);
+    const unsigned vote_at = (unsigned)(PD_BUF - 2 * PD_CHUNK) * 128u;
+
+    // full groups of 8 staged indices to the row, the remainder moved to the
+    // front of the column
+    auto drain = [&](int* buf, unsigned base, unsigned& w, int& done, int* row) {
+        const int pend = (int)((w - base) >> 7);
+        const int groups = pend >> 3;
+        for (int g = 0; g < groups; ++g) {
+            const int* src = buf + g * 256;
+            if (A.vec8 && done + 8 <= cap) {
+                st_global_v8(row + done, src[0], src[32], src[64], src[96], src[128], src[160], src[192], src[224]);
+            } else {
+                for (int e = 0; e < 8; ++e)
+                    if (done + e < cap) row[done + e] = src[e * 32];
+            }
+            done += 8;
+        }
+        const int rest = pend - groups * 8;
+        if (groups > 0)
+            for (int e = 0; e < rest; ++e) buf[e * 32] = buf[(groups * 8 + e) * 32];
+        w = base + 128u * (unsigned)rest;
+    };
+    // the last staged indices (a group completed with pads where the row is
+    // pad-filled and has room), the count, and the pads
+    auto finish = [&](int* buf, unsigned base, unsigned w, int done, int* row, bool valid, int idx) {
+        drain(buf, base, w, done, row);
+        const int pend = (int)((w - base) >> 7);
+        int filled;
+        if (A.pad_fill && A.vec8 && pend > 0 && done + 8 <= cap) {
+            int v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = e < pend ? buf[e * 32] : -1;
+            st_global_v8(row + done, v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+            filled = done + 8;
+        } else {
+            for (int e = 0; e < pend; ++e)
+                if (done + e < cap) row[done + e] = buf[e * 32];
+            filled = min(done + pend, cap);
+        }
+        const int cnt = done + pend;
+        if (valid) {
+            A.counts[idx] = cnt;
+            if (A.pad_fill) {
+                int e = filled;
+                if (A.vec8) {
+                    for (; e < cap && (e & 7); ++e) row[e] = -1;
+                    for (; e + 8 <= cap; e += 8) st_global_v8(row + e, -1, -1, -1, -1, -1, -1, -1, -1);
+                }
+                for (; e < cap; ++e) row[e] = -1;
+            }
+        }
+        return cnt;
+    };
+
+    u64 cx[PD_CHUNK], cy2[PD_CHUNK], cz2[PD_CHUNK], cj[PD_CHUNK];
+#pragma unroll
+    for (int u = 0; u < PD_CHUNK; ++u) cx[u] = cy2[u] = cz2[u] = cj[u] = 0ull;
+
+    for (long long pos = (long long)blockIdx.x * PD_WARPS + warp; pos < ntiles;
+         pos += (long long)gridDim.x * PD_WARPS) {
+        // the warps of a block take tiles about one cell row apart (row_tiles
+        // tiles per row on average): the same x range of adjacent rows, whose
+        // stencils share most of their cell rows in L1
+        long long tile = pos;
+        if (TESS_PD_GROUP) {
+            const long long span = (long long)PD_WARPS * A.row_tiles, g = pos / span;
+            if ((g + 1) * span <= ntiles) {
+                const long long r = pos - g * span;
+                tile = g * span + (r % PD_WARPS) * A.row_tiles + r / PD_WARPS;
+            }
+        }
+        const int m = (int)(tile * 32) + lane;
+        u64 ox = 0ull, oy = 0ull, oz = 0ull, oj = ~0ull;
+        ld_pair_if(m < nrec, A.pairs + m, ox, oy, oz, oj);
+        const int ia = (int)(unsigned)oj, ib = (int)(oj >> 32);
+        const bool va = ia >= 0, vb = ib >= 0;
+        // test coordinates as given (NaN for a pad); the windows use them too,
+        // with x clamped into the box (y and z only enter through distances
+        // to cell rows, where a NaN or distant value just empties the row)
+        const float3 pa = make_float3(__uint_as_float((unsigned)ox), __uint_as_float((unsigned)oy),
+                                      __uint_as_float((unsigned)oz));
+        const float3 pb = make_float3(__uint_as_float((unsigned)(ox >> 32)), __uint_as_float((unsigned)(oy >> 32)),
+                                      __uint_as_float((unsigned)(oz >> 32)));
+        const float xa = fminf(fmaxf(pa.x, 0.f), A.L.x), xb = fminf(fmaxf(pb.x, 0.f), A.L.x);
+        int* const rowa = A.nbr + (size_t)(va ? ia : 0) * cap;
+        int* const rowb = A.nbr + (size_t)(vb ? ib : 0) * cap;
+        const int cyc = cell_coord(pa.y, A.inv_w.y, A.nc.y);
+        const int czc = cell_coord(pa.z, A.inv_w.z, A.nc.z);
+        const int own = 2 * m;
+        // a window reaches at most 3 cells either side of its atom's cell; two
+        // atoms whose windows together could exceed nc.x + 1 cells (far apart
+        // in a sparse row) are walked one after the other, b in a second pass
+        const bool far = vb && cell_coord(xb, A.inv_w.x, ncx) - cell_coord(xa, A.inv_w.x, ncx) > ncx - 6;
+        const int passes = __any_sync(FULL, far) ? 2 : 1;
+
+        int donea = 0, doneb = 0;
+        unsigned wa = basea, wb = baseb;
+
+        for (int pass = 0; pass < passes; ++pass) {
+            const bool usea = va && pass == 0, useb = vb && (pass == 0) != far;
+            for (int dz = -CELL_DIV; dz <= CELL_DIV; ++dz) {
+                int wz_i = czc + dz, kz = 0;
+                while (wz_i < 0) { wz_i += A.nc.z; --kz; }
+                while (wz_i >= A.nc.z) { wz_i -= A.nc.z; ++kz; }
+                const float zlo = (float)(czc + dz) * wz;
+                const float dza = fmaxf(fmaxf(zlo - pa.z, pa.z - (zlo + wz)), 0.f);
+                const float dzb = fmaxf(fmaxf(zlo - pb.z, pb.z - (zlo + wz)), 0.f);
+                const u64 qaz = pk2(pa.z - (float)kz * A.L.z), qbz = pk2(pb.z - (float)kz * A.L.z);
+                for (int dy = -CELL_DIV; dy <= CELL_DIV; ++dy) {
+                    int wy_i = cyc + dy, ky = 0;
+                    while (wy_i < 0) { wy_i += A.nc.y; --ky; }
+                    while (wy_i >= A.nc.y) { wy_i -= A.nc.y; ++ky; }
+                    const float ylo = (float)(cyc + dy) * wy;
+                    const float dya = fmaxf(fmaxf(ylo - pa.y, pa.y - (ylo + wy)), 0.f);
+                    const float dyb = fmaxf(fmaxf(ylo - pb.y, pb.y - (ylo + wy)), 0.f);
+                    const float ch2a = reach2 - dya * dya - dza * dza;
+                    const float ch2b = reach2 - dyb * dyb - dzb * dzb;
+                    const u64 qay = pk2(pa.y - (float)ky * A.L.y), qby = pk2(pb.y - (float)ky * A.L.y);
+                    const bool ina = usea && ch2a > 0.f, inb = useb && ch2b > 0.f;
+                    // the union of the two x windows, in unwrapped cells
+                    // (chords approximate, widened)
+                    int lo = INT_MAX, hi = INT_MIN;
+                    if (ina) {
+                        const float ch = fmaf(ch2a * rsqrtf(ch2a), 1.0001f, 1e-4f);
+                        lo = (int)floorf((xa - ch) * A.inv_w.x);
+                        hi = (int)floorf((xa + ch) * A.inv_w.x);
+                    }
+                    if (inb) {
+                        const float ch = fmaf(ch2b * rsqrtf(ch2b), 1.0001f, 1e-4f);
+                        lo = min(lo, (int)floorf((xb - ch) * A.inv_w.x));
+                        hi = max(hi, (int)floorf((xb + ch) * A.inv_w.x));
+                    }
+                    // as up to two ranges of slots; the second (wrapped) one
+                    // has image shift kx + 1.  Slots just outside a range (a
+                    // record's other half) lie in the same cell row beyond the
+                    // window, so the distance test rejects them.
+                    int B0 = 0, E0 = 0, B1 = 0, E1 = 0, kx = 0;
+                    if (ina || inb) {
+                        const int rowbase = (wz_i * A.nc.y + wy_i) * ncx;
+                        while (lo < 0) { lo += ncx; hi += ncx; --kx; }
+                        while (lo >= ncx) { lo -= ncx; hi -= ncx; ++kx; }
+                        B0 = A.cell_start[rowbase + lo];
+                        E0 = A.cell_start[rowbase + min(hi, ncx - 1) + 1];
+                        if (hi >= ncx) {
+                            B1 = A.cell_start[rowbase];
+                            E1 = A.cell_start[rowbase + min(hi - ncx, ncx - 1) + 1];
+                        }
+                    }
+
+                    auto run = [&](auto self_tag) {
+                        constexpr bool SELF = decltype(self_tag)::value;
+#pragma unroll
+                        for (int pc = 0; pc < 2; ++pc) {
+                            const int beg = pc ? B1 : B0, end = pc ? E1 : E0;
+                            const int kb = beg & ~1;
+                            const int np = end > beg ? (end - kb + 1) >> 1 : 0;
+                            const int maxp = (int)__reduce_max_sync(FULL, (unsigned)np);
+                            if (maxp == 0) continue;
+                            const float sx = (float)(kx + pc) * A.L.x;
+                            const u64 qax = pk2(usea ? pa.x - sx : nan), qbx = pk2(useb ? pb.x - sx : nan);
+                            const SlotPair* src = A.pairs + (kb >> 1);
+                            for (int t0 = 0; t0 < maxp; t0 += PD_CHUNK) {
+                                if (__any_sync(FULL, max(wa - basea, wb - baseb) > vote_at)) {
+                                    drain(bufa, basea, wa, donea, rowa);
+                                    drain(bufb, baseb, wb, doneb, rowb);
+                                }
+#pragma unroll
+                                for (int u = 0; u < PD_CHUNK; ++u)
+                                    ld_pair_if(t0 + u < np, src + t0 + u, cx[u], cy2[u], cz2[u], cj[u]);
+#pragma unroll
+                                for (int u = 0; u < PD_CHUNK; ++u)
+                                    duo_test<SELF>(wa, wb, cx[u], cy2[u], cz2[u], cj[u], qax, qay, qaz, qbx, qby,
+                                                   qbz, A.rs2, t0 + u < np, kb + 2 * (t0 + u), own);
+                            }
+                        }
+                    };
+                    if (dz == 0 && dy == 0) run(std::true_type{});
+                    else run(std::false_type{});
+                }
+            }
+        }
+        const int cnta = finish(bufa, basea, wa, donea, rowa, va, ia);
+        const int cntb = finish(bufb, baseb, wb, doneb, rowb, vb, ib);
+        const unsigned ov = __ballot_sync(FULL, (va && cnta > cap) || (vb && cntb > cap));
+        if (ov && lane == 0) atomicOr(A.status, TESS_DEV_OVERFLOW);
+        __syncwarp();
+    }
+}
+
 // ---------------------------------------------------------------- host
 
 struct NbrLayout {
@@ -905,7 +1338,9 @@ struct NbrLayout {
     int* cell_start;
     int* sums;
     int* slot_atom;
-    float4* pos_cell;
+    int* rowpad;
+    float4* pos_cell;      // cell order as float4, or (same storage) as two-slot records
+    SlotPair* pairs;
     int32_t* status;
     size_t total;
 };
@@ -914,13 +1349,17 @@ static NbrLayout nbr_layout(void* ws, int n, const Grid& g) {
     Carve c(ws);
     NbrLayout L{};
     const long long m = g.ncell;
+    const long long nrows = (long long)g.nc[1] * g.nc[2];
+    const long long slots = (long long)n + nrows;          // the record layout's pads included
     L.cell_id = c.take<int>((size_t)n);
     L.cell_rank = c.take<int>((size_t)n);
     L.cnt = c.take<int>((size_t)m);
     L.cell_start = c.take<int>((size_t)m + 1);
     L.sums = c.take<int>((size_t)((m + SCAN_TILE - 1) / SCAN_TILE) + 1);
-    L.slot_atom = c.take<int>((size_t)n);
-    L.pos_cell = c.take<float4>((size_t)n);
+    L.slot_atom = c.take<int>((size_t)slots);
+    L.rowpad = c.take<int>((size_t)nrows);
+    L.pairs = c.take<SlotPair>((size_t)((slots + 1) / 2));
+    L.pos_cell = reinterpret_cast<float4*>(L.pairs);
     L.status = c.take<int32_t>(1);
     L.total = align_up(c.off, 256);
     return L;
@@ -940,8 +1379,8 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
     if (n <= 0 || !pos || !ws || !nbr || !counts || !overflow || cap < 1) return TESS_ERR_INVALID_ARG;
     if (!box_ok(box) || !(rc > 0.f) || !(skin >= 0.f) || !std::isfinite(rc) || !std::isfinite(skin))
         return TESS_ERR_INVALID_ARG;
-    if ((flags & ~(TESS_NO_PAD_FILL | TESS_LANE_SEARCH | TESS_TILE_SEARCH)) != 0) return TESS_ERR_INVALID_ARG;
-    if ((flags & TESS_LANE_SEARCH) && (flags & TESS_TILE_SEARCH)) return TESS_ERR_INVALID_ARG;
+    const int kinds = flags & (TESS_LANE_SEARCH | TESS_TILE_SEARCH | TESS_LANE2_SEARCH);
+    if ((flags & ~(TESS_NO_PAD_FILL | kinds)) != 0 || (kinds & (kinds - 1)) != 0) return TESS_ERR_INVALID_ARG;
     if (!aligned(pos, 16) || !aligned(ws, 256) || !aligned(nbr, 4) || !aligned(counts, 4)) return TESS_ERR_INVALID_ARG;
     const float rs = rc + skin;
     if (box.lx < 2.f * rs || box.ly < 2.f * rs || box.lz < 2.f * rs) return TESS_ERR_BOX_TOO_SMALL;
@@ -959,45 +1398,68 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
     const long long m = g.ncell;
     const long long scan_tiles = (m + SCAN_TILE - 1) / SCAN_TILE;
 
+    // which search: the per-lane kinds need every box length >= 2 reach (a
+    // window then wraps at most once); otherwise the tile search runs
+    const float lmax = std::max(box.lx, std::max(box.ly, box.lz));
+    const float reach = rs + 1e-3f + 4e-6f * lmax;
+    const bool lane_ok = box.lx >= 2.f * reach && box.ly >= 2.f * reach && box.lz >= 2.f * reach;
+    int kind = kinds ? kinds : TESS_DEFAULT_SEARCH;
+    if (kind != TESS_TILE_SEARCH && !lane_ok) kind = TESS_TILE_SEARCH;
+    const bool records = kind == TESS_LANE2_SEARCH;
+
     cudaMemsetAsync(overflow, 0, sizeof(int32_t), s);
     {
         StageScope sc(ST_CELLS, s);
         cudaMemsetAsync(L.cnt, 0, sizeof(int) * (size_t)m, s);
         const int blocks = (int)std::min<long long>(((long long)n + 255) / 256, (long long)sms * 16);
         cell_count_kernel<<<blocks, 256, 0, s>>>(pos4, n, nc, inv_w, Lb, L.cell_id, L.cell_rank, L.cnt, overflow);
+        const long long nrows = (long long)nc.y * nc.z;
+        if (records) {
+            const long long rb = std::min<long long>((nrows + 7) / 8, (long long)sms * 32);
+            row_pad_kernel<<<(unsigned)rb, 256, 0, s>>>(L.cnt, nc.x, nrows, L.rowpad);
+        }
         scan_reduce_kernel<<<(unsigned)scan_tiles, SCAN_THREADS, 0, s>>>(L.cnt, m, L.sums);
         scan_sums_kernel<<<1, SCAN_THREADS, 0, s>>>(L.sums, scan_tiles);
         scan_apply_kernel<<<(unsigned)scan_tiles, SCAN_THREADS, 0, s>>>(L.cnt, m, L.sums, L.cell_start);
-        cell_scatter_kernel<<<blocks, 256, 0, s>>>(L.cell_id, L.cell_rank, n, L.cell_start, L.slot_atom, overflow);
-        cell_order_kernel<<<(int)std::min<long long>((m + 255) / 256, (long long)sms * 16), 256, 0, s>>>(
-            L.slot_atom, m, L.cell_start, pos4, L.pos_cell);
-        count_launch(6);
+        cell_scatter_kernel<<<blocks, 256, 0, s>>>(L.cell_id, L.cell_rank, n, (long long)n + nrows, L.cell_start,
+                                                   L.slot_atom, overflow);
+        const int oblocks = (int)std::min<long long>((m + 255) / 256, (long long)sms * 16);
+        if (records)
+            cell_order_pairs_kernel<<<oblocks, 256, 0, s>>>(L.slot_atom, m, nc.x, L.cell_start, L.rowpad, pos4,
+                                                            L.pairs);
+        else
+            cell_order_kernel<<<oblocks, 256, 0, s>>>(L.slot_atom, m, L.cell_start, pos4, L.pos_cell);
+        count_launch(records ? 7 : 6);
     }
     {
         StageScope sc(ST_PAIRS, s);
         PairArgs A;
         A.pos = pos4;
         A.pos_cell = L.pos_cell;
+        A.pairs = L.pairs;
+        A.nslots = L.cell_start + m;
         A.cell_start = L.cell_start;
         A.n = n;
         A.cap = cap;
         A.pad_fill = (flags & TESS_NO_PAD_FILL) ? 0 : 1;
         A.vec_rows = (cap % 4 == 0 && aligned(nbr, 16)) ? 1 : 0;
+        A.vec8 = (cap % 8 == 0 && aligned(nbr, 32)) ? 1 : 0;
+        A.row_tiles = 1;
         A.nc = nc;
         A.inv_w = inv_w;
         A.L = Lb;
         A.rs2 = rs * rs;
-        const float lmax = std::max(box.lx, std::max(box.ly, box.lz));
-        A.reach = rs + 1e-3f + 4e-6f * lmax;
+        A.reach = reach;
         A.nbr = nbr;
         A.counts = counts;
         A.status = overflow;
         const long long ntiles = ((long long)n + 31) / 32;
-        // the per-lane search needs every box length >= 2 reach (a window
-        // then wraps at most once); otherwise the tile search handles it
-        const bool lane_ok = box.lx >= 2.f * A.reach && box.ly >= 2.f * A.reach && box.lz >= 2.f * A.reach;
-        const bool want_lane = (flags & TESS_LANE_SEARCH) || (!(flags & TESS_TILE_SEARCH) && TESS_DEFAULT_LANE);
-        if (want_lane && lane_ok) {
+        if (kind == TESS_LANE2_SEARCH) {
+            const long long recs = ((long long)n + (long long)nc.y * nc.z + 1) / 2;
+            A.row_tiles = (int)std::max<long long>(1, std::llround((double)n / ((double)nc.y * nc.z) / 64.0));
+            const long long blocks = ((recs + 31) / 32 + PD_WARPS - 1) / PD_WARPS;
+            pair_search_duo_kernel<<<(unsigned)std::min<long long>(blocks, 1LL << 30), PD_WARPS * 32, 0, s>>>(A);
+        } else if (kind == TESS_LANE_SEARCH) {
             const long long blocks = (ntiles + PL_WARPS - 1) / PL_WARPS;
             pair_search_lane_kernel<<<(unsigned)std::min<long long>(blocks, 1LL << 30), PL_WARPS * 32, 0, s>>>(A);
         } else {

@@ -63,8 +63,9 @@ def test_argument_errors_are_reported_before_any_launch(lib):
     assert tess.tess_build_neighbors(p, 10, (12.0, 30.0, 30.0), 6.0, 0.5, 16, 0, p, 1 << 30, p, p, p, null) == 2
     # workspace too small
     assert tess.tess_build_neighbors(p, 10, box, 6.0, 0.5, 16, 0, p, 16, p, p, p, null) == 3
-    # unknown flag
-    assert tess.tess_build_neighbors(p, 10, box, 6.0, 0.5, 16, 8, p, 1 << 30, p, p, p, null) == 1
+    # unknown flag, or two search kinds at once
+    for flags in (16, 64, 1 << 30, 2 | 4, 2 | 8, 4 | 8, 2 | 4 | 8):
+        assert tess.tess_build_neighbors(p, 10, box, 6.0, 0.5, 16, flags, p, 1 << 30, p, p, p, null) == 1
     assert tess.tess_skin_check(p, p, 10, box, -0.5, p, null, null) == 1
     assert tess.tess_edge_aggregate(p, 10, box, 6.0, p, p, 16, p, 0, p, null, null, null, null) == 1
     # backward: F not a multiple of 4, cap above 512, box below 2 rc

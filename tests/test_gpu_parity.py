@@ -14,6 +14,8 @@ from gpu_util import agg_error, agg_error_geom, canon_rows, canon_rows_gpu, geom
 pytestmark = pytest.mark.gpu
 
 AGG_TOL = 1e-5
+# the three pair-search kernels (same sets, rows in different orders)
+SEARCHES = ["tile", "lane", "lane2"]
 
 
 def _tess():
@@ -94,15 +96,15 @@ def test_sort_configs(cfg):
 # ------------------------------------------------------------------ neighbors
 
 
-def _gpu_list(pos4, box, rc, skin, cap, pad_fill=True, lane=False):
+def _gpu_list(pos4, box, rc, skin, cap, pad_fill=True, search="tile"):
     tess = _tess()
-    nbr, cnt, ov = tess.build_neighbors(_dev(pos4), box, rc, skin, cap, pad_fill=pad_fill, search="lane" if lane else "tile")
+    nbr, cnt, ov = tess.build_neighbors(_dev(pos4), box, rc, skin, cap, pad_fill=pad_fill, search=search)
     torch_cuda().cuda.synchronize()
     return nbr, cnt, int(ov.item())
 
 
-def _check_list(pos4, box, rc, skin, cap, pad_fill=True, method="cells", lane=False):
-    nbr_d, cnt_d, ov = _gpu_list(pos4, box, rc, skin, cap, pad_fill, lane)
+def _check_list(pos4, box, rc, skin, cap, pad_fill=True, method="cells", search="tile"):
+    nbr_d, cnt_d, ov = _gpu_list(pos4, box, rc, skin, cap, pad_fill, search)
     fn = oracle.neighbors_cells if method == "cells" else oracle.neighbors_brute
     onbr, ocnt, oov = fn(pos4, box, rc, skin, cap)
     cnt = cnt_d.cpu().numpy()
@@ -125,40 +127,56 @@ def _check_list(pos4, box, rc, skin, cap, pad_fill=True, method="cells", lane=Fa
     return nbr_d, cnt
 
 
-@pytest.mark.parametrize("lane", [False, True])
+@pytest.mark.parametrize("search", SEARCHES)
 @pytest.mark.parametrize("cfg", [1, 2])
-def test_neighbors_configs_sorted_order(cfg, lane):
+def test_neighbors_configs_sorted_order(cfg, search):
     s = synth.system(cfg)
     perm, _ = oracle.hilbert_sort(s.pos, s.box, 10)
     p4 = s.pos4()[perm]
-    _check_list(p4, s.box, s.rc, s.skin, s.cap, lane=lane)
+    _check_list(p4, s.box, s.rc, s.skin, s.cap, search=search)
 
 
-def test_neighbors_config3():
+@pytest.mark.parametrize("search", ["default", "lane2"])
+def test_neighbors_config3(search):
     s = synth.system(3)
     perm, _ = oracle.hilbert_sort(s.pos, s.box, 10)
-    _check_list(s.pos4()[perm], s.box, s.rc, s.skin, s.cap)
+    _check_list(s.pos4()[perm], s.box, s.rc, s.skin, s.cap, search=search)
 
 
-@pytest.mark.parametrize("lane", [False, True])
-def test_neighbors_unsorted_input_gives_the_same_sets(lane):
+@pytest.mark.parametrize("search", SEARCHES)
+@pytest.mark.parametrize("n,L", [(40, 60.0), (300, 60.0), (3000, 31.0)])
+def test_neighbors_sparse_rows(n, L, search):
+    # dilute systems: cell rows with one atom (a pad slot beside it in the
+    # record layout) or with two atoms far apart along x, whose windows
+    # together span more than the row
+    rng = np.random.default_rng(n)
+    p = np.zeros((n, 4), np.float32)
+    p[:, :3] = rng.uniform(0, L, (n, 3))
+    p = synth.band_clean(p, (L, L, L), 6.5)
+    _check_list(p, (L, L, L), 6.0, 0.5, 64, method="brute", search=search)
+    p = p[oracle.hilbert_sort(p, (L, L, L), 10)[0]]
+    _check_list(p, (L, L, L), 6.0, 0.5, 64, method="brute", search=search)
+
+
+@pytest.mark.parametrize("search", SEARCHES)
+def test_neighbors_unsorted_input_gives_the_same_sets(search):
     s = synth.system(1)
-    _check_list(s.pos4(), s.box, s.rc, s.skin, s.cap, method="brute", lane=lane)
+    _check_list(s.pos4(), s.box, s.rc, s.skin, s.cap, method="brute", search=search)
 
 
-@pytest.mark.parametrize("lane", [False, True])
+@pytest.mark.parametrize("search", SEARCHES)
 @pytest.mark.parametrize("n", [1, 2, 31, 32, 33, 97, 1000])
-def test_neighbors_ragged(n, lane):
+def test_neighbors_ragged(n, search):
     rng = np.random.default_rng(100 + n)
     L = 30.0
     p = np.zeros((n, 4), np.float32)
     p[:, :3] = rng.uniform(0, L, (n, 3))
     p = synth.band_clean(p, (L, L, L), 4.5)       # no pair within 1e-4 A of rs, like every generated input
-    _check_list(p, (L, L, L), 4.0, 0.5, 64, method="brute", lane=lane)
+    _check_list(p, (L, L, L), 4.0, 0.5, 64, method="brute", search=search)
 
 
-@pytest.mark.parametrize("lane", [False, True])
-def test_neighbors_flag_invalid_positions(lane):
+@pytest.mark.parametrize("search", SEARCHES)
+def test_neighbors_flag_invalid_positions(search):
     """A NaN atom and atoms outside [0, L) are flagged in the overflow word
     (TESS_DEV_BAD_INPUT) without a fault; rows away from them are exact."""
     tess = _tess()
@@ -172,7 +190,7 @@ def test_neighbors_flag_invalid_positions(lane):
     p[9, 0] = -0.5
     p[13, 1] = L + 1.0
     nbr_d, cnt_d, ov = tess.build_neighbors(_dev(p), (L, L, L), rc, skin, 128,
-                                            search="lane" if lane else "tile")
+                                            search=search)
     assert int(ov.item()) & 2
     onbr, ocnt, _ = oracle.neighbors_brute(p, (L, L, L), rc, skin, 128)
     good = np.ones(n, bool)
@@ -187,20 +205,20 @@ def test_neighbors_flag_invalid_positions(lane):
     assert np.array_equal(g[good], o[good])
 
 
-@pytest.mark.parametrize("lane", [False, True])
-def test_neighbors_no_pad_fill_and_overflow(lane):
+@pytest.mark.parametrize("search", SEARCHES)
+def test_neighbors_no_pad_fill_and_overflow(search):
     s = synth.system(1)
     perm, _ = oracle.hilbert_sort(s.pos, s.box, 10)
     p4 = s.pos4()[perm]
-    _check_list(p4, s.box, s.rc, s.skin, s.cap, pad_fill=False, lane=lane)
-    _check_list(p4, s.box, s.rc, s.skin, 40, lane=lane)                 # overflow: flag, true counts
-    _check_list(p4, s.box, s.rc, s.skin, 40, pad_fill=False, lane=lane)
-    _check_list(p4, s.box, s.rc, s.skin, 37, lane=lane)                 # cap not a multiple of 4
+    _check_list(p4, s.box, s.rc, s.skin, s.cap, pad_fill=False, search=search)
+    _check_list(p4, s.box, s.rc, s.skin, 40, search=search)                 # overflow: flag, true counts
+    _check_list(p4, s.box, s.rc, s.skin, 40, pad_fill=False, search=search)
+    _check_list(p4, s.box, s.rc, s.skin, 37, search=search)                 # cap not a multiple of 4
 
 
-@pytest.mark.parametrize("lane", [False, True])
+@pytest.mark.parametrize("search", SEARCHES)
 @pytest.mark.parametrize("L,rc", [(13.0, 6.0), (13.1, 6.0), (19.6, 6.0), (25.0, 5.75)])
-def test_neighbors_small_boxes(L, rc, lane):
+def test_neighbors_small_boxes(L, rc, search):
     # boxes of 2 to 4 list radii: cell ranges and windows wrap onto themselves
     rng = np.random.default_rng(int(L * 10))
     n = int(0.1 * L ** 3)
@@ -208,14 +226,14 @@ def test_neighbors_small_boxes(L, rc, lane):
     p[:, :3] = rng.uniform(0, L, (n, 3))
     p = synth.band_clean(p, (L, L, L), float(np.float32(rc) + np.float32(0.5)))
     p = p[oracle.hilbert_sort(p, (L, L, L), 10)[0]]
-    _check_list(p, (L, L, L), rc, 0.5, 256, method="brute", lane=lane)
+    _check_list(p, (L, L, L), rc, 0.5, 256, method="brute", search=search)
 
 
-@pytest.mark.parametrize("lane", [False, True])
-def test_neighbors_large_cap(lane):
+@pytest.mark.parametrize("search", SEARCHES)
+def test_neighbors_large_cap(search):
     s = synth.system(1)
     perm, _ = oracle.hilbert_sort(s.pos, s.box, 10)
-    _check_list(s.pos4()[perm], s.box, s.rc, s.skin, 1024, lane=lane)
+    _check_list(s.pos4()[perm], s.box, s.rc, s.skin, 1024, search=search)
 
 
 def test_neighbors_dense_rows_drain_the_buffer():
@@ -227,8 +245,8 @@ def test_neighbors_dense_rows_drain_the_buffer():
     p[:, :3] = rng.uniform(0, 1, (n, 3)) * np.array([L, L, 6.0]) + np.array([0, 0, 10.0])
     p = synth.band_clean(p, (L, L, L), 5.5)
     p = p[oracle.hilbert_sort(p, (L, L, L), 10)[0]]
-    for lane in (False, True):
-        _check_list(p, (L, L, L), 5.0, 0.5, 512, method="brute", lane=lane)
+    for search in SEARCHES:
+        _check_list(p, (L, L, L), 5.0, 0.5, 512, method="brute", search=search)
 
 
 def test_neighbors_box_errors():
@@ -237,6 +255,22 @@ def test_neighbors_box_errors():
     with pytest.raises(tess.TessError) as e:
         tess.build_neighbors(p, (12.9, 30, 30), 6.0, 0.5, 16)
     assert e.value.code == 2
+
+
+def test_neighbors_flag_errors():
+    # at most one search kind; unknown bits are refused before any launch
+    tess = _tess()
+    torch = torch_cuda()
+    n, box = 10, (30.0, 30.0, 30.0)
+    p = _dev(np.zeros((n, 4), np.float32))
+    ws = torch.empty(tess.tess_build_neighbors_workspace(n, box, 6.0, 0.5), dtype=torch.uint8, device="cuda")
+    nbr = torch.empty((n, 16), dtype=torch.int32, device="cuda")
+    cnt = torch.empty(n, dtype=torch.int32, device="cuda")
+    ov = torch.empty(1, dtype=torch.int32, device="cuda")
+    for flags in (2 | 4, 2 | 8, 4 | 8, 16, 1 << 30):
+        code = tess.tess_build_neighbors(tess._ptr(p), n, box, 6.0, 0.5, 16, flags, tess._ptr(ws), ws.numel(),
+                                         tess._ptr(nbr), tess._ptr(cnt), tess._ptr(ov), None)
+        assert code == 1, flags
 
 
 # ------------------------------------------------------------------ skin check + rebuild loop
