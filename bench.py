@@ -153,7 +153,15 @@ class Step:
         self.feat = torch.randn((n, F), generator=g, device=device, dtype=torch.float32)
         self.out = torch.empty((n, F), dtype=torch.float32, device=device)
         self.flags = (0 if pad_fill else tess.TESS_NO_PAD_FILL) | tess.SEARCH_FLAGS[search]
-        self.sort_fn = tess.tess_hilbert_sort if curve == "hilbert" else tess.tess_morton_sort
+        # curve "none": no sort at all; the atoms stay in a fixed random order
+        # (the locality baseline: what the list and the aggregation cost
+        # without a space-filling-curve order)
+        self.sort_fn = {"hilbert": tess.tess_hilbert_sort, "morton": tess.tess_morton_sort, "none": None}[curve]
+        if self.sort_fn is None:
+            shuffle = torch.randperm(n, generator=torch.Generator().manual_seed(s.seed)).to(device)
+            self.perm.copy_(shuffle.int())
+            self.pos_sorted.zero_()
+            self.pos_sorted[:, :3] = self.pos3[shuffle]
         # the next frame of the trajectory, in the sorted order of frame 0
         t1 = next(iter(s.trajectory(1, condition=False)))[1]
         self.frame1 = torch.from_numpy(t1).to(device)
@@ -178,9 +186,10 @@ class Step:
         """The timed unit: Hilbert sort, then the padded neighbor list."""
         tess, s, P, st = self.tess, self.s, self._ptr, self._stream()
         pos3 = self.pos3 if pos3 is None else pos3
-        c = self.sort_fn(P(pos3), self.n, s.box, 10, P(self.ws_sort), self.ws_sort.numel(),
-                         P(self.perm), P(self.keys), P(self.pos_sorted), P(self.status), st)
-        assert c == 0, c
+        if self.sort_fn is not None:
+            c = self.sort_fn(P(pos3), self.n, s.box, 10, P(self.ws_sort), self.ws_sort.numel(),
+                             P(self.perm), P(self.keys), P(self.pos_sorted), P(self.status), st)
+            assert c == 0, c
         c = tess.tess_build_neighbors(P(self.pos_sorted), self.n, s.box, s.rc, s.skin, s.cap, self.flags,
                                       P(self.ws_nbr), self.ws_nbr.numel(), P(self.nbr), P(self.counts),
                                       P(self.overflow), st)
@@ -741,8 +750,9 @@ def main(argv=None):
     ap.add_argument("--no-pad-fill", action="store_true")
     ap.add_argument("--search", choices=["default", "tile", "lane", "lane2"], default="default",
                     help="pair search kernel (default: the library's choice)")
-    ap.add_argument("--curve", choices=["hilbert", "morton"], default="hilbert",
-                    help="space-filling curve of the sort (morton: the comparison curve)")
+    ap.add_argument("--curve", choices=["hilbert", "morton", "none"], default="hilbert",
+                    help="space-filling curve of the sort (morton: the comparison curve; none: no sort, atoms "
+                         "in a fixed random order -- a locality baseline, not a rebuild)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--graph", action="store_true", help="also time the step captured as one CUDA graph")
     ap.add_argument("--backward", action="store_true", help="also time the aggregation's backward on the same list")

@@ -77,6 +77,27 @@ __device__ __forceinline__ unsigned lanemask_lt() {
     return m;
 }
 
+// Runs of equal consecutive values among the valid lanes of a warp (the
+// valid lanes must be a prefix of the warp, as in a loop over i < n with
+// consecutive lanes on consecutive i): the first lane of this lane's run,
+// the run's length and this lane's rank in it.  Inputs in curve or cell
+// order put equal bins in long runs, so one atomic per run serves as a
+// warp-aggregated histogram update; all 32 lanes must call it.
+struct WarpRun {
+    int leader, len, rank;
+};
+__device__ __forceinline__ WarpRun warp_run(unsigned v, bool valid) {
+    const int lane = threadIdx.x & 31;
+    const unsigned prev = __shfl_up_sync(0xffffffffu, v, 1);
+    const unsigned heads = __ballot_sync(0xffffffffu, valid && (lane == 0 || v != prev));
+    const int nvalid = __popc(__ballot_sync(0xffffffffu, valid));
+    const unsigned le = lanemask_lt() | (1u << lane);
+    const int leader = 31 - __clz(heads & le);
+    const unsigned after = heads & ~le;
+    const int end = after ? __ffs(after) - 1 : nvalid;
+    return WarpRun{leader, end - leader, lane - leader};
+}
+
 // Checked builds (-DTESS_CHECK): an index that a kernel scatters to or
 // gathers from is tested against its bound; a bad one sets TESS_DEV_CHECK in
 // the status word given and the access is skipped.  In the product build the

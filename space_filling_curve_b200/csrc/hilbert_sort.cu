@@ -318,6 +318,11 @@ __global__ __launch_bounds__(SORT_THREADS, TESS_SORT_MINB) void onesweep_pass(co
 // sets a device flag, and the LSD onesweep sort above -- launched gated on
 // that flag -- then writes every output instead (no host synchronisation).
 
+// Histogram and scatter aggregate the lanes of a warp by runs of equal
+// buckets (1) or by warp match (0).
+#ifndef TESS_BK_RUNS
+#define TESS_BK_RUNS 1
+#endif
 constexpr int BK_THREADS = 256;
 constexpr int BK_LOCAL_MAX = 256;    // largest bucket a warp sorts (8 elements per lane)
 constexpr int BK_WARPS = 8;          // warps per block of the local sort
@@ -352,12 +357,18 @@ __global__ __launch_bounds__(BK_THREADS) void bucket_keys_kernel(const float* __
             elems[i] = ((unsigned long long)key << 32) | (unsigned)i;
             b = key >> bshift;
         }
+#if TESS_BK_RUNS
+        // one atomic per run of lanes in the same bucket
+        const WarpRun g = warp_run(b, valid);
+        if (valid && (int)(threadIdx.x & 31) == g.leader) atomicAdd(&bcount[b], g.len);
+#else
         const unsigned act = __ballot_sync(FULL, valid);
         if (valid) {
             // one atomic per group of lanes in the same bucket
             const unsigned peers = __match_any_sync(act, b);
             if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&bcount[b], __popc(peers));
         }
+#endif
     }
     if (__any_sync(FULL, bad) && (threadIdx.x & 31) == 0 && status) atomicOr(status, TESS_DEV_BAD_INPUT);
 }
@@ -374,6 +385,16 @@ __global__ __launch_bounds__(BK_THREADS) void bucket_scatter_kernel(const unsign
         const bool valid = i < n;
         const unsigned long long e = valid ? in[i] : 0ull;
         const uint32_t b = (uint32_t)(e >> 32) >> bshift;
+#if TESS_BK_RUNS
+        const WarpRun g = warp_run(b, valid);
+        int off = 0;
+        if (valid && lane == g.leader) off = atomicAdd(&cursor[b], g.len);
+        off = __shfl_sync(FULL, off, valid ? g.leader : lane) + g.rank;
+        if (valid) {
+            const long long slot = (long long)bstart[b] + off;
+            if (check_index(slot, n, status)) out[slot] = e;
+        }
+#else
         const unsigned act = __ballot_sync(FULL, valid);
         if (valid) {
             const unsigned peers = __match_any_sync(act, b);
@@ -384,6 +405,7 @@ __global__ __launch_bounds__(BK_THREADS) void bucket_scatter_kernel(const unsign
             const long long slot = (long long)bstart[b] + off;
             if (check_index(slot, n, status)) out[slot] = e;
         }
+#endif
     }
 }
 

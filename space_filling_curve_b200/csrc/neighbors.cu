@@ -94,17 +94,14 @@ __global__ void cell_count_kernel(const float4* __restrict__ pos, int n, int3 nc
             c = (cz * nc.y + cy) * nc.x + cx;
             cell_id[i] = c;
         }
-        const unsigned act = __ballot_sync(FULL, valid);
-        if (valid) {
-            // one atomic per group of lanes in the same cell; each lane keeps its
-            // slot among the cell's atoms (any order: cell_order fixes it)
-            const unsigned peers = __match_any_sync(act, c);
-            const int lane = threadIdx.x & 31, leader = __ffs(peers) - 1;
-            int b0 = 0;
-            if (lane == leader) b0 = atomicAdd(&cnt[c], __popc(peers));
-            b0 = __shfl_sync(peers, b0, leader);
-            cell_rank[i] = b0 + __popc(peers & lanemask_lt());
-        }
+        // one atomic per run of lanes in the same cell; each lane keeps its
+        // slot among the cell's atoms (any order: cell_order fixes it)
+        const WarpRun g = warp_run((unsigned)c, valid);
+        const int lane = threadIdx.x & 31;
+        int b0 = 0;
+        if (valid && lane == g.leader) b0 = atomicAdd(&cnt[c], g.len);
+        b0 = __shfl_sync(FULL, b0, valid ? g.leader : lane);
+        if (valid) cell_rank[i] = b0 + g.rank;
     }
     if (__any_sync(FULL, bad) && (threadIdx.x & 31) == 0 && status) atomicOr(status, TESS_DEV_BAD_INPUT);
 }

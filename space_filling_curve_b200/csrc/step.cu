@@ -661,10 +661,9 @@ bool by_shape(int q, Launch&& launch) {
 // F is a multiple of 8 and every array is 32-byte aligned, else 4 (the
 // callers require 16-byte alignment and F % 4 == 0 for either).
 inline int pick_width(int F, std::initializer_list<const void*> ptrs) {
-    if (TESS_EV_W != 8 || F % 8 != 0) return 4;
-    for (const void* p : ptrs)
-        if (!aligned(p, 32)) return 4;
-    return 8;
+    bool wide = TESS_EV_W == 8 && F % 8 == 0;
+    for (const void* p : ptrs) wide = wide && aligned(p, 32);
+    return wide ? 8 : 4;
 }
 
 tess_status edge_backward(const float* pos, int n, tess_box box, float rc, const int32_t* nbr, const int32_t* counts,
