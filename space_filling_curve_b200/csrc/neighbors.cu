@@ -45,16 +45,18 @@ struct Grid {
 };
 
 // Cells of width about rs/CELL_DIV (the tile search adapts to any width; the
-// per-lane stencil relies on width >= rs/CELL_DIV, which coarsening keeps),
-// coarsened when that would give more than ~2 cells per atom.
-static Grid make_grid(int n, tess_box box, float rs) {
+// per-lane stencils rely on width >= rs/CELL_DIV along y and z, which
+// coarsening keeps), xfine times narrower along x (the per-lane searches clip
+// each cell row to a chord along x, so narrower x cells mean fewer
+// candidates), coarsened when that would give more than ~2 cells per atom.
+static Grid make_grid(int n, tess_box box, float rs, double xfine) {
     Grid g{};
     const float L[3] = {box.lx, box.ly, box.lz};
     double w = (double)rs * 1.0001 / (double)CELL_DIV;
     for (int it = 0; it < 64; ++it) {
         long long tot = 1;
         for (int d = 0; d < 3; ++d) {
-            long long c = (long long)std::floor((double)L[d] / w);
+            long long c = (long long)std::floor((double)L[d] / (d == 0 ? w / xfine : w));
             if (c < 1) c = 1;
             if (c > (1 << 20)) c = 1 << 20;
             g.nc[d] = (int)c;
@@ -293,6 +295,7 @@ struct PairArgs {
     int vec_rows;      // rows can take 16-byte stores (cap % 4 == 0, 16-byte aligned nbr)
     int vec8;          // rows can take 32-byte stores (cap % 8 == 0, 32-byte aligned nbr)
     int row_tiles;     // tiles of 32 records per cell row, on average (at least 1)
+    int far_cells;     // two atoms of one row more than this many cells apart take two passes
     int3 nc;
     float3 inv_w;
     float3 L;
@@ -1226,10 +1229,10 @@ __global__ __launch_bounds__(PD_WARPS * 32, TESS_PD_MINB) void pair_search_duo_k
         const int cyc = cell_coord(pa.y, A.inv_w.y, A.nc.y);
         const int czc = cell_coord(pa.z, A.inv_w.z, A.nc.z);
         const int own = 2 * m;
-        // a window reaches at most 3 cells either side of its atom's cell; two
-        // atoms whose windows together could exceed nc.x + 1 cells (far apart
-        // in a sparse row) are walked one after the other, b in a second pass
-        const bool far = vb && cell_coord(xb, A.inv_w.x, ncx) - cell_coord(xa, A.inv_w.x, ncx) > ncx - 6;
+        // two atoms whose windows together could exceed nc.x + 1 cells (far
+        // apart in a sparse row) are walked one after the other, b in a
+        // second pass
+        const bool far = vb && cell_coord(xb, A.inv_w.x, ncx) - cell_coord(xa, A.inv_w.x, ncx) > A.far_cells;
         const int passes = __any_sync(FULL, far) ? 2 : 1;
 
         int donea = 0, doneb = 0;
@@ -1273,16 +1276,28 @@ __global__ __launch_bounds__(PD_WARPS * 32, TESS_PD_MINB) void pair_search_duo_k
                     // has image shift kx + 1.  Slots just outside a range (a
                     // record's other half) lie in the same cell row beyond the
                     // window, so the distance test rejects them.
-                    int B0 = 0, E0 = 0, B1 = 0, E1 = 0, kx = 0;
+                    int B0 = 0, E0 = 0, B1 = 0, E1 = 0, k0 = 0, k1 = 0;
                     if (ina || inb) {
                         const int rowbase = (wz_i * A.nc.y + wy_i) * ncx;
+                        int kx = 0;
                         while (lo < 0) { lo += ncx; hi += ncx; --kx; }
                         while (lo >= ncx) { lo -= ncx; hi -= ncx; ++kx; }
                         B0 = A.cell_start[rowbase + lo];
                         E0 = A.cell_start[rowbase + min(hi, ncx - 1) + 1];
+                        k0 = kx;
                         if (hi >= ncx) {
                             B1 = A.cell_start[rowbase];
                             E1 = A.cell_start[rowbase + min(hi - ncx, ncx - 1) + 1];
+                            k1 = kx + 1;
+                            if (kx < 0) {
+                                // the second range (image shift 0) holds the
+                                // atoms' own cells: walk it first, in step with
+                                // the main ranges of the other lanes
+                                int t = B0; B0 = B1; B1 = t;
+                                t = E0; E0 = E1; E1 = t;
+                                k0 = kx + 1;
+                                k1 = kx;
+                            }
                         }
                     }
 
@@ -1295,7 +1310,7 @@ __global__ __launch_bounds__(PD_WARPS * 32, TESS_PD_MINB) void pair_search_duo_k
                             const int np = end > beg ? (end - kb + 1) >> 1 : 0;
                             const int maxp = (int)__reduce_max_sync(FULL, (unsigned)np);
                             if (maxp == 0) continue;
-                            const float sx = (float)(kx + pc) * A.L.x;
+                            const float sx = (float)(pc ? k1 : k0) * A.L.x;
                             const u64 qax = pk2(usea ? pa.x - sx : nan), qbx = pk2(useb ? pb.x - sx : nan);
                             const SlotPair* src = A.pairs + (kb >> 1);
                             for (int t0 = 0; t0 < maxp; t0 += PD_CHUNK) {
@@ -1364,10 +1379,17 @@ static NbrLayout nbr_layout(void* ws, int n, const Grid& g) {
 
 static bool box_ok(tess_box b) { return finite_pos(b.lx) && finite_pos(b.ly) && finite_pos(b.lz); }
 
+// x cells per y/z cell width for the two-atoms-per-lane search
+#ifndef TESS_DUO_XFINE
+#define TESS_DUO_XFINE 2.0
+#endif
+
 size_t build_neighbors_workspace(int n, tess_box box, float rc, float skin) {
     if (n <= 0 || !box_ok(box) || !(rc > 0.f) || !(skin >= 0.f)) return 0;
     const float rs = rc + skin;
-    return nbr_layout(nullptr, n, make_grid(n, box, rs)).total;
+    // enough for either grid (the search kind is chosen per call)
+    return std::max(nbr_layout(nullptr, n, make_grid(n, box, rs, 1.0)).total,
+                    nbr_layout(nullptr, n, make_grid(n, box, rs, TESS_DUO_XFINE)).total);
 }
 
 tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, float skin, int cap, int flags,
@@ -1381,7 +1403,16 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
     if (!aligned(pos, 16) || !aligned(ws, 256) || !aligned(nbr, 4) || !aligned(counts, 4)) return TESS_ERR_INVALID_ARG;
     const float rs = rc + skin;
     if (box.lx < 2.f * rs || box.ly < 2.f * rs || box.lz < 2.f * rs) return TESS_ERR_BOX_TOO_SMALL;
-    const Grid g = make_grid(n, box, rs);
+    // which search: the per-lane kinds need every box length >= 2 reach (a
+    // window then wraps at most once); otherwise the tile search runs
+    const float lmax = std::max(box.lx, std::max(box.ly, box.lz));
+    const float reach = rs + 1e-3f + 4e-6f * lmax;
+    const bool lane_ok = box.lx >= 2.f * reach && box.ly >= 2.f * reach && box.lz >= 2.f * reach;
+    int kind = kinds ? kinds : TESS_DEFAULT_SEARCH;
+    if (kind != TESS_TILE_SEARCH && !lane_ok) kind = TESS_TILE_SEARCH;
+    const bool records = kind == TESS_LANE2_SEARCH;
+
+    const Grid g = make_grid(n, box, rs, records ? TESS_DUO_XFINE : 1.0);
     NbrLayout L = nbr_layout(ws, n, g);
     if (ws_bytes < L.total) return TESS_ERR_WORKSPACE_TOO_SMALL;
 
@@ -1394,15 +1425,6 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
     const float3 Lb = make_float3(box.lx, box.ly, box.lz);
     const long long m = g.ncell;
     const long long scan_tiles = (m + SCAN_TILE - 1) / SCAN_TILE;
-
-    // which search: the per-lane kinds need every box length >= 2 reach (a
-    // window then wraps at most once); otherwise the tile search runs
-    const float lmax = std::max(box.lx, std::max(box.ly, box.lz));
-    const float reach = rs + 1e-3f + 4e-6f * lmax;
-    const bool lane_ok = box.lx >= 2.f * reach && box.ly >= 2.f * reach && box.lz >= 2.f * reach;
-    int kind = kinds ? kinds : TESS_DEFAULT_SEARCH;
-    if (kind != TESS_TILE_SEARCH && !lane_ok) kind = TESS_TILE_SEARCH;
-    const bool records = kind == TESS_LANE2_SEARCH;
 
     cudaMemsetAsync(overflow, 0, sizeof(int32_t), s);
     {
@@ -1442,6 +1464,7 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
         A.vec_rows = (cap % 4 == 0 && aligned(nbr, 16)) ? 1 : 0;
         A.vec8 = (cap % 8 == 0 && aligned(nbr, 32)) ? 1 : 0;
         A.row_tiles = 1;
+        A.far_cells = 0;
         A.nc = nc;
         A.inv_w = inv_w;
         A.L = Lb;
@@ -1454,6 +1477,9 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
         if (kind == TESS_LANE2_SEARCH) {
             const long long recs = ((long long)n + (long long)nc.y * nc.z + 1) / 2;
             A.row_tiles = (int)std::max<long long>(1, std::llround((double)n / ((double)nc.y * nc.z) / 64.0));
+            // a window reaches at most R cells either side of its atom's cell
+            const double chmax = (double)reach * 1.0001 + 1e-4;
+            A.far_cells = nc.x - 2 * ((int)std::ceil(chmax * (double)inv_w.x) + 1);
             const long long blocks = ((recs + 31) / 32 + PD_WARPS - 1) / PD_WARPS;
             pair_search_duo_kernel<<<(unsigned)std::min<long long>(blocks, 1LL << 30), PD_WARPS * 32, 0, s>>>(A);
         } else if (kind == TESS_LANE_SEARCH) {
