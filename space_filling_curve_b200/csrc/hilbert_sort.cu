@@ -318,11 +318,6 @@ __global__ __launch_bounds__(SORT_THREADS, TESS_SORT_MINB) void onesweep_pass(co
 // sets a device flag, and the LSD onesweep sort above -- launched gated on
 // that flag -- then writes every output instead (no host synchronisation).
 
-// Histogram and scatter aggregate the lanes of a warp by runs of equal
-// buckets (1) or by warp match (0).
-#ifndef TESS_BK_RUNS
-#define TESS_BK_RUNS 1
-#endif
 constexpr int BK_THREADS = 256;
 constexpr int BK_LOCAL_MAX = 256;    // largest bucket a warp sorts (8 elements per lane)
 constexpr int BK_WARPS = 8;          // warps per block of the local sort
@@ -340,10 +335,12 @@ template <int CURVE>
 __global__ __launch_bounds__(BK_THREADS) void bucket_keys_kernel(const float* __restrict__ pos, int n, float3 scale,
                                                                  float3 L, int bits, int bshift,
                                                                  unsigned long long* __restrict__ elems,
-                                                                 int* __restrict__ bcount, int32_t* status) {
+                                                                 int* __restrict__ bcount, int* __restrict__ rank,
+                                                                 int32_t* status) {
     const uint32_t top = (1u << bits) - 1u;
     bool bad = false;
     const int stride = gridDim.x * blockDim.x;
+    const int lane = threadIdx.x & 31;
     for (int base = blockIdx.x * blockDim.x; base < n; base += stride) {
         const int i = base + (int)threadIdx.x;
         const bool valid = i < n;
@@ -357,55 +354,29 @@ __global__ __launch_bounds__(BK_THREADS) void bucket_keys_kernel(const float* __
             elems[i] = ((unsigned long long)key << 32) | (unsigned)i;
             b = key >> bshift;
         }
-#if TESS_BK_RUNS
-        // one atomic per run of lanes in the same bucket
+        // one atomic per run of lanes in the same bucket; each element keeps
+        // its place among the bucket's elements (any order: the local sort
+        // fixes it), so the scatter needs no atomics of its own
         const WarpRun g = warp_run(b, valid);
-        if (valid && (int)(threadIdx.x & 31) == g.leader) atomicAdd(&bcount[b], g.len);
-#else
-        const unsigned act = __ballot_sync(FULL, valid);
-        if (valid) {
-            // one atomic per group of lanes in the same bucket
-            const unsigned peers = __match_any_sync(act, b);
-            if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&bcount[b], __popc(peers));
-        }
-#endif
+        int r0 = 0;
+        if (valid && lane == g.leader) r0 = atomicAdd(&bcount[b], g.len);
+        r0 = __shfl_sync(FULL, r0, valid ? g.leader : lane);
+        if (valid) rank[i] = r0 + g.rank;
     }
-    if (__any_sync(FULL, bad) && (threadIdx.x & 31) == 0 && status) atomicOr(status, TESS_DEV_BAD_INPUT);
+    if (__any_sync(FULL, bad) && lane == 0 && status) atomicOr(status, TESS_DEV_BAD_INPUT);
 }
 
 __global__ __launch_bounds__(BK_THREADS) void bucket_scatter_kernel(const unsigned long long* __restrict__ in, int n,
                                                                     int bshift, const int* __restrict__ bstart,
-                                                                    int* __restrict__ cursor,
+                                                                    const int* __restrict__ rank,
                                                                     unsigned long long* __restrict__ out,
                                                                     int32_t* status) {
     const int stride = gridDim.x * blockDim.x;
-    const int lane = threadIdx.x & 31;
-    for (int base = blockIdx.x * blockDim.x; base < n; base += stride) {
-        const int i = base + (int)threadIdx.x;
-        const bool valid = i < n;
-        const unsigned long long e = valid ? in[i] : 0ull;
+    for (int i = blockIdx.x * blockDim.x + (int)threadIdx.x; i < n; i += stride) {
+        const unsigned long long e = in[i];
         const uint32_t b = (uint32_t)(e >> 32) >> bshift;
-#if TESS_BK_RUNS
-        const WarpRun g = warp_run(b, valid);
-        int off = 0;
-        if (valid && lane == g.leader) off = atomicAdd(&cursor[b], g.len);
-        off = __shfl_sync(FULL, off, valid ? g.leader : lane) + g.rank;
-        if (valid) {
-            const long long slot = (long long)bstart[b] + off;
-            if (check_index(slot, n, status)) out[slot] = e;
-        }
-#else
-        const unsigned act = __ballot_sync(FULL, valid);
-        if (valid) {
-            const unsigned peers = __match_any_sync(act, b);
-            const int leader = __ffs(peers) - 1;
-            int off = 0;
-            if (lane == leader) off = atomicAdd(&cursor[b], __popc(peers));
-            off = __shfl_sync(peers, off, leader) + __popc(peers & lanemask_lt());
-            const long long slot = (long long)bstart[b] + off;
-            if (check_index(slot, n, status)) out[slot] = e;
-        }
-#endif
+        const long long slot = (long long)bstart[b] + rank[i];
+        if (check_index(slot, n, status)) out[slot] = e;
     }
 }
 
@@ -590,7 +561,9 @@ static void sfc_sort_launch(const float* pos, int n, tess_box box, int bits, int
 // buffers also carry the bucket pass), then the bucket counts / offsets.
 struct BucketLayout {
     SortLayout lsd;
-    int* bcount;             // [nb] counts, then scatter cursors
+    int* bcount;             // [nb] counts
+    int* rank;               // [n] place of each element in its bucket (in the LSD sort's
+                             // look-back states, which the fallback zeroes before use)
     int32_t* flag;           // 1: some bucket too large for the local sort
     int* bstart;             // [nb + 1]
     int* sums;               // scan scratch
@@ -611,6 +584,9 @@ static BucketLayout bucket_layout(void* ws, int n) {
     B.bstart = c.take<int>((size_t)nb + 1);
     B.sums = c.take<int>((size_t)scan_sums_len(nb));
     B.total = align_up(c.off, 256);
+    // 4 passes x tiles of 2048 x 256 eight-byte states hold n ints
+    static_assert((size_t)MAX_PASSES * RADIX * 8 >= (size_t)SORT_TILE * 4, "rank storage");
+    B.rank = reinterpret_cast<int*>(B.lsd.states);
     return B;
 }
 
@@ -644,16 +620,16 @@ tess_status sfc_sort(const float* pos, int n, tess_box box, int bits, int curve,
         StageScope sc(ST_KEYS, s);
         if (curve == 0)
             bucket_keys_kernel<0><<<blocks, BK_THREADS, 0, s>>>(pos, n, scale, Lb, bits, bshift, L.a, B.bcount,
-                                                                 status);
+                                                                 B.rank, status);
         else
             bucket_keys_kernel<1><<<blocks, BK_THREADS, 0, s>>>(pos, n, scale, Lb, bits, bshift, L.a, B.bcount,
-                                                                 status);
+                                                                 B.rank, status);
         count_launch();
     }
     {
         StageScope sc(ST_SORT, s);
         exclusive_scan(B.bcount, nb, B.sums, B.bstart, s);
-        bucket_scatter_kernel<<<blocks, BK_THREADS, 0, s>>>(L.a, n, bshift, B.bstart, B.bcount, L.b, status);
+        bucket_scatter_kernel<<<blocks, BK_THREADS, 0, s>>>(L.a, n, bshift, B.bstart, B.rank, L.b, status);
         const int lblocks = (int)std::min<long long>((nb + BK_WARPS - 1) / BK_WARPS, (long long)sms * 16);
         bucket_local_sort<<<lblocks, BK_WARPS * 32, 0, s>>>(L.b, B.bstart, (int)nb, pos, perm, keys_sorted,
                                                            reinterpret_cast<float4*>(pos_sorted), B.flag, n, status);

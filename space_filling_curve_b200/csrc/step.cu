@@ -242,6 +242,12 @@ constexpr int EV_MAXCAP = 512;       // live edges of one row staged in shared m
 // in space and share most of their neighbors.  All blocks together sweep a
 // front of gridDim * chunk rows, which bounds the L2 working set.
 constexpr int EV_CHUNK = TESS_EV_CHUNK;
+// the shape for dense rows: caps above EV_DENSE_CAP (the row capacity stands
+// in for the mean row length, which the host does not know)
+constexpr int EV_DENSE_CAP = 192;
+constexpr int EV_DENSE_WARPS = 8;
+constexpr int EV_DENSE_MINB = 3;
+constexpr int EV_DENSE_CHUNK = 256;
 constexpr int EV_GEO_UNROLL = TESS_EV_GEO_UNROLL;     // neighbor/position loads in flight per lane
 constexpr int EV_ACC_UNROLL = TESS_EV_ACC_UNROLL;     // feature rows in flight per lane group
 
@@ -342,16 +348,20 @@ __device__ __forceinline__ FVec<8> ld_vec<8>(const float* p) {
 // phase 2 accumulates f_c * h_j with several rows in flight; the lane groups
 // are then summed with shuffles.  Shared memory: EV_WARPS * cap int2
 // (dynamic, so that what a small cap leaves over serves as L1).
-template <int W, int LPE, int VPL>
-__global__ __launch_bounds__(EV_WARPS * 32, TESS_EV_MINB) void edge_vec_kernel(EdgeArgs A) {
+// Block shape (WARPS per block, MINB resident blocks, rows per CHUNK): one
+// block of 24 warps per SM over 768-row chunks for rows of up to ~100 live
+// edges; dense rows (caps above 192) fill L1 faster and run best as 3 blocks
+// of 8 warps over 256-row chunks.
+template <int W, int LPE, int VPL, int WARPS = EV_WARPS, int MINB = TESS_EV_MINB, int CHUNK = EV_CHUNK>
+__global__ __launch_bounds__(WARPS * 32, MINB) void edge_vec_kernel(EdgeArgs A) {
     constexpr int EPI = 32 / LPE;
     extern __shared__ int2 s_edge[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int2* live_e = s_edge + (size_t)warp * A.cap;
     const int g = lane / LPE, fl = lane % LPE;
     const bool edges = A.edge_vec || A.edge_fc || A.edge_unit;
-    for (long long c0 = (long long)blockIdx.x * EV_CHUNK; c0 < A.n; c0 += (long long)gridDim.x * EV_CHUNK)
-    for (long long i = c0 + warp, c1 = min((long long)A.n, c0 + EV_CHUNK); i < c1; i += EV_WARPS) {
+    for (long long c0 = (long long)blockIdx.x * CHUNK; c0 < A.n; c0 += (long long)gridDim.x * CHUNK)
+    for (long long i = c0 + warp, c1 = min((long long)A.n, c0 + CHUNK); i < c1; i += WARPS) {
         const float4 pi = A.pos[i];
         const int m = max(min(A.counts[i], A.cap), 0);
         const int limit = edges ? A.cap : m;
@@ -739,13 +749,20 @@ tess_status edge_aggregate(const float* pos, int n, tess_box box, float rc, cons
     const long long rows_blocks = ((long long)n + EDGE_WARPS - 1) / EDGE_WARPS;
     const int blocks = (int)std::min<long long>(rows_blocks, (long long)sms * 64);
     const bool vec = (F % 4 == 0) && F <= 256 && aligned(feat, 16) && aligned(out, 16) && cap <= EV_MAXCAP;
-    const size_t vsmem = (size_t)EV_WARPS * cap * sizeof(int2);
+    const bool dense = cap > EV_DENSE_CAP;
+    const int warps = dense ? EV_DENSE_WARPS : EV_WARPS;
+    const size_t vsmem = (size_t)warps * cap * sizeof(int2);
     bool launched = false;
     if (vec) {
         auto launch = [&](auto w, auto lpe, auto vpl) {
-            auto* k = edge_vec_kernel<decltype(w)::value, decltype(lpe)::value, decltype(vpl)::value>;
-            if (vsmem > 48 * 1024) cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)vsmem);
-            k<<<chunk_grid(k, EV_WARPS * 32, vsmem, n, sms, EV_CHUNK), EV_WARPS * 32, vsmem, s>>>(A);
+            constexpr int Wv = decltype(w)::value, Lv = decltype(lpe)::value, Vv = decltype(vpl)::value;
+            auto go = [&](auto* k, int chunk) {
+                if (vsmem > 48 * 1024)
+                    cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)vsmem);
+                k<<<chunk_grid(k, warps * 32, vsmem, n, sms, chunk), warps * 32, vsmem, s>>>(A);
+            };
+            if (dense) go(edge_vec_kernel<Wv, Lv, Vv, EV_DENSE_WARPS, EV_DENSE_MINB, EV_DENSE_CHUNK>, EV_DENSE_CHUNK);
+            else go(edge_vec_kernel<Wv, Lv, Vv>, EV_CHUNK);
         };
         const int W = pick_width(F, {feat, out});
         launched = W == 8 ? by_shape<8>(F / 8, launch) : by_shape<4>(F / 4, launch);
