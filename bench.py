@@ -58,7 +58,7 @@ class ClockSampler:
              "clocks_event_reasons.sw_power_cap")
         try:
             self._proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + q,
-                                           "--format=csv,noheader,nounits", "-lms", "100"],
+                                           "--format=csv,noheader,nounits", "-lms", "50"],
                                           stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self._t = threading.Thread(target=self._read, daemon=True)
             self._t.start()
@@ -322,8 +322,10 @@ def run_cuda(args, world, rank, local):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        reb = _timed(step.rebuild, args.steps, flush)
+    # clocks are sampled over the timed rebuilds and the timed loops right
+    # after them (same load), so that a short timed region still gets samples
+    clk = ClockSampler(local).__enter__()
+    reb = _timed(step.rebuild, args.steps, flush)
     if world > 1:
         torch.distributed.barrier()
     launches = tess.tess_kernel_launch_count() - launches0
@@ -343,6 +345,7 @@ def run_cuda(args, world, rank, local):
     whole_stages = _stage_ms(tess.tess_stage_times())
     tess.tess_stage_timing(False)
     whole_ms = sum(whole) / args.steps
+    clk.__exit__(None, None, None)
 
     extras = _extras(args, step, flush, dev, world, ms_max)
 

@@ -1123,12 +1123,34 @@ __device__ __forceinline__ void duo_test(unsigned& wa, unsigned& wb, u64 x, u64 
 }
 #undef TESS_DUO_BODY
 
+#ifndef TESS_PD_BULKPAD
+#define TESS_PD_BULKPAD 1
+#endif
+constexpr int PD_PADS = 256;               // ints of -1 that the pad copies read
+
+// bytes (a multiple of 16) from shared address src to global dst (both 16-byte
+// aligned) by the bulk copy engine, as one bulk group of this thread
+__device__ __forceinline__ void bulk_store(int* dst, unsigned src, unsigned bytes) {
+    asm volatile(
+        "cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n\t"
+        "cp.async.bulk.commit_group;" ::"l"(dst), "r"(src), "r"(bytes)
+        : "memory");
+}
+
 #ifndef TESS_PD_MINB
 #define TESS_PD_MINB 6
 #endif
 
 __global__ __launch_bounds__(PD_WARPS * 32, TESS_PD_MINB) void pair_search_duo_kernel(PairArgs A) {
     __shared__ int s_buf[PD_WARPS][2][32 * PD_BUF];
+#if TESS_PD_BULKPAD
+    __shared__ __align__(16) int s_pads[PD_PADS];
+    for (int k = threadIdx.x; k < PD_PADS; k += blockDim.x) s_pads[k] = -1;
+    // the bulk copies read s_pads through the async proxy
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+    const unsigned pads_sa = (unsigned)__cvta_generic_to_shared(s_pads);
+#endif
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int* const bufa = &s_buf[warp][0][lane];
     int* const bufb = &s_buf[warp][1][lane];
@@ -1186,7 +1208,17 @@ __global__ __launch_bounds__(PD_WARPS * 32, TESS_PD_MINB) void pair_search_duo_k
                 int e = filled;
                 if (A.vec8) {
                     for (; e < cap && (e & 7); ++e) row[e] = -1;
+#if TESS_PD_BULKPAD
+                    // the pads as bulk copies of a shared block of -1 (the copy
+                    // engine writes them, not the lane's load/store path)
+                    while (e + 8 <= cap) {
+                        const int m8 = min((cap - e) >> 3, PD_PADS >> 3);
+                        bulk_store(row + e, pads_sa, (unsigned)m8 * 32u);
+                        e += m8 * 8;
+                    }
+#else
                     for (; e + 8 <= cap; e += 8) st_global_v8(row + e, -1, -1, -1, -1, -1, -1, -1, -1);
+#endif
                 }
                 for (; e < cap; ++e) row[e] = -1;
             }
@@ -1339,6 +1371,10 @@ __global__ __launch_bounds__(PD_WARPS * 32, TESS_PD_MINB) void pair_search_duo_k
         if (ov && lane == 0) atomicOr(A.status, TESS_DEV_OVERFLOW);
         __syncwarp();
     }
+#if TESS_PD_BULKPAD
+    // s_pads must outlive the reads of this thread's bulk copies
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+#endif
 }
 
 // ---------------------------------------------------------------- host
