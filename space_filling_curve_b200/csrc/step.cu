@@ -242,6 +242,7 @@ constexpr int EV_MAXCAP = 512;       // live edges of one row staged in shared m
 // in space and share most of their neighbors.  All blocks together sweep a
 // front of gridDim * chunk rows, which bounds the L2 working set.
 constexpr int EV_CHUNK = TESS_EV_CHUNK;
+
 // the shape for dense rows: caps above EV_DENSE_CAP (the row capacity stands
 // in for the mean row length, which the host does not know)
 constexpr int EV_DENSE_CAP = 192;
@@ -486,6 +487,13 @@ constexpr int BK_MAXCAP = 512;
 #define TESS_BK_MINB 3
 #endif
 constexpr int BK_CHUNK = TESS_BK_CHUNK;
+#ifndef TESS_BK_ACC_UNROLL
+#define TESS_BK_ACC_UNROLL 2
+#endif
+constexpr int BK_ACC_UNROLL = TESS_BK_ACC_UNROLL;   // edge steps in flight per lane group
+#ifndef TESS_BK_PREFETCH
+#define TESS_BK_PREFETCH 1
+#endif
 
 template <int W, int LPE, int VPL>
 __global__ __launch_bounds__(BK_WARPS * 32, TESS_BK_MINB) void edge_backward_kernel(BackArgs A) {
@@ -537,31 +545,51 @@ __global__ __launch_bounds__(BK_WARPS * 32, TESS_BK_MINB) void edge_backward_ker
             hi[v] = ld_vec<W>(A.feat + own + v * LPE * W);
             acc[v].zero();
         }
+#if TESS_BK_PREFETCH
+        {
+            // the next row of this warp: its list entries into L2 meanwhile
+            long long in = i + BK_WARPS;
+            if (in >= c1) in = c0 + (long long)gridDim.x * BK_CHUNK + warp;
+            if (in < A.n && lane * 32 < A.cap)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(A.nbr + (size_t)in * A.cap + lane * 32));
+        }
+#endif
         float fx = 0.f, fy = 0.f, fz = 0.f;
-        for (int e0 = 0; e0 < nlive; e0 += EPI) {
-            const int e = e0 + g;
-            const bool ok = e < nlive;
-            const int j = ok ? s_j[e] : (int)i;
-            const float4 w = ok ? s_w[e] : make_float4(0.f, 0.f, 0.f, 0.f);
-            const size_t base = (size_t)j * A.F + fl * W;
-            FVec<W> hj[VPL], gj[VPL];
+        // BK_ACC_UNROLL steps of EPI edges in flight per lane group
+        for (int e0 = 0; e0 < nlive; e0 += EPI * BK_ACC_UNROLL) {
+            int jj[BK_ACC_UNROLL];
+            float4 ww[BK_ACC_UNROLL];
 #pragma unroll
-            for (int v = 0; v < VPL; ++v) {
-                hj[v] = ld_vec<W>(A.feat + base + v * LPE * W);
-                gj[v] = ld_vec<W>(A.grad_out + base + v * LPE * W);
+            for (int u = 0; u < BK_ACC_UNROLL; ++u) {
+                const int e = e0 + u * EPI + g;
+                const bool ok = e < nlive;
+                jj[u] = ok ? s_j[e] : -1;
+                ww[u] = ok ? s_w[e] : make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            if (ok) {
+            FVec<W> hj[BK_ACC_UNROLL][VPL], gj[BK_ACC_UNROLL][VPL];
+#pragma unroll
+            for (int u = 0; u < BK_ACC_UNROLL; ++u) {
+                const size_t base = (size_t)(jj[u] >= 0 ? jj[u] : (int)i) * A.F + fl * W;
+#pragma unroll
+                for (int v = 0; v < VPL; ++v) {
+                    hj[u][v] = ld_vec<W>(A.feat + base + v * LPE * W);
+                    gj[u][v] = ld_vec<W>(A.grad_out + base + v * LPE * W);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < BK_ACC_UNROLL; ++u) {
+                if (jj[u] < 0) continue;
                 unsigned long long d2 = 0ull;
 #pragma unroll
                 for (int v = 0; v < VPL; ++v) {
-                    acc[v].fma(w.x, gj[v]);
-                    d2 = FVec<W>::dot2(gi[v], hj[v], d2);
-                    d2 = FVec<W>::dot2(gj[v], hi[v], d2);
+                    acc[v].fma(ww[u].x, gj[u][v]);
+                    d2 = FVec<W>::dot2(gi[v], hj[u][v], d2);
+                    d2 = FVec<W>::dot2(gj[u][v], hi[v], d2);
                 }
                 const float dot = f2_sum(d2);
-                fx = fmaf(dot, w.y, fx);
-                fy = fmaf(dot, w.z, fy);
-                fz = fmaf(dot, w.w, fz);
+                fx = fmaf(dot, ww[u].y, fx);
+                fy = fmaf(dot, ww[u].z, fy);
+                fz = fmaf(dot, ww[u].w, fz);
             }
         }
         // feature gradient: lane groups hold disjoint edges of the same
