@@ -3,28 +3,29 @@
 // abstract).
 //
 // Level 0 (binning, deterministic):
-//   cell_count     cell id per atom, warp-aggregated histogram
+//   cell_count     cell id per atom, histogram (one atomic per run of equal
+//                  cells in a warp)
+//   row_pad        (record layout) an odd cell row gets a pad slot
 //   scan_*         exclusive scan of the cell counts -> cell_start
 //   cell_scatter   atom indices into their cells (any order within a cell)
 //   cell_order     within each cell, order by atom index and write the
-//                  positions in cell order as float4 (x, y, z, index bits)
-// Levels 1-3 (pair_tile_kernel, the default; one warp per tile of 32
-// consecutive atoms, lane = atom i):
-//   1. tile: bounding box of the 32 atoms (Hilbert-consecutive, so compact)
-//      and a frame centred on it
-//   2. cells: the cell rows within reach of the box, each clipped to the
-//      box's chord at its distance; each piece of a row is one contiguous
-//      range of the cell-ordered positions, shifted by its periodic image;
-//      candidates are culled against the rounded box and compacted (ballot
-//      + popc) into a shared-memory chunk
-//   3. pairs: every lane tests its atom against the chunk (broadcast reads,
-//      packed f32x2), 32 candidates per accept mask, and turns the set bits
-//      into indices that leave for its row in aligned 32-byte groups.
-// pair_search_lane_kernel (TESS_LANE_SEARCH) walks a stencil of cell rows
-// per lane instead, and pair_search_duo_kernel (TESS_LANE2_SEARCH) does so
-// with two atoms per lane over a record layout of the cell order; all three
-// give the same lists (in different orders).  Which one runs when the caller
-// names none is TESS_DEFAULT_SEARCH.
+//                  positions in cell order: as two-slot records (x0 x1 | y0 y1
+//                  | z0 z1 | i0 i1) with every cell row starting at an even
+//                  slot for the default search, as float4 (x, y, z, index
+//                  bits) for the other two
+// Levels 1-3, three kernels with the same lists (rows in different orders):
+//   pair_search_duo_kernel (TESS_LANE2_SEARCH, the default): two atoms per
+//     lane; each walks the 5 x 5 cell rows around its row, clipped to the
+//     atoms' chords (level 1-2), and tests every record of the windows
+//     against both atoms in packed f32x2 (level 3), accepted indices staged
+//     per atom in shared memory and drained to the rows in 32-byte groups
+//   pair_search_lane_kernel (TESS_LANE_SEARCH): the same walk with one atom
+//     per lane over float4 candidates
+//   pair_tile_kernel (TESS_TILE_SEARCH; boxes shorter than 2 reach): one warp
+//     per 32 Hilbert-consecutive atoms; the cell rows within reach of their
+//     bounding box, culled against it and compacted into a shared chunk,
+//     tested by every lane (broadcast reads), 32 candidates per accept mask.
+// Which one runs when the caller names none is TESS_DEFAULT_SEARCH.
 #include <climits>
 #include <type_traits>
 
