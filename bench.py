@@ -22,7 +22,6 @@ import os
 import subprocess
 import sys
 import threading
-import time
 
 import numpy as np
 
@@ -65,6 +64,15 @@ class ClockSampler:
         except (OSError, FileNotFoundError):
             self._proc = None
         return self
+
+    def running(self):
+        return self._proc is not None and self._proc.poll() is None
+
+    def mark(self):
+        """Start of the timed region: drop the samples taken so far (the
+        sampler is started earlier, during the warm-up, because nvidia-smi
+        can take a while to print its first line)."""
+        self.samples.clear()
 
     def _read(self):
         for line in self._proc.stdout:
@@ -302,6 +310,9 @@ def run_cuda(args, world, rank, local):
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     peak, peak_kind = _peaks()
 
+    # clocks: the sampler starts with the warm-up and keeps the samples from
+    # the timed rebuilds and the timed loops right after them (same load)
+    clk = ClockSampler(local).__enter__()
     # warm-up (W whole steps); stage timing on so that its event pool fills
     tess.tess_stage_times()
     tess.tess_stage_timing(True)
@@ -318,13 +329,17 @@ def run_cuda(args, world, rank, local):
     # timed region: K rebuilds (sort + list), per-rebuild events on the
     # launching stream, L2 flushed before each, the library's stage timing off
     tess.tess_stage_timing(False)
-    launches0 = tess.tess_kernel_launch_count()
+    # keep the GPU busy until the clock sampler has printed (at most ~3 s more)
+    extra = 0
+    while clk.running() and not clk.samples and extra < 600:
+        step.rebuild()
+        torch.cuda.synchronize()
+        extra += 1
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    # clocks are sampled over the timed rebuilds and the timed loops right
-    # after them (same load), so that a short timed region still gets samples
-    clk = ClockSampler(local).__enter__()
+    launches0 = tess.tess_kernel_launch_count()
+    clk.mark()
     reb = _timed(step.rebuild, args.steps, flush)
     if world > 1:
         torch.distributed.barrier()
