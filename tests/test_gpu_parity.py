@@ -236,6 +236,29 @@ def test_neighbors_large_cap(search):
     _check_list(s.pos4()[perm], s.box, s.rc, s.skin, 1024, search=search)
 
 
+@pytest.mark.parametrize("search", SEARCHES)
+def test_neighbors_rows_not_vector_aligned(search):
+    # a list buffer that starts 4 bytes past an aligned address: no 16- or
+    # 32-byte row stores (nor bulk pad copies) may be used, whatever the cap
+    tess = _tess()
+    torch = torch_cuda()
+    s = synth.system(1)
+    perm, _ = oracle.hilbert_sort(s.pos, s.box, 10)
+    p4 = s.pos4()[perm]
+    cap = s.cap                      # 192: a multiple of 8, rows without overflow
+    raw = torch.full((s.n * cap + 8,), 7, dtype=torch.int32, device="cuda")
+    nbr = raw[1:1 + s.n * cap].view(s.n, cap)
+    nbr_d, cnt_d, ov = tess.build_neighbors(_dev(p4), s.box, s.rc, s.skin, cap, search=search, nbr=nbr)
+    onbr, ocnt, oov = oracle.neighbors_cells(p4, s.box, s.rc, s.skin, cap)
+    cnt = cnt_d.cpu().numpy()
+    assert np.array_equal(cnt, ocnt) and int(ov.item()) == oov
+    assert np.array_equal(canon_rows_gpu(nbr_d, cnt_d), onbr)
+    nb = nbr_d.cpu().numpy()
+    assert np.all(nb[np.arange(cap)[None, :] >= np.minimum(cnt, cap)[:, None]] == -1)
+    # nothing outside the list was written
+    assert int(raw[0].item()) == 7 and bool((raw[1 + s.n * cap:] == 7).all())
+
+
 def test_neighbors_dense_rows_drain_the_buffer():
     # a dense cluster: rows far longer than the per-lane staging buffer
     rng = np.random.default_rng(5)
