@@ -22,6 +22,7 @@ import os
 import subprocess
 import sys
 import threading
+import time
 
 import numpy as np
 
