@@ -350,7 +350,9 @@ __global__ __launch_bounds__(BK_THREADS) void bucket_keys_kernel(const float* __
             bad |= !(x >= 0.0f && x < L.x && y >= 0.0f && y < L.y && z >= 0.0f && z < L.z);
             const uint32_t qx = quantize(x, scale.x, top), qy = quantize(y, scale.y, top),
                            qz = quantize(z, scale.z, top);
-            const uint32_t key = CURVE == 0 ? hilbert_key(qx, qy, qz, bits) : morton_key(qx, qy, qz);
+            // the default 10 bits with the level loop unrolled at compile time
+            const uint32_t key = CURVE == 0 ? (bits == 10 ? hilbert_key(qx, qy, qz, 10) : hilbert_key(qx, qy, qz, bits))
+                                            : morton_key(qx, qy, qz);
             elems[i] = ((unsigned long long)key << 32) | (unsigned)i;
             b = key >> bshift;
         }
