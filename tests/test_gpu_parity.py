@@ -230,6 +230,21 @@ def test_neighbors_small_boxes(L, rc, search):
 
 
 @pytest.mark.parametrize("search", SEARCHES)
+@pytest.mark.parametrize("box", [(13.5, 30.0, 60.0), (60.0, 13.5, 30.0), (30.0, 60.0, 13.5), (80.0, 14.0, 14.0)])
+def test_neighbors_elongated_boxes(box, search):
+    # one axis just above two list radii (its cell rows wrap onto themselves,
+    # the two-atoms-per-lane search walks far-apart pairs in two passes when
+    # that axis is x), the others long
+    rng = np.random.default_rng(int(sum(box)))
+    n = int(0.05 * box[0] * box[1] * box[2])
+    p = np.zeros((n, 4), np.float32)
+    p[:, :3] = rng.uniform(0, 1, (n, 3)) * np.array(box)
+    p = synth.band_clean(p, box, 6.5)
+    p = p[oracle.hilbert_sort(p, box, 10)[0]]
+    _check_list(p, box, 6.0, 0.5, 128, method="brute", search=search)
+
+
+@pytest.mark.parametrize("search", SEARCHES)
 def test_neighbors_large_cap(search):
     s = synth.system(1)
     perm, _ = oracle.hilbert_sort(s.pos, s.box, 10)
