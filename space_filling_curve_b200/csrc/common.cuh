@@ -8,6 +8,7 @@
 #include <cmath>
 
 #include "tess.h"
+#include <utility>
 
 // The pair search that tess_build_neighbors runs when its flags name none
 // (TESS_LANE2_SEARCH, TESS_LANE_SEARCH or TESS_TILE_SEARCH): the fastest on
@@ -75,6 +76,39 @@ __device__ __forceinline__ unsigned lanemask_lt() {
     unsigned m;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
     return m;
+}
+
+// Programmatic dependent launch: kernels of the rebuild path are launched so
+// that each may be scheduled while the one before it drains, and each waits
+// at its first line (griddepcontrol.wait) until the grids it depends on have
+// completed and their memory is visible.  The wait is a no-op for a grid
+// launched without the attribute.
+#ifndef TESS_PDL
+#define TESS_PDL 1
+#endif
+__device__ __forceinline__ void pdl_wait() {
+#if TESS_PDL
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+#endif
+}
+
+template <typename... P, typename... A>
+inline void launch_pdl(void (*k)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, A&&... args) {
+#if TESS_PDL
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, k, std::forward<A>(args)...);
+#else
+    k<<<grid, block, smem, s>>>(std::forward<A>(args)...);
+#endif
 }
 
 // Runs of equal consecutive values among the valid lanes of a warp (the

@@ -337,6 +337,7 @@ __global__ __launch_bounds__(BK_THREADS) void bucket_keys_kernel(const float* __
                                                                  unsigned long long* __restrict__ elems,
                                                                  int* __restrict__ bcount, int* __restrict__ rank,
                                                                  int32_t* status) {
+    pdl_wait();
     const uint32_t top = (1u << bits) - 1u;
     bool bad = false;
     const int stride = gridDim.x * blockDim.x;
@@ -373,6 +374,7 @@ __global__ __launch_bounds__(BK_THREADS) void bucket_scatter_kernel(const unsign
                                                                     const int* __restrict__ rank,
                                                                     unsigned long long* __restrict__ out,
                                                                     int32_t* status) {
+    pdl_wait();
     const int stride = gridDim.x * blockDim.x;
     for (int i = blockIdx.x * blockDim.x + (int)threadIdx.x; i < n; i += stride) {
         const unsigned long long e = in[i];
@@ -443,6 +445,7 @@ __global__ __launch_bounds__(BK_WARPS * 32, 4) void bucket_local_sort(const unsi
                                                                    uint32_t* __restrict__ keys_out,
                                                                    float4* __restrict__ pos_sorted,
                                                                    int32_t* fallback, int n, int32_t* status) {
+    pdl_wait();
     __shared__ unsigned long long s_el[BK_WARPS][BK_LOCAL_MAX];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     unsigned long long* s = s_el[warp];
@@ -620,6 +623,7 @@ tess_status sfc_sort(const float* pos, int n, tess_box box, int bits, int curve,
     if (dev_status) cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s);
     {
         StageScope sc(ST_KEYS, s);
+        // after the memsets: a plain launch (programmatic launch only follows kernels)
         if (curve == 0)
             bucket_keys_kernel<0><<<blocks, BK_THREADS, 0, s>>>(pos, n, scale, Lb, bits, bshift, L.a, B.bcount,
                                                                  B.rank, status);
@@ -631,10 +635,12 @@ tess_status sfc_sort(const float* pos, int n, tess_box box, int bits, int curve,
     {
         StageScope sc(ST_SORT, s);
         exclusive_scan(B.bcount, nb, B.sums, B.bstart, s);
-        bucket_scatter_kernel<<<blocks, BK_THREADS, 0, s>>>(L.a, n, bshift, B.bstart, B.rank, L.b, status);
+        launch_pdl(bucket_scatter_kernel, dim3(blocks), dim3(BK_THREADS), 0, s, (const unsigned long long*)L.a, n,
+                   bshift, (const int*)B.bstart, (const int*)B.rank, L.b, status);
         const int lblocks = (int)std::min<long long>((nb + BK_WARPS - 1) / BK_WARPS, (long long)sms * 16);
-        bucket_local_sort<<<lblocks, BK_WARPS * 32, 0, s>>>(L.b, B.bstart, (int)nb, pos, perm, keys_sorted,
-                                                           reinterpret_cast<float4*>(pos_sorted), B.flag, n, status);
+        launch_pdl(bucket_local_sort, dim3(lblocks), dim3(BK_WARPS * 32), 0, s, (const unsigned long long*)L.b,
+                   (const int*)B.bstart, (int)nb, pos, perm, keys_sorted, reinterpret_cast<float4*>(pos_sorted),
+                   B.flag, n, status);
         count_launch(2);
         // a bucket too large for the local sort: the LSD sort, gated on the flag
         zero_if_kernel<<<sms * 2, 256, 0, s>>>(reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) +

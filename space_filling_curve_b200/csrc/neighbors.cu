@@ -82,6 +82,7 @@ __device__ __forceinline__ int cell_coord(float x, float inv_w, int nc) {
 __global__ void cell_count_kernel(const float4* __restrict__ pos, int n, int3 nc, float3 inv_w, float3 L,
                                   int* __restrict__ cell_id, int* __restrict__ cell_rank, int* __restrict__ cnt,
                                   int32_t* status) {
+    pdl_wait();
     bool bad = false;
     const int stride = gridDim.x * blockDim.x;
     for (int base = blockIdx.x * blockDim.x; base < n; base += stride) {
@@ -112,6 +113,7 @@ __global__ void cell_count_kernel(const float4* __restrict__ pos, int n, int3 nc
 __global__ void cell_scatter_kernel(const int* __restrict__ cell_id, const int* __restrict__ cell_rank, int n,
                                     long long nslots, const int* __restrict__ cell_start,
                                     int* __restrict__ slot_atom, int32_t* status) {
+    pdl_wait();
     const int stride = gridDim.x * blockDim.x;
     for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
         const long long slot = (long long)cell_start[cell_id[i]] + cell_rank[i];
@@ -185,6 +187,7 @@ struct alignas(32) SlotPair {
 // slot counted in the row's last cell, so the scan of the counts starts every
 // row at an even slot.  rowpad[r] = 1 marks such a row.
 __global__ void row_pad_kernel(int* __restrict__ cnt, int ncx, long long nrows, int* __restrict__ rowpad) {
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
     for (long long r = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < nrows; r += warps) {
@@ -224,6 +227,7 @@ __device__ __forceinline__ void put_record(SlotPair* pairs, int r, float4 p0, in
 __global__ void cell_order_pairs_kernel(const int* __restrict__ slot_atom, long long ncell, int ncx,
                                         const int* __restrict__ cell_start, const int* __restrict__ rowpad,
                                         const float4* __restrict__ pos, SlotPair* __restrict__ pairs) {
+    pdl_wait();
     const long long stride = (long long)gridDim.x * blockDim.x;
     const float nan = __int_as_float(0x7fc00000);
     const float4 pnan = make_float4(nan, nan, nan, nan);
@@ -1143,6 +1147,7 @@ __device__ __forceinline__ void bulk_store(int* dst, unsigned src, unsigned byte
 #endif
 
 __global__ __launch_bounds__(PD_WARPS * 32, TESS_PD_MINB) void pair_search_duo_kernel(PairArgs A) {
+    pdl_wait();
     __shared__ int s_buf[PD_WARPS][2][32 * PD_BUF];
 #if TESS_PD_BULKPAD
     __shared__ __align__(16) int s_pads[PD_PADS];
@@ -1468,21 +1473,24 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
         StageScope sc(ST_CELLS, s);
         cudaMemsetAsync(L.cnt, 0, sizeof(int) * (size_t)m, s);
         const int blocks = (int)std::min<long long>(((long long)n + 255) / 256, (long long)sms * 16);
+        // after the memsets: a plain launch (programmatic launch only follows kernels)
         cell_count_kernel<<<blocks, 256, 0, s>>>(pos4, n, nc, inv_w, Lb, L.cell_id, L.cell_rank, L.cnt, overflow);
         const long long nrows = (long long)nc.y * nc.z;
         if (records) {
             const long long rb = std::min<long long>((nrows + 7) / 8, (long long)sms * 32);
-            row_pad_kernel<<<(unsigned)rb, 256, 0, s>>>(L.cnt, nc.x, nrows, L.rowpad);
+            launch_pdl(row_pad_kernel, dim3((unsigned)rb), dim3(256), 0, s, L.cnt, nc.x, nrows, L.rowpad);
         }
-        scan_reduce_kernel<<<(unsigned)scan_tiles, SCAN_THREADS, 0, s>>>(L.cnt, m, L.sums);
-        scan_sums_kernel<<<1, SCAN_THREADS, 0, s>>>(L.sums, scan_tiles);
-        scan_apply_kernel<<<(unsigned)scan_tiles, SCAN_THREADS, 0, s>>>(L.cnt, m, L.sums, L.cell_start);
-        cell_scatter_kernel<<<blocks, 256, 0, s>>>(L.cell_id, L.cell_rank, n, (long long)n + nrows, L.cell_start,
-                                                   L.slot_atom, overflow);
+        launch_pdl(scan_reduce_kernel, dim3((unsigned)scan_tiles), dim3(SCAN_THREADS), 0, s, (const int*)L.cnt, m,
+                   L.sums);
+        launch_pdl(scan_sums_kernel, dim3(1), dim3(SCAN_THREADS), 0, s, L.sums, scan_tiles);
+        launch_pdl(scan_apply_kernel, dim3((unsigned)scan_tiles), dim3(SCAN_THREADS), 0, s, L.cnt, m,
+                   (const int*)L.sums, L.cell_start);
+        launch_pdl(cell_scatter_kernel, dim3(blocks), dim3(256), 0, s, (const int*)L.cell_id, (const int*)L.cell_rank,
+                   n, (long long)n + nrows, (const int*)L.cell_start, L.slot_atom, overflow);
         const int oblocks = (int)std::min<long long>((m + 255) / 256, (long long)sms * 16);
         if (records)
-            cell_order_pairs_kernel<<<oblocks, 256, 0, s>>>(L.slot_atom, m, nc.x, L.cell_start, L.rowpad, pos4,
-                                                            L.pairs);
+            launch_pdl(cell_order_pairs_kernel, dim3(oblocks), dim3(256), 0, s, (const int*)L.slot_atom, m, nc.x,
+                       (const int*)L.cell_start, (const int*)L.rowpad, pos4, L.pairs);
         else
             cell_order_kernel<<<oblocks, 256, 0, s>>>(L.slot_atom, m, L.cell_start, pos4, L.pos_cell);
         count_launch(records ? 7 : 6);
@@ -1518,7 +1526,8 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
             const double chmax = (double)reach * 1.0001 + 1e-4;
             A.far_cells = nc.x - 2 * ((int)std::ceil(chmax * (double)inv_w.x) + 1);
             const long long blocks = ((recs + 31) / 32 + PD_WARPS - 1) / PD_WARPS;
-            pair_search_duo_kernel<<<(unsigned)std::min<long long>(blocks, 1LL << 30), PD_WARPS * 32, 0, s>>>(A);
+            launch_pdl(pair_search_duo_kernel, dim3((unsigned)std::min<long long>(blocks, 1LL << 30)),
+                       dim3(PD_WARPS * 32), 0, s, A);
         } else if (kind == TESS_LANE_SEARCH) {
             const long long blocks = (ntiles + PL_WARPS - 1) / PL_WARPS;
             pair_search_lane_kernel<<<(unsigned)std::min<long long>(blocks, 1LL << 30), PL_WARPS * 32, 0, s>>>(A);

@@ -41,6 +41,7 @@ __device__ __forceinline__ int block_scan_incl(int v, int* s_warp) {
 __global__ __launch_bounds__(SCAN_THREADS) void scan_reduce_kernel(const int* __restrict__ cnt, long long m,
                                                                    int* __restrict__ sums) {
     __shared__ int s_warp[32];
+    pdl_wait();
     const long long b = (long long)blockIdx.x * SCAN_TILE + (long long)threadIdx.x * SCAN_ITEMS;
     int v = 0;
 #pragma unroll
@@ -52,6 +53,7 @@ __global__ __launch_bounds__(SCAN_THREADS) void scan_reduce_kernel(const int* __
 // exclusive scan of the per-tile sums, one block, any length
 __global__ __launch_bounds__(SCAN_THREADS) void scan_sums_kernel(int* sums, long long nt) {
     __shared__ int s_warp[32];
+    pdl_wait();
     __shared__ int s_carry;
     if (threadIdx.x == 0) s_carry = 0;
     __syncthreads();
@@ -72,6 +74,7 @@ __global__ __launch_bounds__(SCAN_THREADS) void scan_apply_kernel(int* __restric
                                                                   const int* __restrict__ sums,
                                                                   int* __restrict__ cell_start) {
     __shared__ int s_warp[32];
+    pdl_wait();
     const long long b = (long long)blockIdx.x * SCAN_TILE + (long long)threadIdx.x * SCAN_ITEMS;
     int v[SCAN_ITEMS];
     int tot = 0;
@@ -99,9 +102,9 @@ __global__ __launch_bounds__(SCAN_THREADS) void scan_apply_kernel(int* __restric
 inline long long scan_sums_len(long long m) { return (m + SCAN_TILE - 1) / SCAN_TILE + 1; }
 inline void exclusive_scan(int* cnt, long long m, int* sums, int* start, cudaStream_t s) {
     const long long tiles = (m + SCAN_TILE - 1) / SCAN_TILE;
-    scan_reduce_kernel<<<(unsigned)tiles, SCAN_THREADS, 0, s>>>(cnt, m, sums);
-    scan_sums_kernel<<<1, SCAN_THREADS, 0, s>>>(sums, tiles);
-    scan_apply_kernel<<<(unsigned)tiles, SCAN_THREADS, 0, s>>>(cnt, m, sums, start);
+    launch_pdl(scan_reduce_kernel, dim3((unsigned)tiles), dim3(SCAN_THREADS), 0, s, (const int*)cnt, m, sums);
+    launch_pdl(scan_sums_kernel, dim3(1), dim3(SCAN_THREADS), 0, s, sums, tiles);
+    launch_pdl(scan_apply_kernel, dim3((unsigned)tiles), dim3(SCAN_THREADS), 0, s, cnt, m, (const int*)sums, start);
     count_launch(3);
 }
 
