@@ -181,6 +181,7 @@ __global__ __launch_bounds__(SORT_THREADS, TESS_SORT_MINB) void onesweep_pass(co
                                                               float4* __restrict__ pos_sorted,
                                                               const float* __restrict__ pos3, const int* n_dev,
                                                               const int32_t* gate, int want) {
+    pdl_wait();
     constexpr int TILE = SORT_THREADS * ITEMS;
     extern __shared__ __align__(16) unsigned char smem_raw[];
     SortSharedT<ITEMS>& S = *reinterpret_cast<SortSharedT<ITEMS>*>(smem_raw);
@@ -468,6 +469,7 @@ __global__ __launch_bounds__(BK_WARPS * 32, 4) void bucket_local_sort(const unsi
 
 // Zeroes `words` 64-bit words when *gate == want (the fallback's state).
 __global__ void zero_if_kernel(unsigned long long* p, size_t words, const int32_t* gate, int want) {
+    pdl_wait();
     if (*gate != want) return;
     for (size_t k = blockIdx.x * (size_t)blockDim.x + threadIdx.x; k < words; k += (size_t)gridDim.x * blockDim.x)
         p[k] = 0ull;
@@ -547,14 +549,15 @@ static void sfc_sort_launch(const float* pos, int n, tess_box box, int bits, int
         unsigned long long* dst = L.b;
         for (int p = 0; p < npass; ++p) {
             unsigned long long* states = L.states + (size_t)p * tiles * RADIX;
+            // each pass follows a kernel (the keys or the previous pass)
             if (p == npass - 1) {
-                onesweep_pass<true><<<grid, SORT_THREADS, smem, s>>>(
-                    src, nullptr, n, 32 + 8 * p, L.hist + p * RADIX, states, L.counters + p, status, perm,
-                    keys_sorted, reinterpret_cast<float4*>(pos_sorted), pos, nullptr, gate, want);
+                launch_pdl(onesweep_pass<true>, dim3(grid), dim3(SORT_THREADS), smem, s, src, nullptr, n, 32 + 8 * p,
+                           L.hist + p * RADIX, states, L.counters + p, status, perm, keys_sorted,
+                           reinterpret_cast<float4*>(pos_sorted), pos, nullptr, gate, want);
             } else {
-                onesweep_pass<false><<<grid, SORT_THREADS, smem, s>>>(
-                    src, dst, n, 32 + 8 * p, L.hist + p * RADIX, states, L.counters + p, status, nullptr, nullptr,
-                    nullptr, nullptr, nullptr, gate, want);
+                launch_pdl(onesweep_pass<false>, dim3(grid), dim3(SORT_THREADS), smem, s, src, dst, n, 32 + 8 * p,
+                           L.hist + p * RADIX, states, L.counters + p, status, nullptr, nullptr, nullptr, nullptr,
+                           nullptr, gate, want);
             }
             count_launch();
             std::swap(src, dst);
@@ -643,9 +646,9 @@ tess_status sfc_sort(const float* pos, int n, tess_box box, int bits, int curve,
                    B.flag, n, status);
         count_launch(2);
         // a bucket too large for the local sort: the LSD sort, gated on the flag
-        zero_if_kernel<<<sms * 2, 256, 0, s>>>(reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) +
-                                                                                     L.zero_begin),
-                                               L.zero_bytes / 8, B.flag, 1);
+        launch_pdl(zero_if_kernel, dim3(sms * 2), dim3(256), 0, s,
+                   reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + L.zero_begin),
+                   (size_t)(L.zero_bytes / 8), (const int32_t*)B.flag, 1);
         count_launch();
     }
     sfc_sort_launch(pos, n, box, bits, curve, L, perm, keys_sorted, pos_sorted, status, B.flag, 1, s);
