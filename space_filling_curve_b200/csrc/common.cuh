@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 
@@ -109,6 +110,23 @@ inline void launch_pdl(void (*k)(P...), dim3 grid, dim3 block, size_t smem, cuda
 #else
     k<<<grid, block, smem, s>>>(std::forward<A>(args)...);
 #endif
+}
+
+// Zeroes two ranges of 32-bit words (either may be empty): the resets at
+// the start of a call, as a kernel so that the call's chain of launches stays
+// programmatic from its first kernel on (a memset would break it).
+namespace {
+__global__ void zero2_kernel(unsigned* a, size_t na, unsigned* b, size_t nb) {
+    pdl_wait();
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    for (size_t k = (size_t)blockIdx.x * blockDim.x + threadIdx.x; k < na; k += stride) a[k] = 0u;
+    for (size_t k = (size_t)blockIdx.x * blockDim.x + threadIdx.x; k < nb; k += stride) b[k] = 0u;
+}
+}  // namespace
+inline void zero2(unsigned* a, size_t na, unsigned* b, size_t nb, int sms, cudaStream_t s) {
+    const size_t words = na > nb ? na : nb;
+    const unsigned blocks = (unsigned)std::max<size_t>(1, std::min<size_t>((words + 1023) / 1024, (size_t)sms * 4));
+    launch_pdl(zero2_kernel, dim3(blocks), dim3(256), 0, s, a, na, b, nb);
 }
 
 // Runs of equal consecutive values among the valid lanes of a warp (the

@@ -622,17 +622,16 @@ tess_status sfc_sort(const float* pos, int n, tess_box box, int bits, int curve,
     const int sms = sm_count();
     const int blocks = (int)std::min<long long>(((long long)n + BK_THREADS - 1) / BK_THREADS, (long long)sms * 8);
 
-    cudaMemsetAsync(static_cast<char*>(ws) + B.zero_begin, 0, B.zero_bytes, s);
-    if (dev_status) cudaMemsetAsync(dev_status, 0, sizeof(int32_t), s);
+    zero2(reinterpret_cast<unsigned*>(static_cast<char*>(ws) + B.zero_begin), B.zero_bytes / 4,
+          reinterpret_cast<unsigned*>(dev_status), dev_status ? 1 : 0, sms, s);
     {
         StageScope sc(ST_KEYS, s);
-        // after the memsets: a plain launch (programmatic launch only follows kernels)
         if (curve == 0)
-            bucket_keys_kernel<0><<<blocks, BK_THREADS, 0, s>>>(pos, n, scale, Lb, bits, bshift, L.a, B.bcount,
-                                                                 B.rank, status);
+            launch_pdl(bucket_keys_kernel<0>, dim3(blocks), dim3(BK_THREADS), 0, s, pos, n, scale, Lb, bits, bshift,
+                       L.a, B.bcount, B.rank, status);
         else
-            bucket_keys_kernel<1><<<blocks, BK_THREADS, 0, s>>>(pos, n, scale, Lb, bits, bshift, L.a, B.bcount,
-                                                                 B.rank, status);
+            launch_pdl(bucket_keys_kernel<1>, dim3(blocks), dim3(BK_THREADS), 0, s, pos, n, scale, Lb, bits, bshift,
+                       L.a, B.bcount, B.rank, status);
         count_launch();
     }
     {

@@ -1423,7 +1423,7 @@ static bool box_ok(tess_box b) { return finite_pos(b.lx) && finite_pos(b.ly) && 
 
 // x cells per y/z cell width for the two-atoms-per-lane search
 #ifndef TESS_DUO_XFINE
-#define TESS_DUO_XFINE 2.0
+#define TESS_DUO_XFINE 2.5
 #endif
 
 size_t build_neighbors_workspace(int n, tess_box box, float rc, float skin) {
@@ -1468,13 +1468,12 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
     const long long m = g.ncell;
     const long long scan_tiles = (m + SCAN_TILE - 1) / SCAN_TILE;
 
-    cudaMemsetAsync(overflow, 0, sizeof(int32_t), s);
     {
         StageScope sc(ST_CELLS, s);
-        cudaMemsetAsync(L.cnt, 0, sizeof(int) * (size_t)m, s);
+        zero2(reinterpret_cast<unsigned*>(overflow), 1, reinterpret_cast<unsigned*>(L.cnt), (size_t)m, sms, s);
         const int blocks = (int)std::min<long long>(((long long)n + 255) / 256, (long long)sms * 16);
-        // after the memsets: a plain launch (programmatic launch only follows kernels)
-        cell_count_kernel<<<blocks, 256, 0, s>>>(pos4, n, nc, inv_w, Lb, L.cell_id, L.cell_rank, L.cnt, overflow);
+        launch_pdl(cell_count_kernel, dim3(blocks), dim3(256), 0, s, (const float4*)pos4, n, nc, inv_w, Lb, L.cell_id,
+                   L.cell_rank, L.cnt, overflow);
         const long long nrows = (long long)nc.y * nc.z;
         if (records) {
             const long long rb = std::min<long long>((nrows + 7) / 8, (long long)sms * 32);
