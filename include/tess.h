@@ -220,7 +220,9 @@ tess_status tess_hilbert_sort_static(const float* pos, int n, tess_box box, int 
  *                  which cap neighbors are stored is unspecified)
  *   overflow       [1] int32 out: 0, or TESS_DEV_OVERFLOW if any count > cap,
  *                  or'ed with TESS_DEV_BAD_INPUT if a position is outside
- *                  [0, L) or not finite (its list is then unspecified)
+ *                  [0, L) or not finite (its list is then unspecified), and
+ *                  with TESS_DEV_TIMEOUT if the cell-offset scan's wait
+ *                  between blocks gave up (every output is then invalid)
  * Errors: INVALID_ARG, BOX_TOO_SMALL (some L_d < 2 * rs, where the minimum
  * image is not unique), WORKSPACE_TOO_SMALL, CUDA.
  * ------------------------------------------------------------------------- */

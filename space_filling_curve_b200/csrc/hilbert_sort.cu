@@ -124,19 +124,6 @@ constexpr int SORT_WARPS = SORT_THREADS / 32;
 #endif
 constexpr int SORT_ITEMS = TESS_SORT_ITEMS;     // elements per thread in one sort tile
 constexpr int SORT_TILE = SORT_THREADS * SORT_ITEMS;
-constexpr unsigned long long ST_AGG = 1ull << 62;
-constexpr unsigned long long ST_INC = 2ull << 62;
-constexpr unsigned long long ST_VAL = (1ull << 62) - 1ull;
-constexpr int LOOKBACK_SPIN_LIMIT = 1 << 22;
-
-__device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long* p) {
-    unsigned long long v;
-    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_relaxed(unsigned long long* p, unsigned long long v) {
-    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
 
 // Exclusive scan of one value per thread over a 256-thread block.
 __device__ __forceinline__ unsigned block_excl_scan256(unsigned v, unsigned* s_warp) {
@@ -573,8 +560,8 @@ struct BucketLayout {
     int* rank;               // [n] place of each element in its bucket (in the LSD sort's
                              // look-back states, which the fallback zeroes before use)
     int32_t* flag;           // 1: some bucket too large for the local sort
+    unsigned long long* scan_state;   // look-back words of the offset scan
     int* bstart;             // [nb + 1]
-    int* sums;               // scan scratch
     size_t zero_begin, zero_bytes, total;
 };
 
@@ -588,9 +575,9 @@ static BucketLayout bucket_layout(void* ws, int n) {
     B.zero_begin = c.off;
     B.bcount = c.take<int>((size_t)nb);
     B.flag = c.take<int32_t>(1);
+    B.scan_state = c.take<unsigned long long>((size_t)scan_state_len(nb));
     B.zero_bytes = c.off - B.zero_begin;
     B.bstart = c.take<int>((size_t)nb + 1);
-    B.sums = c.take<int>((size_t)scan_sums_len(nb));
     B.total = align_up(c.off, 256);
     // 4 passes x tiles of 2048 x 256 eight-byte states hold n ints
     static_assert((size_t)MAX_PASSES * RADIX * 8 >= (size_t)SORT_TILE * 4, "rank storage");
@@ -636,7 +623,7 @@ tess_status sfc_sort(const float* pos, int n, tess_box box, int bits, int curve,
     }
     {
         StageScope sc(ST_SORT, s);
-        exclusive_scan(B.bcount, nb, B.sums, B.bstart, s);
+        exclusive_scan(B.bcount, nb, B.scan_state, B.bstart, status, s);
         launch_pdl(bucket_scatter_kernel, dim3(blocks), dim3(BK_THREADS), 0, s, (const unsigned long long*)L.a, n,
                    bshift, (const int*)B.bstart, (const int*)B.rank, L.b, status);
         const int lblocks = (int)std::min<long long>((nb + BK_WARPS - 1) / BK_WARPS, (long long)sms * 16);

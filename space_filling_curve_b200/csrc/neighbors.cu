@@ -1389,8 +1389,9 @@ struct NbrLayout {
     int* cell_id;
     int* cell_rank;
     int* cnt;
+    unsigned long long* scan_state;   // look-back words of the offset scan
+    size_t zero_words;                // cnt .. end of scan_state, zeroed per call
     int* cell_start;
-    int* sums;
     int* slot_atom;
     int* rowpad;
     float4* pos_cell;      // cell order as float4, or (same storage) as two-slot records
@@ -1408,8 +1409,10 @@ static NbrLayout nbr_layout(void* ws, int n, const Grid& g) {
     L.cell_id = c.take<int>((size_t)n);
     L.cell_rank = c.take<int>((size_t)n);
     L.cnt = c.take<int>((size_t)m);
+    L.scan_state = c.take<unsigned long long>((size_t)scan_state_len(m));   // zeroed with cnt
+    L.zero_words = (size_t)(reinterpret_cast<char*>(L.scan_state + scan_state_len(m)) -
+                            reinterpret_cast<char*>(L.cnt)) / 4;
     L.cell_start = c.take<int>((size_t)m + 1);
-    L.sums = c.take<int>((size_t)((m + SCAN_TILE - 1) / SCAN_TILE) + 1);
     L.slot_atom = c.take<int>((size_t)slots);
     L.rowpad = c.take<int>((size_t)nrows);
     L.pairs = c.take<SlotPair>((size_t)((slots + 1) / 2));
@@ -1466,11 +1469,10 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
     const float3 inv_w = make_float3(g.inv_w[0], g.inv_w[1], g.inv_w[2]);
     const float3 Lb = make_float3(box.lx, box.ly, box.lz);
     const long long m = g.ncell;
-    const long long scan_tiles = (m + SCAN_TILE - 1) / SCAN_TILE;
 
     {
         StageScope sc(ST_CELLS, s);
-        zero2(reinterpret_cast<unsigned*>(overflow), 1, reinterpret_cast<unsigned*>(L.cnt), (size_t)m, sms, s);
+        zero2(reinterpret_cast<unsigned*>(overflow), 1, reinterpret_cast<unsigned*>(L.cnt), L.zero_words, sms, s);
         const int blocks = (int)std::min<long long>(((long long)n + 255) / 256, (long long)sms * 16);
         launch_pdl(cell_count_kernel, dim3(blocks), dim3(256), 0, s, (const float4*)pos4, n, nc, inv_w, Lb, L.cell_id,
                    L.cell_rank, L.cnt, overflow);
@@ -1479,11 +1481,7 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
             const long long rb = std::min<long long>((nrows + 7) / 8, (long long)sms * 32);
             launch_pdl(row_pad_kernel, dim3((unsigned)rb), dim3(256), 0, s, L.cnt, nc.x, nrows, L.rowpad);
         }
-        launch_pdl(scan_reduce_kernel, dim3((unsigned)scan_tiles), dim3(SCAN_THREADS), 0, s, (const int*)L.cnt, m,
-                   L.sums);
-        launch_pdl(scan_sums_kernel, dim3(1), dim3(SCAN_THREADS), 0, s, L.sums, scan_tiles);
-        launch_pdl(scan_apply_kernel, dim3((unsigned)scan_tiles), dim3(SCAN_THREADS), 0, s, L.cnt, m,
-                   (const int*)L.sums, L.cell_start);
+        exclusive_scan(L.cnt, m, L.scan_state, L.cell_start, overflow, s);
         launch_pdl(cell_scatter_kernel, dim3(blocks), dim3(256), 0, s, (const int*)L.cell_id, (const int*)L.cell_rank,
                    n, (long long)n + nrows, (const int*)L.cell_start, L.slot_atom, overflow);
         const int oblocks = (int)std::min<long long>((m + 255) / 256, (long long)sms * 16);

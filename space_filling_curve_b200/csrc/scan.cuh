@@ -1,7 +1,8 @@
 // scan.cuh -- exclusive scan of an int array of any length on the device
-// (three launches: per-tile sums, a scan of the sums, per-tile scans), used
-// for the cell offsets of the neighbor list and the bucket offsets of the
-// sort.  Internal; each translation unit that includes it gets its own copy.
+// (one launch, decoupled look-back between tiles), used for the cell offsets
+// of the neighbor list and the bucket offsets of the sort.  Also the
+// look-back word format the radix sort shares.  Internal; each translation
+// unit that includes it gets its own copy.
 #pragma once
 
 #include "common.cuh"
@@ -37,75 +38,109 @@ __device__ __forceinline__ int block_scan_incl(int v, int* s_warp) {
     return v + add;
 }
 
-// per-tile sums of the counts
-__global__ __launch_bounds__(SCAN_THREADS) void scan_reduce_kernel(const int* __restrict__ cnt, long long m,
-                                                                   int* __restrict__ sums) {
-    __shared__ int s_warp[32];
-    pdl_wait();
-    const long long b = (long long)blockIdx.x * SCAN_TILE + (long long)threadIdx.x * SCAN_ITEMS;
-    int v = 0;
-#pragma unroll
-    for (int k = 0; k < SCAN_ITEMS; ++k) v += (b + k < m) ? cnt[b + k] : 0;
-    const int tot = block_scan_incl(v, s_warp);
-    if (threadIdx.x == blockDim.x - 1) sums[blockIdx.x] = tot;
+// Decoupled look-back state of one tile: a flag in the top two bits (0: not
+// yet published), the value below it.
+constexpr unsigned long long ST_AGG = 1ull << 62;   // the tile's own total
+constexpr unsigned long long ST_INC = 2ull << 62;   // the tile's inclusive prefix
+constexpr unsigned long long ST_VAL = (1ull << 62) - 1ull;
+constexpr int LOOKBACK_SPIN_LIMIT = 1 << 22;         // polls before a wait gives up
+
+__device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long* p) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_relaxed(unsigned long long* p, unsigned long long v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
-// exclusive scan of the per-tile sums, one block, any length
-__global__ __launch_bounds__(SCAN_THREADS) void scan_sums_kernel(int* sums, long long nt) {
+// One pass: start[c] = cnt[0] + ... + cnt[c - 1] for c <= m.  Each block
+// takes the next tile from a counter (so every lower tile has started),
+// scans it, publishes its total, then looks back over the lower tiles'
+// words -- 32 at a time, one per lane of the last warp -- summing totals
+// until it meets an inclusive prefix, and publishes its own.  A wait that
+// outlasts LOOKBACK_SPIN_LIMIT polls sets TESS_DEV_TIMEOUT and reads the
+// tile as 0, so the kernel always ends.  state: tiles words + 1 (the
+// counter), all zero on entry.
+__global__ __launch_bounds__(SCAN_THREADS) void scan_lookback_kernel(const int* __restrict__ cnt, long long m,
+                                                                     unsigned long long* state,
+                                                                     int* __restrict__ start, int32_t* status) {
     __shared__ int s_warp[32];
+    __shared__ int s_tile, s_excl;
     pdl_wait();
-    __shared__ int s_carry;
-    if (threadIdx.x == 0) s_carry = 0;
+    const long long tiles = (m + SCAN_TILE - 1) / SCAN_TILE;
+    if (threadIdx.x == 0) s_tile = atomicAdd(reinterpret_cast<unsigned*>(state + tiles), 1u);
     __syncthreads();
-    for (long long b = 0; b < nt; b += SCAN_THREADS) {
-        const long long k = b + threadIdx.x;
-        const int v = k < nt ? sums[k] : 0;
-        const int inc = block_scan_incl(v, s_warp);
-        const int carry = s_carry;
-        if (k < nt) sums[k] = carry + inc - v;
-        __syncthreads();
-        if (threadIdx.x == blockDim.x - 1) s_carry = carry + inc;
-        __syncthreads();
-    }
-}
-
-// cell_start[c] = exclusive prefix; cnt[c] reset to 0 for the scatter cursor
-__global__ __launch_bounds__(SCAN_THREADS) void scan_apply_kernel(int* __restrict__ cnt, long long m,
-                                                                  const int* __restrict__ sums,
-                                                                  int* __restrict__ cell_start) {
-    __shared__ int s_warp[32];
-    pdl_wait();
-    const long long b = (long long)blockIdx.x * SCAN_TILE + (long long)threadIdx.x * SCAN_ITEMS;
+    const long long t = s_tile;
+    const long long b = t * SCAN_TILE + (long long)threadIdx.x * SCAN_ITEMS;
+    static_assert(SCAN_ITEMS == 4, "one int4 per thread");
     int v[SCAN_ITEMS];
-    int tot = 0;
+    if (b + SCAN_ITEMS <= m) {
+        const int4 q = *reinterpret_cast<const int4*>(cnt + b);
+        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+    } else {
 #pragma unroll
-    for (int k = 0; k < SCAN_ITEMS; ++k) {
-        v[k] = (b + k < m) ? cnt[b + k] : 0;
-        tot += v[k];
+        for (int k = 0; k < SCAN_ITEMS; ++k) v[k] = (b + k < m) ? cnt[b + k] : 0;
     }
-    const int inc = block_scan_incl(tot, s_warp);
-    int run = sums[blockIdx.x] + inc - tot;
+    const int sum = v[0] + v[1] + v[2] + v[3];
+    const int inc = block_scan_incl(sum, s_warp);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (warp == (int)(blockDim.x >> 5) - 1) {
+        const int tot = __shfl_sync(FULL, inc, 31);
+        if (lane == 0) st_relaxed(state + t, (t == 0 ? ST_INC : ST_AGG) | (unsigned)tot);
+        int excl = 0;
+        bool timed_out = false;
+        for (long long top = t - 1; top >= 0; top -= 32) {
+            const long long p = top - lane;
+            unsigned long long w = ST_INC;   // below tile 0: an inclusive prefix of 0
+            if (p >= 0) {
+                int spins = 0;
+                while (((w = ld_relaxed(state + p)) & ~ST_VAL) == 0) {
+                    if (++spins > LOOKBACK_SPIN_LIMIT) {
+                        timed_out = true;
+                        w = ST_INC;
+                        break;
+                    }
+                    __nanosleep(32);
+                }
+            }
+            const unsigned incl = __ballot_sync(FULL, (w & ~ST_VAL) == ST_INC);
+            const int last = incl ? __ffs(incl) - 1 : 31;   // nearest inclusive word
+            excl += __reduce_add_sync(FULL, lane <= last ? (unsigned)(w & ST_VAL) : 0u);
+            if (incl) break;
+        }
+        if (t > 0 && lane == 0) st_relaxed(state + t, ST_INC | (unsigned)(excl + tot));
+        if (__any_sync(FULL, timed_out) && lane == 0 && status) atomicOr(status, TESS_DEV_TIMEOUT);
+        if (lane == 0) s_excl = excl;
+    }
+    __syncthreads();
+    int run = s_excl + inc - sum;
+    int o[SCAN_ITEMS];
 #pragma unroll
     for (int k = 0; k < SCAN_ITEMS; ++k) {
-        if (b + k < m) {
-            cell_start[b + k] = run;
-            cnt[b + k] = 0;
-        }
+        o[k] = run;
         run += v[k];
     }
-    if (b < m && b + SCAN_ITEMS >= m) cell_start[m] = run;   // the thread holding the last cell
+    if (b + SCAN_ITEMS <= m) {
+        *reinterpret_cast<int4*>(start + b) = make_int4(o[0], o[1], o[2], o[3]);
+    } else {
+#pragma unroll
+        for (int k = 0; k < SCAN_ITEMS; ++k)
+            if (b + k < m) start[b + k] = o[k];
+    }
+    if (b < m && b + SCAN_ITEMS >= m) start[m] = run;   // the thread holding the last element
 }
 
+// Words of look-back state exclusive_scan needs for m elements (zero them
+// before each call).
+inline long long scan_state_len(long long m) { return (m + SCAN_TILE - 1) / SCAN_TILE + 1; }
 
-// Launches the three kernels: start[c] = sum of cnt[0 .. c) for c <= m, and
-// cnt is reset to 0 (a scatter cursor).  sums holds scan_sums_len(m) ints.
-inline long long scan_sums_len(long long m) { return (m + SCAN_TILE - 1) / SCAN_TILE + 1; }
-inline void exclusive_scan(int* cnt, long long m, int* sums, int* start, cudaStream_t s) {
+// start[c] = sum of cnt[0 .. c) for c <= m; cnt and start 16-byte aligned.
+inline void exclusive_scan(const int* cnt, long long m, unsigned long long* state, int* start, int32_t* status,
+                           cudaStream_t s) {
     const long long tiles = (m + SCAN_TILE - 1) / SCAN_TILE;
-    launch_pdl(scan_reduce_kernel, dim3((unsigned)tiles), dim3(SCAN_THREADS), 0, s, (const int*)cnt, m, sums);
-    launch_pdl(scan_sums_kernel, dim3(1), dim3(SCAN_THREADS), 0, s, sums, tiles);
-    launch_pdl(scan_apply_kernel, dim3((unsigned)tiles), dim3(SCAN_THREADS), 0, s, cnt, m, (const int*)sums, start);
-    count_launch(3);
+    launch_pdl(scan_lookback_kernel, dim3((unsigned)tiles), dim3(SCAN_THREADS), 0, s, cnt, m, state, start, status);
+    count_launch();
 }
 
 }  // namespace
