@@ -90,6 +90,7 @@ __global__ __launch_bounds__(KEYS_THREADS) void keys_kernel(const float* __restr
                                                             unsigned* __restrict__ hist, int32_t* status,
                                                             const int32_t* gate, int want) {
     // gate: when given, the kernel runs only if *gate == want
+    pdl_wait();
     if (gate && *gate != want) return;
     __shared__ unsigned sh[MAX_PASSES][RADIX];
     for (int k = threadIdx.x; k < MAX_PASSES * RADIX; k += blockDim.x) (&sh[0][0])[k] = 0u;
@@ -518,11 +519,11 @@ static void sfc_sort_launch(const float* pos, int n, tess_box box, int bits, int
         StageScope sc(ST_KEYS, s);
         const int blocks = (int)std::min<long long>(((long long)n + KEYS_THREADS - 1) / KEYS_THREADS, (long long)sms * 8);
         if (curve == 0)
-            keys_kernel<0><<<blocks, KEYS_THREADS, 0, s>>>(pos, n, scale, make_float3(box.lx, box.ly, box.lz), bits,
-                                                           npass, L.a, L.hist, status, gate, want);
+            launch_pdl(keys_kernel<0>, dim3(blocks), dim3(KEYS_THREADS), 0, s, pos, n, scale,
+                       make_float3(box.lx, box.ly, box.lz), bits, npass, L.a, L.hist, status, gate, want);
         else
-            keys_kernel<1><<<blocks, KEYS_THREADS, 0, s>>>(pos, n, scale, make_float3(box.lx, box.ly, box.lz), bits,
-                                                           npass, L.a, L.hist, status, gate, want);
+            launch_pdl(keys_kernel<1>, dim3(blocks), dim3(KEYS_THREADS), 0, s, pos, n, scale,
+                       make_float3(box.lx, box.ly, box.lz), bits, npass, L.a, L.hist, status, gate, want);
         count_launch();
     }
     {
