@@ -15,6 +15,7 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "hilbert_table.cuh"
 #include "scan.cuh"
 
 namespace tess {
@@ -31,40 +32,6 @@ __device__ __forceinline__ uint32_t spread3(uint32_t v) {
     return v;
 }
 
-// 3-D Hilbert index of grid point (x, y, z) with `bits` bits per axis,
-// following Skilling's transform ("Programming the Hilbert curve", 2004):
-// undo the sub-cube rotations/reflections level by level from the top, Gray
-// encode across axes, fold in the parity of the last axis, and interleave
-// the three words most-significant level first (x's bit highest in each
-// triple).  Written branch-free: each per-level choice between "invert" and
-// "exchange" becomes a mask, and the parity fold is a suffix-XOR scan.
-__device__ __forceinline__ uint32_t hilbert_key(uint32_t x, uint32_t y, uint32_t z, int bits) {
-    for (int l = bits - 1; l >= 1; --l) {
-        const uint32_t low = (1u << l) - 1u;
-        x ^= low & (0u - ((x >> l) & 1u));              // axis 0: invert or no-op
-        uint32_t m = 0u - ((y >> l) & 1u);
-        uint32_t t = (x ^ y) & low & ~m;                // exchange part (bit clear)
-        x ^= (low & m) ^ t;                             // invert (bit set) or exchange
-        y ^= t;
-        m = 0u - ((z >> l) & 1u);
-        t = (x ^ z) & low & ~m;
-        x ^= (low & m) ^ t;
-        z ^= t;
-    }
-    y ^= x;
-    z ^= y;
-    // bit k of the fold = XOR of z's bits above k
-    uint32_t f = z >> 1;
-    f ^= f >> 1;
-    f ^= f >> 2;
-    f ^= f >> 4;
-    f ^= f >> 8;
-    x ^= f;
-    y ^= f;
-    z ^= f;
-    return (spread3(x) << 2) | (spread3(y) << 1) | spread3(z);
-}
-
 // Grid cell of one coordinate: floor(x * scale) with one fp32 multiply,
 // clamped into [0, top]; products below 1 (negative, NaN) give 0.
 __device__ __forceinline__ uint32_t quantize(float x, float scale, uint32_t top) {
@@ -72,6 +39,43 @@ __device__ __forceinline__ uint32_t quantize(float x, float scale, uint32_t top)
     if (!(prod >= 1.0f)) return 0u;
     float fl = floorf(prod);
     return fl >= (float)top ? top : (uint32_t)fl;
+}
+
+// The same index from the Morton code m of the point by the state machine of
+// hilbert_table.cuh: one shared-memory lookup per two levels (and one for
+// the top level when bits is odd).
+constexpr int HT_STATES = kHilbertTables.nstates;
+struct alignas(16) HilbertSmem {
+    uint16_t two[HT_STATES * 64];
+    uint16_t one[HT_STATES * 8];
+};
+static_assert(sizeof(HilbertSmem) % 4 == 0, "copied as words");
+__device__ const HilbertTables d_hilbert_tables = kHilbertTables;
+
+__device__ __forceinline__ void load_hilbert_tables(HilbertSmem& S) {
+    const uint32_t* two = reinterpret_cast<const uint32_t*>(d_hilbert_tables.two);
+    const uint32_t* one = reinterpret_cast<const uint32_t*>(d_hilbert_tables.one);
+    uint32_t* d2 = reinterpret_cast<uint32_t*>(S.two);
+    uint32_t* d1 = reinterpret_cast<uint32_t*>(S.one);
+    for (int k = threadIdx.x; k < HT_STATES * 32; k += blockDim.x) d2[k] = two[k];
+    for (int k = threadIdx.x; k < HT_STATES * 4; k += blockDim.x) d1[k] = one[k];
+}
+
+__device__ __forceinline__ uint32_t hilbert_key_fsm(uint32_t m, int bits, const HilbertSmem& S) {
+    uint32_t st = 0u, key = 0u;
+    int l = bits;
+    if (l & 1) {
+        const uint32_t e = S.one[(m >> (3 * (l - 1))) & 7u];
+        key = e & 7u;
+        st = e >> 6;
+        --l;
+    }
+    for (; l > 0; l -= 2) {
+        const uint32_t e = S.two[(st << 6) | ((m >> (3 * (l - 2))) & 63u)];
+        key = (key << 6) | (e & 63u);
+        st = e >> 6;
+    }
+    return key;
 }
 
 constexpr int KEYS_THREADS = 256;
@@ -93,7 +97,9 @@ __global__ __launch_bounds__(KEYS_THREADS) void keys_kernel(const float* __restr
     pdl_wait();
     if (gate && *gate != want) return;
     __shared__ unsigned sh[MAX_PASSES][RADIX];
+    __shared__ HilbertSmem s_ht;
     for (int k = threadIdx.x; k < MAX_PASSES * RADIX; k += blockDim.x) (&sh[0][0])[k] = 0u;
+    if (CURVE == 0) load_hilbert_tables(s_ht);
     __syncthreads();
     const uint32_t top = (1u << bits) - 1u;
     bool bad = false;
@@ -101,7 +107,8 @@ __global__ __launch_bounds__(KEYS_THREADS) void keys_kernel(const float* __restr
         const float x = pos[3 * (size_t)i], y = pos[3 * (size_t)i + 1], z = pos[3 * (size_t)i + 2];
         bad |= !(x >= 0.0f && x < L.x && y >= 0.0f && y < L.y && z >= 0.0f && z < L.z);
         const uint32_t qx = quantize(x, scale.x, top), qy = quantize(y, scale.y, top), qz = quantize(z, scale.z, top);
-        const uint32_t key = CURVE == 0 ? hilbert_key(qx, qy, qz, bits) : morton_key(qx, qy, qz);
+        const uint32_t mk = morton_key(qx, qy, qz);
+        const uint32_t key = CURVE == 0 ? hilbert_key_fsm(mk, bits, s_ht) : mk;
         elems[i] = ((unsigned long long)key << 32) | (unsigned)i;
         for (int p = 0; p < npass; ++p) atomicAdd(&sh[p][(key >> (8 * p)) & 0xffu], 1u);
     }
@@ -326,6 +333,9 @@ __global__ __launch_bounds__(BK_THREADS) void bucket_keys_kernel(const float* __
                                                                  unsigned long long* __restrict__ elems,
                                                                  int* __restrict__ bcount, int* __restrict__ rank,
                                                                  int32_t* status) {
+    __shared__ HilbertSmem s_ht;
+    if (CURVE == 0) load_hilbert_tables(s_ht);
+    __syncthreads();
     pdl_wait();
     const uint32_t top = (1u << bits) - 1u;
     bool bad = false;
@@ -341,8 +351,9 @@ __global__ __launch_bounds__(BK_THREADS) void bucket_keys_kernel(const float* __
             const uint32_t qx = quantize(x, scale.x, top), qy = quantize(y, scale.y, top),
                            qz = quantize(z, scale.z, top);
             // the default 10 bits with the level loop unrolled at compile time
-            const uint32_t key = CURVE == 0 ? (bits == 10 ? hilbert_key(qx, qy, qz, 10) : hilbert_key(qx, qy, qz, bits))
-                                            : morton_key(qx, qy, qz);
+            const uint32_t mk = morton_key(qx, qy, qz);
+            const uint32_t key = CURVE == 0 ? (bits == 10 ? hilbert_key_fsm(mk, 10, s_ht) : hilbert_key_fsm(mk, bits, s_ht))
+                                            : mk;
             elems[i] = ((unsigned long long)key << 32) | (unsigned)i;
             b = key >> bshift;
         }
@@ -624,7 +635,7 @@ tess_status sfc_sort(const float* pos, int n, tess_box box, int bits, int curve,
     }
     {
         StageScope sc(ST_SORT, s);
-        exclusive_scan(B.bcount, nb, B.scan_state, B.bstart, status, s);
+        exclusive_scan(B.bcount, nb, B.scan_state, B.bstart, status, sms, s);
         launch_pdl(bucket_scatter_kernel, dim3(blocks), dim3(BK_THREADS), 0, s, (const unsigned long long*)L.a, n,
                    bshift, (const int*)B.bstart, (const int*)B.rank, L.b, status);
         const int lblocks = (int)std::min<long long>((nb + BK_WARPS - 1) / BK_WARPS, (long long)sms * 16);
@@ -710,6 +721,9 @@ __global__ __launch_bounds__(RS_THREADS) void resort_classify(const float* __res
                                                               int* __restrict__ tile_cnt, ResortCtl* ctl,
                                                               int32_t* status) {
     __shared__ int s_red[RS_THREADS / 32];
+    __shared__ HilbertSmem s_ht;
+    load_hilbert_tables(s_ht);
+    __syncthreads();
     const long long base = (long long)blockIdx.x * RS_TILE;
     const uint32_t top = (1u << bits) - 1u;
     constexpr int U = RS_TILE / RS_THREADS;
@@ -744,8 +758,8 @@ __global__ __launch_bounds__(RS_THREADS) void resort_classify(const float* __res
         if (k >= n) break;
         const float x = px[u], y = py[u], z = pz[u];
         bad |= !(x >= 0.0f && x < L.x && y >= 0.0f && y < L.y && z >= 0.0f && z < L.z);
-        const uint32_t key =
-            hilbert_key(quantize(x, scale.x, top), quantize(y, scale.y, top), quantize(z, scale.z, top), bits);
+        const uint32_t key = hilbert_key_fsm(
+            morton_key(quantize(x, scale.x, top), quantize(y, scale.y, top), quantize(z, scale.z, top)), bits, s_ht);
         elems[k] = ((unsigned long long)key << 32) | (unsigned)idx[u];
         const bool loc = key >= lo[u] && key <= hi[u];
         local[k] = loc ? 1 : 0;

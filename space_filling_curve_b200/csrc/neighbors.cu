@@ -1481,7 +1481,7 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
             const long long rb = std::min<long long>((nrows + 7) / 8, (long long)sms * 32);
             launch_pdl(row_pad_kernel, dim3((unsigned)rb), dim3(256), 0, s, L.cnt, nc.x, nrows, L.rowpad);
         }
-        exclusive_scan(L.cnt, m, L.scan_state, L.cell_start, overflow, s);
+        exclusive_scan(L.cnt, m, L.scan_state, L.cell_start, overflow, sms, s);
         launch_pdl(cell_scatter_kernel, dim3(blocks), dim3(256), 0, s, (const int*)L.cell_id, (const int*)L.cell_rank,
                    n, (long long)n + nrows, (const int*)L.cell_start, L.slot_atom, overflow);
         const int oblocks = (int)std::min<long long>((m + 255) / 256, (long long)sms * 16);

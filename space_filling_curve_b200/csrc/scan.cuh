@@ -1,5 +1,5 @@
 // scan.cuh -- exclusive scan of an int array of any length on the device
-// (one launch, decoupled look-back between tiles), used for the cell offsets
+// (one launch, decoupled look-back between chunks), used for the cell offsets
 // of the neighbor list and the bucket offsets of the sort.  Also the
 // look-back word format the radix sort shares.  Internal; each translation
 // unit that includes it gets its own copy.
@@ -10,12 +10,14 @@
 namespace tess {
 namespace {
 
-constexpr int SCAN_THREADS = 1024;
-constexpr int SCAN_ITEMS = 4;
-constexpr int SCAN_TILE = SCAN_THREADS * SCAN_ITEMS;
+constexpr int SCAN_THREADS = 512;
+constexpr int SCAN_SUB = SCAN_THREADS * 4;     // elements per block step (one int4 per thread)
+constexpr int SCAN_MAX_CHUNKS = 1024;          // blocks of one scan at most
 
-__device__ __forceinline__ int block_scan_incl(int v, int* s_warp) {
+// Inclusive scan of one value per thread over the block; *tot = block total.
+__device__ __forceinline__ int block_scan_incl(int v, int* s_warp, int* tot) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nw = (int)(blockDim.x >> 5);
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         int y = __shfl_up_sync(FULL, v, o);
@@ -24,7 +26,7 @@ __device__ __forceinline__ int block_scan_incl(int v, int* s_warp) {
     if (lane == 31) s_warp[warp] = v;
     __syncthreads();
     if (warp == 0) {
-        int w = (lane < (int)(blockDim.x >> 5)) ? s_warp[lane] : 0;
+        int w = (lane < nw) ? s_warp[lane] : 0;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             int y = __shfl_up_sync(FULL, w, o);
@@ -34,6 +36,7 @@ __device__ __forceinline__ int block_scan_incl(int v, int* s_warp) {
     }
     __syncthreads();
     const int add = warp > 0 ? s_warp[warp - 1] : 0;
+    *tot = s_warp[nw - 1];
     __syncthreads();
     return v + add;
 }
@@ -54,45 +57,48 @@ __device__ __forceinline__ void st_relaxed(unsigned long long* p, unsigned long 
     asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
-// One pass: start[c] = cnt[0] + ... + cnt[c - 1] for c <= m.  Each block
-// takes the next tile from a counter (so every lower tile has started),
-// scans it, publishes its total, then looks back over the lower tiles'
-// words -- 32 at a time, one per lane of the last warp -- summing totals
-// until it meets an inclusive prefix, and publishes its own.  A wait that
-// outlasts LOOKBACK_SPIN_LIMIT polls sets TESS_DEV_TIMEOUT and reads the
-// tile as 0, so the kernel always ends.  state: tiles words + 1 (the
-// counter), all zero on entry.
+// One launch: start[c] = cnt[0] + ... + cnt[c - 1] for c <= m.  The array
+// is cut into chunks, one per block, taken in order from a counter (so every
+// lower chunk's block has started).  A block sums its chunk, publishes the
+// total, looks back over the lower chunks' words -- 32 at a time, one per
+// lane of warp 0 -- summing totals until it meets an inclusive prefix,
+// publishes its own, then scans its chunk (a second read, from L2).  A wait
+// that outlasts LOOKBACK_SPIN_LIMIT polls sets TESS_DEV_TIMEOUT and reads
+// the chunk as 0, so the kernel always ends.  state: nchunks words + 1 (the
+// counter), all zero on entry; chunk a multiple of 4.
 __global__ __launch_bounds__(SCAN_THREADS) void scan_lookback_kernel(const int* __restrict__ cnt, long long m,
+                                                                     long long chunk, int nchunks,
                                                                      unsigned long long* state,
                                                                      int* __restrict__ start, int32_t* status) {
     __shared__ int s_warp[32];
     __shared__ int s_tile, s_excl;
     pdl_wait();
-    const long long tiles = (m + SCAN_TILE - 1) / SCAN_TILE;
-    if (threadIdx.x == 0) s_tile = atomicAdd(reinterpret_cast<unsigned*>(state + tiles), 1u);
+    if (threadIdx.x == 0) s_tile = atomicAdd(reinterpret_cast<unsigned*>(state + nchunks), 1u);
     __syncthreads();
-    const long long t = s_tile;
-    const long long b = t * SCAN_TILE + (long long)threadIdx.x * SCAN_ITEMS;
-    static_assert(SCAN_ITEMS == 4, "one int4 per thread");
-    int v[SCAN_ITEMS];
-    if (b + SCAN_ITEMS <= m) {
-        const int4 q = *reinterpret_cast<const int4*>(cnt + b);
-        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
-    } else {
-#pragma unroll
-        for (int k = 0; k < SCAN_ITEMS; ++k) v[k] = (b + k < m) ? cnt[b + k] : 0;
-    }
-    const int sum = v[0] + v[1] + v[2] + v[3];
-    const int inc = block_scan_incl(sum, s_warp);
+    const int t = s_tile;
+    const long long beg = (long long)t * chunk, end = beg + chunk < m ? beg + chunk : m;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    if (warp == (int)(blockDim.x >> 5) - 1) {
-        const int tot = __shfl_sync(FULL, inc, 31);
+
+    int sum = 0;
+    for (long long b = beg + 4 * (long long)threadIdx.x; b < end; b += SCAN_SUB) {
+        if (b + 4 <= end) {
+            const int4 q = *reinterpret_cast<const int4*>(cnt + b);
+            sum += q.x + q.y + q.z + q.w;
+        } else {
+            for (long long k = b; k < end; ++k) sum += cnt[k];
+        }
+    }
+    sum = (int)__reduce_add_sync(FULL, (unsigned)sum);
+    if (lane == 0) s_warp[warp] = sum;
+    __syncthreads();
+    if (warp == 0) {
+        const int tot = (int)__reduce_add_sync(FULL, lane < (int)(blockDim.x >> 5) ? (unsigned)s_warp[lane] : 0u);
         if (lane == 0) st_relaxed(state + t, (t == 0 ? ST_INC : ST_AGG) | (unsigned)tot);
         int excl = 0;
         bool timed_out = false;
-        for (long long top = t - 1; top >= 0; top -= 32) {
+        for (long long top = (long long)t - 1; top >= 0; top -= 32) {
             const long long p = top - lane;
-            unsigned long long w = ST_INC;   // below tile 0: an inclusive prefix of 0
+            unsigned long long w = ST_INC;   // below chunk 0: an inclusive prefix of 0
             if (p >= 0) {
                 int spins = 0;
                 while (((w = ld_relaxed(state + p)) & ~ST_VAL) == 0) {
@@ -106,7 +112,7 @@ __global__ __launch_bounds__(SCAN_THREADS) void scan_lookback_kernel(const int* 
             }
             const unsigned incl = __ballot_sync(FULL, (w & ~ST_VAL) == ST_INC);
             const int last = incl ? __ffs(incl) - 1 : 31;   // nearest inclusive word
-            excl += __reduce_add_sync(FULL, lane <= last ? (unsigned)(w & ST_VAL) : 0u);
+            excl += (int)__reduce_add_sync(FULL, lane <= last ? (unsigned)(w & ST_VAL) : 0u);
             if (incl) break;
         }
         if (t > 0 && lane == 0) st_relaxed(state + t, ST_INC | (unsigned)(excl + tot));
@@ -114,32 +120,66 @@ __global__ __launch_bounds__(SCAN_THREADS) void scan_lookback_kernel(const int* 
         if (lane == 0) s_excl = excl;
     }
     __syncthreads();
-    int run = s_excl + inc - sum;
-    int o[SCAN_ITEMS];
+
+    int carry = s_excl;
+    for (long long b0 = beg; b0 < end; b0 += SCAN_SUB) {
+        const long long b = b0 + 4 * (long long)threadIdx.x;
+        int v[4] = {0, 0, 0, 0};
+        if (b + 4 <= end) {
+            const int4 q = *reinterpret_cast<const int4*>(cnt + b);
+            v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+        } else {
 #pragma unroll
-    for (int k = 0; k < SCAN_ITEMS; ++k) {
-        o[k] = run;
-        run += v[k];
-    }
-    if (b + SCAN_ITEMS <= m) {
-        *reinterpret_cast<int4*>(start + b) = make_int4(o[0], o[1], o[2], o[3]);
-    } else {
+            for (int k = 0; k < 4; ++k) v[k] = (b + k < end) ? cnt[b + k] : 0;
+        }
+        const int own = v[0] + v[1] + v[2] + v[3];
+        int tot;
+        const int inc = block_scan_incl(own, s_warp, &tot);
+        int o[4];
+        int run = carry + inc - own;
 #pragma unroll
-        for (int k = 0; k < SCAN_ITEMS; ++k)
-            if (b + k < m) start[b + k] = o[k];
+        for (int k = 0; k < 4; ++k) {
+            o[k] = run;
+            run += v[k];
+        }
+        if (b + 4 <= end) {
+            *reinterpret_cast<int4*>(start + b) = make_int4(o[0], o[1], o[2], o[3]);
+        } else {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                if (b + k < end) start[b + k] = o[k];
+        }
+        if (b < m && b + 4 >= m) start[m] = run;   // the thread holding the last element
+        carry += tot;
     }
-    if (b < m && b + SCAN_ITEMS >= m) start[m] = run;   // the thread holding the last element
+    if (m == 0 && threadIdx.x == 0) start[0] = 0;
+}
+
+// Chunks of a scan of m elements on sms SMs (a multiple of 4 elements each).
+struct ScanPlan {
+    long long chunk;
+    int nchunks;
+};
+inline ScanPlan scan_plan(long long m, int sms) {
+    const long long subs = (m + SCAN_SUB - 1) / SCAN_SUB;
+    const long long want = std::max<long long>(1, std::min<long long>(subs, std::min(sms * 4, SCAN_MAX_CHUNKS)));
+    long long chunk = (m + want - 1) / want;
+    chunk = std::max<long long>(4, (chunk + 3) / 4 * 4);
+    return ScanPlan{chunk, (int)std::max<long long>(1, (m + chunk - 1) / chunk)};
 }
 
 // Words of look-back state exclusive_scan needs for m elements (zero them
 // before each call).
-inline long long scan_state_len(long long m) { return (m + SCAN_TILE - 1) / SCAN_TILE + 1; }
+inline long long scan_state_len(long long m) {
+    return std::max<long long>(1, std::min<long long>((m + SCAN_SUB - 1) / SCAN_SUB, SCAN_MAX_CHUNKS)) + 1;
+}
 
 // start[c] = sum of cnt[0 .. c) for c <= m; cnt and start 16-byte aligned.
 inline void exclusive_scan(const int* cnt, long long m, unsigned long long* state, int* start, int32_t* status,
-                           cudaStream_t s) {
-    const long long tiles = (m + SCAN_TILE - 1) / SCAN_TILE;
-    launch_pdl(scan_lookback_kernel, dim3((unsigned)tiles), dim3(SCAN_THREADS), 0, s, cnt, m, state, start, status);
+                           int sms, cudaStream_t s) {
+    const ScanPlan P = scan_plan(m, sms);
+    launch_pdl(scan_lookback_kernel, dim3((unsigned)P.nchunks), dim3(SCAN_THREADS), 0, s, cnt, m, P.chunk,
+               P.nchunks, state, start, status);
     count_launch();
 }
 
