@@ -223,61 +223,92 @@ __device__ __forceinline__ void put_record(SlotPair* pairs, int r, float4 p0, in
 // positions written as two-slot records (a record whose two slots both
 // belong to the cell, its pad slot included, in one store; a record shared
 // with a neighboring cell half by half), and the pad slot of an odd row
-// (the last slot of the row's last cell) filled.
-__global__ void cell_order_pairs_kernel(const int* __restrict__ slot_atom, long long ncell, int ncx,
-                                        const int* __restrict__ cell_start, const int* __restrict__ rowpad,
-                                        const float4* __restrict__ pos, SlotPair* __restrict__ pairs) {
-    pdl_wait();
-    const long long stride = (long long)gridDim.x * blockDim.x;
+// (the last slot of the row's last cell) filled.  One thread per cell; the
+// range and the first two atom indices are loaded first (most cells hold at
+// most two atoms), the others only for a larger cell.
+struct CellLoad {
+    int b, e, m;
+    bool pad;
+    int v0, v1;   // the cell's first two atom indices (most cells hold at most two)
+};
+
+__device__ __forceinline__ void cell_load(CellLoad& L, long long c, const int* __restrict__ slot_atom, int ncx,
+                                          const int* __restrict__ cell_start, const int* __restrict__ rowpad) {
+    L.b = cell_start[c];
+    L.e = cell_start[c + 1];
+    const long long r = c / ncx;
+    L.pad = c - r * ncx == ncx - 1 && rowpad[r];
+    if (L.pad) --L.e;                  // slot e is the row's pad
+    L.m = L.e - L.b;
+    L.v0 = L.m > 0 ? slot_atom[L.b] : INT_MAX;
+    L.v1 = L.m > 1 ? slot_atom[L.b + 1] : INT_MAX;
+}
+
+__device__ __forceinline__ void cell_emit(const CellLoad& L, const int* __restrict__ slot_atom,
+                                          const float4* __restrict__ pos, SlotPair* __restrict__ pairs) {
     const float nan = __int_as_float(0x7fc00000);
     const float4 pnan = make_float4(nan, nan, nan, nan);
-    for (long long c = (long long)blockIdx.x * blockDim.x + threadIdx.x; c < ncell; c += stride) {
-        const int b = cell_start[c];
-        int e = cell_start[c + 1];
-        const long long r = c / ncx;
-        const bool pad = c - r * ncx == ncx - 1 && rowpad[r];
-        if (pad) --e;                      // slot e is the row's pad
-        const int m = e - b;
-        if (m <= 0) {
-            if (pad) put_slot(pairs, e, nan, nan, nan, -1);
-            continue;
-        }
-        if (m <= 8) {
-            int v[8];
+    const int b = L.b, e = L.e, m = L.m;
+    const bool pad = L.pad;
+    if (m <= 0) {
+        if (pad) put_slot(pairs, e, nan, nan, nan, -1);
+        return;
+    }
+    if (m <= 8) {
+        int v[8];
+        v[0] = L.v0;
+        v[1] = L.v1;
 #pragma unroll
-            for (int k = 0; k < 8; ++k) v[k] = k < m ? slot_atom[b + k] : INT_MAX;
-            sort8(v);
-            // slots b .. e-1 hold v[0 .. m-1], slot e the pad when there is one
-            // (the pad is always the second half of its record)
-            auto emit = [&](auto first) {
-                constexpr int K0 = decltype(first)::value;
-                if (K0 == 1) {             // slot b: the second half of a record shared with the cell before
-                    const float4 p = pos[v[0]];
-                    put_slot(pairs, b, p.x, p.y, p.z, v[0]);
-                }
-#pragma unroll
-                for (int kk = K0; kk < 8; kk += 2) {
-                    if (kk + 1 < m) {
-                        put_record(pairs, (b + kk) >> 1, pos[v[kk]], v[kk], pos[v[kk + 1]], v[kk + 1]);
-                    } else if (kk + 1 == m) {
-                        const float4 p = pos[v[kk]];
-                        if (pad) put_record(pairs, (b + kk) >> 1, p, v[kk], pnan, -1);
-                        else put_slot(pairs, b + kk, p.x, p.y, p.z, v[kk]);   // shared with the cell after
-                    }
-                }
-            };
-            if (b & 1) emit(std::integral_constant<int, 1>{});
-            else emit(std::integral_constant<int, 0>{});
-        } else {
-            for (int s = b; s < e; ++s) {
-                const int i = slot_atom[s];
-                int rk = 0;
-                for (int t = b; t < e; ++t) rk += slot_atom[t] < i;
-                const float4 p = pos[i];
-                put_slot(pairs, b + rk, p.x, p.y, p.z, i);
+        for (int k = 2; k < 8; ++k) v[k] = k < m ? slot_atom[b + k] : INT_MAX;
+        if (m <= 2) cswap(v[0], v[1]);
+        else sort8(v);
+        // slots b .. e-1 hold v[0 .. m-1], slot e the pad when there is one
+        // (the pad is always the second half of its record)
+        auto emit = [&](auto first) {
+            constexpr int K0 = decltype(first)::value;
+            if (K0 == 1) {             // slot b: the second half of a record shared with the cell before
+                const float4 p = pos[v[0]];
+                put_slot(pairs, b, p.x, p.y, p.z, v[0]);
             }
-            if (pad) put_slot(pairs, e, nan, nan, nan, -1);
+#pragma unroll
+            for (int kk = K0; kk < 8; kk += 2) {
+                if (kk + 1 < m) {
+                    put_record(pairs, (b + kk) >> 1, pos[v[kk]], v[kk], pos[v[kk + 1]], v[kk + 1]);
+                } else if (kk + 1 == m) {
+                    const float4 p = pos[v[kk]];
+                    if (pad) put_record(pairs, (b + kk) >> 1, p, v[kk], pnan, -1);
+                    else put_slot(pairs, b + kk, p.x, p.y, p.z, v[kk]);   // shared with the cell after
+                }
+            }
+        };
+        if (b & 1) emit(std::integral_constant<int, 1>{});
+        else emit(std::integral_constant<int, 0>{});
+    } else {
+        for (int s = b; s < e; ++s) {
+            const int i = slot_atom[s];
+            int rk = 0;
+            for (int t = b; t < e; ++t) rk += slot_atom[t] < i;
+            const float4 p = pos[i];
+            put_slot(pairs, b + rk, p.x, p.y, p.z, i);
         }
+        if (pad) put_slot(pairs, e, nan, nan, nan, -1);
+    }
+}
+
+// 32 registers, so that 8 blocks of 256 threads fit an SM: the kernel waits
+// on its chain of dependent loads (range, indices, positions), and more
+// threads in flight beat holding two cells per thread.
+__global__ __launch_bounds__(256, 8) void cell_order_pairs_kernel(const int* __restrict__ slot_atom, long long ncell,
+                                                                 int ncx, const int* __restrict__ cell_start,
+                                                                 const int* __restrict__ rowpad,
+                                                                 const float4* __restrict__ pos,
+                                                                 SlotPair* __restrict__ pairs) {
+    pdl_wait();
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long c = (long long)blockIdx.x * blockDim.x + threadIdx.x; c < ncell; c += stride) {
+        CellLoad L;
+        cell_load(L, c, slot_atom, ncx, cell_start, rowpad);
+        cell_emit(L, slot_atom, pos, pairs);
     }
 }
 

@@ -287,6 +287,21 @@ def test_neighbors_dense_rows_drain_the_buffer():
         _check_list(p, (L, L, L), 5.0, 0.5, 512, method="brute", search=search)
 
 
+def test_neighbors_clustered_cells():
+    # a dense blob: cells of far more than 8 atoms, and runs of 32 cells that
+    # hold more slots than the record ordering stages per warp
+    rng = np.random.default_rng(11)
+    L = 30.0
+    p = np.zeros((3000, 4), np.float32)
+    p[:1500, :3] = rng.uniform(0, 3.0, (1500, 3)) + 12.0
+    p[1500:, :3] = rng.uniform(0, L, (1500, 3))
+    p = synth.band_clean(p, (L, L, L), 4.5)
+    p = p[oracle.hilbert_sort(p, (L, L, L), 10)[0]]
+    for search in SEARCHES:
+        _check_list(p, (L, L, L), 4.0, 0.5, 2048, method="brute", search=search)
+    _check_list(p[::-1].copy(), (L, L, L), 4.0, 0.5, 2048, method="brute", search="lane2")
+
+
 def test_neighbors_box_errors():
     tess = _tess()
     p = _dev(np.zeros((10, 4), np.float32))
