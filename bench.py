@@ -718,13 +718,19 @@ def _sample_system(budget_steps: int):
 def cpu_baseline(args):
     import oracle
     s = _sample_system(1)
+    # repeated rebuilds of the sample for about 10 s of CPU work
+    reps = 0
     t = time.perf_counter()
-    _oracle_step(s)
-    dt = time.perf_counter() - t
-    return {"value": s.n / dt, "unit": "atoms/s", "cores": oracle.get_threads(), "kind": "oracle",
-            "sample": "one full rebuild (Hilbert sort, cell-list Verlet list) of %s "
+    while True:
+        _oracle_step(s)
+        reps += 1
+        dt = time.perf_counter() - t
+        if dt >= 10.0 or reps >= 100:
+            break
+    return {"value": s.n * reps / dt, "unit": "atoms/s", "cores": oracle.get_threads(), "kind": "oracle",
+            "sample": "%d full rebuilds (Hilbert sort, cell-list Verlet list) of %s "
                       "(%d atoms, same generator and rc/skin/cap/F family as the 10.24M workload), %.1f s"
-                      % (s.name, s.n, dt)}
+                      % (reps, s.name, s.n, dt)}
 
 
 def run_reference(args, world, rank):
