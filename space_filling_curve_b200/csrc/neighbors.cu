@@ -1201,13 +1201,15 @@ __global__ __launch_bounds__(PD_WARPS * 32, TESS_PD_MINB) void pair_search_duo_k
     const float nan = __int_as_float(0x7fc00000);
     const unsigned vote_at = (unsigned)(PD_BUF - 2 * PD_CHUNK) * 128u;
 
-    // full groups of 8 staged indices to the row, the remainder moved to the
-    // front of the column
+    // full groups of 8 staged indices to the row: the newest ones, so that
+    // the remainder (the oldest, fewer than 8) stays at the front of the
+    // column and nothing moves (the order within a row is free)
     auto drain = [&](int* buf, unsigned base, unsigned& w, int& done, int* row) {
         const int pend = (int)((w - base) >> 7);
         const int groups = pend >> 3;
+        const int rest = pend - groups * 8;
         for (int g = 0; g < groups; ++g) {
-            const int* src = buf + g * 256;
+            const int* src = buf + (rest + g * 8) * 32;
             if (A.vec8 && done + 8 <= cap) {
                 st_global_v8(row + done, src[0], src[32], src[64], src[96], src[128], src[160], src[192], src[224]);
             } else {
@@ -1216,9 +1218,6 @@ __global__ __launch_bounds__(PD_WARPS * 32, TESS_PD_MINB) void pair_search_duo_k
             }
             done += 8;
         }
-        const int rest = pend - groups * 8;
-        if (groups > 0)
-            for (int e = 0; e < rest; ++e) buf[e * 32] = buf[(groups * 8 + e) * 32];
         w = base + 128u * (unsigned)rest;
     };
     // the last staged indices (a group completed with pads where the row is
