@@ -622,12 +622,14 @@ __global__ __launch_bounds__(TM_WARPS * 32, 4) void pair_tile_kernel(PairArgs A)
         int pend = 0;      // indices waiting in this lane's buffer
         int ncand = 0;     // staged candidates (warp-uniform)
 
-        // write the complete groups of TM_GROUP buffered indices to the row;
-        // the rest moves to the front of the buffer
+        // the complete groups of TM_GROUP buffered indices to the row, the
+        // newest first: the remainder (the oldest) stays at the front of the
+        // buffer (the order within a row is free)
         auto drain = [&]() {
             const int groups = pend / TM_GROUP;
+            const int rest = pend - groups * TM_GROUP;
             for (int gi = 0; gi < groups; ++gi) {
-                const int* src = buf + gi * TM_GROUP * 32;
+                const int* src = buf + (rest + gi * TM_GROUP) * 32;
                 if (VW == 8 && done + TM_GROUP <= cap) {
                     st_global_v8(row + done, src[0], src[32], src[64], src[96], src[128], src[160], src[192],
                                  src[224]);
@@ -641,8 +643,6 @@ __global__ __launch_bounds__(TM_WARPS * 32, 4) void pair_tile_kernel(PairArgs A)
                 }
                 done += TM_GROUP;
             }
-            const int rest = pend - groups * TM_GROUP;
-            for (int e = 0; e < rest; ++e) buf[e * 32] = buf[(groups * TM_GROUP + e) * 32];
             pend = rest;
         };
 
@@ -939,11 +939,14 @@ __global__ __launch_bounds__(PL_WARPS * 32, 6) void pair_search_lane_kernel(Pair
 
         int done = 0;
         unsigned wsa = buf_sa;
+        // full groups to the row, the newest first: the remainder (the oldest)
+        // stays at the front of the column (the order within a row is free)
         auto drain = [&](bool all) {
             const int pend = (int)((wsa - buf_sa) >> 7);
             const int groups = pend / PS_GROUP;
+            const int rest = pend - groups * PS_GROUP;
             for (int gi = 0; gi < groups; ++gi) {
-                const int* src = buf + gi * PS_GROUP * 32;
+                const int* src = buf + (rest + gi * PS_GROUP) * 32;
                 if (done + PS_GROUP <= cap && A.vec_rows) {
                     const int4 a = make_int4(src[0], src[32], src[64], src[96]);
                     const int4 b = make_int4(src[128], src[160], src[192], src[224]);
@@ -955,14 +958,12 @@ __global__ __launch_bounds__(PL_WARPS * 32, 6) void pair_search_lane_kernel(Pair
                 }
                 done += PS_GROUP;
             }
-            const int rest = pend - groups * PS_GROUP;
             if (all) {
                 for (int e = 0; e < rest; ++e)
-                    if (done + e < cap) row[done + e] = buf[(groups * PS_GROUP + e) * 32];
+                    if (done + e < cap) row[done + e] = buf[e * 32];
                 done += rest;
                 wsa = buf_sa;
             } else {
-                for (int e = 0; e < rest; ++e) buf[e * 32] = buf[(groups * PS_GROUP + e) * 32];
                 wsa = buf_sa + 128u * (unsigned)rest;
             }
         };
