@@ -1072,7 +1072,7 @@ __global__ __launch_bounds__(PL_WARPS * 32, 6) void pair_search_lane_kernel(Pair
 #define TESS_PD_WARPS 4
 #endif
 #ifndef TESS_PD_BUF
-#define TESS_PD_BUF 24
+#define TESS_PD_BUF 20
 #endif
 #ifndef TESS_PD_GROUP
 #define TESS_PD_GROUP 1
@@ -1175,7 +1175,7 @@ __device__ __forceinline__ void bulk_store(int* dst, unsigned src, unsigned byte
 }
 
 #ifndef TESS_PD_MINB
-#define TESS_PD_MINB 6
+#define TESS_PD_MINB 7
 #endif
 
 __global__ __launch_bounds__(PD_WARPS * 32, TESS_PD_MINB) void pair_search_duo_kernel(PairArgs A) {
