@@ -371,8 +371,9 @@ def run_cuda(args, world, rank, local):
     # e2e: through the C ABI with host buffers (pinned); every rebuild's
     # copies (positions in; perm, counts and the status words out -- the list
     # itself stays on the device for the steps that use it) are inside the
-    # timed region, issued on a second stream with double buffers so that
-    # they overlap the neighboring rebuilds, as a stream-ordered caller would
+    # timed region, issued on two copy streams (one per direction) with double
+    # buffers so that they overlap the neighboring rebuilds and each other, as
+    # a stream-ordered caller would
     e2e_val, e2e_steps = _e2e(step, s, args.steps, world, dev)
 
     nbytes = _algorithmic_bytes(s.n, mean_count, s.F)
@@ -473,7 +474,8 @@ def _e2e(step, s, steps, world, dev):
     st_counts = [torch.empty_like(step.counts) for _ in range(2)]
     st_flags = [torch.empty(2, dtype=torch.int32, device=dev) for _ in range(2)]
     cs = torch.cuda.current_stream()
-    xs = torch.cuda.Stream(device=dev)
+    xs = torch.cuda.Stream(device=dev)       # host -> device copies
+    ys = torch.cuda.Stream(device=dev)       # device -> host copies (the other direction of the link)
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_out = [torch.cuda.Event() for _ in range(2)]
     ev_read = [torch.cuda.Event() for _ in range(2)]
@@ -497,16 +499,19 @@ def _e2e(step, s, steps, world, dev):
         st_flags[b][0:1].copy_(step.overflow)
         st_flags[b][1:2].copy_(step.status)
         ev_out[b].record(cs)
-        with torch.cuda.stream(xs):
-            xs.wait_event(ev_out[b])
+        with torch.cuda.stream(ys):
+            ys.wait_event(ev_out[b])
             host_perm[b].copy_(st_perm[b], non_blocking=True)
             host_counts[b].copy_(st_counts[b], non_blocking=True)
             host_flags[b].copy_(st_flags[b], non_blocking=True)
-            ev_read[b].record(xs)
-            if t + 2 < e2e_steps:                  # rebuild t has read pos_in[b]: load t+2's positions
+            ev_read[b].record(ys)
+        if t + 2 < e2e_steps:                      # rebuild t has read pos_in[b]: load t+2's positions
+            with torch.cuda.stream(xs):
+                xs.wait_event(ev_out[b])
                 pos_in[b].copy_(host_pos, non_blocking=True)
                 ev_in[b].record(xs)
     cs.wait_stream(xs)
+    cs.wait_stream(ys)
     e1.record(cs)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
