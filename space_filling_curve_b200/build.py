@@ -11,7 +11,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libtess.so")
 SOURCES = ["capi.cu", "hilbert_sort.cu", "neighbors.cu", "step.cu", "static_scratch.cu", "step_graph.cu"]
-HEADERS = ["common.cuh", "scan.cuh"]
+HEADERS = ["common.cuh", "scan.cuh", "hilbert_table.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
