@@ -479,7 +479,9 @@ def _e2e(step, s, steps, world, dev):
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_out = [torch.cuda.Event() for _ in range(2)]
     ev_read = [torch.cuda.Event() for _ in range(2)]
-    e2e_steps = max(1, steps)
+    # at least 30 rebuilds, so that filling and draining the copy pipeline
+    # (the first positions in, the last results out) weighs as in a long run
+    e2e_steps = max(30, steps)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(cs)
