@@ -288,8 +288,8 @@ def test_neighbors_dense_rows_drain_the_buffer():
 
 
 def test_neighbors_clustered_cells():
-    # a dense blob: cells of far more than 8 atoms, and runs of 32 cells that
-    # hold more slots than the record ordering stages per warp
+    # a dense blob: cells of far more than 8 atoms (the record ordering ranks
+    # those by counting instead of its sorting network)
     rng = np.random.default_rng(11)
     L = 30.0
     p = np.zeros((3000, 4), np.float32)
