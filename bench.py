@@ -191,17 +191,23 @@ class Step:
         import torch
         return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
 
-    def rebuild(self, pos3=None):
-        """The timed unit: Hilbert sort, then the padded neighbor list."""
+    def rebuild(self, pos3=None, perm=None, counts=None, overflow=None, status=None):
+        """The timed unit: Hilbert sort, then the padded neighbor list.  The
+        outputs a caller copies out (perm, counts, the two status words) may
+        be given as other buffers."""
         tess, s, P, st = self.tess, self.s, self._ptr, self._stream()
         pos3 = self.pos3 if pos3 is None else pos3
+        perm = self.perm if perm is None else perm
+        counts = self.counts if counts is None else counts
+        overflow = self.overflow if overflow is None else overflow
+        status = self.status if status is None else status
         if self.sort_fn is not None:
             c = self.sort_fn(P(pos3), self.n, s.box, 10, P(self.ws_sort), self.ws_sort.numel(),
-                             P(self.perm), P(self.keys), P(self.pos_sorted), P(self.status), st)
+                             P(perm), P(self.keys), P(self.pos_sorted), P(status), st)
             assert c == 0, c
         c = tess.tess_build_neighbors(P(self.pos_sorted), self.n, s.box, s.rc, s.skin, s.cap, self.flags,
-                                      P(self.ws_nbr), self.ws_nbr.numel(), P(self.nbr), P(self.counts),
-                                      P(self.overflow), st)
+                                      P(self.ws_nbr), self.ws_nbr.numel(), P(self.nbr), P(counts),
+                                      P(overflow), st)
         assert c == 0, c
 
     def per_step(self):
@@ -493,13 +499,11 @@ def _e2e(step, s, steps, world, dev):
     for t in range(e2e_steps):
         b = t % 2
         cs.wait_event(ev_in[b])
-        step.rebuild(pos3=pos_in[b])
         if t >= 2:
-            cs.wait_event(ev_read[b])            # rebuild t-2's results have left the staging buffers
-        st_perm[b].copy_(step.perm)
-        st_counts[b].copy_(step.counts)
-        st_flags[b][0:1].copy_(step.overflow)
-        st_flags[b][1:2].copy_(step.status)
+            cs.wait_event(ev_read[b])            # rebuild t-2's results have left output buffer set b
+        # the rebuild writes its perm, counts and status words straight into buffer set b
+        step.rebuild(pos3=pos_in[b], perm=st_perm[b], counts=st_counts[b], overflow=st_flags[b][0:1],
+                     status=st_flags[b][1:2])
         ev_out[b].record(cs)
         with torch.cuda.stream(ys):
             ys.wait_event(ev_out[b])
