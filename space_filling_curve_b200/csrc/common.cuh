@@ -127,6 +127,7 @@ inline void zero2(unsigned* a, size_t na, unsigned* b, size_t nb, int sms, cudaS
     const size_t words = na > nb ? na : nb;
     const unsigned blocks = (unsigned)std::max<size_t>(1, std::min<size_t>((words + 1023) / 1024, (size_t)sms * 4));
     launch_pdl(zero2_kernel, dim3(blocks), dim3(256), 0, s, a, na, b, nb);
+    count_launch();
 }
 
 // Runs of equal consecutive values among the valid lanes of a warp (the

@@ -1521,7 +1521,7 @@ tess_status build_neighbors(const float* pos, int n, tess_box box, float rc, flo
                        (const int*)L.cell_start, (const int*)L.rowpad, pos4, L.pairs);
         else
             cell_order_kernel<<<oblocks, 256, 0, s>>>(L.slot_atom, m, L.cell_start, pos4, L.pos_cell);
-        count_launch(records ? 7 : 6);
+        count_launch(records ? 4 : 3);   // count, row pads, scatter, ordering (zero2 and the scan count themselves)
     }
     {
         StageScope sc(ST_PAIRS, s);
